@@ -1,0 +1,151 @@
+"""Workload shapes and seeded synthetic inputs.
+
+This module holds no arithmetic of the method: only the decoder shapes the
+pages describe and seeded random draws.  Both the CUDA path and the CPU oracle
+are fed from here (the oracle through host copies of the same tensors), and
+nothing here quantizes, dequantizes or multiplies.
+
+Shapes:
+  * "Qwen3-VL (2B / 4B / 8B, vision-language) -- Core AI", architecture
+    paragraph and size table: vocab 151 936, head_dim 128, 8 KV heads,
+    SwiGLU; 2B = 28 layers, hidden 2048, 16 q-heads, SwiGLU 6144; 4B = 36
+    layers, hidden 2560, 32 q-heads, SwiGLU 9728; 8B = 36 layers, hidden 4096,
+    32 q-heads, SwiGLU 12288.  2B/4B tie the LM head to the embedding, 8B is
+    untied ("Qwen3-VL 4B & 8B -- Core ML stateful", Gotchas).
+  * "Qwen3.8-27B (VLM: text decoder + vision path) -- Core AI", intro: 64
+    layers, 24 q / 4 KV heads of head_dim 256, a swish output gate (a q-sized
+    projection), dense MLP 17408, untied 248 320-vocab head.  The page gives no
+    hidden size; 5120 is taken, and every layer gets full-attention shapes.
+
+Synthetic data: weights are fp32 N(0, 0.02), activations fp16 = RNE(fp32
+N(0, 1)), drawn with torch.Generator on the requested device.  The pages use
+real checkpoints and prompts; these seeded tensors stand in for them.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import List, Optional, Tuple
+
+import torch
+
+W_STD = 0.02
+
+# proj ids used in weight seeds
+PROJ_ID = {"q": 0, "k": 1, "v": 2, "o": 3, "gate": 4, "up": 5, "down": 6,
+           "outgate": 7, "head": 15}
+
+
+@dataclass(frozen=True)
+class Decoder:
+    """Decoder shape: the weight matrices one decode token reads."""
+    name: str
+    seed_id: int
+    layers: int
+    hidden: int
+    q_dim: int
+    kv_dim: int
+    inter: int
+    vocab: int
+    tied_head: bool
+    out_gate: bool = False  # extra q-sized projection fused with q
+
+    # --- fused row-concatenations used by the sweep -----------------------
+    def qkv_parts(self) -> List[Tuple[str, int]]:
+        """Row blocks of the fused q|(outgate)|k|v projection, in order."""
+        parts = [("q", self.q_dim)]
+        if self.out_gate:
+            parts.append(("outgate", self.q_dim))
+        parts += [("k", self.kv_dim), ("v", self.kv_dim)]
+        return parts
+
+    @property
+    def qkv_rows(self) -> int:
+        return sum(n for _, n in self.qkv_parts())
+
+    def layer_matrices(self) -> List[Tuple[str, int, int]]:
+        """(name, rows N, cols K) of every weight matrix of one layer."""
+        mats = [(p, n, self.hidden) for p, n in self.qkv_parts()]
+        mats += [("o", self.hidden, self.q_dim),
+                 ("gate", self.inter, self.hidden),
+                 ("up", self.inter, self.hidden),
+                 ("down", self.hidden, self.inter)]
+        return mats
+
+    def all_matrices(self) -> List[Tuple[int, str, int, int]]:
+        """(layer or -1 for the head, name, N, K) for the whole sweep."""
+        out = []
+        for l in range(self.layers):
+            out += [(l, n, r, c) for n, r, c in self.layer_matrices()]
+        out.append((-1, "head", self.vocab, self.hidden))
+        return out
+
+    def weight_count(self, include_head: bool = True) -> int:
+        body = self.layers * sum(r * c for _, r, c in self.layer_matrices())
+        return body + (self.vocab * self.hidden if include_head else 0)
+
+    # --- seeds ------------------------------------------------------------
+    def weight_seed(self, layer: int, proj: str) -> int:
+        if proj == "head":
+            return 1000 * self.seed_id + PROJ_ID["head"]
+        return 1000 * self.seed_id + 16 * layer + PROJ_ID[proj]
+
+    def x_seed(self, layer: int) -> int:
+        """Seed of the fresh fp16 activation of layer ``layer`` (-1: head)."""
+        return 500000 + 1000 * self.seed_id + (layer if layer >= 0 else 999)
+
+    def chunk_seed(self, layer: int) -> int:
+        """Seed of the S=16 activation chunk of layer ``layer`` (-1: head)."""
+        return 600000 + 1000 * self.seed_id + (layer if layer >= 0 else 999)
+
+
+QWEN3VL_2B = Decoder("qwen3vl-2b", 2, layers=28, hidden=2048, q_dim=2048,
+                     kv_dim=1024, inter=6144, vocab=151936, tied_head=True)
+QWEN3VL_4B = Decoder("qwen3vl-4b", 3, layers=36, hidden=2560, q_dim=4096,
+                     kv_dim=1024, inter=9728, vocab=151936, tied_head=True)
+QWEN3VL_8B = Decoder("qwen3vl-8b", 4, layers=36, hidden=4096, q_dim=4096,
+                     kv_dim=1024, inter=12288, vocab=151936, tied_head=False)
+DENSE_27B = Decoder("dense-27b", 5, layers=64, hidden=5120, q_dim=6144,
+                    kv_dim=1024, inter=17408, vocab=248320, tied_head=False,
+                    out_gate=True)
+
+DECODERS = {d.name: d for d in (QWEN3VL_2B, QWEN3VL_4B, QWEN3VL_8B, DENSE_27B)}
+
+# Single 2048 x 2048 int8 block-32 GEMV: W seed 0, x seed 1.
+GEMV_2048 = dict(name="gemv-2048", n=2048, k=2048, w_seed=0, x_seed=1)
+
+
+# ----------------------------------------------------------- generators ----
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def weight_fp32(n: int, k: int, seed: int, device="cpu") -> torch.Tensor:
+    """fp32 N(0, 0.02) weight [n, k] (row-major, Linear.weight order)."""
+    w = torch.randn((n, k), generator=_gen(seed, device), device=device,
+                    dtype=torch.float32)
+    return w.mul_(W_STD)
+
+
+def act_fp16(shape, seed: int, device="cpu", std: float = 1.0) -> torch.Tensor:
+    """fp16 activation: fp32 N(0, std) rounded to fp16 (torch's RNE cast)."""
+    if isinstance(shape, int):
+        shape = (shape,)
+    x = torch.randn(shape, generator=_gen(seed, device), device=device,
+                    dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(torch.float16)
+
+
+def sample_rows(n: int, count: int, seed: int) -> torch.Tensor:
+    """Sorted distinct row indices for sampled full-size checks, always
+    including the first and last row (int64, CPU)."""
+    g = _gen(seed, "cpu")
+    if count >= n:
+        return torch.arange(n, dtype=torch.int64)
+    idx = torch.randperm(n, generator=g)[: max(count - 2, 0)]
+    idx = torch.cat([idx, torch.tensor([0, n - 1])])
+    return torch.unique(idx).sort().values

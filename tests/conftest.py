@@ -1,0 +1,21 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line(
+        "markers", "gpu: needs a CUDA GPU (B200, sm_100a) and the built libqgemv.so")
+
+
+@pytest.fixture(scope="session")
+def cuda():
+    """The CUDA device for -m gpu tests; fails (never skips) without one."""
+    import torch
+    assert torch.cuda.is_available(), "gpu-marked test run without a CUDA device"
+    return torch.device("cuda:0")
