@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Benchmark the decode weight sweep through libqgemv.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+A step is one full sweep of the decoder's weights (every layer's q|k|v, o,
+gate/up + SwiGLU and down, then the LM head + argmax) replayed from a CUDA
+graph.  The default workload is the Qwen3-VL-2B-shaped int8 block-32 S=1
+sweep (1.83 GB per sweep, far larger than the 126 MB L2, so no flush is
+needed between steps).  N > 1 runs one replica per GPU (launch with torchrun):
+decode sweeps are independent, so nothing is exchanged and the time is the
+max over ranks.
+
+`--impl reference` times the CPU oracle (fp64 dequantize-then-matvec, on the
+host's cores) on a bounded sample of the same workload, for the driver's
+ratio; it never touches the GPU.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "weight-stream GB/s (% of HBM peak) and decode sweeps/s, S=1 int8 block-32"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+
+# name -> (decoder, body format, head format, S)
+WORKLOADS = {
+    "qwen3vl-2b": ("QWEN3VL_2B", 0, 0, 1),
+    "qwen3vl-4b": ("QWEN3VL_4B", 0, 0, 1),
+    "qwen3vl-4b-int4": ("QWEN3VL_4B", 1, 0, 1),
+    "qwen3vl-8b": ("QWEN3VL_8B", 0, 0, 1),
+    "qwen3vl-8b-s16": ("QWEN3VL_8B", 0, 0, 16),
+    "dense-27b": ("DENSE_27B", 0, 0, 1),
+}
+DEFAULT_WORKLOAD = "qwen3vl-2b"
+FMT_NAME = {0: "int8 block-32", 1: "int4 group-64"}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--graph-sweeps", type=int, default=1,
+                    help="sweeps captured per CUDA graph (steps are rounded up to a multiple)")
+    ap.add_argument("--cpu-budget-s", type=float, default=10.0,
+                    help="seconds of oracle work for the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    return a
+
+
+# --------------------------------------------------------------- helpers ----
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The maximum of `value` over all ranks (identity when world == 1)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(units_per_rank: float, elapsed_s_max: float, world: int) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest
+    rank's time (weak scaling: each rank runs the same fixed work)."""
+    return units_per_rank * world / elapsed_s_max
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def csrc_digest() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "int4_quantized_decode_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            for line in f:
+                if line.startswith("#") or "=" not in line:
+                    continue
+                kv = dict(p.split("=", 1) for p in line.split())
+                if (kv.get("kernel") == kernel and kv.get("workload") == workload
+                        and kv.get("csrc") == csrc_digest()):
+                    return float(kv["bytes_per_launch"])
+    except (OSError, ValueError, KeyError):
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.out = tempfile.NamedTemporaryFile("w+", delete=False, suffix=".csv")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu)], stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        rows = [r.strip().split(", ") for r in self.out.read().splitlines() if r.strip()]
+        self.out.close()
+        os.unlink(self.out.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------- CPU oracle ----
+
+def oracle_sample(dec, body_fmt, S, budget_s, max_passes=None):
+    """Time the CPU oracle (test infrastructure) on a bounded sample of the
+    workload: one decoder layer's projections, quantized by the oracle from
+    CPU-drawn weights, run as fp64 dequantize-then-matvec (+ SwiGLU) for S
+    tokens, repeated until `budget_s` (or `max_passes`).  Returns
+    (passes, seconds, bytes per pass, threads)."""
+    import numpy as np
+
+    import oracle
+    from int4_quantized_decode_b200 import workloads as wl
+
+    fmt = body_fmt
+    qz = oracle.quantize_block32 if fmt == 0 else oracle.quantize_int4_g64
+    mats = {}
+    for name, n, k in dec.layer_matrices():
+        w = wl.weight_fp32(n, k, dec.weight_seed(0, name), "cpu").numpy()
+        q = qz(w)
+        mats[name] = (q[0], q[1], q[2] if fmt == 1 else None, k)
+    nbytes = sum(c.nbytes + s.nbytes + (b.nbytes if b is not None else 0)
+                 for c, s, b, _ in mats.values())
+    xs = [wl.act_fp16(dec.hidden, dec.x_seed(0) + s, "cpu").numpy().view(np.uint16)
+          for s in range(S)]
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        for x in xs:
+            for name in ("q", "k", "v") + (("outgate",) if dec.out_gate else ()):
+                c, s, b, _ = mats[name]
+                y, _ = oracle.matvec(fmt, c, s, b, x)
+            c, s, b, _ = mats["o"]
+            oracle.matvec(fmt, c, s, b, xs[0] if dec.q_dim == dec.hidden else
+                          np.resize(x, dec.q_dim))
+            g, mg = oracle.matvec(fmt, *mats["gate"][:3], x)
+            u, mu = oracle.matvec(fmt, *mats["up"][:3], x)
+            h, _ = oracle.swiglu(g, u, mg, mu, oracle.GEMV_TOL)
+            h16 = h.astype(np.float16).view(np.uint16)
+            oracle.matvec(fmt, *mats["down"][:3], h16)
+        passes += 1
+        el = time.perf_counter() - t0
+        if (max_passes is not None and passes >= max_passes) or \
+                (max_passes is None and el >= budget_s):
+            return passes, el, nbytes, oracle.num_threads()
+
+
+def cpu_baseline(dec, body_fmt, S, budget_s, sweep_bytes):
+    passes, el, nbytes, threads = oracle_sample(dec, body_fmt, S, budget_s)
+    gbs = passes * nbytes / el / 1e9
+    return {"value": round(gbs, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sweeps_per_s": round(gbs * 1e9 / sweep_bytes, 4),
+            "sample": (f"layer 0 of the {dec.name} sweep ({nbytes / 1e6:.1f} MB of "
+                       f"{FMT_NAME[body_fmt]} codes+scales, S={S}) x {passes} passes, "
+                       f"fp64 dequantize-then-matvec + SwiGLU, {el:.1f} s")}
+
+
+# ------------------------------------------------------------ reference ----
+
+def run_reference(a):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    from int4_quantized_decode_b200 import workloads as wl
+    dname, body_fmt, head_fmt, S = WORKLOADS[a.workload]
+    dec = getattr(wl, dname)
+    sweep_bytes = _sweep_bytes(dec, body_fmt, head_fmt)
+    oracle_sample(dec, body_fmt, S, 0, max_passes=a.warmup)
+    passes, el, nbytes, threads = oracle_sample(dec, body_fmt, S, 0, max_passes=a.steps)
+    gbs = passes * nbytes / el / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": UNIT,
+        "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": round(el / passes * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config(a, dec, body_fmt, head_fmt, S, sweep_bytes),
+        "sweeps_per_s": round(gbs * 1e9 / sweep_bytes, 5),
+        "cpu_baseline": {"value": round(gbs, 4), "unit": UNIT, "cores": threads,
+                         "kind": "oracle",
+                         "sample": (f"each step: layer 0 of the sweep ({nbytes / 1e6:.1f} MB "
+                                    f"quantized), fp64 dequantize-then-matvec + SwiGLU, S={S}")},
+        "e2e": {"value": round(gbs, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def _sweep_bytes(dec, body_fmt, head_fmt):
+    bpw = {0: 1.0625, 1: 0.5625}
+    return int(dec.weight_count(include_head=False) * bpw[body_fmt] +
+               dec.vocab * dec.hidden * bpw[head_fmt])
+
+
+def _config(a, dec, body_fmt, head_fmt, S, sweep_bytes):
+    return {
+        "workload": (f"{dec.name}-shaped decode weight sweep, {FMT_NAME[body_fmt]} body + "
+                     f"{FMT_NAME[head_fmt]} head{' (tied)' if dec.tied_head else ''}, "
+                     f"S={S}"),
+        "layers": dec.layers, "hidden": dec.hidden, "inter": dec.inter,
+        "vocab": dec.vocab, "S": S, "sweep_bytes": sweep_bytes,
+        "parallelism": f"replicas x{a.gpus}",
+        "l2": "inputs larger than L2 (no flush needed)",
+    }
+
+
+# ------------------------------------------------------------------- ours --
+
+def run_ours(a):
+    import torch
+
+    from int4_quantized_decode_b200 import qgemv as qg
+    from int4_quantized_decode_b200 import workloads as wl
+    from int4_quantized_decode_b200.sweep import DecodeSweep
+
+    rank, local, world = dist_env()
+    if world != a.gpus:
+        raise SystemExit(f"--gpus {a.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier(device_ids=[local])
+
+    dname, body_fmt, head_fmt, S = WORKLOADS[a.workload]
+    dec = getattr(wl, dname)
+    sw = DecodeSweep(dec, body_fmt, head_fmt, S=S, device=dev)
+    G = max(1, a.graph_sweeps)
+    graph = sw.capture(sweeps_per_graph=G)
+    steps = ((a.steps + G - 1) // G) * G
+    stream = torch.cuda.current_stream(dev)
+    sweep_bytes = sw.weight_bytes
+
+    # --- device-timed sweeps (inputs resident in HBM) ----------------------
+    for _ in range((a.warmup + G - 1) // G):
+        graph.replay()
+    qg.qg_stream_check()
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local).start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps // G):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    qg.qg_stream_check()
+    el_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    el_s = el_ms / 1e3
+    value = aggregate(steps * sweep_bytes / 1e9, el_s, world)
+    sweeps_s = aggregate(steps, el_s, world)
+
+    # --- dominant kernel: the fused gate/up SwiGLU over every layer --------
+    dom = _time_gate_up(sw, stream, dev, qg, torch)
+
+    # --- end to end: pinned host inputs -> sweep -> greedy token to host ---
+    e2e = _time_e2e(sw, graph, G, steps, a.warmup, stream, dev, world, torch)
+
+    peak, peak_kind = hbm_peak()
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": steps, "warmup": a.warmup, "ms_per_step": round(el_ms / steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "i8/i4 x f16 -> f32" if S == 1 else "i8 x f16 -> f32 (mma f16)",
+        "data": "synthetic (seeded N(0,0.02) weights, N(0,1) fp16 activations)",
+        "config": _config(a, dec, body_fmt, head_fmt, S, sweep_bytes),
+        "sweeps_per_s": round(sweeps_s, 2),
+        "tokens_per_s": round(sweeps_s * S, 2),
+        "hbm_frac": round(value / world / peak, 4),
+        "roofline": {
+            "bound": "hbm", "kernel": dom["kernel"], "achieved": round(dom["gbs"], 1),
+            "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy, MEASURED_PEAKS.json)"
+            if peak_kind == "measured" else "fallback 6650 GB/s",
+            "unit": "GB/s", "frac": round(dom["gbs"] / peak, 4),
+            "traffic": profiled_traffic(dom["kernel"], a.workload),
+            "algorithmic_bytes_per_launch": dom["bytes"],
+            "launch_us": round(dom["us"], 3), "launches": dom["launches"]},
+        "e2e": e2e,
+        "gpu_launches": steps * sw.launches_per_sweep,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(dec, body_fmt, S, a.cpu_budget_s, sweep_bytes)
+    if rank == 0:
+        print(json.dumps(line))
+    del graph, sw
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def _time_gate_up(sw, stream, dev, qg, torch):
+    """Average duration of the fused gate/up SwiGLU launch, timed with CUDA
+    events on its stream over a graph of every layer's launch (the weights of
+    all layers together are far larger than L2)."""
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(stream)
+    with torch.cuda.graph(g, stream=s):
+        for l, L in enumerate(sw.layers):
+            x = sw.x[l]
+            qg.qg_gate_up_swiglu(L.gate, L.up, x, sw.h if sw.S > 1 else sw.h[0])
+    stream.wait_stream(s)
+    reps = max(3, int(2e9 // (sw.layers[0].gate.nbytes * 2 * len(sw.layers))) + 3)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = reps * len(sw.layers)
+    us = e0.elapsed_time(e1) * 1e3 / launches
+    nbytes = sw.layers[0].gate.nbytes + sw.layers[0].up.nbytes
+    del g
+    return {"kernel": "gemv_s1_kernel<swiglu>" if sw.S == 1 else "gemm_s16_kernel<swiglu>",
+            "gbs": nbytes / (us * 1e-6) / 1e9, "us": us, "bytes": nbytes,
+            "launches": launches}
+
+
+def _time_e2e(sw, graph, G, steps, warmup, stream, dev, world, torch):
+    """Same metric through the public path with host buffers: each step copies
+    that step's activations from pinned host memory, replays the sweep, and
+    reads the greedy token back."""
+    x_host = [x.cpu().pin_memory() for x in sw.inputs()]
+    idx_host = torch.empty(1, dtype=torch.int32).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in x_host)
+    d2h = idx_host.numel() * idx_host.element_size()
+    single = sw.capture(sweeps_per_graph=1) if G != 1 else graph
+    sw.graph = graph
+
+    def one():
+        for xd, xh in zip(sw.inputs(), x_host):
+            xd.copy_(xh, non_blocking=True)
+        single.replay()
+        idx_host.copy_(sw.idx, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize(dev)
+    n = max(10, steps // 4)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    el_s = max_over_ranks(e0.elapsed_time(e1), world, dev) / 1e3
+    return {"value": round(aggregate(n * sw.weight_bytes / 1e9, el_s, world), 2),
+            "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": n}
+
+
+def main(argv=None):
+    a = parse_args(argv)
+    if a.impl == "reference":
+        return run_reference(a)
+    return run_ours(a)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,197 @@
+/*
+ * qgemv.h -- C ABI of libqgemv: weight-only quantized GEMV for LLM decode on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation, as the pages describe it: single-token decode reads every
+ * decoder weight once per token and is bound by memory bandwidth ("Qwen3-VL 4B
+ * -- Core AI (.aimodel)", section Measured: the int8hu decoder reads its whole
+ * size per token).  The shipped format is an int8 per-block-32 symmetric body
+ * and an absmax int8 LM head ("Qwen3-VL (2B / 4B / 8B, vision-language) --
+ * Core AI", Measured table), with an INT4 group-64 variant ("Qwen3-VL 4B & 8B
+ * -- Core ML stateful", Architecture) and a 16-token chunked-prefill function
+ * beside the one-token step ("Qwen3.8-27B ... -- Core AI", The vision path).
+ *
+ * Conventions for every call below
+ *   - Weights are row-major [n, k] (rows = outputs, k = the reduction axis,
+ *     Linear.weight order); quantization blocks run along k.
+ *   - fp16 values travel as their IEEE binary16 bit patterns (uint16_t).
+ *   - Every pointer argument except `W` / `Wg` / `Wu` (host pointers to a
+ *     qg_weight the call reads before returning) is DEVICE memory owned by the
+ *     caller.  The library allocates nothing.
+ *   - Calls validate their arguments synchronously, on the host, before any
+ *     launch; on an error nothing is enqueued.  On success the work is
+ *     enqueued on `stream` and the call returns at once (asynchronous).
+ *   - Buffer rows are contiguous: row r of codes starts at r*k bytes (int8) or
+ *     r*k/2 bytes (int4), row r of scales/biases at r*(k/32) or r*(k/64)
+ *     elements.  A row range of a larger matrix is a valid weight on its own.
+ *   - Outputs are unspecified after an error.  Non-finite inputs (NaN/Inf in
+ *     weights or activations) give unspecified results.
+ */
+#ifndef QGEMV_H
+#define QGEMV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define QG_API __attribute__((visibility("default")))
+#else
+#define QG_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QG_OK = 0,
+    QG_ERR_NULL = 1,      /* a required pointer is NULL */
+    QG_ERR_SHAPE = 2,     /* n < 1, k < 1, k not a multiple of the block, S out of range */
+    QG_ERR_ALIGN = 3,     /* a pointer is not aligned as documented */
+    QG_ERR_FORMAT = 4,    /* unknown format, or gate/up weights that disagree */
+    QG_ERR_WORKSPACE = 5, /* workspace NULL or smaller than required */
+    QG_ERR_CUDA = 6,      /* a CUDA runtime call or launch failed */
+    QG_ERR_TIMEOUT = 7    /* a device-side bounded wait expired (see qg_stream_check) */
+} qg_status;
+
+typedef enum {
+    /* int8 codes, one fp16 scale per 32 consecutive k:  w ~= q * s */
+    QG_FMT_I8_B32 = 0,
+    /* int4 codes (two per byte, even k in the low nibble), one fp16 scale and
+     * one fp16 bias per 64 consecutive k:  w ~= q * s + b */
+    QG_FMT_I4_G64 = 1
+} qg_format;
+
+/* A quantized weight matrix [n, k].
+ *   fmt    : a qg_format value.
+ *   codes  : QG_FMT_I8_B32: int8 [n, k]; QG_FMT_I4_G64: uint8 [n, k/2].
+ *            16-byte aligned.  k % 32 == 0 (int8) or k % 64 == 0 (int4).
+ *   scales : fp16 [n, k/32] (int8) or [n, k/64] (int4); 16-byte aligned.
+ *   biases : fp16 [n, k/64] for int4, 16-byte aligned; ignored for int8. */
+typedef struct {
+    int32_t fmt;
+    int32_t reserved;
+    int64_t n;
+    int64_t k;
+    const void* codes;
+    const uint16_t* scales;
+    const uint16_t* biases;
+} qg_weight;
+
+/* ---------------------------------------------------------------------------
+ * qg_quantize_block32 -- int8 per-block-32 symmetric absmax quantization
+ * ("Qwen3-VL 4B -- Core AI (.aimodel)", Files: int8 per-block-32 body +
+ * absmax int8 head; "Qwen3.8-27B ... -- Core AI", Verified: the absmax
+ * symmetric per-block-32 rule, no clipping).
+ * For each row and each block of 32 consecutive k:
+ *   s = fp16_rne( absmax_fp32 / 127 )          (IEEE fp32 division)
+ *   q = clamp( round_half_even( w / float(s) ), -127, 127 ), all q = 0 if s == 0
+ * w      : fp32 [n, k], 16-byte aligned.      k % 32 == 0, n >= 1.
+ * codes  : int8 [n, k] out, 16-byte aligned.
+ * scales : fp16 [n, k/32] out, 2-byte aligned.
+ * Bit-exact with the CPU oracle.  Blocks with absmax/127 above the fp16
+ * range give an Inf scale (unspecified codes).
+ * ------------------------------------------------------------------------- */
+QG_API qg_status qg_quantize_block32(const float* w, int64_t n, int64_t k,
+                              int8_t* codes, uint16_t* scales,
+                              cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * qg_quantize_int4_g64 -- int4 group-64 affine quantization ("Qwen3-VL 4B &
+ * 8B -- Core ML stateful", Architecture: INT4 per-grouped-channel, group size
+ * 64).  The pages name no formula; this is the plain affine reading:
+ *   s = fp16_rne( (max - min) / 15 ),  b = fp16_rne( min )   (fp32 ops)
+ *   q = clamp( round_half_even( (w - float(b)) / float(s) ), 0, 15 ),
+ *   all q = 0 if s == 0
+ * w       : fp32 [n, k], 16-byte aligned.    k % 64 == 0, n >= 1.
+ * codes   : uint8 [n, k/2] out (low nibble = even k), 16-byte aligned.
+ * scales, biases : fp16 [n, k/64] out, 2-byte aligned.
+ * Bit-exact with the CPU oracle.
+ * ------------------------------------------------------------------------- */
+QG_API qg_status qg_quantize_int4_g64(const float* w, int64_t n, int64_t k,
+                               uint8_t* codes, uint16_t* scales,
+                               uint16_t* biases, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * qg_gemv_s1 -- one-token (S=1) quantized GEMV, the decode weight stream
+ * ("Qwen3-VL 4B -- Core AI (.aimodel)", Measured: decode is bandwidth-bound).
+ *   y[r] = sum_k w_dq[r, k] * x[k]     (fp32 accumulation)
+ * W   : the weight (int8 block-32 or int4 group-64).
+ * x   : fp16 [k], 16-byte aligned.
+ * y   : fp32 [n] out (4-byte aligned), or NULL.
+ * y16 : fp16 [n] out = fp16_rne(y) (2-byte aligned), or NULL.
+ * At least one of y, y16 must be non-NULL.  x must not overlap the outputs.
+ * Accuracy: |y - y_ref| <= 2e-3 * sum_k |w_dq x| per row (fp64 oracle).
+ * ------------------------------------------------------------------------- */
+QG_API qg_status qg_gemv_s1(const qg_weight* W, const uint16_t* x, float* y,
+                     uint16_t* y16, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * qg_gemm_s16 -- chunked-prefill skinny GEMM on the tensor cores, S tokens
+ * through the same weights ("Qwen3.8-27B ... -- Core AI", The vision path:
+ * a static S=16 'prefill' chunk beside the S=1 'main' decode).
+ *   Y[s, r] = sum_k X[s, k] * w_dq[r, k],   0 <= s < S
+ * W : the weight (int8 block-32 only; QG_ERR_FORMAT for int4).
+ * X : fp16 [S, k] row-major, 16-byte aligned.   1 <= S <= 16.
+ * Y : fp32 [S, n] out, 4-byte aligned.
+ * Accuracy: each row s obeys the qg_gemv_s1 bound for x = X[s].
+ * ------------------------------------------------------------------------- */
+QG_API qg_status qg_gemm_s16(const qg_weight* W, const uint16_t* X, int S, float* Y,
+                      cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * qg_gate_up_swiglu -- fused gate/up projections with the SwiGLU epilogue
+ * ("Qwen3-VL (2B / 4B / 8B, vision-language) -- Core AI", architecture: a
+ * SwiGLU MLP):
+ *   g = W_g x,  u = W_u x,  H[s, i] = fp16_rne( silu(g_i) * u_i ),
+ *   silu(g) = g / (1 + exp(-g))
+ * Wg, Wu : weights of identical format and shape [n = intermediate, k].
+ *          S == 1 accepts int8 or int4; S > 1 (tensor cores) int8 only.
+ * X      : fp16 [S, k], 16-byte aligned.   1 <= S <= 16.
+ * H      : fp16 [S, n] out, 2-byte aligned.
+ * ------------------------------------------------------------------------- */
+QG_API qg_status qg_gate_up_swiglu(const qg_weight* Wg, const qg_weight* Wu,
+                            const uint16_t* X, int S, uint16_t* H,
+                            cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * qg_head_argmax -- LM head GEMV fused with the greedy argmax
+ * ("Qwen3.8-27B ... -- Core AI", Verified: absmax int8 head, greedy
+ * teacher-forced argmax).
+ *   logits[v] = sum_k w_dq[v, k] x[k];   idx = the smallest v of the max
+ * W         : the head weight [vocab, hidden] (int8 or int4).
+ * x         : fp16 [k], 16-byte aligned.
+ * logits    : fp32 [n] out (4-byte aligned) or NULL.
+ * idx       : int32 [1] out, device memory.
+ * workspace : device memory of at least qg_head_argmax_workspace_bytes(n)
+ *             bytes, 16-byte aligned.  It must be all zero before its first
+ *             use; every call that returns QG_OK and runs to completion
+ *             leaves it all zero again, so it can be reused without clearing.
+ *             Calls that share a workspace must not overlap on the GPU.
+ * ------------------------------------------------------------------------- */
+QG_API size_t qg_head_argmax_workspace_bytes(int64_t n);
+QG_API qg_status qg_head_argmax(const qg_weight* W, const uint16_t* x, float* logits,
+                         int32_t* idx, void* workspace, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * qg_stream_check -- synchronize `stream` and report asynchronous failures:
+ * QG_ERR_CUDA for a CUDA error, QG_ERR_TIMEOUT if a kernel's bounded wait on
+ * its own bulk copies expired since the last check (the flag is then
+ * cleared).  Kernels never spin without a limit.
+ * ------------------------------------------------------------------------- */
+QG_API qg_status qg_stream_check(cudaStream_t stream);
+
+/* Human-readable name of a status code (static string). */
+QG_API const char* qg_status_string(qg_status status);
+
+/* ABI version of this header (major * 100 + minor). */
+QG_API int qg_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QGEMV_H */

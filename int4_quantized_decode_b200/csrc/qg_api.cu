@@ -1,0 +1,218 @@
+// qg_api.cu -- the extern "C" entry points of libqgemv: argument validation
+// (synchronous, before any launch) and dispatch to the kernel launchers.
+#include <cstdint>
+
+#include "qg_internal.h"
+
+namespace qg {
+
+qg_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return QG_OK;
+    (void)cudaGetLastError();  // clear a non-sticky error
+    return QG_ERR_CUDA;
+}
+
+qg_status device_info(DeviceInfo* out) {
+    static DeviceInfo cache[64];
+    static bool valid[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cuda_status(cudaErrorInvalidDevice);
+    if (dev >= 0 && dev < 64 && valid[dev]) {
+        *out = cache[dev];
+        return QG_OK;
+    }
+    DeviceInfo d;
+    d.device = dev;
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+        return cuda_status(cudaErrorInvalidDevice);
+    if (dev >= 0 && dev < 64) {
+        cache[dev] = d;
+        valid[dev] = true;
+    }
+    *out = d;
+    return QG_OK;
+}
+
+}  // namespace qg
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int64_t block_of(int fmt) { return fmt == QG_FMT_I8_B32 ? 32 : 64; }
+
+// Shape, format and alignment of one weight descriptor.
+qg_status check_weight(const qg_weight* W) {
+    if (!W) return QG_ERR_NULL;
+    if (W->fmt != QG_FMT_I8_B32 && W->fmt != QG_FMT_I4_G64) return QG_ERR_FORMAT;
+    if (!W->codes || !W->scales) return QG_ERR_NULL;
+    if (W->fmt == QG_FMT_I4_G64 && !W->biases) return QG_ERR_NULL;
+    if (W->n < 1 || W->k < 1 || W->k % block_of(W->fmt) != 0) return QG_ERR_SHAPE;
+    if (W->n > (int64_t(1) << 31) - 1) return QG_ERR_SHAPE;  // row indices are int32 in argmax
+    if (!aligned(W->codes, 16) || !aligned(W->scales, 16)) return QG_ERR_ALIGN;
+    if (W->fmt == QG_FMT_I4_G64 && !aligned(W->biases, 16)) return QG_ERR_ALIGN;
+    return QG_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qg_abi_version(void) { return 100; }
+
+const char* qg_status_string(qg_status s) {
+    switch (s) {
+        case QG_OK: return "QG_OK";
+        case QG_ERR_NULL: return "QG_ERR_NULL: a required pointer is NULL";
+        case QG_ERR_SHAPE: return "QG_ERR_SHAPE: unsupported n, k or S";
+        case QG_ERR_ALIGN: return "QG_ERR_ALIGN: pointer not aligned as documented";
+        case QG_ERR_FORMAT: return "QG_ERR_FORMAT: unknown or mismatched weight format";
+        case QG_ERR_WORKSPACE: return "QG_ERR_WORKSPACE: workspace NULL or too small";
+        case QG_ERR_CUDA: return "QG_ERR_CUDA: CUDA runtime error";
+        case QG_ERR_TIMEOUT: return "QG_ERR_TIMEOUT: a device-side bounded wait expired";
+    }
+    return "QG_ERR_UNKNOWN";
+}
+
+qg_status qg_quantize_block32(const float* w, int64_t n, int64_t k, int8_t* codes,
+                              uint16_t* scales, cudaStream_t stream) {
+    if (!w || !codes || !scales) return QG_ERR_NULL;
+    if (n < 1 || k < 32 || k % 32 != 0) return QG_ERR_SHAPE;
+    if (!aligned(w, 16) || !aligned(codes, 16) || !aligned(scales, 2)) return QG_ERR_ALIGN;
+    return qg::launch_quantize_block32(w, n, k, codes, scales, stream);
+}
+
+qg_status qg_quantize_int4_g64(const float* w, int64_t n, int64_t k, uint8_t* codes,
+                               uint16_t* scales, uint16_t* biases, cudaStream_t stream) {
+    if (!w || !codes || !scales || !biases) return QG_ERR_NULL;
+    if (n < 1 || k < 64 || k % 64 != 0) return QG_ERR_SHAPE;
+    if (!aligned(w, 16) || !aligned(codes, 16) || !aligned(scales, 2) || !aligned(biases, 2))
+        return QG_ERR_ALIGN;
+    return qg::launch_quantize_int4_g64(w, n, k, codes, scales, biases, stream);
+}
+
+qg_status qg_gemv_s1(const qg_weight* W, const uint16_t* x, float* y, uint16_t* y16,
+                     cudaStream_t stream) {
+    qg_status st = check_weight(W);
+    if (st != QG_OK) return st;
+    if (!x || (!y && !y16)) return QG_ERR_NULL;
+    if (!aligned(x, 16) || (y && !aligned(y, 4)) || (y16 && !aligned(y16, 2))) return QG_ERR_ALIGN;
+    qg::GemvLaunch L = {};
+    L.fmt = W->fmt;
+    L.epilogue = qg::kEpiPlain;
+    L.nmat = 1;
+    L.n = W->n;
+    L.k = W->k;
+    L.codes[0] = W->codes;
+    L.scales[0] = W->scales;
+    L.biases[0] = W->biases;
+    L.x = x;
+    L.y = y;
+    L.y16 = y16;
+    return qg::launch_gemv_s1(L, stream);
+}
+
+qg_status qg_gemm_s16(const qg_weight* W, const uint16_t* X, int S, float* Y,
+                      cudaStream_t stream) {
+    qg_status st = check_weight(W);
+    if (st != QG_OK) return st;
+    if (!X || !Y) return QG_ERR_NULL;
+    if (S < 1 || S > 16) return QG_ERR_SHAPE;
+    if (!aligned(X, 16) || !aligned(Y, 4)) return QG_ERR_ALIGN;
+    if (S == 1) return qg_gemv_s1(W, X, Y, nullptr, stream);
+    if (W->fmt != QG_FMT_I8_B32) return QG_ERR_FORMAT;
+    qg::GemmS16Launch L = {};
+    L.epilogue = qg::kEpiPlain;
+    L.S = S;
+    L.n = W->n;
+    L.k = W->k;
+    L.codes[0] = L.codes[1] = static_cast<const int8_t*>(W->codes);
+    L.scales[0] = L.scales[1] = W->scales;
+    L.X = X;
+    L.Y = Y;
+    return qg::launch_gemm_s16(L, stream);
+}
+
+qg_status qg_gate_up_swiglu(const qg_weight* Wg, const qg_weight* Wu, const uint16_t* X, int S,
+                            uint16_t* H, cudaStream_t stream) {
+    qg_status st = check_weight(Wg);
+    if (st != QG_OK) return st;
+    st = check_weight(Wu);
+    if (st != QG_OK) return st;
+    if (Wg->fmt != Wu->fmt) return QG_ERR_FORMAT;
+    if (Wg->n != Wu->n || Wg->k != Wu->k) return QG_ERR_SHAPE;
+    if (!X || !H) return QG_ERR_NULL;
+    if (S < 1 || S > 16) return QG_ERR_SHAPE;
+    if (!aligned(X, 16) || !aligned(H, 2)) return QG_ERR_ALIGN;
+    if (S == 1) {
+        qg::GemvLaunch L = {};
+        L.fmt = Wg->fmt;
+        L.epilogue = qg::kEpiSwiglu;
+        L.nmat = 2;
+        L.n = Wg->n;
+        L.k = Wg->k;
+        L.codes[0] = Wg->codes;
+        L.scales[0] = Wg->scales;
+        L.biases[0] = Wg->biases;
+        L.codes[1] = Wu->codes;
+        L.scales[1] = Wu->scales;
+        L.biases[1] = Wu->biases;
+        L.x = X;
+        L.h = H;
+        return qg::launch_gemv_s1(L, stream);
+    }
+    if (Wg->fmt != QG_FMT_I8_B32) return QG_ERR_FORMAT;
+    qg::GemmS16Launch L = {};
+    L.epilogue = qg::kEpiSwiglu;
+    L.S = S;
+    L.n = Wg->n;
+    L.k = Wg->k;
+    L.codes[0] = static_cast<const int8_t*>(Wg->codes);
+    L.scales[0] = Wg->scales;
+    L.codes[1] = static_cast<const int8_t*>(Wu->codes);
+    L.scales[1] = Wu->scales;
+    L.X = X;
+    L.H = H;
+    return qg::launch_gemm_s16(L, stream);
+}
+
+size_t qg_head_argmax_workspace_bytes(int64_t n) {
+    (void)n;
+    return qg::kHeadWorkspaceBytes;
+}
+
+qg_status qg_head_argmax(const qg_weight* W, const uint16_t* x, float* logits, int32_t* idx,
+                         void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    qg_status st = check_weight(W);
+    if (st != QG_OK) return st;
+    if (!x || !idx) return QG_ERR_NULL;
+    if (!workspace || ws_bytes < qg::kHeadWorkspaceBytes) return QG_ERR_WORKSPACE;
+    if (!aligned(x, 16) || (logits && !aligned(logits, 4)) || !aligned(idx, 4) ||
+        !aligned(workspace, 16))
+        return QG_ERR_ALIGN;
+    qg::GemvLaunch L = {};
+    L.fmt = W->fmt;
+    L.epilogue = qg::kEpiHead;
+    L.nmat = 1;
+    L.n = W->n;
+    L.k = W->k;
+    L.codes[0] = W->codes;
+    L.scales[0] = W->scales;
+    L.biases[0] = W->biases;
+    L.x = x;
+    L.logits = logits;
+    L.idx = idx;
+    L.workspace = workspace;
+    return qg::launch_gemv_s1(L, stream);
+}
+
+qg_status qg_stream_check(cudaStream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return qg::cuda_status(e);
+    const unsigned int f = qg::gemv_read_and_clear_error() | qg::gemm_s16_read_and_clear_error();
+    return f ? QG_ERR_TIMEOUT : QG_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// qg_internal.h -- host-side interfaces between the C-ABI layer (qg_api.cu)
+// and the kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cstdint>
+
+#include "qgemv.h"
+
+namespace qg {
+
+// Cached per-device properties.
+struct DeviceInfo {
+    int device;
+    int num_sms;
+    int max_smem_optin;  // bytes of dynamic shared memory a CTA may opt into
+};
+qg_status device_info(DeviceInfo* out);
+
+// Map the last CUDA error (if any) to a status, clearing it.
+qg_status cuda_status(cudaError_t e);
+
+// Epilogues of the S=1 streaming kernel.
+enum GemvEpilogue : int { kEpiPlain = 0, kEpiSwiglu = 1, kEpiHead = 2 };
+
+// One S=1 streaming launch: NMAT (1 or 2) weights of identical format and
+// shape, one fp16 activation, one of three epilogues.
+struct GemvLaunch {
+    int fmt;  // qg_format
+    int epilogue;
+    int nmat;
+    int64_t n, k;
+    const void* codes[2];
+    const uint16_t* scales[2];
+    const uint16_t* biases[2];
+    const uint16_t* x;
+    float* y;             // plain: fp32 out or NULL
+    uint16_t* y16;        // plain: fp16 out or NULL
+    uint16_t* h;          // swiglu: fp16 out
+    float* logits;        // head: fp32 out or NULL
+    int32_t* idx;         // head: argmax out
+    void* workspace;      // head: zeroed scratch (key + ticket)
+};
+qg_status launch_gemv_s1(const GemvLaunch& L, cudaStream_t stream);
+unsigned int gemv_read_and_clear_error();
+
+// Quantizers.
+qg_status launch_quantize_block32(const float* w, int64_t n, int64_t k, int8_t* codes,
+                                  uint16_t* scales, cudaStream_t stream);
+qg_status launch_quantize_int4_g64(const float* w, int64_t n, int64_t k, uint8_t* codes,
+                                   uint16_t* scales, uint16_t* biases, cudaStream_t stream);
+
+// S <= 16 tensor-core path (int8 block-32): plain (Y fp32) or SwiGLU (H fp16).
+struct GemmS16Launch {
+    int epilogue;  // kEpiPlain or kEpiSwiglu
+    int S;
+    int64_t n, k;
+    const int8_t* codes[2];
+    const uint16_t* scales[2];
+    const uint16_t* X;
+    float* Y;
+    uint16_t* H;
+};
+qg_status launch_gemm_s16(const GemmS16Launch& L, cudaStream_t stream);
+unsigned int gemm_s16_read_and_clear_error();
+
+// Head-argmax workspace layout (bytes).
+constexpr size_t kHeadWorkspaceBytes = 256;
+
+}  // namespace qg

@@ -1,0 +1,231 @@
+"""Python binding of libqgemv's C ABI (include/qgemv.h).
+
+Argument marshalling only: every function takes torch CUDA tensors, checks
+dtypes and shapes, and calls the C entry point of the same name on the current
+torch stream.  All arithmetic runs in the library's kernels; there is no CPU
+or PyTorch fallback, and importing a function without the built library
+raises at once.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqgemv.so")
+
+QG_OK = 0
+STATUS_NAMES = {0: "QG_OK", 1: "QG_ERR_NULL", 2: "QG_ERR_SHAPE", 3: "QG_ERR_ALIGN",
+                4: "QG_ERR_FORMAT", 5: "QG_ERR_WORKSPACE", 6: "QG_ERR_CUDA",
+                7: "QG_ERR_TIMEOUT"}
+FMT_I8_B32 = 0
+FMT_I4_G64 = 1
+
+# every symbol include/qgemv.h declares
+ABI_SYMBOLS = ("qg_quantize_block32", "qg_quantize_int4_g64", "qg_gemv_s1",
+               "qg_gemm_s16", "qg_gate_up_swiglu", "qg_head_argmax_workspace_bytes",
+               "qg_head_argmax", "qg_stream_check", "qg_status_string", "qg_abi_version")
+
+
+class QgError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_string(status)}")
+
+
+class CWeight(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("n", ctypes.c_int64), ("k", ctypes.c_int64),
+                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("biases", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libqgemv.so (built by int4_quantized_decode_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"libqgemv.so is not built ({LIB_PATH}); run "
+                "`python -m int4_quantized_decode_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        W = ctypes.POINTER(CWeight)
+        L.qg_quantize_block32.argtypes = [P, I64, I64, P, P, P]
+        L.qg_quantize_int4_g64.argtypes = [P, I64, I64, P, P, P, P]
+        L.qg_gemv_s1.argtypes = [W, P, P, P, P]
+        L.qg_gemm_s16.argtypes = [W, P, I, P, P]
+        L.qg_gate_up_swiglu.argtypes = [W, W, P, I, P, P]
+        L.qg_head_argmax_workspace_bytes.argtypes = [I64]
+        L.qg_head_argmax_workspace_bytes.restype = ctypes.c_size_t
+        L.qg_head_argmax.argtypes = [W, P, P, P, P, ctypes.c_size_t, P]
+        L.qg_stream_check.argtypes = [P]
+        L.qg_status_string.argtypes = [I]
+        L.qg_status_string.restype = ctypes.c_char_p
+        L.qg_abi_version.argtypes = []
+        for name in ABI_SYMBOLS:
+            if name not in ("qg_head_argmax_workspace_bytes", "qg_status_string"):
+                getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().qg_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != QG_OK:
+        raise QgError(fn, status)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _cuda(t: torch.Tensor, dtype, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+@dataclass
+class QWeight:
+    """A quantized weight [n, k] held in torch CUDA tensors."""
+    fmt: int
+    n: int
+    k: int
+    codes: torch.Tensor            # int8 [n, k] or uint8 [n, k/2]
+    scales: torch.Tensor           # int16 (fp16 bits) [n, k/block]
+    biases: Optional[torch.Tensor] = None
+
+    @staticmethod
+    def empty(fmt: int, n: int, k: int, device="cuda") -> "QWeight":
+        if fmt == FMT_I8_B32:
+            return QWeight(fmt, n, k, torch.empty((n, k), dtype=torch.int8, device=device),
+                           torch.empty((n, k // 32), dtype=torch.int16, device=device))
+        return QWeight(fmt, n, k, torch.empty((n, k // 2), dtype=torch.uint8, device=device),
+                       torch.empty((n, k // 64), dtype=torch.int16, device=device),
+                       torch.empty((n, k // 64), dtype=torch.int16, device=device))
+
+    def rows(self, r0: int, r1: int) -> "QWeight":
+        """View of rows [r0, r1) (row ranges are valid weights on their own)."""
+        return QWeight(self.fmt, r1 - r0, self.k, self.codes[r0:r1], self.scales[r0:r1],
+                       None if self.biases is None else self.biases[r0:r1])
+
+    @property
+    def nbytes(self) -> int:
+        b = self.codes.numel() * self.codes.element_size()
+        b += self.scales.numel() * 2
+        if self.biases is not None:
+            b += self.biases.numel() * 2
+        return b
+
+    def c(self) -> CWeight:
+        return CWeight(self.fmt, 0, self.n, self.k, self.codes.data_ptr(),
+                       self.scales.data_ptr(),
+                       self.biases.data_ptr() if self.biases is not None else None)
+
+
+# ------------------------------------------------------------ entry points --
+
+def qg_quantize_block32(w: torch.Tensor, out: QWeight, stream=None) -> QWeight:
+    _cuda(w, torch.float32, "w")
+    n, k = w.shape
+    assert out.fmt == FMT_I8_B32 and out.n == n and out.k == k
+    _check("qg_quantize_block32",
+           lib().qg_quantize_block32(_ptr(w), n, k, _ptr(out.codes), _ptr(out.scales),
+                                     _stream(stream)))
+    return out
+
+
+def qg_quantize_int4_g64(w: torch.Tensor, out: QWeight, stream=None) -> QWeight:
+    _cuda(w, torch.float32, "w")
+    n, k = w.shape
+    assert out.fmt == FMT_I4_G64 and out.n == n and out.k == k
+    _check("qg_quantize_int4_g64",
+           lib().qg_quantize_int4_g64(_ptr(w), n, k, _ptr(out.codes), _ptr(out.scales),
+                                      _ptr(out.biases), _stream(stream)))
+    return out
+
+
+def quantize(w: torch.Tensor, fmt: int, out: Optional[QWeight] = None, stream=None) -> QWeight:
+    n, k = w.shape
+    out = out if out is not None else QWeight.empty(fmt, n, k, device=w.device)
+    if fmt == FMT_I8_B32:
+        return qg_quantize_block32(w, out, stream)
+    return qg_quantize_int4_g64(w, out, stream)
+
+
+def qg_gemv_s1(W: QWeight, x: torch.Tensor, y: Optional[torch.Tensor] = None,
+               y16: Optional[torch.Tensor] = None, stream=None) -> None:
+    _cuda(x, torch.float16, "x")
+    if y is not None:
+        _cuda(y, torch.float32, "y")
+    if y16 is not None:
+        _cuda(y16, torch.float16, "y16")
+    cw = W.c()
+    _check("qg_gemv_s1", lib().qg_gemv_s1(ctypes.byref(cw), _ptr(x), _ptr(y), _ptr(y16),
+                                          _stream(stream)))
+
+
+def qg_gemm_s16(W: QWeight, X: torch.Tensor, Y: torch.Tensor, stream=None) -> None:
+    _cuda(X, torch.float16, "X")
+    _cuda(Y, torch.float32, "Y")
+    S = X.shape[0]
+    cw = W.c()
+    _check("qg_gemm_s16", lib().qg_gemm_s16(ctypes.byref(cw), _ptr(X), S, _ptr(Y),
+                                            _stream(stream)))
+
+
+def qg_gate_up_swiglu(Wg: QWeight, Wu: QWeight, X: torch.Tensor, H: torch.Tensor,
+                      stream=None) -> None:
+    _cuda(X, torch.float16, "X")
+    _cuda(H, torch.float16, "H")
+    S = X.shape[0] if X.dim() == 2 else 1
+    cg, cu = Wg.c(), Wu.c()
+    _check("qg_gate_up_swiglu",
+           lib().qg_gate_up_swiglu(ctypes.byref(cg), ctypes.byref(cu), _ptr(X), S, _ptr(H),
+                                   _stream(stream)))
+
+
+def qg_head_argmax_workspace_bytes(n: int) -> int:
+    return int(lib().qg_head_argmax_workspace_bytes(int(n)))
+
+
+def head_workspace(n: int, device="cuda") -> torch.Tensor:
+    """A zeroed workspace for qg_head_argmax (it stays zeroed between calls)."""
+    return torch.zeros(qg_head_argmax_workspace_bytes(n), dtype=torch.uint8, device=device)
+
+
+def qg_head_argmax(W: QWeight, x: torch.Tensor, idx: torch.Tensor, workspace: torch.Tensor,
+                   logits: Optional[torch.Tensor] = None, stream=None) -> None:
+    _cuda(x, torch.float16, "x")
+    _cuda(idx, torch.int32, "idx")
+    _cuda(workspace, torch.uint8, "workspace")
+    if logits is not None:
+        _cuda(logits, torch.float32, "logits")
+    cw = W.c()
+    _check("qg_head_argmax",
+           lib().qg_head_argmax(ctypes.byref(cw), _ptr(x), _ptr(logits), _ptr(idx),
+                                _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def qg_stream_check(stream=None) -> None:
+    _check("qg_stream_check", lib().qg_stream_check(_stream(stream)))

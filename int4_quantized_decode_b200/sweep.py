@@ -1,0 +1,169 @@
+"""One decode step's weight sweep through libqgemv, captured in a CUDA graph.
+
+"Decode reads the whole model per token" ("Qwen3.8-27B ... -- Core AI", The
+vision path / bandwidth note; "Qwen3-VL 4B -- Core AI (.aimodel)", Measured):
+a sweep reads every decoder weight once.  Per layer it runs
+
+    qkv(+output gate) GEMV  ->  o GEMV  ->  gate/up + SwiGLU  ->  down GEMV
+
+and finishes with the LM head fused with the greedy argmax.  q|(gate)|k|v are
+row-concatenated into one weight (rows are independent, so the fused matrix is
+just the projections' rows one after another).  Attention and norms are not
+part of the weight stream; as their stand-in, o reads fp16(q_out), each layer
+takes a fresh seeded activation for qkv and gate/up, and down reads the SwiGLU
+output.  With S = 16 (chunked prefill) every projection runs on the tensor-core
+path with a [16, K] chunk, o reads a fresh seeded chunk, and the head reads the
+chunk's last row.
+
+All work is enqueued through the C ABI on the current stream; this module only
+allocates buffers, draws the seeded weights, and replays the graph.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import List, Optional
+
+import torch
+
+from . import qgemv as qg
+from . import workloads as wl
+
+
+@dataclass
+class LayerWeights:
+    qkv: qg.QWeight
+    o: qg.QWeight
+    gate: qg.QWeight
+    up: qg.QWeight
+    down: qg.QWeight
+
+
+class DecodeSweep:
+    """Quantized weights of a decoder plus the buffers of one sweep."""
+
+    def __init__(self, dec: wl.Decoder, body_fmt: int = qg.FMT_I8_B32,
+                 head_fmt: int = qg.FMT_I8_B32, S: int = 1, device="cuda",
+                 keep_logits: bool = False):
+        assert 1 <= S <= 16
+        self.dec, self.S, self.device = dec, S, torch.device(device)
+        self.body_fmt, self.head_fmt = body_fmt, head_fmt
+        if S > 1:
+            assert body_fmt == qg.FMT_I8_B32 and head_fmt == qg.FMT_I8_B32
+        self.layers: List[LayerWeights] = []
+        for l in range(dec.layers):
+            self.layers.append(self._make_layer(l))
+        self.head = self._quantized("head", -1, dec.vocab, dec.hidden, head_fmt)
+        self._make_buffers(keep_logits)
+        self.graph: Optional[torch.cuda.CUDAGraph] = None
+
+    # ------------------------------------------------------------ weights --
+    def _quantized(self, proj: str, layer: int, n: int, k: int, fmt: int,
+                   out: Optional[qg.QWeight] = None) -> qg.QWeight:
+        w = wl.weight_fp32(n, k, self.dec.weight_seed(layer, proj), self.device)
+        q = qg.quantize(w, fmt, out)
+        del w
+        return q
+
+    def _make_layer(self, l: int) -> LayerWeights:
+        d, f = self.dec, self.body_fmt
+        qkv = qg.QWeight.empty(f, d.qkv_rows, d.hidden, self.device)
+        r = 0
+        for name, rows in d.qkv_parts():
+            self._quantized(name, l, rows, d.hidden, f, qkv.rows(r, r + rows))
+            r += rows
+        return LayerWeights(
+            qkv=qkv,
+            o=self._quantized("o", l, d.hidden, d.q_dim, f),
+            gate=self._quantized("gate", l, d.inter, d.hidden, f),
+            up=self._quantized("up", l, d.inter, d.hidden, f),
+            down=self._quantized("down", l, d.hidden, d.inter, f))
+
+    # ------------------------------------------------------------ buffers --
+    def _make_buffers(self, keep_logits: bool) -> None:
+        d, S, dev = self.dec, self.S, self.device
+        # every activation of a sweep lives in one or two contiguous tensors so
+        # a host caller can refresh them with one copy each
+        if S == 1:
+            self.x_all = torch.empty((d.layers + 1, d.hidden), dtype=torch.float16, device=dev)
+            for l in range(d.layers):
+                self.x_all[l] = wl.act_fp16(d.hidden, d.x_seed(l), dev)
+            self.x_all[d.layers] = wl.act_fp16(d.hidden, d.x_seed(-1), dev)
+            self.x_o_all = None
+        else:
+            self.x_all = torch.empty((d.layers + 1, S, d.hidden), dtype=torch.float16, device=dev)
+            for l in range(d.layers):
+                self.x_all[l] = wl.act_fp16((S, d.hidden), d.chunk_seed(l), dev)
+            self.x_all[d.layers] = wl.act_fp16((S, d.hidden), d.chunk_seed(-1), dev)
+            self.x_o_all = torch.empty((d.layers, S, d.q_dim), dtype=torch.float16, device=dev)
+            for l in range(d.layers):
+                self.x_o_all[l] = wl.act_fp16((S, d.q_dim), d.chunk_seed(l) + 100000, dev)
+        self.x = [self.x_all[l] for l in range(d.layers)]
+        self.x_head = self.x_all[d.layers]
+        self.x_o = None if self.x_o_all is None else [self.x_o_all[l] for l in range(d.layers)]
+        self.y_qkv = torch.empty((S, d.qkv_rows), dtype=torch.float32, device=dev)
+        self.y16_qkv = torch.empty((d.qkv_rows,), dtype=torch.float16, device=dev)
+        self.y_o = torch.empty((S, d.hidden), dtype=torch.float32, device=dev)
+        self.h = torch.empty((S, d.inter), dtype=torch.float16, device=dev)
+        self.y_down = torch.empty((S, d.hidden), dtype=torch.float32, device=dev)
+        self.logits = (torch.empty(d.vocab, dtype=torch.float32, device=dev)
+                       if keep_logits else None)
+        self.idx = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.ws = qg.head_workspace(d.vocab, dev)
+
+    # ------------------------------------------------------------- sweep --
+    @property
+    def weight_bytes(self) -> int:
+        """Algorithmic bytes one sweep streams: codes + scales (+ biases)."""
+        b = sum(L.qkv.nbytes + L.o.nbytes + L.gate.nbytes + L.up.nbytes + L.down.nbytes
+                for L in self.layers)
+        return b + self.head.nbytes
+
+    @property
+    def launches_per_sweep(self) -> int:
+        return 4 * self.dec.layers + 1
+
+    def inputs(self) -> List[torch.Tensor]:
+        """The per-step activation tensors (contiguous), in a fixed order."""
+        return [self.x_all] if self.x_o_all is None else [self.x_all, self.x_o_all]
+
+    def head_input(self) -> torch.Tensor:
+        return self.x_head if self.S == 1 else self.x_head[self.S - 1]
+
+    def run_layer(self, l: int, stream=None) -> None:
+        """Enqueue layer l's four launches on `stream` (default: current)."""
+        d, L = self.dec, self.layers[l]
+        if self.S == 1:
+            qg.qg_gemv_s1(L.qkv, self.x[l], self.y_qkv[0], self.y16_qkv, stream)
+            qg.qg_gemv_s1(L.o, self.y16_qkv[: d.q_dim], self.y_o[0], None, stream)
+            qg.qg_gate_up_swiglu(L.gate, L.up, self.x[l], self.h[0], stream)
+            qg.qg_gemv_s1(L.down, self.h[0], self.y_down[0], None, stream)
+        else:
+            qg.qg_gemm_s16(L.qkv, self.x[l], self.y_qkv, stream)
+            qg.qg_gemm_s16(L.o, self.x_o[l], self.y_o, stream)
+            qg.qg_gate_up_swiglu(L.gate, L.up, self.x[l], self.h, stream)
+            qg.qg_gemm_s16(L.down, self.h, self.y_down, stream)
+
+    def run_head(self, stream=None) -> None:
+        qg.qg_head_argmax(self.head, self.head_input(), self.idx, self.ws, self.logits, stream)
+
+    def step(self, stream=None) -> None:
+        """Enqueue one sweep on `stream` (default: the current stream)."""
+        for l in range(self.dec.layers):
+            self.run_layer(l, stream)
+        self.run_head(stream)
+
+    def capture(self, sweeps_per_graph: int = 1) -> torch.cuda.CUDAGraph:
+        """Capture `sweeps_per_graph` back-to-back sweeps into one CUDA graph."""
+        s = torch.cuda.Stream(device=self.device)
+        s.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(s):
+            self.step()  # warm the launch paths (function attributes) outside capture
+        torch.cuda.current_stream(self.device).wait_stream(s)
+        torch.cuda.synchronize(self.device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(sweeps_per_graph):
+                self.step()
+        self.graph = g
+        self.sweeps_per_graph = sweeps_per_graph
+        return g

@@ -78,6 +78,8 @@ def lib():
         L.orc_swiglu.restype = None
         L.orc_argmax.argtypes = [P, I64]
         L.orc_argmax.restype = I64
+        L.orc_num_threads.argtypes = []
+        L.orc_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -213,6 +215,10 @@ def swiglu(g, u, mag_g, mag_u, tol: float):
     bound = np.empty(n, dtype=np.float64)
     lib().orc_swiglu(_p(g), _p(u), _p(mag_g), _p(mag_u), n, float(tol), _p(h), _p(bound))
     return h, bound
+
+
+def num_threads() -> int:
+    return int(lib().orc_num_threads())
 
 
 def argmax(v) -> int:

@@ -10,6 +10,8 @@
 #include "oracle.h"
 
 #include <math.h>
+#include <omp.h>
+#include <stdlib.h>
 #include <string.h>
 
 /* ---------------------------------------------------------------- fp16 --- */
@@ -129,6 +131,11 @@ void orc_quantize_int4_g64(const float* w, int64_t n, int64_t k, uint8_t* codes,
                 if (wg[j] > mx) mx = wg[j];
                 if (wg[j] < mn) mn = wg[j];
             }
+            /* a signed-zero extreme counts as +0 (x + 0 maps -0 to +0 and
+             * leaves every other value unchanged) */
+            volatile float zero = 0.0f;
+            mx = mx + zero;
+            mn = mn + zero;
             /* scale = (max - min) / 15 and bias = min, both fp16 (RNE);
              * each fp32 operation rounded on its own */
             volatile float range = mx - mn;
@@ -187,29 +194,45 @@ void orc_dequant_row_i4(const uint8_t* codes, const uint16_t* scales,
 void orc_matvec(int fmt, const void* codes, const uint16_t* scales,
                 const uint16_t* biases, int64_t n, int64_t k, const uint16_t* x,
                 double* y, double* mag) {
-#pragma omp parallel for schedule(static)
+    /* x and the per-row side data are converted to fp64 once (exact); the
+     * sums run in index order. */
+    double* xd = (double*)malloc(sizeof(double) * (size_t)k);
+    for (int64_t j = 0; j < k; ++j) xd[j] = orc_f16_to_f64(x[j]);
+    const int64_t blk = fmt == 0 ? 32 : 64;
+    const int64_t nb = k / blk;
+#pragma omp parallel
+    {
+        double* sd = (double*)malloc(sizeof(double) * (size_t)nb);
+        double* bd = (double*)malloc(sizeof(double) * (size_t)nb);
+#pragma omp for schedule(static)
         for (int64_t r = 0; r < n; ++r) {
+            for (int64_t b = 0; b < nb; ++b) {
+                sd[b] = orc_f16_to_f64(scales[r * nb + b]);
+                bd[b] = fmt == 0 ? 0.0 : orc_f16_to_f64(biases[r * nb + b]);
+            }
             double acc = 0.0, am = 0.0;
             for (int64_t j = 0; j < k; ++j) {
                 double wdq;
                 if (fmt == 0) {
                     const int8_t* c = (const int8_t*)codes;
-                    wdq = (double)c[r * k + j] *
-                          orc_f16_to_f64(scales[r * (k / 32) + j / 32]);
+                    wdq = (double)c[r * k + j] * sd[j / 32];
                 } else {
                     const uint8_t* c = (const uint8_t*)codes;
                     uint8_t byte = c[r * (k / 2) + j / 2];
                     int q = (j & 1) ? (byte >> 4) : (byte & 0x0F);
-                    wdq = (double)q * orc_f16_to_f64(scales[r * (k / 64) + j / 64]) +
-                          orc_f16_to_f64(biases[r * (k / 64) + j / 64]);
+                    wdq = (double)q * sd[j / 64] + bd[j / 64];
                 }
-                double p = wdq * orc_f16_to_f64(x[j]);
+                double p = wdq * xd[j];
                 acc += p;
                 am += fabs(p);
             }
             if (y) y[r] = acc;
             if (mag) mag[r] = am;
         }
+        free(sd);
+        free(bd);
+    }
+    free(xd);
 }
 
 /* ------------------------------------------------------------- SwiGLU --- */
@@ -251,3 +274,7 @@ int64_t orc_argmax(const double* v, int64_t n) {
         if (v[i] > v[best]) best = i;
     return best;
 }
+
+/* ------------------------------------------------------------ threads --- */
+
+int orc_num_threads(void) { return omp_get_max_threads(); }

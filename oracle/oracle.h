@@ -95,6 +95,9 @@ double orc_ulp_f16(double v);
 /* Greedy argmax: the smallest index holding the largest value. */
 int64_t orc_argmax(const double* v, int64_t n);
 
+/* Threads the parallel row loops use (OpenMP). */
+int orc_num_threads(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,101 @@
+"""The C-ABI library without a GPU: it loads, exports exactly what
+include/qgemv.h declares, and rejects bad arguments synchronously with a status
+code (validation runs on the host before any CUDA call, so these calls never
+launch anything)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from int4_quantized_decode_b200 import build as qbuild
+from int4_quantized_decode_b200 import qgemv as qg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qgemv.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    qbuild.build()
+    return qg.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"QG_API\s+[\w\s\*]+?\b(qg_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert header_functions() == sorted(qg.ABI_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in header_functions():
+        assert hasattr(L, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", qg.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = sorted(set(m for m in re.findall(r" T (qg_\w+)", out)))
+    assert exported == header_functions()
+
+
+def test_status_strings_and_version(L):
+    for code, name in qg.STATUS_NAMES.items():
+        assert qg.status_string(code).startswith(name)
+    assert qg.status_string(99) == "QG_ERR_UNKNOWN"
+    assert L.qg_abi_version() == 100
+    assert L.qg_head_argmax_workspace_bytes(151936) >= 16
+
+
+def W(fmt=0, n=8, k=64, codes=0x1000, scales=0x2000, biases=0x3000):
+    return qg.CWeight(fmt, 0, n, k, codes, scales, biases)
+
+
+def gemv(L, w, x=0x4000, y=0x5000, y16=None):
+    return L.qg_gemv_s1(ctypes.byref(w) if w is not None else None, x, y, y16, None)
+
+
+def test_gemv_validation(L):
+    assert gemv(L, None) == 1                                  # NULL weight
+    assert gemv(L, W(fmt=7)) == 4                              # unknown format
+    assert gemv(L, W(codes=0)) == 1
+    assert gemv(L, W(scales=0)) == 1
+    assert gemv(L, W(fmt=1, k=128, biases=0)) == 1             # int4 needs biases
+    assert gemv(L, W(k=48)) == 2                               # k % 32
+    assert gemv(L, W(fmt=1, k=96)) == 2                        # k % 64
+    assert gemv(L, W(n=0)) == 2
+    assert gemv(L, W(codes=0x1008)) == 3                       # 16-byte codes
+    assert gemv(L, W(scales=0x2002)) == 3
+    assert gemv(L, W(), x=0) == 1
+    assert gemv(L, W(), y=0, y16=None) == 1                    # need an output
+    assert gemv(L, W(), x=0x4008) == 3
+    assert gemv(L, W(), y=0x5002) == 3
+
+
+def test_gemm_s16_and_swiglu_validation(L):
+    w = W()
+    assert L.qg_gemm_s16(ctypes.byref(w), 0x4000, 0, 0x5000, None) == 2
+    assert L.qg_gemm_s16(ctypes.byref(w), 0x4000, 17, 0x5000, None) == 2
+    assert L.qg_gemm_s16(ctypes.byref(w), None, 4, 0x5000, None) == 1
+    w4 = W(fmt=1, k=256)
+    assert L.qg_gemm_s16(ctypes.byref(w4), 0x4000, 4, 0x5000, None) == 4
+    wg, wu = W(), W(fmt=1, k=64)
+    assert L.qg_gate_up_swiglu(ctypes.byref(wg), ctypes.byref(wu), 0x4000, 1, 0x6000, None) == 4
+    wu2 = W(n=16)
+    assert L.qg_gate_up_swiglu(ctypes.byref(wg), ctypes.byref(wu2), 0x4000, 1, 0x6000, None) == 2
+    assert L.qg_gate_up_swiglu(ctypes.byref(wg), ctypes.byref(wg), 0x4000, 1, None, None) == 1
+
+
+def test_head_and_quantize_validation(L):
+    w = W()
+    assert L.qg_head_argmax(ctypes.byref(w), 0x4000, None, 0x5000, None, 256, None) == 5
+    assert L.qg_head_argmax(ctypes.byref(w), 0x4000, None, 0x5000, 0x7000, 8, None) == 5
+    assert L.qg_head_argmax(ctypes.byref(w), 0x4000, None, None, 0x7000, 256, None) == 1
+    assert L.qg_head_argmax(ctypes.byref(w), 0x4000, None, 0x5000, 0x7008, 256, None) == 3
+    assert L.qg_quantize_block32(None, 4, 64, 0x1000, 0x2000, None) == 1
+    assert L.qg_quantize_block32(0x1000, 4, 40, 0x1000, 0x2000, None) == 2
+    assert L.qg_quantize_block32(0x1004, 4, 64, 0x1000, 0x2000, None) == 3
+    assert L.qg_quantize_int4_g64(0x1000, 4, 64, 0x1000, 0x2000, None, None) == 1
+    assert L.qg_quantize_int4_g64(0x1000, 4, 96, 0x1000, 0x2000, 0x3000, None) == 2

@@ -1,0 +1,86 @@
+"""S <= 16 chunked-prefill GEMM (tensor cores) vs the fp64 oracle, and the
+chunk-consistency invariant: every row of the chunk agrees with the S=1 GEMV
+within the same bound, and the head argmax of the last row is the same
+("Qwen3.8-27B ... -- Core AI", The vision path: chunked vs S=1 prefill must
+give the same greedy tokens)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import assert_codes_equal, assert_within_bound, oracle_gemv
+from int4_quantized_decode_b200 import qgemv as qg
+from int4_quantized_decode_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+I8 = qg.FMT_I8_B32
+
+
+@pytest.mark.parametrize("n,k,S", [(1, 256, 16), (64, 256, 16), (100, 512, 3), (1000, 2048, 16),
+                                   (4096, 4096, 16), (6144, 4096, 7), (4096, 12288, 16),
+                                   (333, 1280, 2), (2050, 768, 16)])
+def test_gemm_s16_parity(cuda, n, k, S):
+    w = wl.weight_fp32(n, k, 300 + S, cuda)
+    W = qg.quantize(w, I8)
+    X = wl.act_fp16((S, k), 400 + n % 13, cuda)
+    Y = torch.full((S, n), float("nan"), dtype=torch.float32, device=cuda)
+    qg.qg_gemm_s16(W, X, Y)
+    qg.qg_stream_check()
+    if n * k <= 16 * 2**20:
+        assert_codes_equal(W, w)
+    Yd = Y.cpu().numpy()
+    y1 = torch.empty(n, dtype=torch.float32, device=cuda)
+    for s in range(S):
+        yr, mag = oracle_gemv(W, X[s])
+        assert_within_bound(Yd[s], yr, mag)
+        # chunk consistency: the S=1 path on the same row is within the bound too
+        qg.qg_gemv_s1(W, X[s], y1)
+        assert_within_bound(y1.cpu().numpy(), yr, mag)
+
+
+def test_gemm_s16_deterministic(cuda):
+    n, k, S = 4096, 4096, 16
+    W = qg.quantize(wl.weight_fp32(n, k, 5, cuda), I8)
+    X = wl.act_fp16((S, k), 6, cuda)
+    Y1 = torch.empty((S, n), dtype=torch.float32, device=cuda)
+    Y2 = torch.empty_like(Y1)
+    qg.qg_gemm_s16(W, X, Y1)
+    qg.qg_gemm_s16(W, X, Y2)
+    qg.qg_stream_check()
+    assert torch.equal(Y1, Y2)
+
+
+@pytest.mark.parametrize("n,k,S", [(12288, 4096, 16), (77, 512, 5), (1000, 2048, 16)])
+def test_swiglu_s16(cuda, n, k, S):
+    Wg = qg.quantize(wl.weight_fp32(n, k, 61, cuda), I8)
+    Wu = qg.quantize(wl.weight_fp32(n, k, 62, cuda), I8)
+    X = wl.act_fp16((S, k), 63, cuda)
+    H = torch.empty((S, n), dtype=torch.float16, device=cuda)
+    qg.qg_gate_up_swiglu(Wg, Wu, X, H)
+    qg.qg_stream_check()
+    Hd = H.cpu().numpy().astype(np.float64)
+    h1 = torch.empty(n, dtype=torch.float16, device=cuda)
+    for s in range(S):
+        gr, mg = oracle_gemv(Wg, X[s])
+        ur, mu = oracle_gemv(Wu, X[s])
+        hr, hb = oracle.swiglu(gr, ur, mg, mu, oracle.GEMV_TOL)
+        assert np.all(np.abs(Hd[s] - hr) <= hb)
+        qg.qg_gate_up_swiglu(Wg, Wu, X[s], h1)               # S=1 path, same row
+        assert np.all(np.abs(h1.cpu().numpy().astype(np.float64) - hr) <= hb)
+
+
+def test_chunk_head_argmax_matches_s1(cuda):
+    """The head argmax of the chunk's last row equals the S=1 decode's."""
+    V, H, S = 151936, 4096, 16
+    Wh = qg.quantize(wl.weight_fp32(V, H, wl.QWEN3VL_8B.weight_seed(-1, "head"), cuda), I8)
+    X = wl.act_fp16((S, H), 71, cuda)
+    ws = qg.head_workspace(V, cuda)
+    i16 = torch.zeros(1, dtype=torch.int32, device=cuda)
+    qg.qg_head_argmax(Wh, X[S - 1], i16, ws)
+    x1 = X[S - 1].clone()                                   # the same token decoded alone
+    i1 = torch.zeros(1, dtype=torch.int32, device=cuda)
+    qg.qg_head_argmax(Wh, x1, i1, ws)
+    qg.qg_stream_check()
+    assert int(i16.item()) == int(i1.item())
+    yr, _ = oracle_gemv(Wh, X[S - 1])
+    assert oracle.argmax_ok(int(i16.item()), yr)

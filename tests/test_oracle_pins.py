@@ -395,3 +395,14 @@ def test_bundle_sizes_printed_on_pages():
     for dec, head, printed in rows:
         if head == "int8":
             assert not _size_matches(_bundle_gib(dec, head, 1.125), printed)
+
+
+def test_int4_signed_zero_group_gives_positive_zero_side_data():
+    """A group of +0 and -0 has min = max = 0; its scale and bias are +0."""
+    w = np.zeros((1, 64), dtype=np.float32)
+    w[0, 1::2] = -0.0
+    codes, scales, biases = oracle.quantize_int4_g64(w)
+    assert scales[0, 0] == 0 and biases[0, 0] == 0 and (codes == 0).all()
+    w2 = -np.zeros((1, 64), dtype=np.float32)
+    codes, scales, biases = oracle.quantize_int4_g64(w2)
+    assert scales[0, 0] == 0 and biases[0, 0] == 0
