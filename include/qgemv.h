@@ -187,6 +187,10 @@ QG_API qg_status qg_stream_check(cudaStream_t stream);
 /* Human-readable name of a status code (static string). */
 QG_API const char* qg_status_string(qg_status status);
 
+/* Name of the CUDA error behind the calling thread's most recent QG_ERR_CUDA
+ * ("cudaSuccess" if there was none); a static string. */
+QG_API const char* qg_last_cuda_error(void);
+
 /* ABI version of this header (major * 100 + minor). */
 QG_API int qg_abi_version(void);
 

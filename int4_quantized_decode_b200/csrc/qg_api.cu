@@ -6,11 +6,18 @@
 
 namespace qg {
 
+namespace {
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+}
+
 qg_status cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return QG_OK;
+    t_last_cuda_error = e;
     (void)cudaGetLastError();  // clear a non-sticky error
     return QG_ERR_CUDA;
 }
+
+const char* last_cuda_error_name() { return cudaGetErrorName(t_last_cuda_error); }
 
 qg_status device_info(DeviceInfo* out) {
     static DeviceInfo cache[64];
@@ -61,6 +68,8 @@ qg_status check_weight(const qg_weight* W) {
 extern "C" {
 
 int qg_abi_version(void) { return 100; }
+
+const char* qg_last_cuda_error(void) { return qg::last_cuda_error_name(); }
 
 const char* qg_status_string(qg_status s) {
     switch (s) {

@@ -417,13 +417,15 @@ template <int FMT, int NMAT, int RG, int EPI, bool SC>
 qg_status launch_t(const Params& p, const DeviceInfo& dev, cudaStream_t stream) {
     auto kern = gemv_s1_kernel<FMT, NMAT, RG, EPI, SC>;
     const size_t smem = smem_bytes<FMT, NMAT, RG, EPI, SC>(p);
-    if (smem > static_cast<size_t>(dev.max_smem_optin)) return QG_ERR_SHAPE;
-    static int attr_done[64] = {0};
-    if (dev.device < 64 && !attr_done[dev.device]) {
+    if (smem + 1024 > static_cast<size_t>(dev.max_smem_optin)) return QG_ERR_SHAPE;
+    // Opt in to exactly the dynamic shared memory this launch needs (static
+    // shared memory counts against the same per-block limit).
+    static size_t attr_set[64] = {0};
+    if (dev.device >= 64 || attr_set[dev.device] < smem) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(dev.max_smem_optin));
+                                             static_cast<int>(smem));
         if (e != cudaSuccess) return cuda_status(e);
-        attr_done[dev.device] = 1;
+        if (dev.device < 64) attr_set[dev.device] = smem;
     }
     const int64_t items = (p.n + RG - 1) / RG;
     int64_t grid = (items + kNumWarps - 1) / kNumWarps;

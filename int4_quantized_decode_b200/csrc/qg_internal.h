@@ -16,8 +16,10 @@ struct DeviceInfo {
 };
 qg_status device_info(DeviceInfo* out);
 
-// Map the last CUDA error (if any) to a status, clearing it.
+// Map a CUDA error (if any) to a status, clearing it and remembering its name
+// for qg_last_cuda_error().
 qg_status cuda_status(cudaError_t e);
+const char* last_cuda_error_name();
 
 // Epilogues of the S=1 streaming kernel.
 enum GemvEpilogue : int { kEpiPlain = 0, kEpiSwiglu = 1, kEpiHead = 2 };

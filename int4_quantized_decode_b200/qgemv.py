@@ -28,13 +28,17 @@ FMT_I4_G64 = 1
 # every symbol include/qgemv.h declares
 ABI_SYMBOLS = ("qg_quantize_block32", "qg_quantize_int4_g64", "qg_gemv_s1",
                "qg_gemm_s16", "qg_gate_up_swiglu", "qg_head_argmax_workspace_bytes",
-               "qg_head_argmax", "qg_stream_check", "qg_status_string", "qg_abi_version")
+               "qg_head_argmax", "qg_stream_check", "qg_status_string", "qg_abi_version",
+               "qg_last_cuda_error")
 
 
 class QgError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} failed: {status_string(status)}")
+        msg = f"{fn} failed: {status_string(status)}"
+        if status == 6:
+            msg += f" ({lib().qg_last_cuda_error().decode()})"
+        super().__init__(msg)
 
 
 class CWeight(ctypes.Structure):
@@ -70,8 +74,11 @@ def lib() -> ctypes.CDLL:
         L.qg_status_string.argtypes = [I]
         L.qg_status_string.restype = ctypes.c_char_p
         L.qg_abi_version.argtypes = []
+        L.qg_last_cuda_error.argtypes = []
+        L.qg_last_cuda_error.restype = ctypes.c_char_p
         for name in ABI_SYMBOLS:
-            if name not in ("qg_head_argmax_workspace_bytes", "qg_status_string"):
+            if name not in ("qg_head_argmax_workspace_bytes", "qg_status_string",
+                            "qg_last_cuda_error"):
                 getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
