@@ -177,6 +177,31 @@ QG_API qg_status qg_head_argmax(const qg_weight* W, const uint16_t* x, float* lo
                          cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * qg_head_argmax_noalloc -- qg_head_argmax for callers that cannot allocate
+ * device memory.  The pages have no counterpart to this call; it exists for
+ * callers that cannot provide a workspace: a plugin or custom operator whose
+ * host framework owns and budgets every device allocation, or a
+ * latency-critical loop where a device allocation is not acceptable.
+ * Same arguments, results and accuracy as qg_head_argmax, minus the workspace:
+ * the reduction scratch is a 256-byte array inside the library that every GPU
+ * loading the library keeps until the process exits.  The call allocates
+ * nothing (no cudaMalloc, no cudaFree, no allocating library routine).
+ *   - The first call on each device looks up that array's device address
+ *     (cudaGetSymbolAddress, with the device current); make that first call
+ *     before capturing any stream into a CUDA graph.
+ *   - Each call clears the scratch on `stream` before the kernel runs (an
+ *     asynchronous memset of 256 bytes), because the array keeps what the
+ *     previous call left there.
+ *   - All calls on a device share the one array: calls that overlap on the
+ *     GPU (different streams without ordering between them) race and give
+ *     wrong indices.  Serialize them.
+ *   - A weight whose argmax would need more scratch than the 256 bytes is
+ *     refused with QG_ERR_WORKSPACE (today every n needs 16 bytes).
+ * ------------------------------------------------------------------------- */
+QG_API qg_status qg_head_argmax_noalloc(const qg_weight* W, const uint16_t* x, float* logits,
+                                        int32_t* idx, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * qg_stream_check -- synchronize `stream` and report asynchronous failures:
  * QG_ERR_CUDA for a CUDA error, QG_ERR_TIMEOUT if a kernel's bounded wait on
  * its own bulk copies expired since the last check (the flag is then

@@ -29,7 +29,7 @@ FMT_I4_G64 = 1
 ABI_SYMBOLS = ("qg_quantize_block32", "qg_quantize_int4_g64", "qg_gemv_s1",
                "qg_gemm_s16", "qg_gate_up_swiglu", "qg_head_argmax_workspace_bytes",
                "qg_head_argmax", "qg_stream_check", "qg_status_string", "qg_abi_version",
-               "qg_last_cuda_error")
+               "qg_last_cuda_error", "qg_head_argmax_noalloc")
 
 
 class QgError(RuntimeError):
@@ -70,6 +70,7 @@ def lib() -> ctypes.CDLL:
         L.qg_head_argmax_workspace_bytes.argtypes = [I64]
         L.qg_head_argmax_workspace_bytes.restype = ctypes.c_size_t
         L.qg_head_argmax.argtypes = [W, P, P, P, P, ctypes.c_size_t, P]
+        L.qg_head_argmax_noalloc.argtypes = [W, P, P, P, P]
         L.qg_stream_check.argtypes = [P]
         L.qg_status_string.argtypes = [I]
         L.qg_status_string.restype = ctypes.c_char_p
@@ -78,7 +79,7 @@ def lib() -> ctypes.CDLL:
         L.qg_last_cuda_error.restype = ctypes.c_char_p
         for name in ABI_SYMBOLS:
             if name not in ("qg_head_argmax_workspace_bytes", "qg_status_string",
-                            "qg_last_cuda_error"):
+                            "qg_last_cuda_error", "qg_head_argmax_noalloc"):
                 getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -232,6 +233,20 @@ def qg_head_argmax(W: QWeight, x: torch.Tensor, idx: torch.Tensor, workspace: to
     _check("qg_head_argmax",
            lib().qg_head_argmax(ctypes.byref(cw), _ptr(x), _ptr(logits), _ptr(idx),
                                 _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def qg_head_argmax_noalloc(W: QWeight, x: torch.Tensor, idx: torch.Tensor,
+                           logits: Optional[torch.Tensor] = None, stream=None) -> None:
+    """qg_head_argmax without a caller workspace (the library's built-in
+    scratch; calls must not overlap on the GPU)."""
+    _cuda(x, torch.float16, "x")
+    _cuda(idx, torch.int32, "idx")
+    if logits is not None:
+        _cuda(logits, torch.float32, "logits")
+    cw = W.c()
+    _check("qg_head_argmax_noalloc",
+           lib().qg_head_argmax_noalloc(ctypes.byref(cw), _ptr(x), _ptr(logits), _ptr(idx),
+                                        _stream(stream)))
 
 
 def qg_stream_check(stream=None) -> None:
