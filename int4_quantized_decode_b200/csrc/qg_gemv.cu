@@ -4,29 +4,31 @@
 // group-64 weight, with three epilogues: plain (fp32 and/or fp16 out), fused
 // gate/up SwiGLU (two weights, fp16 h out) and fused LM-head argmax.  The
 // pages ("Qwen3-VL 4B -- Core AI (.aimodel)", Measured) state that decode is
-// bound by reading the weights once per token, so the design goal is to keep
-// HBM busy:
+// bound by reading every weight once per token, so the kernel is built to keep
+// HBM saturated:
 //
-//  * Persistent CTAs (one per SM, 8 warps).  Every warp owns a private ring of
-//    STAGES shared-memory stages and streams its rows through it with 1-D bulk
-//    async copies (cp.async.bulk, mbarrier completion, L2 evict-first, never
-//    multicast).  A stage is RG rows (x NMAT weights) by 512 code bytes plus
-//    the matching fp16 scales (and biases).  Bytes in flight per SM =
-//    8 warps x STAGES x stage size, independent of registers.
-//  * The activation x (fp16) is staged once per CTA into shared memory as
-//    fp32, laid out so that each lane's 16-byte reads are bank-conflict free.
+//  * Codes and scales stream straight from HBM into registers with 16-byte
+//    coalesced vector loads (L1 bypassed, L2 evict-first).  Each lane keeps
+//    DEPTH-1 steps of loads in flight while it computes; a warp owns RG rows
+//    (x NMAT weights) at a time, so 64-128 bytes per lane are outstanding.
+//    (On this GPU a plain 16-byte load stream reaches ~7.3 TB/s, while 1-D
+//    bulk copies need >= 16 KB per copy to get there: every bulk copy carries
+//    a fixed cost, and rows of 2-6 KB would pay it too often.)
+//  * x (fp16) is staged once per CTA into shared memory as fp32, in a layout
+//    where each 8-lane phase of a 16-byte read hits distinct banks; one x read
+//    serves all RG rows of the warp.
 //  * Dequantization happens in registers with no int->float conversion
-//    instruction: int8 codes become floats by byte-permuting them into the
-//    mantissa of 2^23 and subtracting the offset; int4 nibbles by masking them
-//    into that mantissa in place.  Products accumulate in fp32 with the packed
-//    sm_100 f32x2 FMA; each block's fp16 scale is applied once per 16/32
-//    codes; the int4 bias uses sum_k (q s + b) x = s sum q x + b sum x with
-//    the per-half-group sum of x computed once per CTA.
+//    instruction: int8 codes are byte-permuted into the mantissa of 2^23 and
+//    the offset subtracted; int4 nibbles are masked in place into that
+//    mantissa.  Products accumulate in fp32 with the packed sm_100 f32x2 FMA;
+//    each block's fp16 scale is applied once per 16 (int8) or 32 (int4)
+//    codes; the int4 bias uses sum_k (q s + b) x = s sum q x + b sum x with the
+//    per-half-group sums of x computed once per CTA.
 //  * Lanes split K within a row; a warp-shuffle reduction finishes each row.
-//  * Programmatic dependent launch: the weight prologue (first STAGES bulk
-//    copies) is issued before griddepcontrol.wait, so a kernel's weight
-//    stream overlaps the tail of the previous kernel in the stream; only the
-//    x staging waits for it.
+//  * Programmatic dependent launch: before waiting on the previous kernel in
+//    the stream, every warp asks L2 to prefetch (cp.async.bulk.prefetch.L2) the
+//    first rows it will read, so a kernel's weight stream overlaps the tail of
+//    the kernel before it; only x waits for that kernel.
 #include <cfloat>
 #include <climits>
 
@@ -40,26 +42,20 @@ QG_DEFINE_ERROR_FLAG(g_gemv_err);
 namespace {
 
 constexpr int kLanes = 32;
-constexpr int kNumWarps = 8;
-constexpr int kStages = 4;
-constexpr int kStageRowBytes = 512;   // code bytes per row per stage
-constexpr int kStageSideBytes = 32;   // scale (or bias) bytes per row per stage
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * kLanes;
+// Two CTAs (16 warps) per SM: measured faster than one CTA per SM that would
+// leave room for the next kernel to become resident early; the latency hiding
+// of 16 warps is worth more than that overlap.
+constexpr int kCtasPerSm = 2;
+constexpr int kPrefetchBytesPerWarp = 12 * 1024;
 
 template <int FMT>
 struct Fmt {
-    static constexpr int kCodesPerStage = FMT == 0 ? 512 : 1024;
-    static constexpr int kCodesPerLane = FMT == 0 ? 16 : 32;
+    static constexpr int kCodesPerLane = FMT == 0 ? 16 : 32;   // one 16-byte vector
     static constexpr int kBlock = FMT == 0 ? 32 : 64;
-    static constexpr int kPieces = kCodesPerLane / 4;  // float4 pieces of x per lane
+    static constexpr int kPieces = kCodesPerLane / 4;           // float4 pieces of x per lane
     static constexpr bool kBias = FMT == 1;
-};
-
-template <int FMT, int ROWS>
-struct Stage {
-    static constexpr int kCodes = ROWS * kStageRowBytes;
-    static constexpr int kScales = ROWS * kStageSideBytes;
-    static constexpr int kBiases = Fmt<FMT>::kBias ? ROWS * kStageSideBytes : 0;
-    static constexpr int kBytes = kCodes + kScales + kBiases;
 };
 
 struct Params {
@@ -75,11 +71,34 @@ struct Params {
     int32_t* idx;
     unsigned long long* ws_key;
     unsigned int* ws_ticket;
-    int x_floats;  // floats reserved for x in shared memory
+    int x_floats;        // floats reserved for x in shared memory
+    int prefetch_items;  // items per warp prefetched into L2 before the wait
 };
 
 __host__ __device__ constexpr int align_up(int v, int a) { return (v + a - 1) / a * a; }
-__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// ------------------------------------------------------------- loads -----
+__device__ __forceinline__ uint4 ldg_stream_v4(const void* p, uint64_t pol) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+
+__device__ __forceinline__ uint16_t ldg_stream_u16(const void* p, uint64_t pol) {
+    uint16_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.u16 %0, [%1], %2;"
+                 : "=h"(v)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+
+// Ask L2 to fetch [p, p + bytes) (16-byte aligned, multiple of 16): a hint
+// that needs no shared memory and no completion tracking.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 
 // ------------------------------------------------------------ dot products --
 // 16 int8 codes (one 16-byte vector) against 16 fp32 activations.
@@ -134,7 +153,7 @@ __device__ __forceinline__ float dot32_i4(const uint4 c, const float4* xv) {
 }
 
 // float4 index of piece `i` of lane-granule `g` in the staged x: the eight
-// granules read by one 8-lane phase of an LDS.128 are adjacent.
+// granules read by one 8-lane phase of a 16-byte shared load are adjacent.
 template <int FMT>
 __device__ __forceinline__ int x_piece(int g, int i) {
     return ((g >> 3) * Fmt<FMT>::kPieces + i) * 8 + (g & 7);
@@ -147,91 +166,128 @@ __device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
            static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(idx));
 }
 
-template <int FMT, int NMAT, int RG, int EPI, bool SC_TMA>
-__global__ void __launch_bounds__(kNumWarps* kLanes, 1) gemv_s1_kernel(const Params p) {
+// Steps of loads kept in the register pipeline: enough that (DEPTH-1) x rows
+// x 16 bytes per lane stay outstanding (an int4 vector carries twice the
+// weights and needs more registers to dequantize, so its pipeline is shorter).
+template <int FMT, int ROWS>
+struct Depth {
+    static constexpr int value = FMT == 0 ? (ROWS >= 8 ? 2 : (ROWS >= 4 ? 3 : (ROWS >= 2 ? 5 : 8)))
+                                          : (ROWS >= 4 ? 2 : (ROWS >= 2 ? 3 : 6));
+};
+
+template <int ROWS>
+struct Frag {
+    uint4 c[ROWS];
+    uint16_t s[ROWS];
+    uint16_t b[ROWS];
+};
+
+template <int FMT, int NMAT, int RG, int EPI>
+__global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
     using F = Fmt<FMT>;
     constexpr int ROWS = NMAT * RG;
-    using L = Stage<FMT, ROWS>;
-    constexpr int kBarBytes = align_up(kNumWarps * kStages * 8, 128);
-
+    constexpr int DEPTH = Depth<FMT, ROWS>::value;
+    constexpr int kStepBytes = kLanes * 16;  // code bytes of one warp step along a row
+    constexpr int kStepSides = kStepBytes * (FMT == 0 ? 1 : 2) / F::kBlock;  // scales per step
     extern __shared__ __align__(128) unsigned char smem[];
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem) + warp * kStages;
-    unsigned char* ring = smem + kBarBytes + warp * kStages * L::kBytes;
-    float* xs = reinterpret_cast<float*>(smem + kBarBytes + kNumWarps * kStages * L::kBytes);
-    float* hsum = xs + p.x_floats;  // int4: per-lane-granule sum of x
-    __shared__ float red_v[kNumWarps];
-    __shared__ int red_i[kNumWarps];
+    float* xs = reinterpret_cast<float*>(smem);
+    float* hsum = xs + p.x_floats;  // int4: per lane-granule sum of x
+    __shared__ float red_v[kWarps];
+    __shared__ int red_i[kWarps];
 
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t N = p.n, K = p.k;
-    const int nst = static_cast<int>((K + F::kCodesPerStage - 1) / F::kCodesPerStage);
+    const int granules = static_cast<int>(K / F::kCodesPerLane);  // 16-byte vectors per row
+    const int nst = (granules + kLanes - 1) / kLanes;              // warp steps per row
     const int64_t items = (N + RG - 1) / RG;
-    const int64_t wg = static_cast<int64_t>(blockIdx.x) * kNumWarps + warp;
-    const int64_t tw = static_cast<int64_t>(gridDim.x) * kNumWarps;
-    const int64_t my_items = wg < items ? (items - wg + tw - 1) / tw : 0;
-    const int64_t total = my_items * nst;
+    const int64_t wg = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+    const int64_t tw = static_cast<int64_t>(gridDim.x) * kWarps;
+    const int my_items = wg < items ? static_cast<int>((items - wg + tw - 1) / tw) : 0;
+    const int total = my_items * nst;
     const int64_t row_bytes = FMT == 0 ? K : K / 2;
     const int64_t side_per_row = K / F::kBlock;  // fp16 scales (biases) per row
-
-    if (lane == 0) {
-#pragma unroll
-        for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
-        fence_mbar_init();
-    }
-    __syncwarp();
     const uint64_t pol = l2_policy_evict_first();
 
-    // Producer step (lane 0): bring stage t of this warp's sequence into slot
-    // t % kStages.  Stage t is (item t / nst, K-chunk t % nst).
-    auto issue = [&](int64_t t) {
-        const int64_t il = t / nst;
-        const int st = static_cast<int>(t - il * nst);
+    // ---- load cursor: per-row pointers of the next step to load (lane offset
+    // included), advanced by a constant per step and rebuilt once per item.
+    const uint8_t* lc[ROWS];
+    const uint16_t* ls[ROWS];
+    const uint16_t* lb[ROWS];
+    int ld_st = 0, ld_item = 0;
+    auto set_item = [&](int il) {
         const int64_t r0 = (wg + il * tw) * RG;
-        const int rows = static_cast<int>(min64(RG, N - r0));
-        const int64_t k0 = static_cast<int64_t>(st) * F::kCodesPerStage;
-        const int kc = static_cast<int>(min64(F::kCodesPerStage, K - k0));
-        const uint32_t cbytes = FMT == 0 ? kc : kc / 2;
-        const uint32_t sbytes = static_cast<uint32_t>(kc / F::kBlock) * 2u;
-        unsigned char* stage = ring + (t % kStages) * L::kBytes;
-        uint64_t* bar = &bars[t % kStages];
-        uint32_t tx = cbytes;
-        if (SC_TMA) tx += F::kBias ? 2u * sbytes : sbytes;
-        mbar_arrive_expect_tx(bar, tx * static_cast<uint32_t>(rows * NMAT));
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
-            for (int j = 0; j < rows; ++j) {
-                const int64_t r = r0 + j;
-                const int slot_row = m * RG + j;
-                bulk_g2s(stage + slot_row * kStageRowBytes,
-                         p.codes[m] + r * row_bytes + (FMT == 0 ? k0 : k0 / 2), cbytes, bar, pol);
-                if (SC_TMA) {
-                    const int64_t so = r * side_per_row + k0 / F::kBlock;
-                    bulk_g2s(stage + L::kCodes + slot_row * kStageSideBytes, p.scales[m] + so,
-                             sbytes, bar, pol);
-                    if (F::kBias)
-                        bulk_g2s(stage + L::kCodes + L::kScales + slot_row * kStageSideBytes,
-                                 p.biases[m] + so, sbytes, bar, pol);
-                }
+            const uint8_t* cm = m == 0 ? p.codes[0] : p.codes[1];
+            const uint16_t* sm = m == 0 ? p.scales[0] : p.scales[1];
+            const uint16_t* bm = m == 0 ? p.biases[0] : p.biases[1];
+#pragma unroll
+            for (int j = 0; j < RG; ++j) {
+                const int64_t r = r0 + j < N ? r0 + j : N - 1;  // tail rows: load, discard
+                lc[m * RG + j] = cm + r * row_bytes + lane * 16;
+                ls[m * RG + j] = sm + r * side_per_row + (lane >> 1);
+                if (F::kBias) lb[m * RG + j] = bm + r * side_per_row + (lane >> 1);
+            }
+        }
+    };
+    auto load = [&](Frag<ROWS>& f) {
+        if (ld_st * kLanes + lane < granules) {
+#pragma unroll
+            for (int j = 0; j < ROWS; ++j) {
+                f.c[j] = ldg_stream_v4(lc[j], pol);
+                f.s[j] = ldg_stream_u16(ls[j], pol);
+                if (F::kBias) f.b[j] = ldg_stream_u16(lb[j], pol);
+            }
+        }
+        if (++ld_st == nst) {
+            ld_st = 0;
+            if (++ld_item < my_items) set_item(ld_item);
+        } else {
+#pragma unroll
+            for (int j = 0; j < ROWS; ++j) {
+                lc[j] += kStepBytes;
+                ls[j] += kStepSides;
+                if (F::kBias) lb[j] += kStepSides;
             }
         }
     };
 
-    // 1) weight prologue: independent of the previous kernel in the stream.
+    // 1) Weight prologue, independent of the previous kernel in the stream:
+    //    the first DEPTH steps go straight into registers, and L2 is asked to
+    //    prefetch the next rows of this warp.
+    Frag<ROWS> buf[DEPTH];
+    if (my_items > 0) set_item(0);
+#pragma unroll
+    for (int d = 0; d < DEPTH; ++d)
+        if (d < total) load(buf[d]);
     if (lane == 0) {
-        const int64_t pre = total < kStages ? total : kStages;
-        for (int64_t t = 0; t < pre; ++t) issue(t);
+        for (int i = 1; i < p.prefetch_items && i < my_items; ++i) {
+            const int64_t r0 = (wg + i * tw) * RG;
+            const int64_t rows = N - r0 < RG ? N - r0 : RG;
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m) {
+                const uint8_t* cm = m == 0 ? p.codes[0] : p.codes[1];
+                prefetch_l2(cm + r0 * row_bytes, static_cast<uint32_t>(rows * row_bytes));
+                const uintptr_t sa = reinterpret_cast<uintptr_t>(
+                    (m == 0 ? p.scales[0] : p.scales[1]) + r0 * side_per_row);
+                const uint32_t sbytes = static_cast<uint32_t>(rows * side_per_row * 2);
+                if (sa % 16 == 0 && sbytes % 16 == 0) {
+                    prefetch_l2(reinterpret_cast<const void*>(sa), sbytes);
+                    if (F::kBias)
+                        prefetch_l2((m == 0 ? p.biases[0] : p.biases[1]) + r0 * side_per_row,
+                                    sbytes);
+                }
+            }
+        }
     }
 
-    // 2) the activation is produced by the previous kernel: wait for it, then
-    //    stage it as fp32 in the conflict-free layout (int4: pair-permuted and
-    //    with the half-group sums).
+    // 2) x is produced by the previous kernel: wait for it, then stage it as
+    //    fp32 (int4: pair-permuted, plus the half-group sums).
     griddep_wait();
     {
-        const int granules = static_cast<int>(K / F::kCodesPerLane);
-        for (int g = threadIdx.x; g < granules; g += blockDim.x) {
+        float4* xs4 = reinterpret_cast<float4*>(xs);
+        for (int g = threadIdx.x; g < granules; g += kThreads) {
             const uint16_t* xg = p.x + static_cast<int64_t>(g) * F::kCodesPerLane;
-            float4* xs4 = reinterpret_cast<float4*>(xs);
             float gsum = 0.f;
 #pragma unroll
             for (int c = 0; c < F::kCodesPerLane / 8; ++c) {
@@ -261,106 +317,75 @@ __global__ void __launch_bounds__(kNumWarps* kLanes, 1) gemv_s1_kernel(const Par
     __syncthreads();
     griddep_launch_dependents();
 
-    // 3) consume.
+    // 3) stream: the loads of steps t+1 .. t+DEPTH-1 are in flight while step
+    //    t is computed.  The x pieces of a lane advance by a constant per step.
+    const float4* xs4 = reinterpret_cast<const float4*>(xs);
+    const int x_lane = ((lane >> 3) * F::kPieces) * 8 + (lane & 7);  // x_piece(lane, 0)
+    constexpr int kXStep = 4 * F::kPieces * 8;                      // x_piece(g + 32) - x_piece(g)
     float acc[ROWS];
 #pragma unroll
     for (int j = 0; j < ROWS; ++j) acc[j] = 0.f;
     float best_v = -FLT_MAX;
     int best_i = INT_MAX;
-    bool failed = false;
-
-    int64_t t = 0;
-    for (int64_t il = 0; il < my_items && !failed; ++il) {
-        const int64_t r0 = (wg + il * tw) * RG;
-        for (int st = 0; st < nst; ++st, ++t) {
-            unsigned char* stage = ring + (t % kStages) * L::kBytes;
-            const bool ok = mbar_wait_bounded(&bars[t % kStages],
-                                              static_cast<uint32_t>((t / kStages) & 1));
-            if (!__all_sync(0xffffffffu, ok)) {
-                failed = true;
-                break;
+    int cu_st = 0, cu_item = 0;
+    auto consume = [&](const Frag<ROWS>& f) {
+        const int g = cu_st * kLanes + lane;
+        if (g < granules) {
+            float4 xv[F::kPieces];
+            const float4* xp = xs4 + x_lane + cu_st * kXStep;
+#pragma unroll
+            for (int i = 0; i < F::kPieces; ++i) xv[i] = xp[i * 8];
+            const float hs = FMT == 1 ? hsum[g] : 0.f;
+#pragma unroll
+            for (int j = 0; j < ROWS; ++j) {
+                if (FMT == 0)
+                    acc[j] = fmaf(h2f(f.s[j]), dot16_i8(f.c[j], xv), acc[j]);
+                else
+                    acc[j] = fmaf(h2f(f.s[j]), dot32_i4(f.c[j], xv), fmaf(h2f(f.b[j]), hs, acc[j]));
             }
-            const int g = st * kLanes + lane;  // lane-granule index within the row
-            if (static_cast<int64_t>(g) * F::kCodesPerLane < K) {
-                float4 xv[F::kPieces];
-                const float4* xs4 = reinterpret_cast<const float4*>(xs);
+        }
+        if (++cu_st == nst) {
+            // item done: finish its rows across lanes
+            const int64_t r0 = (wg + cu_item * tw) * RG;
 #pragma unroll
-                for (int i = 0; i < F::kPieces; ++i) xv[i] = xs4[x_piece<FMT>(g, i)];
-                const float hs = FMT == 1 ? hsum[g] : 0.f;
+            for (int j = 0; j < ROWS; ++j) acc[j] = warp_sum(acc[j]);
+            if (lane < RG && r0 + lane < N) {
+                const int64_t r = r0 + lane;
+                float v0 = acc[0], v1 = 0.f;
 #pragma unroll
-                for (int j = 0; j < ROWS; ++j) {
-                    const uint4 c =
-                        *reinterpret_cast<const uint4*>(stage + j * kStageRowBytes + lane * 16);
-                    uint16_t sb, bb = 0;
-                    if (SC_TMA) {
-                        sb = *reinterpret_cast<const uint16_t*>(stage + L::kCodes +
-                                                                j * kStageSideBytes + (lane >> 1) * 2);
-                        if (F::kBias)
-                            bb = *reinterpret_cast<const uint16_t*>(
-                                stage + L::kCodes + L::kScales + j * kStageSideBytes + (lane >> 1) * 2);
-                    } else {
-                        const int m = j / RG;
-                        const int64_t r = min64(r0 + (j % RG), N - 1);
-                        const int64_t so = r * side_per_row +
-                                           (static_cast<int64_t>(g) * F::kCodesPerLane) / F::kBlock;
-                        sb = ldg_nc_u16(p.scales[m] + so);
-                        if (F::kBias) bb = ldg_nc_u16(p.biases[m] + so);
+                for (int j = 0; j < RG; ++j)
+                    if (lane == j) {
+                        v0 = acc[j];
+                        if (NMAT == 2) v1 = acc[(NMAT - 1) * RG + j];
                     }
-                    if (FMT == 0) {
-                        acc[j] = fmaf(h2f(sb), dot16_i8(c, xv), acc[j]);
-                    } else {
-                        acc[j] = fmaf(h2f(sb), dot32_i4(c, xv), fmaf(h2f(bb), hs, acc[j]));
+                if (EPI == kEpiPlain) {
+                    if (p.y) p.y[r] = v0;
+                    if (p.y16) p.y16[r] = f2h_rn(v0);
+                } else if (EPI == kEpiSwiglu) {
+                    p.h[r] = f2h_rn(v0 / (1.0f + expf(-v0)) * v1);
+                } else {
+                    if (p.logits) p.logits[r] = v0;
+                    if (v0 > best_v) {  // rows arrive in increasing order per lane
+                        best_v = v0;
+                        best_i = static_cast<int>(r);
                     }
                 }
             }
-            __syncwarp();
-            if (lane == 0 && t + kStages < total) {
-                fence_proxy_async_smem();
-                issue(t + kStages);
+#pragma unroll
+            for (int j = 0; j < ROWS; ++j) acc[j] = 0.f;
+            cu_st = 0;
+            ++cu_item;
+        }
+    };
+
+    for (int t = 0; t < total; t += DEPTH) {
+#pragma unroll
+        for (int d = 0; d < DEPTH; ++d) {
+            if (t + d < total) {
+                consume(buf[d]);
+                if (t + d + DEPTH < total) load(buf[d]);
             }
         }
-        if (failed) break;
-
-        // item epilogue: finish the rows across lanes.
-#pragma unroll
-        for (int j = 0; j < ROWS; ++j) acc[j] = warp_sum(acc[j]);
-        if (lane < RG && r0 + lane < N) {
-            const int64_t r = r0 + lane;
-            float v0 = acc[0], v1 = 0.f;
-#pragma unroll
-            for (int j = 0; j < RG; ++j)
-                if (lane == j) {
-                    v0 = acc[j];
-                    if (NMAT == 2) v1 = acc[(NMAT - 1) * RG + j];
-                }
-            if (EPI == kEpiPlain) {
-                if (p.y) p.y[r] = v0;
-                if (p.y16) p.y16[r] = f2h_rn(v0);
-            } else if (EPI == kEpiSwiglu) {
-                const float sg = v0 / (1.0f + expf(-v0));
-                p.h[r] = f2h_rn(sg * v1);
-            } else {
-                if (p.logits) p.logits[r] = v0;
-                if (v0 > best_v) {  // rows arrive in increasing order per lane
-                    best_v = v0;
-                    best_i = static_cast<int>(r);
-                }
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < ROWS; ++j) acc[j] = 0.f;
-    }
-
-    if (failed) {
-        // Drain: wait (bounded) for this warp's copies still in flight so no
-        // bulk copy targets shared memory after the CTA exits.
-        if (lane == 0) {
-            atomicOr(&g_gemv_err, 1u);
-            const int64_t issued_end = min64(total, t + kStages);
-            for (int64_t u = t; u < issued_end; ++u)
-                mbar_wait_bounded(&bars[u % kStages], static_cast<uint32_t>((u / kStages) & 1));
-        }
-        __syncwarp();
     }
 
     if (EPI == kEpiHead) {
@@ -384,7 +409,7 @@ __global__ void __launch_bounds__(kNumWarps* kLanes, 1) gemv_s1_kernel(const Par
         if (threadIdx.x == 0) {
             float bv = red_v[0];
             int bi = red_i[0];
-            for (int w = 1; w < kNumWarps; ++w)
+            for (int w = 1; w < kWarps; ++w)
                 if (red_v[w] > bv || (red_v[w] == bv && red_i[w] < bi)) {
                     bv = red_v[w];
                     bi = red_i[w];
@@ -403,37 +428,32 @@ __global__ void __launch_bounds__(kNumWarps* kLanes, 1) gemv_s1_kernel(const Par
     }
 }
 
-template <int FMT, int NMAT, int RG, int EPI, bool SC>
-size_t smem_bytes(const Params& p) {
-    using L = Stage<FMT, NMAT * RG>;
-    size_t b = align_up(kNumWarps * kStages * 8, 128);
-    b += static_cast<size_t>(kNumWarps) * kStages * L::kBytes;
-    b += static_cast<size_t>(p.x_floats) * 4;
-    if (FMT == 1) b += static_cast<size_t>(p.k / Fmt<1>::kCodesPerLane) * 4;
-    return b;
-}
-
-template <int FMT, int NMAT, int RG, int EPI, bool SC>
-qg_status launch_t(const Params& p, const DeviceInfo& dev, cudaStream_t stream) {
-    auto kern = gemv_s1_kernel<FMT, NMAT, RG, EPI, SC>;
-    const size_t smem = smem_bytes<FMT, NMAT, RG, EPI, SC>(p);
+template <int FMT, int NMAT, int RG, int EPI>
+qg_status launch_t(Params p, const DeviceInfo& dev, cudaStream_t stream) {
+    auto kern = gemv_kernel<FMT, NMAT, RG, EPI>;
+    size_t smem = static_cast<size_t>(p.x_floats) * 4;
+    if (FMT == 1) smem += static_cast<size_t>(p.k / Fmt<1>::kCodesPerLane) * 4;
     if (smem + 1024 > static_cast<size_t>(dev.max_smem_optin)) return QG_ERR_SHAPE;
     // Opt in to exactly the dynamic shared memory this launch needs (static
     // shared memory counts against the same per-block limit).
     static size_t attr_set[64] = {0};
-    if (dev.device >= 64 || attr_set[dev.device] < smem) {
+    if (smem > 48 * 1024 && (dev.device >= 64 || attr_set[dev.device] < smem)) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return cuda_status(e);
         if (dev.device < 64) attr_set[dev.device] = smem;
     }
     const int64_t items = (p.n + RG - 1) / RG;
-    int64_t grid = (items + kNumWarps - 1) / kNumWarps;
-    if (grid > dev.num_sms) grid = dev.num_sms;
+    int64_t grid = (items + kWarps - 1) / kWarps;
+    const int64_t max_grid = static_cast<int64_t>(dev.num_sms) * kCtasPerSm;
+    if (grid > max_grid) grid = max_grid;
+    const int64_t item_bytes = static_cast<int64_t>(NMAT) * RG * (FMT == 0 ? p.k : p.k / 2);
+    p.prefetch_items = static_cast<int>(kPrefetchBytesPerWarp / item_bytes);
+    if (p.prefetch_items < 1) p.prefetch_items = 1;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    cfg.blockDim = dim3(kNumWarps * kLanes);
+    cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -444,32 +464,31 @@ qg_status launch_t(const Params& p, const DeviceInfo& dev, cudaStream_t stream) 
     return cuda_status(cudaLaunchKernelEx(&cfg, kern, p));
 }
 
-// Rows per warp item: as many as still leave every warp of the grid at least
-// two items, so small matrices spread over all SMs.
+// Rows per warp item: the most that still gives every warp of the grid work.
 int pick_rg(int64_t n, int max_rg, int total_warps) {
-    if (max_rg >= 4 && n >= 8LL * total_warps) return 4;
+    if (max_rg >= 4 && n >= 4LL * 2 * total_warps) return 4;
     if (max_rg >= 2 && n >= 2LL * total_warps) return 2;
     return 1;
 }
 
-template <int FMT, bool SC>
+template <int FMT>
 qg_status dispatch_fmt(const GemvLaunch& L, const Params& p, const DeviceInfo& dev,
                        cudaStream_t stream) {
-    const int tw = dev.num_sms * kNumWarps;
+    const int tw = dev.num_sms * kCtasPerSm * kWarps;
     if (L.epilogue == kEpiSwiglu) {
         const int rg = pick_rg(L.n, 2, tw);
-        if (rg == 2) return launch_t<FMT, 2, 2, kEpiSwiglu, SC>(p, dev, stream);
-        return launch_t<FMT, 2, 1, kEpiSwiglu, SC>(p, dev, stream);
+        if (rg == 2) return launch_t<FMT, 2, 2, kEpiSwiglu>(p, dev, stream);
+        return launch_t<FMT, 2, 1, kEpiSwiglu>(p, dev, stream);
     }
     const int rg = pick_rg(L.n, 4, tw);
     if (L.epilogue == kEpiHead) {
-        if (rg == 4) return launch_t<FMT, 1, 4, kEpiHead, SC>(p, dev, stream);
-        if (rg == 2) return launch_t<FMT, 1, 2, kEpiHead, SC>(p, dev, stream);
-        return launch_t<FMT, 1, 1, kEpiHead, SC>(p, dev, stream);
+        if (rg == 4) return launch_t<FMT, 1, 4, kEpiHead>(p, dev, stream);
+        if (rg == 2) return launch_t<FMT, 1, 2, kEpiHead>(p, dev, stream);
+        return launch_t<FMT, 1, 1, kEpiHead>(p, dev, stream);
     }
-    if (rg == 4) return launch_t<FMT, 1, 4, kEpiPlain, SC>(p, dev, stream);
-    if (rg == 2) return launch_t<FMT, 1, 2, kEpiPlain, SC>(p, dev, stream);
-    return launch_t<FMT, 1, 1, kEpiPlain, SC>(p, dev, stream);
+    if (rg == 4) return launch_t<FMT, 1, 4, kEpiPlain>(p, dev, stream);
+    if (rg == 2) return launch_t<FMT, 1, 2, kEpiPlain>(p, dev, stream);
+    return launch_t<FMT, 1, 1, kEpiPlain>(p, dev, stream);
 }
 
 }  // namespace
@@ -500,15 +519,8 @@ qg_status launch_gemv_s1(const GemvLaunch& L, cudaStream_t stream) {
     const int cpl = L.fmt == QG_FMT_I8_B32 ? Fmt<0>::kCodesPerLane : Fmt<1>::kCodesPerLane;
     const int granules = static_cast<int>(L.k / cpl);
     p.x_floats = align_up(granules, 8) * cpl;
-
-    // Scales (and biases) ride the bulk copies when every per-row, per-stage
-    // window of them is 16-byte aligned; otherwise lanes load them directly.
-    if (L.fmt == QG_FMT_I8_B32) {
-        if (L.k % 256 == 0) return dispatch_fmt<0, true>(L, p, dev, stream);
-        return dispatch_fmt<0, false>(L, p, dev, stream);
-    }
-    if (L.k % 512 == 0) return dispatch_fmt<1, true>(L, p, dev, stream);
-    return dispatch_fmt<1, false>(L, p, dev, stream);
+    if (L.fmt == QG_FMT_I8_B32) return dispatch_fmt<0>(L, p, dev, stream);
+    return dispatch_fmt<1>(L, p, dev, stream);
 }
 
 unsigned int gemv_read_and_clear_error() {
