@@ -182,6 +182,149 @@ struct Frag {
     uint16_t b[ROWS];
 };
 
+// ------------------------------------------------------ shared kernel parts --
+// Stage x (fp16 in global memory, written by the previous kernel) into shared
+// memory as fp32 in the conflict-free piece layout; int4 also gets the sum of
+// x over each 32-code lane granule and the pair-permuted order dot32_i4 uses.
+template <int FMT>
+__device__ __forceinline__ void stage_x(const uint16_t* __restrict__ x, float* xs, float* hsum,
+                                        int granules) {
+    using F = Fmt<FMT>;
+    float4* xs4 = reinterpret_cast<float4*>(xs);
+    for (int g = threadIdx.x; g < granules; g += blockDim.x) {
+        const uint16_t* xg = x + static_cast<int64_t>(g) * F::kCodesPerLane;
+        float gsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < F::kCodesPerLane / 8; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(xg + 8 * c);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            float a[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                a[2 * e] = h2f(static_cast<uint16_t>(w[e] & 0xFFFFu));
+                a[2 * e + 1] = h2f(static_cast<uint16_t>(w[e] >> 16));
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) gsum += a[e];
+            if (FMT == 0) {
+                xs4[x_piece<FMT>(g, 2 * c)] = make_float4(a[0], a[1], a[2], a[3]);
+                xs4[x_piece<FMT>(g, 2 * c + 1)] = make_float4(a[4], a[5], a[6], a[7]);
+            } else {
+                // one 8-code word: (x0, x5, x1, x6) (x2, x7, x3, x4/16)
+                xs4[x_piece<FMT>(g, 2 * c)] = make_float4(a[0], a[5], a[1], a[6]);
+                xs4[x_piece<FMT>(g, 2 * c + 1)] = make_float4(a[2], a[7], a[3], a[4] * 0.0625f);
+            }
+        }
+        if (FMT == 1) hsum[g] = gsum;
+    }
+}
+
+// Finish the RG rows (x NMAT weights) of one warp item: reduce across lanes
+// and apply the epilogue; lane j writes row r0 + j.
+template <int NMAT, int RG, int EPI>
+__device__ __forceinline__ void finish_item(float (&acc)[NMAT * RG], int64_t r0, int64_t N,
+                                            const Params& p, int lane, float& best_v,
+                                            int& best_i) {
+#pragma unroll
+    for (int j = 0; j < NMAT * RG; ++j) acc[j] = warp_sum(acc[j]);
+    if (lane < RG && r0 + lane < N) {
+        const int64_t r = r0 + lane;
+        float v0 = acc[0], v1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < RG; ++j)
+            if (lane == j) {
+                v0 = acc[j];
+                if (NMAT == 2) v1 = acc[(NMAT - 1) * RG + j];
+            }
+        if (EPI == kEpiPlain) {
+            if (p.y) p.y[r] = v0;
+            if (p.y16) p.y16[r] = f2h_rn(v0);
+        } else if (EPI == kEpiSwiglu) {
+            p.h[r] = f2h_rn(v0 / (1.0f + expf(-v0)) * v1);
+        } else {
+            if (p.logits) p.logits[r] = v0;
+            if (v0 > best_v) {  // rows arrive in increasing order per lane
+                best_v = v0;
+                best_i = static_cast<int>(r);
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < NMAT * RG; ++j) acc[j] = 0.f;
+}
+
+// Head epilogue of a whole CTA: lane -> warp -> CTA (value, lowest index),
+// then one atomicMax per CTA and a ticket; the last CTA publishes the index
+// and re-zeroes the workspace.  No CTA ever waits on another.
+__device__ __forceinline__ void head_finish(const Params& p, float best_v, int best_i, int warp,
+                                            int lane, float* red_v, int* red_i, int nwarps) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, best_v, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, best_i, o);
+        if (ov > best_v || (ov == best_v && oi < best_i)) {
+            best_v = ov;
+            best_i = oi;
+        }
+    }
+    if (lane == 0) {
+        red_v[warp] = best_v;
+        red_i[warp] = best_i;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float bv = red_v[0];
+        int bi = red_i[0];
+        for (int w = 1; w < nwarps; ++w)
+            if (red_v[w] > bv || (red_v[w] == bv && red_i[w] < bi)) {
+                bv = red_v[w];
+                bi = red_i[w];
+            }
+        if (bi != INT_MAX) atomicMax(p.ws_key, argmax_key(bv, bi));
+        __threadfence();
+        const unsigned int ticket = atomicAdd(p.ws_ticket, 1u);
+        if (ticket == gridDim.x - 1) {
+            __threadfence();
+            const unsigned long long key = atomicAdd(p.ws_key, 0ull);
+            *p.idx = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(key & 0xFFFFFFFFull));
+            *p.ws_key = 0ull;
+            *p.ws_ticket = 0u;
+        }
+    }
+}
+
+// L2 prefetch of items [first, first + count) of a warp (bulk prefetch hint).
+template <int FMT, int NMAT, int RG>
+__device__ __forceinline__ void prefetch_items(const Params& p, int64_t wg, int64_t tw,
+                                               int first, int count, int my_items) {
+    using F = Fmt<FMT>;
+    const int64_t N = p.n, K = p.k;
+    const int64_t row_bytes = FMT == 0 ? K : K / 2;
+    const int64_t side_per_row = K / F::kBlock;
+    for (int i = first; i < first + count && i < my_items; ++i) {
+        const int64_t r0 = (wg + i * tw) * RG;
+        const int64_t rows = N - r0 < RG ? N - r0 : RG;
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) {
+            const uint8_t* cm = m == 0 ? p.codes[0] : p.codes[1];
+            prefetch_l2(cm + r0 * row_bytes, static_cast<uint32_t>(rows * row_bytes));
+            const uintptr_t sa = reinterpret_cast<uintptr_t>(
+                (m == 0 ? p.scales[0] : p.scales[1]) + r0 * side_per_row);
+            const uint32_t sbytes = static_cast<uint32_t>(rows * side_per_row * 2);
+            if (sa % 16 == 0 && sbytes % 16 == 0) {
+                prefetch_l2(reinterpret_cast<const void*>(sa), sbytes);
+                if (F::kBias)
+                    prefetch_l2((m == 0 ? p.biases[0] : p.biases[1]) + r0 * side_per_row, sbytes);
+            }
+        }
+    }
+}
+
+// ----------------------------------------------------------------------- //
+// Register-pipeline kernel: loads land in registers DEPTH-1 steps ahead.    //
+// Used when a row's scale count is odd (the shared-memory ring below copies //
+// scales as aligned 4-byte words).                                          //
+// ----------------------------------------------------------------------- //
 template <int FMT, int NMAT, int RG, int EPI>
 __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
     using F = Fmt<FMT>;
@@ -191,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
     constexpr int kStepSides = kStepBytes * (FMT == 0 ? 1 : 2) / F::kBlock;  // scales per step
     extern __shared__ __align__(128) unsigned char smem[];
     float* xs = reinterpret_cast<float*>(smem);
-    float* hsum = xs + p.x_floats;  // int4: per lane-granule sum of x
+    float* hsum = xs + p.x_floats;
     __shared__ float red_v[kWarps];
     __shared__ int red_i[kWarps];
 
@@ -205,11 +348,10 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
     const int my_items = wg < items ? static_cast<int>((items - wg + tw - 1) / tw) : 0;
     const int total = my_items * nst;
     const int64_t row_bytes = FMT == 0 ? K : K / 2;
-    const int64_t side_per_row = K / F::kBlock;  // fp16 scales (biases) per row
+    const int64_t side_per_row = K / F::kBlock;
     const uint64_t pol = l2_policy_evict_first();
 
-    // ---- load cursor: per-row pointers of the next step to load (lane offset
-    // included), advanced by a constant per step and rebuilt once per item.
+    // load cursor: per-row pointers of the next step (lane offset included)
     const uint8_t* lc[ROWS];
     const uint16_t* ls[ROWS];
     const uint16_t* lb[ROWS];
@@ -252,76 +394,25 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
         }
     };
 
-    // 1) Weight prologue, independent of the previous kernel in the stream:
-    //    the first DEPTH steps go straight into registers, and L2 is asked to
-    //    prefetch the next rows of this warp.
+    // 1) weight prologue (independent of the previous kernel): the first
+    //    DEPTH steps into registers, the next items into L2.
     Frag<ROWS> buf[DEPTH];
     if (my_items > 0) set_item(0);
 #pragma unroll
     for (int d = 0; d < DEPTH; ++d)
         if (d < total) load(buf[d]);
-    if (lane == 0) {
-        for (int i = 1; i < p.prefetch_items && i < my_items; ++i) {
-            const int64_t r0 = (wg + i * tw) * RG;
-            const int64_t rows = N - r0 < RG ? N - r0 : RG;
-#pragma unroll
-            for (int m = 0; m < NMAT; ++m) {
-                const uint8_t* cm = m == 0 ? p.codes[0] : p.codes[1];
-                prefetch_l2(cm + r0 * row_bytes, static_cast<uint32_t>(rows * row_bytes));
-                const uintptr_t sa = reinterpret_cast<uintptr_t>(
-                    (m == 0 ? p.scales[0] : p.scales[1]) + r0 * side_per_row);
-                const uint32_t sbytes = static_cast<uint32_t>(rows * side_per_row * 2);
-                if (sa % 16 == 0 && sbytes % 16 == 0) {
-                    prefetch_l2(reinterpret_cast<const void*>(sa), sbytes);
-                    if (F::kBias)
-                        prefetch_l2((m == 0 ? p.biases[0] : p.biases[1]) + r0 * side_per_row,
-                                    sbytes);
-                }
-            }
-        }
-    }
+    if (lane == 0) prefetch_items<FMT, NMAT, RG>(p, wg, tw, 1, p.prefetch_items - 1, my_items);
 
-    // 2) x is produced by the previous kernel: wait for it, then stage it as
-    //    fp32 (int4: pair-permuted, plus the half-group sums).
+    // 2) x from the previous kernel
     griddep_wait();
-    {
-        float4* xs4 = reinterpret_cast<float4*>(xs);
-        for (int g = threadIdx.x; g < granules; g += kThreads) {
-            const uint16_t* xg = p.x + static_cast<int64_t>(g) * F::kCodesPerLane;
-            float gsum = 0.f;
-#pragma unroll
-            for (int c = 0; c < F::kCodesPerLane / 8; ++c) {
-                const uint4 v = *reinterpret_cast<const uint4*>(xg + 8 * c);
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                float a[8];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    a[2 * e] = h2f(static_cast<uint16_t>(w[e] & 0xFFFFu));
-                    a[2 * e + 1] = h2f(static_cast<uint16_t>(w[e] >> 16));
-                }
-#pragma unroll
-                for (int e = 0; e < 8; ++e) gsum += a[e];
-                if (FMT == 0) {
-                    xs4[x_piece<FMT>(g, 2 * c)] = make_float4(a[0], a[1], a[2], a[3]);
-                    xs4[x_piece<FMT>(g, 2 * c + 1)] = make_float4(a[4], a[5], a[6], a[7]);
-                } else {
-                    // one 8-code word: (x0, x5, x1, x6) (x2, x7, x3, x4/16)
-                    xs4[x_piece<FMT>(g, 2 * c)] = make_float4(a[0], a[5], a[1], a[6]);
-                    xs4[x_piece<FMT>(g, 2 * c + 1)] =
-                        make_float4(a[2], a[7], a[3], a[4] * 0.0625f);
-                }
-            }
-            if (FMT == 1) hsum[g] = gsum;
-        }
-    }
+    stage_x<FMT>(p.x, xs, hsum, granules);
     __syncthreads();
     griddep_launch_dependents();
 
-    // 3) stream: the loads of steps t+1 .. t+DEPTH-1 are in flight while step
-    //    t is computed.  The x pieces of a lane advance by a constant per step.
+    // 3) stream
     const float4* xs4 = reinterpret_cast<const float4*>(xs);
     const int x_lane = ((lane >> 3) * F::kPieces) * 8 + (lane & 7);  // x_piece(lane, 0)
-    constexpr int kXStep = 4 * F::kPieces * 8;                      // x_piece(g + 32) - x_piece(g)
+    constexpr int kXStep = 4 * F::kPieces * 8;                      // per 32 granules
     float acc[ROWS];
 #pragma unroll
     for (int j = 0; j < ROWS; ++j) acc[j] = 0.f;
@@ -345,39 +436,11 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
             }
         }
         if (++cu_st == nst) {
-            // item done: finish its rows across lanes
-            const int64_t r0 = (wg + cu_item * tw) * RG;
-#pragma unroll
-            for (int j = 0; j < ROWS; ++j) acc[j] = warp_sum(acc[j]);
-            if (lane < RG && r0 + lane < N) {
-                const int64_t r = r0 + lane;
-                float v0 = acc[0], v1 = 0.f;
-#pragma unroll
-                for (int j = 0; j < RG; ++j)
-                    if (lane == j) {
-                        v0 = acc[j];
-                        if (NMAT == 2) v1 = acc[(NMAT - 1) * RG + j];
-                    }
-                if (EPI == kEpiPlain) {
-                    if (p.y) p.y[r] = v0;
-                    if (p.y16) p.y16[r] = f2h_rn(v0);
-                } else if (EPI == kEpiSwiglu) {
-                    p.h[r] = f2h_rn(v0 / (1.0f + expf(-v0)) * v1);
-                } else {
-                    if (p.logits) p.logits[r] = v0;
-                    if (v0 > best_v) {  // rows arrive in increasing order per lane
-                        best_v = v0;
-                        best_i = static_cast<int>(r);
-                    }
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < ROWS; ++j) acc[j] = 0.f;
+            finish_item<NMAT, RG, EPI>(acc, (wg + cu_item * tw) * RG, N, p, lane, best_v, best_i);
             cu_st = 0;
             ++cu_item;
         }
     };
-
     for (int t = 0; t < total; t += DEPTH) {
 #pragma unroll
         for (int d = 0; d < DEPTH; ++d) {
@@ -387,57 +450,221 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
             }
         }
     }
-
-    if (EPI == kEpiHead) {
-        // lane -> warp -> CTA (value, lowest index), then one atomicMax per CTA
-        // and a ticket: the last CTA publishes the index and re-zeroes the
-        // workspace.  No CTA ever waits on another.
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, best_v, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, best_i, o);
-            if (ov > best_v || (ov == best_v && oi < best_i)) {
-                best_v = ov;
-                best_i = oi;
-            }
-        }
-        if (lane == 0) {
-            red_v[warp] = best_v;
-            red_i[warp] = best_i;
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            float bv = red_v[0];
-            int bi = red_i[0];
-            for (int w = 1; w < kWarps; ++w)
-                if (red_v[w] > bv || (red_v[w] == bv && red_i[w] < bi)) {
-                    bv = red_v[w];
-                    bi = red_i[w];
-                }
-            if (bi != INT_MAX) atomicMax(p.ws_key, argmax_key(bv, bi));
-            __threadfence();
-            const unsigned int ticket = atomicAdd(p.ws_ticket, 1u);
-            if (ticket == gridDim.x - 1) {
-                __threadfence();
-                const unsigned long long key = atomicAdd(p.ws_key, 0ull);
-                *p.idx = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(key & 0xFFFFFFFFull));
-                *p.ws_key = 0ull;
-                *p.ws_ticket = 0u;
-            }
-        }
-    }
+    if (EPI == kEpiHead) head_finish(p, best_v, best_i, warp, lane, red_v, red_i, kWarps);
 }
 
+// ----------------------------------------------------------------------- //
+// Shared-memory-ring kernel: every lane copies the 16-byte code vectors    //
+// (and the 4-byte scale words) it will consume with cp.async into its own  //
+// ring slots, kRing-1 steps ahead.  A lane reads only what it copied, so   //
+// no cross-lane synchronization is needed, and the bytes in flight cost no //
+// registers: 3 steps x RG rows x 16 B per lane stay outstanding.          //
+// Requires an even number of scales per row (aligned 4-byte scale words).  //
+// ----------------------------------------------------------------------- //
+constexpr int kRing = 4;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint64_t pol) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst),
+                 "l"(src), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+
+template <int FMT, int NMAT>
+struct RingLayout {
+    // bytes per (slot, row) for the 32 lanes of a warp
+    static constexpr int kCodes = kLanes * 16;
+    static constexpr int kSide = kLanes * 4;
+    static constexpr int kPerRow = kCodes + kSide * (FMT == 1 ? 2 : 1);
+};
+
 template <int FMT, int NMAT, int RG, int EPI>
+__global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) {
+    using F = Fmt<FMT>;
+    using RL = RingLayout<FMT, NMAT>;
+    constexpr int ROWS = NMAT * RG;
+    constexpr int kStepBytes = kLanes * 16;
+    constexpr int kStepSides = kStepBytes * (FMT == 0 ? 1 : 2) / F::kBlock;
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ float red_v[kWarps];
+    __shared__ int red_i[kWarps];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t N = p.n, K = p.k;
+    const int granules = static_cast<int>(K / F::kCodesPerLane);
+    const int nst = (granules + kLanes - 1) / kLanes;
+    const int64_t items = (N + RG - 1) / RG;
+    const int64_t wg = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+    const int64_t tw = static_cast<int64_t>(gridDim.x) * kWarps;
+    const int my_items = wg < items ? static_cast<int>((items - wg + tw - 1) / tw) : 0;
+    const int total = my_items * nst;
+    const int64_t row_bytes = FMT == 0 ? K : K / 2;
+    const int64_t side_per_row = K / F::kBlock;
+    const uint64_t pol = l2_policy_evict_first();
+
+    // shared memory: [ring of this CTA's warps][x fp32][hsum]
+    const uint32_t ring = smem_u32(smem) + warp * (kRing * ROWS * RL::kPerRow);
+    float* xs = reinterpret_cast<float*>(smem + kWarps * kRing * ROWS * RL::kPerRow);
+    float* hsum = xs + p.x_floats;
+    // this lane's address inside slot s, row j
+    auto slot_codes = [&](int s, int j) -> uint32_t {
+        return ring + (s * ROWS + j) * RL::kPerRow + lane * 16;
+    };
+    auto slot_side = [&](int s, int j, int which) -> uint32_t {
+        return ring + (s * ROWS + j) * RL::kPerRow + RL::kCodes + which * RL::kSide + lane * 4;
+    };
+
+    // load cursor (global addresses of the next step; the 4-byte scale word
+    // holding this lane's scale starts at an even scale index)
+    const uint8_t* lc[ROWS];
+    const uint16_t* ls[ROWS];
+    const uint16_t* lb[ROWS];
+    int ld_st = 0, ld_item = 0, ld_slot = 0;
+    auto set_item = [&](int il) {
+        const int64_t r0 = (wg + il * tw) * RG;
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) {
+            const uint8_t* cm = m == 0 ? p.codes[0] : p.codes[1];
+            const uint16_t* sm = m == 0 ? p.scales[0] : p.scales[1];
+            const uint16_t* bm = m == 0 ? p.biases[0] : p.biases[1];
+#pragma unroll
+            for (int j = 0; j < RG; ++j) {
+                const int64_t r = r0 + j < N ? r0 + j : N - 1;
+                lc[m * RG + j] = cm + r * row_bytes + lane * 16;
+                ls[m * RG + j] = sm + r * side_per_row + ((lane >> 2) << 1);
+                if (F::kBias) lb[m * RG + j] = bm + r * side_per_row + ((lane >> 2) << 1);
+            }
+        }
+    };
+    auto issue = [&]() {
+        if (ld_st * kLanes + lane < granules) {
+#pragma unroll
+            for (int j = 0; j < ROWS; ++j) {
+                cp_async16(slot_codes(ld_slot, j), lc[j], pol);
+                cp_async4(slot_side(ld_slot, j, 0), ls[j]);
+                if (F::kBias) cp_async4(slot_side(ld_slot, j, 1), lb[j]);
+            }
+        }
+        cp_async_commit();
+        if (++ld_slot == kRing) ld_slot = 0;
+        if (++ld_st == nst) {
+            ld_st = 0;
+            if (++ld_item < my_items) set_item(ld_item);
+        } else {
+#pragma unroll
+            for (int j = 0; j < ROWS; ++j) {
+                lc[j] += kStepBytes;
+                ls[j] += kStepSides;
+                if (F::kBias) lb[j] += kStepSides;
+            }
+        }
+    };
+
+    // 1) weight prologue (independent of the previous kernel)
+    if (my_items > 0) set_item(0);
+#pragma unroll
+    for (int d = 0; d < kRing - 1; ++d) {
+        if (d < total) issue();
+        else cp_async_commit();
+    }
+    if (lane == 0) prefetch_items<FMT, NMAT, RG>(p, wg, tw, 1, p.prefetch_items - 1, my_items);
+
+    // 2) x from the previous kernel
+    griddep_wait();
+    stage_x<FMT>(p.x, xs, hsum, granules);
+    __syncthreads();
+    griddep_launch_dependents();
+
+    // 3) stream: issue step t + kRing - 1, wait for step t, compute it
+    const float4* xs4 = reinterpret_cast<const float4*>(xs);
+    const int x_lane = ((lane >> 3) * F::kPieces) * 8 + (lane & 7);
+    constexpr int kXStep = 4 * F::kPieces * 8;
+    const int half = ((lane >> 1) & 1) * 16;  // this lane's scale inside its word
+    float acc[ROWS];
+#pragma unroll
+    for (int j = 0; j < ROWS; ++j) acc[j] = 0.f;
+    float best_v = -FLT_MAX;
+    int best_i = INT_MAX;
+    int cu_st = 0, cu_item = 0, cu_slot = 0;
+    for (int t = 0; t < total; ++t) {
+        if (t + kRing - 1 < total) issue();
+        else cp_async_commit();
+        cp_async_wait<kRing - 1>();
+        const int g = cu_st * kLanes + lane;
+        if (g < granules) {
+            float4 xv[F::kPieces];
+            const float4* xp = xs4 + x_lane + cu_st * kXStep;
+#pragma unroll
+            for (int i = 0; i < F::kPieces; ++i) xv[i] = xp[i * 8];
+            const float hs = FMT == 1 ? hsum[g] : 0.f;
+#pragma unroll
+            for (int j = 0; j < ROWS; ++j) {
+                const uint4 c = lds128(slot_codes(cu_slot, j));
+                const float sc = h2f(static_cast<uint16_t>(lds32(slot_side(cu_slot, j, 0)) >> half));
+                if (FMT == 0) {
+                    acc[j] = fmaf(sc, dot16_i8(c, xv), acc[j]);
+                } else {
+                    const float bi =
+                        h2f(static_cast<uint16_t>(lds32(slot_side(cu_slot, j, 1)) >> half));
+                    acc[j] = fmaf(sc, dot32_i4(c, xv), fmaf(bi, hs, acc[j]));
+                }
+            }
+        }
+        if (++cu_slot == kRing) cu_slot = 0;
+        if (++cu_st == nst) {
+            finish_item<NMAT, RG, EPI>(acc, (wg + cu_item * tw) * RG, N, p, lane, best_v, best_i);
+            cu_st = 0;
+            ++cu_item;
+        }
+    }
+    cp_async_wait<0>();
+    if (EPI == kEpiHead) head_finish(p, best_v, best_i, warp, lane, red_v, red_i, kWarps);
+}
+
+size_t x_smem_bytes(int fmt, const Params& p) {
+    size_t b = static_cast<size_t>(p.x_floats) * 4;
+    if (fmt == QG_FMT_I4_G64) b += static_cast<size_t>(p.k / Fmt<1>::kCodesPerLane) * 4;
+    return b;
+}
+
+template <int FMT, int NMAT, int RG>
+constexpr size_t ring_smem_bytes() {
+    return static_cast<size_t>(kWarps) * kRing * NMAT * RG * RingLayout<FMT, NMAT>::kPerRow;
+}
+
+// Per-CTA shared memory that still lets two CTAs share an SM.
+constexpr size_t kSmemPerCtaBudget = 110 * 1024;
+
+template <int FMT, int NMAT, int RG, int EPI, bool RING>
 qg_status launch_t(Params p, const DeviceInfo& dev, cudaStream_t stream) {
-    auto kern = gemv_kernel<FMT, NMAT, RG, EPI>;
-    size_t smem = static_cast<size_t>(p.x_floats) * 4;
-    if (FMT == 1) smem += static_cast<size_t>(p.k / Fmt<1>::kCodesPerLane) * 4;
+    auto kern = RING ? gemv_ring_kernel<FMT, NMAT, RG, EPI> : gemv_kernel<FMT, NMAT, RG, EPI>;
+    size_t smem = x_smem_bytes(FMT, p) + (RING ? ring_smem_bytes<FMT, NMAT, RG>() : 0);
     if (smem + 1024 > static_cast<size_t>(dev.max_smem_optin)) return QG_ERR_SHAPE;
     // Opt in to exactly the dynamic shared memory this launch needs (static
     // shared memory counts against the same per-block limit).
     static size_t attr_set[64] = {0};
-    if (smem > 48 * 1024 && (dev.device >= 64 || attr_set[dev.device] < smem)) {
+    if (dev.device >= 64 || attr_set[dev.device] < smem) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return cuda_status(e);
@@ -471,24 +698,34 @@ int pick_rg(int64_t n, int max_rg, int total_warps) {
     return 1;
 }
 
+template <int FMT, int NMAT, int RG, int EPI>
+qg_status launch_pick(const Params& p, const DeviceInfo& dev, cudaStream_t stream) {
+    // The ring kernel copies scale words of two scales: rows need an even
+    // scale count; its ring must fit beside x in the per-CTA budget.
+    const bool even_sides = (p.k / Fmt<FMT>::kBlock) % 2 == 0;
+    const bool fits = x_smem_bytes(FMT, p) + ring_smem_bytes<FMT, NMAT, RG>() <= kSmemPerCtaBudget;
+    if (even_sides && fits) return launch_t<FMT, NMAT, RG, EPI, true>(p, dev, stream);
+    return launch_t<FMT, NMAT, RG, EPI, false>(p, dev, stream);
+}
+
 template <int FMT>
 qg_status dispatch_fmt(const GemvLaunch& L, const Params& p, const DeviceInfo& dev,
                        cudaStream_t stream) {
     const int tw = dev.num_sms * kCtasPerSm * kWarps;
     if (L.epilogue == kEpiSwiglu) {
         const int rg = pick_rg(L.n, 2, tw);
-        if (rg == 2) return launch_t<FMT, 2, 2, kEpiSwiglu>(p, dev, stream);
-        return launch_t<FMT, 2, 1, kEpiSwiglu>(p, dev, stream);
+        if (rg == 2) return launch_pick<FMT, 2, 2, kEpiSwiglu>(p, dev, stream);
+        return launch_pick<FMT, 2, 1, kEpiSwiglu>(p, dev, stream);
     }
     const int rg = pick_rg(L.n, 4, tw);
     if (L.epilogue == kEpiHead) {
-        if (rg == 4) return launch_t<FMT, 1, 4, kEpiHead>(p, dev, stream);
-        if (rg == 2) return launch_t<FMT, 1, 2, kEpiHead>(p, dev, stream);
-        return launch_t<FMT, 1, 1, kEpiHead>(p, dev, stream);
+        if (rg == 4) return launch_pick<FMT, 1, 4, kEpiHead>(p, dev, stream);
+        if (rg == 2) return launch_pick<FMT, 1, 2, kEpiHead>(p, dev, stream);
+        return launch_pick<FMT, 1, 1, kEpiHead>(p, dev, stream);
     }
-    if (rg == 4) return launch_t<FMT, 1, 4, kEpiPlain>(p, dev, stream);
-    if (rg == 2) return launch_t<FMT, 1, 2, kEpiPlain>(p, dev, stream);
-    return launch_t<FMT, 1, 1, kEpiPlain>(p, dev, stream);
+    if (rg == 4) return launch_pick<FMT, 1, 4, kEpiPlain>(p, dev, stream);
+    if (rg == 2) return launch_pick<FMT, 1, 2, kEpiPlain>(p, dev, stream);
+    return launch_pick<FMT, 1, 1, kEpiPlain>(p, dev, stream);
 }
 
 }  // namespace
