@@ -405,7 +405,8 @@ def _time_gate_up(sw, stream, dev, qg, torch):
     us = e0.elapsed_time(e1) * 1e3 / launches
     nbytes = sw.layers[0].gate.nbytes + sw.layers[0].up.nbytes
     del g
-    return {"kernel": "gemv_s1_kernel<swiglu>" if sw.S == 1 else "gemm_s16_kernel<swiglu>",
+    return {"kernel": ("gemv_ring_kernel (fused gate/up + SwiGLU)" if sw.S == 1
+                       else "gemm_s16_kernel (fused gate/up + SwiGLU)"),
             "gbs": nbytes / (us * 1e-6) / 1e9, "us": us, "bytes": nbytes,
             "launches": launches}
 
