@@ -322,8 +322,8 @@ __device__ __forceinline__ void prefetch_items(const Params& p, int64_t wg, int6
 
 // ----------------------------------------------------------------------- //
 // Register-pipeline kernel: loads land in registers DEPTH-1 steps ahead.    //
-// Used when a row's scale count is odd (the shared-memory ring below copies //
-// scales as aligned 4-byte words).                                          //
+// Used when a row's scale count is not a multiple of 8 (the shared-memory   //
+// ring below copies scales as 16-byte pieces).                              //
 // ----------------------------------------------------------------------- //
 template <int FMT, int NMAT, int RG, int EPI>
 __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
@@ -455,11 +455,11 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
 
 // ----------------------------------------------------------------------- //
 // Shared-memory-ring kernel: every lane copies the 16-byte code vectors    //
-// (and the 4-byte scale words) it will consume with cp.async into its own  //
-// ring slots, kRing-1 steps ahead.  A lane reads only what it copied, so   //
-// no cross-lane synchronization is needed, and the bytes in flight cost no //
+// it will consume with cp.async into its own ring slots, kRing-1 steps     //
+// ahead; a few lanes copy each step's scales (and biases) as 16-byte       //
+// pieces, read by the warp after a __syncwarp.  Bytes in flight cost no    //
 // registers: 3 steps x RG rows x 16 B per lane stay outstanding.          //
-// Requires an even number of scales per row (aligned 4-byte scale words).  //
+// Requires a multiple of 8 scales per row (16-byte pieces).                //
 // ----------------------------------------------------------------------- //
 constexpr int kRing = 4;
 
@@ -467,9 +467,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint64
     asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst),
                  "l"(src), "l"(pol)
                  : "memory");
-}
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() {
     asm volatile("cp.async.commit_group;" ::: "memory");
@@ -485,17 +482,18 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
                  : "r"(a));
     return v;
 }
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+__device__ __forceinline__ uint16_t lds16(uint32_t a) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
     return v;
 }
 
 template <int FMT, int NMAT>
 struct RingLayout {
-    // bytes per (slot, row) for the 32 lanes of a warp
+    // bytes per (slot, row): the 32 lanes' code vectors, then the step's 16
+    // fp16 scales (and 16 biases for int4)
     static constexpr int kCodes = kLanes * 16;
-    static constexpr int kSide = kLanes * 4;
+    static constexpr int kSide = 32;
     static constexpr int kPerRow = kCodes + kSide * (FMT == 1 ? 2 : 1);
 };
 
@@ -505,7 +503,8 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) 
     using RL = RingLayout<FMT, NMAT>;
     constexpr int ROWS = NMAT * RG;
     constexpr int kStepBytes = kLanes * 16;
-    constexpr int kStepSides = kStepBytes * (FMT == 0 ? 1 : 2) / F::kBlock;
+    constexpr int kStepSides = kStepBytes * (FMT == 0 ? 1 : 2) / F::kBlock;  // 16
+    constexpr int kSideLanes = 2 * ROWS * (F::kBias ? 2 : 1);  // lanes that copy side data
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ float red_v[kWarps];
     __shared__ int red_i[kWarps];
@@ -520,52 +519,60 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) 
     const int my_items = wg < items ? static_cast<int>((items - wg + tw - 1) / tw) : 0;
     const int total = my_items * nst;
     const int64_t row_bytes = FMT == 0 ? K : K / 2;
-    const int64_t side_per_row = K / F::kBlock;
+    const int64_t side_per_row = K / F::kBlock;  // a multiple of 8 (16-byte pieces)
     const uint64_t pol = l2_policy_evict_first();
 
     // shared memory: [ring of this CTA's warps][x fp32][hsum]
     const uint32_t ring = smem_u32(smem) + warp * (kRing * ROWS * RL::kPerRow);
     float* xs = reinterpret_cast<float*>(smem + kWarps * kRing * ROWS * RL::kPerRow);
     float* hsum = xs + p.x_floats;
-    // this lane's address inside slot s, row j
-    auto slot_codes = [&](int s, int j) -> uint32_t {
+    auto slot_codes = [&](int s, int j) -> uint32_t {  // this lane's code vector
         return ring + (s * ROWS + j) * RL::kPerRow + lane * 16;
     };
-    auto slot_side = [&](int s, int j, int which) -> uint32_t {
-        return ring + (s * ROWS + j) * RL::kPerRow + RL::kCodes + which * RL::kSide + lane * 4;
+    auto slot_side = [&](int s, int j, int which) -> uint32_t {  // the step's 16 sides
+        return ring + (s * ROWS + j) * RL::kPerRow + RL::kCodes + which * RL::kSide;
     };
 
-    // load cursor (global addresses of the next step; the 4-byte scale word
-    // holding this lane's scale starts at an even scale index)
+    // Side data: each step of a row needs 16 consecutive scales (32 B) and,
+    // for int4, 16 biases.  Lane l < kSideLanes copies one 16-byte piece of
+    // one of them (no two lanes copy the same bytes); the warp then
+    // synchronizes before reading.
+    const bool side_lane = lane < kSideLanes;
+    const int side_which = lane / (2 * ROWS);          // 0: scales, 1: biases
+    const int side_row = (lane % (2 * ROWS)) >> 1;     // row slot 0..ROWS-1
+    const int side_half = lane & 1;                    // which 16-byte piece
+    const int side_m = side_row / RG, side_j = side_row % RG;
+
+    // load cursor (global addresses of the next step)
     const uint8_t* lc[ROWS];
-    const uint16_t* ls[ROWS];
-    const uint16_t* lb[ROWS];
+    const uint16_t* lside = nullptr;
     int ld_st = 0, ld_item = 0, ld_slot = 0;
     auto set_item = [&](int il) {
         const int64_t r0 = (wg + il * tw) * RG;
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
             const uint8_t* cm = m == 0 ? p.codes[0] : p.codes[1];
-            const uint16_t* sm = m == 0 ? p.scales[0] : p.scales[1];
-            const uint16_t* bm = m == 0 ? p.biases[0] : p.biases[1];
 #pragma unroll
             for (int j = 0; j < RG; ++j) {
-                const int64_t r = r0 + j < N ? r0 + j : N - 1;
+                const int64_t r = r0 + j < N ? r0 + j : N - 1;  // tail rows: copy, discard
                 lc[m * RG + j] = cm + r * row_bytes + lane * 16;
-                ls[m * RG + j] = sm + r * side_per_row + ((lane >> 2) << 1);
-                if (F::kBias) lb[m * RG + j] = bm + r * side_per_row + ((lane >> 2) << 1);
             }
+        }
+        if (side_lane) {
+            const int64_t r = r0 + side_j < N ? r0 + side_j : N - 1;
+            const uint16_t* base =
+                side_which == 0 ? (side_m == 0 ? p.scales[0] : p.scales[1])
+                                : (side_m == 0 ? p.biases[0] : p.biases[1]);
+            lside = base + r * side_per_row + side_half * 8;
         }
     };
     auto issue = [&]() {
         if (ld_st * kLanes + lane < granules) {
 #pragma unroll
-            for (int j = 0; j < ROWS; ++j) {
-                cp_async16(slot_codes(ld_slot, j), lc[j], pol);
-                cp_async4(slot_side(ld_slot, j, 0), ls[j]);
-                if (F::kBias) cp_async4(slot_side(ld_slot, j, 1), lb[j]);
-            }
+            for (int j = 0; j < ROWS; ++j) cp_async16(slot_codes(ld_slot, j), lc[j], pol);
         }
+        if (side_lane && ld_st * kStepSides + side_half * 8 + 8 <= side_per_row)
+            cp_async16(slot_side(ld_slot, side_row, side_which) + side_half * 16, lside, pol);
         cp_async_commit();
         if (++ld_slot == kRing) ld_slot = 0;
         if (++ld_st == nst) {
@@ -573,11 +580,8 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) 
             if (++ld_item < my_items) set_item(ld_item);
         } else {
 #pragma unroll
-            for (int j = 0; j < ROWS; ++j) {
-                lc[j] += kStepBytes;
-                ls[j] += kStepSides;
-                if (F::kBias) lb[j] += kStepSides;
-            }
+            for (int j = 0; j < ROWS; ++j) lc[j] += kStepBytes;
+            if (side_lane) lside += kStepSides;
         }
     };
 
@@ -600,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) 
     const float4* xs4 = reinterpret_cast<const float4*>(xs);
     const int x_lane = ((lane >> 3) * F::kPieces) * 8 + (lane & 7);
     constexpr int kXStep = 4 * F::kPieces * 8;
-    const int half = ((lane >> 1) & 1) * 16;  // this lane's scale inside its word
+    const int side_off = (lane >> 1) * 2;  // this lane's scale (bias) inside the step's 16
     float acc[ROWS];
 #pragma unroll
     for (int j = 0; j < ROWS; ++j) acc[j] = 0.f;
@@ -611,6 +615,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) 
         if (t + kRing - 1 < total) issue();
         else cp_async_commit();
         cp_async_wait<kRing - 1>();
+        __syncwarp();  // side pieces copied by other lanes are now visible
         const int g = cu_st * kLanes + lane;
         if (g < granules) {
             float4 xv[F::kPieces];
@@ -621,16 +626,16 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) 
 #pragma unroll
             for (int j = 0; j < ROWS; ++j) {
                 const uint4 c = lds128(slot_codes(cu_slot, j));
-                const float sc = h2f(static_cast<uint16_t>(lds32(slot_side(cu_slot, j, 0)) >> half));
+                const float sc = h2f(lds16(slot_side(cu_slot, j, 0) + side_off));
                 if (FMT == 0) {
                     acc[j] = fmaf(sc, dot16_i8(c, xv), acc[j]);
                 } else {
-                    const float bi =
-                        h2f(static_cast<uint16_t>(lds32(slot_side(cu_slot, j, 1)) >> half));
+                    const float bi = h2f(lds16(slot_side(cu_slot, j, 1) + side_off));
                     acc[j] = fmaf(sc, dot32_i4(c, xv), fmaf(bi, hs, acc[j]));
                 }
             }
         }
+        __syncwarp();  // every lane is done with this slot before it is refilled
         if (++cu_slot == kRing) cu_slot = 0;
         if (++cu_st == nst) {
             finish_item<NMAT, RG, EPI>(acc, (wg + cu_item * tw) * RG, N, p, lane, best_v, best_i);
@@ -700,9 +705,10 @@ int pick_rg(int64_t n, int max_rg, int total_warps) {
 
 template <int FMT, int NMAT, int RG, int EPI>
 qg_status launch_pick(const Params& p, const DeviceInfo& dev, cudaStream_t stream) {
-    // The ring kernel copies scale words of two scales: rows need an even
-    // scale count; its ring must fit beside x in the per-CTA budget.
-    const bool even_sides = (p.k / Fmt<FMT>::kBlock) % 2 == 0;
+    // The ring kernel copies side data (scales, biases) as 16-byte pieces of 8:
+    // a row's count must be a multiple of 8; its ring must fit beside x in the
+    // per-CTA budget.
+    const bool even_sides = (p.k / Fmt<FMT>::kBlock) % 8 == 0;
     const bool fits = x_smem_bytes(FMT, p) + ring_smem_bytes<FMT, NMAT, RG>() <= kSmemPerCtaBudget;
     if (even_sides && fits) return launch_t<FMT, NMAT, RG, EPI, true>(p, dev, stream);
     return launch_t<FMT, NMAT, RG, EPI, false>(p, dev, stream);

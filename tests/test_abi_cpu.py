@@ -81,6 +81,8 @@ def test_gemm_s16_and_swiglu_validation(L):
     assert L.qg_gemm_s16(ctypes.byref(w), None, 4, 0x5000, None) == 1
     w4 = W(fmt=1, k=256)
     assert L.qg_gemm_s16(ctypes.byref(w4), 0x4000, 4, 0x5000, None) == 4
+    w256 = W(k=256)                                            # S > 1 needs k % 512 == 0
+    assert L.qg_gemm_s16(ctypes.byref(w256), 0x4000, 4, 0x5000, None) == 2
     wg, wu = W(), W(fmt=1, k=64)
     assert L.qg_gate_up_swiglu(ctypes.byref(wg), ctypes.byref(wu), 0x4000, 1, 0x6000, None) == 4
     wu2 = W(n=16)

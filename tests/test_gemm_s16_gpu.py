@@ -16,9 +16,9 @@ pytestmark = pytest.mark.gpu
 I8 = qg.FMT_I8_B32
 
 
-@pytest.mark.parametrize("n,k,S", [(1, 256, 16), (64, 256, 16), (100, 512, 3), (1000, 2048, 16),
+@pytest.mark.parametrize("n,k,S", [(1, 512, 16), (64, 512, 16), (100, 512, 3), (1000, 2048, 16),
                                    (4096, 4096, 16), (6144, 4096, 7), (4096, 12288, 16),
-                                   (333, 1280, 2), (2050, 768, 16)])
+                                   (333, 1536, 2), (2050, 1024, 16), (130, 2560, 16)])
 def test_gemm_s16_parity(cuda, n, k, S):
     w = wl.weight_fp32(n, k, 300 + S, cuda)
     W = qg.quantize(w, I8)
