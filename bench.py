@@ -113,14 +113,15 @@ def csrc_digest() -> str:
 
 def profiled_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+    the current kernel sources (else None).  Kernel names are stored with
+    spaces written as underscores."""
     try:
         with open(PROFILE_TRAFFIC) as f:
             for line in f:
                 if line.startswith("#") or "=" not in line:
                     continue
                 kv = dict(p.split("=", 1) for p in line.split())
-                if (kv.get("kernel") == kernel and kv.get("workload") == workload
+                if (kv.get("kernel") == kernel.replace(" ", "_") and kv.get("workload") == workload
                         and kv.get("csrc") == csrc_digest()):
                     return float(kv["bytes_per_launch"])
     except (OSError, ValueError, KeyError):
