@@ -2,11 +2,13 @@
 """Benchmark the decode weight sweep through libqgemv.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl ours|reference]
+                    [--impl ours|reference] [--path auto|persistent|launches]
 
 A step is one full sweep of the decoder's weights (every layer's q|k|v, o,
 gate/up + SwiGLU and down, then the LM head + argmax) replayed from a CUDA
-graph.  The default workload is the Qwen3-VL-2B-shaped int8 block-32 S=1
+graph.  At S=1 the sweep runs by default as one persistent launch
+(qg_sweep_run); `--path launches` times the same stages as one launch per
+call instead (S=16 always runs that way).  The default workload is the Qwen3-VL-2B-shaped int8 block-32 S=1
 sweep (1.83 GB per sweep, far larger than the 126 MB L2, so no flush is
 needed between steps).  N > 1 runs one replica per GPU (launch with torchrun):
 decode sweeps are independent, so nothing is exchanged and the time is the
@@ -58,6 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="auto", choices=["auto", "persistent", "launches"],
+                    help="S=1 sweep as one persistent launch (auto) or one launch per call")
     ap.add_argument("--graph-sweeps", type=int, default=1,
                     help="sweeps captured per CUDA graph (steps are rounded up to a multiple)")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0,
@@ -313,8 +317,11 @@ def run_ours(a):
     dname, body_fmt, head_fmt, S = WORKLOADS[a.workload]
     dec = getattr(wl, dname)
     sw = DecodeSweep(dec, body_fmt, head_fmt, S=S, device=dev)
+    persistent = S == 1 and a.path != "launches"
+    if a.path == "persistent" and S != 1:
+        raise SystemExit("--path persistent needs an S=1 workload")
     G = max(1, a.graph_sweeps)
-    graph = sw.capture(sweeps_per_graph=G)
+    graph = sw.capture(sweeps_per_graph=G, persistent=persistent)
     steps = ((a.steps + G - 1) // G) * G
     stream = torch.cuda.current_stream(dev)
     sweep_bytes = sw.weight_bytes
@@ -340,11 +347,18 @@ def run_ours(a):
     value = aggregate(steps * sweep_bytes / 1e9, el_s, world)
     sweeps_s = aggregate(steps, el_s, world)
 
-    # --- dominant kernel: the fused gate/up SwiGLU over every layer --------
-    dom = _time_gate_up(sw, stream, dev, qg, torch)
+    # --- dominant kernel --------------------------------------------------
+    if persistent:
+        # the persistent sweep kernel is every launch of the timed region; its
+        # average duration comes from the same CUDA events on its stream
+        dom = {"kernel": "sweep_kernel (persistent sweep)", "us": el_ms * 1e3 / steps,
+               "gbs": sweep_bytes / (el_ms * 1e-3 / steps) / 1e9, "bytes": sweep_bytes,
+               "launches": steps}
+    else:
+        dom = _time_gate_up(sw, stream, dev, qg, torch)
 
     # --- end to end: pinned host inputs -> sweep -> greedy token to host ---
-    e2e = _time_e2e(sw, graph, G, steps, a.warmup, stream, dev, world, torch)
+    e2e = _time_e2e(sw, graph, G, steps, a.warmup, stream, dev, world, torch, persistent)
 
     peak, peak_kind = hbm_peak()
     line = {
@@ -353,7 +367,9 @@ def run_ours(a):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "i8/i4 x f16 -> f32" if S == 1 else "i8 x f16 -> f32 (mma f16)",
         "data": "synthetic (seeded N(0,0.02) weights, N(0,1) fp16 activations)",
-        "config": _config(a, dec, body_fmt, head_fmt, S, sweep_bytes),
+        "config": dict(_config(a, dec, body_fmt, head_fmt, S, sweep_bytes),
+                       path="persistent (one launch per sweep)" if persistent
+                       else "one launch per call"),
         "sweeps_per_s": round(sweeps_s, 2),
         "tokens_per_s": round(sweeps_s * S, 2),
         "hbm_frac": round(value / world / peak, 4),
@@ -366,7 +382,7 @@ def run_ours(a):
             "algorithmic_bytes_per_launch": dom["bytes"],
             "launch_us": round(dom["us"], 3), "launches": dom["launches"]},
         "e2e": e2e,
-        "gpu_launches": steps * sw.launches_per_sweep,
+        "gpu_launches": steps * sw.launches_per_sweep(persistent),
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -412,7 +428,7 @@ def _time_gate_up(sw, stream, dev, qg, torch):
             "launches": launches}
 
 
-def _time_e2e(sw, graph, G, steps, warmup, stream, dev, world, torch):
+def _time_e2e(sw, graph, G, steps, warmup, stream, dev, world, torch, persistent):
     """Same metric through the public path with host buffers: each step copies
     that step's activations from pinned host memory, replays the sweep, and
     reads the greedy token back."""
@@ -420,7 +436,7 @@ def _time_e2e(sw, graph, G, steps, warmup, stream, dev, world, torch):
     idx_host = torch.empty(1, dtype=torch.int32).pin_memory()
     h2d = sum(x.numel() * x.element_size() for x in x_host)
     d2h = idx_host.numel() * idx_host.element_size()
-    single = sw.capture(sweeps_per_graph=1) if G != 1 else graph
+    single = sw.capture(sweeps_per_graph=1, persistent=persistent) if G != 1 else graph
     sw.graph = graph
 
     def one():

@@ -53,7 +53,9 @@ typedef enum {
     QG_ERR_FORMAT = 4,    /* unknown format, or gate/up weights that disagree */
     QG_ERR_WORKSPACE = 5, /* workspace NULL or smaller than required */
     QG_ERR_CUDA = 6,      /* a CUDA runtime call or launch failed */
-    QG_ERR_TIMEOUT = 7    /* a device-side bounded wait expired (see qg_stream_check) */
+    QG_ERR_TIMEOUT = 7,   /* a device-side bounded wait expired (see qg_stream_check) */
+    QG_ERR_PLAN = 8       /* qg_sweep_run found no plan of that many stages in its
+                             workspace (reported by qg_stream_check) */
 } qg_status;
 
 typedef enum {
@@ -204,10 +206,100 @@ QG_API qg_status qg_head_argmax_noalloc(const qg_weight* W, const uint16_t* x, f
                                         int32_t* idx, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * qg_sweep_* -- a whole one-token decode step as ONE persistent launch.
+ * A decode step reads every decoder weight once ("Qwen3-VL 4B -- Core AI
+ * (.aimodel)", Measured), as an ordered chain of S=1 projections per layer
+ * (qkv -> o -> gate/up + SwiGLU -> down) and the LM head with the greedy
+ * argmax ("Qwen3.8-27B ... -- Core AI", The vision path: prefill runs as
+ * pipelined S=1 steps).  A sweep is that chain: an ordered list of stages,
+ * each one of the S=1 calls above with the same arguments, results and
+ * accuracy (the results are bit-identical to those calls).
+ *
+ * Order: stage i + 1 reads its x only after every part of stage i is done,
+ * exactly as if the calls were enqueued one after another on one stream, so
+ * a stage may read what an earlier stage wrote.  What the single launch adds
+ * is that the WEIGHTS of stage i + 1 (which no stage writes) start streaming
+ * while the GPU waits for the last parts of stage i, and no launch gaps.
+ *
+ *   op     : QG_STAGE_GEMV        y = W x  (y and/or y16, as qg_gemv_s1)
+ *            QG_STAGE_SWIGLU      h = fp16(silu(W x) * (w_up x))
+ *                                 (as qg_gate_up_swiglu with S = 1)
+ *            QG_STAGE_HEAD_ARGMAX logits = W x (optional), idx = argmax
+ *                                 (as qg_head_argmax; the workspace is part
+ *                                 of the sweep's)
+ *   w      : the weight (the gate weight for QG_STAGE_SWIGLU), a copy.
+ *   w_up   : QG_STAGE_SWIGLU only: the up weight (same format and shape).
+ *   x      : fp16 [k], 16-byte aligned, device.
+ *   y, y16 : QG_STAGE_GEMV outputs (at least one), as qg_gemv_s1.
+ *   h      : QG_STAGE_SWIGLU output fp16 [n], 2-byte aligned.
+ *   logits, idx : QG_STAGE_HEAD_ARGMAX outputs, as qg_head_argmax.
+ * Unused pointers must be NULL.  Every pointer stays owned by the caller and
+ * must stay valid while a run that uses the plan can execute.
+ *
+ * Formats: a plan is either all int8, or the int4 run's layout -- every
+ *   GEMV and SwiGLU stage int4 and every head int8 (the pages pair an int4
+ *   body with an absmax int8 head); other mixes give QG_ERR_FORMAT.
+ *
+ * qg_sweep_workspace_bytes(n) -- device bytes a plan of n stages needs.
+ * qg_sweep_plan -- validates every stage (the same checks, with the same
+ *   status codes, as the single calls; QG_ERR_FORMAT for an unknown op or a
+ *   format mix above; QG_ERR_SHAPE if a stage's rows do not hold a multiple
+ *   of 8 scales, i.e. k % 256 (int8) or k % 512 (int4), or its x does not
+ *   fit the launch's shared memory, k <= 17408 for every shape the pages
+ *   use), writes the plan into `workspace` (device memory, 256-byte aligned,
+ *   at least qg_sweep_workspace_bytes(n) bytes) with a synchronous
+ *   host-to-device copy, and fills `*sweep` (host memory owned by the
+ *   caller), which qg_sweep_run reads.  Call it outside stream capture, and
+ *   never while a run that uses the same workspace may still execute.
+ *   1 <= n_stages <= 65536.
+ * qg_sweep_run -- enqueues one run of the plan on `stream` (asynchronous;
+ *   safe to capture in a CUDA graph).  It is a cooperative launch of two
+ *   CTAs per SM that must all be resident at once: it fails with
+ *   QG_ERR_CUDA if the device cannot host them, and runs must not overlap
+ *   other runs of the same workspace.  Between stages the CTAs wait on
+ *   counters in the workspace; a wait that has not finished after ~2 s gives
+ *   up, and qg_stream_check then reports QG_ERR_TIMEOUT; a workspace that
+ *   does not hold the plan `sweep` describes is reported as QG_ERR_PLAN.  After either
+ *   error, plan the workspace again before the next run.  Every run that
+ *   completes leaves the counters zero for the next one.
+ * ------------------------------------------------------------------------- */
+typedef enum {
+    QG_STAGE_GEMV = 0,
+    QG_STAGE_SWIGLU = 1,
+    QG_STAGE_HEAD_ARGMAX = 2
+} qg_stage_op;
+
+typedef struct {
+    int32_t op;
+    int32_t reserved;
+    qg_weight w;
+    qg_weight w_up;
+    const uint16_t* x;
+    float* y;
+    uint16_t* y16;
+    uint16_t* h;
+    float* logits;
+    int32_t* idx;
+} qg_stage;
+
+/* What qg_sweep_run needs to know about a plan on the host. */
+typedef struct {
+    int32_t n_stages; /* stages in the plan */
+    int32_t kernel;   /* the persistent kernel that runs it: 0 int8, 1 int4 */
+    int64_t reserved[3];
+} qg_sweep;
+
+QG_API size_t qg_sweep_workspace_bytes(int n_stages);
+QG_API qg_status qg_sweep_plan(const qg_stage* stages, int n_stages, void* workspace,
+                               size_t ws_bytes, qg_sweep* sweep);
+QG_API qg_status qg_sweep_run(const qg_sweep* sweep, void* workspace, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * qg_stream_check -- synchronize `stream` and report asynchronous failures:
- * QG_ERR_CUDA for a CUDA error, QG_ERR_TIMEOUT if a kernel's bounded wait on
- * its own bulk copies expired since the last check (the flag is then
- * cleared).  Kernels never spin without a limit.
+ * QG_ERR_CUDA for a CUDA error, QG_ERR_PLAN if a sweep ran on a workspace
+ * without its plan, QG_ERR_TIMEOUT if a kernel's bounded wait (on its own
+ * copies, or a sweep's wait between stages) expired since the last check
+ * (the flags are then cleared).  Kernels never spin without a limit.
  * ------------------------------------------------------------------------- */
 QG_API qg_status qg_stream_check(cudaStream_t stream);
 

@@ -1,6 +1,7 @@
 // qg_api.cu -- the extern "C" entry points of libqgemv: argument validation
 // (synchronous, before any launch) and dispatch to the kernel launchers.
 #include <cstdint>
+#include <vector>
 
 #include "qg_internal.h"
 
@@ -63,11 +64,65 @@ qg_status check_weight(const qg_weight* W) {
     return QG_OK;
 }
 
+constexpr int kMaxSweepStages = 65536;
+
+// One sweep stage -> the launch description of the S=1 call it stands for,
+// with that call's checks.
+qg_status stage_launch(const qg_stage& S, qg::GemvLaunch* out) {
+    qg::GemvLaunch L = {};
+    qg_status st = check_weight(&S.w);
+    if (st != QG_OK) return st;
+    if (!S.x) return QG_ERR_NULL;
+    if (!aligned(S.x, 16)) return QG_ERR_ALIGN;
+    L.fmt = S.w.fmt;
+    L.nmat = 1;
+    L.n = S.w.n;
+    L.k = S.w.k;
+    L.codes[0] = S.w.codes;
+    L.scales[0] = S.w.scales;
+    L.biases[0] = S.w.biases;
+    L.x = S.x;
+    switch (S.op) {
+        case QG_STAGE_GEMV:
+            if (!S.y && !S.y16) return QG_ERR_NULL;
+            if ((S.y && !aligned(S.y, 4)) || (S.y16 && !aligned(S.y16, 2))) return QG_ERR_ALIGN;
+            L.epilogue = qg::kEpiPlain;
+            L.y = S.y;
+            L.y16 = S.y16;
+            break;
+        case QG_STAGE_SWIGLU:
+            st = check_weight(&S.w_up);
+            if (st != QG_OK) return st;
+            if (S.w_up.fmt != S.w.fmt) return QG_ERR_FORMAT;
+            if (S.w_up.n != S.w.n || S.w_up.k != S.w.k) return QG_ERR_SHAPE;
+            if (!S.h) return QG_ERR_NULL;
+            if (!aligned(S.h, 2)) return QG_ERR_ALIGN;
+            L.epilogue = qg::kEpiSwiglu;
+            L.nmat = 2;
+            L.codes[1] = S.w_up.codes;
+            L.scales[1] = S.w_up.scales;
+            L.biases[1] = S.w_up.biases;
+            L.h = S.h;
+            break;
+        case QG_STAGE_HEAD_ARGMAX:
+            if (!S.idx) return QG_ERR_NULL;
+            if ((S.logits && !aligned(S.logits, 4)) || !aligned(S.idx, 4)) return QG_ERR_ALIGN;
+            L.epilogue = qg::kEpiHead;
+            L.logits = S.logits;
+            L.idx = S.idx;
+            break;
+        default:
+            return QG_ERR_FORMAT;
+    }
+    *out = L;
+    return QG_OK;
+}
+
 }  // namespace
 
 extern "C" {
 
-int qg_abi_version(void) { return 100; }
+int qg_abi_version(void) { return 101; }
 
 const char* qg_last_cuda_error(void) { return qg::last_cuda_error_name(); }
 
@@ -81,6 +136,7 @@ const char* qg_status_string(qg_status s) {
         case QG_ERR_WORKSPACE: return "QG_ERR_WORKSPACE: workspace NULL or too small";
         case QG_ERR_CUDA: return "QG_ERR_CUDA: CUDA runtime error";
         case QG_ERR_TIMEOUT: return "QG_ERR_TIMEOUT: a device-side bounded wait expired";
+        case QG_ERR_PLAN: return "QG_ERR_PLAN: the workspace holds no sweep plan of that size";
     }
     return "QG_ERR_UNKNOWN";
 }
@@ -217,10 +273,45 @@ qg_status qg_head_argmax(const qg_weight* W, const uint16_t* x, float* logits, i
     return qg::launch_gemv_s1(L, stream);
 }
 
+size_t qg_sweep_workspace_bytes(int n_stages) {
+    if (n_stages < 1 || n_stages > kMaxSweepStages) return 0;
+    return qg::sweep_workspace_bytes(n_stages);
+}
+
+qg_status qg_sweep_plan(const qg_stage* stages, int n_stages, void* workspace, size_t ws_bytes,
+                        qg_sweep* sweep) {
+    if (!stages || !sweep) return QG_ERR_NULL;
+    if (n_stages < 1 || n_stages > kMaxSweepStages) return QG_ERR_SHAPE;
+    if (!workspace || ws_bytes < qg::sweep_workspace_bytes(n_stages)) return QG_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return QG_ERR_ALIGN;
+    std::vector<qg::GemvLaunch> L(static_cast<size_t>(n_stages));
+    for (int i = 0; i < n_stages; ++i) {
+        qg_status st = stage_launch(stages[i], &L[i]);
+        if (st != QG_OK) return st;
+    }
+    int kernel = -1;
+    qg_status st = qg::plan_sweep(L.data(), n_stages, workspace, ws_bytes, &kernel);
+    if (st != QG_OK) return st;
+    qg_sweep out = {};
+    out.n_stages = n_stages;
+    out.kernel = kernel;
+    *sweep = out;
+    return QG_OK;
+}
+
+qg_status qg_sweep_run(const qg_sweep* sweep, void* workspace, cudaStream_t stream) {
+    if (!sweep || !workspace) return QG_ERR_NULL;
+    if (sweep->n_stages < 1 || sweep->n_stages > kMaxSweepStages) return QG_ERR_SHAPE;
+    if (!aligned(workspace, 256)) return QG_ERR_ALIGN;
+    return qg::launch_sweep(sweep->kernel, workspace, sweep->n_stages, stream);
+}
+
 qg_status qg_stream_check(cudaStream_t stream) {
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return qg::cuda_status(e);
-    const unsigned int f = qg::gemv_read_and_clear_error() | qg::gemm_s16_read_and_clear_error();
+    const unsigned int g = qg::gemv_read_and_clear_error();
+    const unsigned int f = g | qg::gemm_s16_read_and_clear_error();
+    if (g & qg::kGemvErrBadPlan) return QG_ERR_PLAN;
     return f ? QG_ERR_TIMEOUT : QG_OK;
 }
 

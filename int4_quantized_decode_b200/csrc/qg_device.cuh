@@ -123,6 +123,37 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
     return v;
 }
 
+// A 16-byte load served by L2 (never from a possibly stale L1 line): for data
+// that other CTAs of the same grid wrote earlier in the launch.
+__device__ __forceinline__ uint4 ldg_cg_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Wait until *counter >= target (a counter other CTAs of this grid increment
+// after a __threadfence).  Gives up after kWaitLimitCycles; returns whether
+// the target was reached.
+__device__ __forceinline__ bool wait_counter_bounded(const unsigned int* counter,
+                                                     unsigned int target) {
+    if (ld_acquire_gpu(counter) >= target) return true;
+    const long long t0 = clock64();
+    while (ld_acquire_gpu(counter) < target) {
+        if (clock64() - t0 > kWaitLimitCycles) return false;
+        __nanosleep(64);
+    }
+    return true;
+}
+
 __device__ __forceinline__ uint16_t ldg_nc_u16(const void* p) {
     uint16_t v;
     asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));

@@ -31,6 +31,7 @@
 //    the kernel before it; only x waits for that kernel.
 #include <cfloat>
 #include <climits>
+#include <vector>
 
 #include "qg_device.cuh"
 #include "qg_internal.h"
@@ -183,9 +184,10 @@ struct Frag {
 };
 
 // ------------------------------------------------------ shared kernel parts --
-// Stage x (fp16 in global memory, written by the previous kernel) into shared
-// memory as fp32 in the conflict-free piece layout; int4 also gets the sum of
-// x over each 32-code lane granule and the pair-permuted order dot32_i4 uses.
+// Stage x (fp16 in global memory, written by the previous kernel or by an
+// earlier stage of the same sweep, hence read through L2) into shared memory
+// as fp32 in the conflict-free piece layout; int4 also gets the sum of x over
+// each 32-code lane granule and the pair-permuted order dot32_i4 uses.
 template <int FMT>
 __device__ __forceinline__ void stage_x(const uint16_t* __restrict__ x, float* xs, float* hsum,
                                         int granules) {
@@ -196,7 +198,7 @@ __device__ __forceinline__ void stage_x(const uint16_t* __restrict__ x, float* x
         float gsum = 0.f;
 #pragma unroll
         for (int c = 0; c < F::kCodesPerLane / 8; ++c) {
-            const uint4 v = *reinterpret_cast<const uint4*>(xg + 8 * c);
+            const uint4 v = ldg_cg_v4(xg + 8 * c);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
             float a[8];
 #pragma unroll
@@ -454,12 +456,8 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
 }
 
 // ----------------------------------------------------------------------- //
-// Shared-memory-ring kernel: every lane copies the 16-byte code vectors    //
-// it will consume with cp.async into its own ring slots, kRing-1 steps     //
-// ahead; a few lanes copy each step's scales (and biases) as 16-byte       //
-// pieces, read by the warp after a __syncwarp.  Bytes in flight cost no    //
-// registers: 3 steps x RG rows x 16 B per lane stay outstanding.          //
-// Requires a multiple of 8 scales per row (16-byte pieces).                //
+// Shared-memory rings: the fast path, as a launch of its own or as one     //
+// stage of a persistent sweep.                                             //
 // ----------------------------------------------------------------------- //
 constexpr int kRing = 4;
 
@@ -497,17 +495,66 @@ struct RingLayout {
     static constexpr int kPerRow = kCodes + kSide * (FMT == 1 ? 2 : 1);
 };
 
-template <int FMT, int NMAT, int RG, int EPI>
-__global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) {
+// Shared memory of one CTA's rings; x (and the int4 sums) follow it.
+__host__ __device__ constexpr uint32_t ring_bytes(int fmt, int rows) {
+    return static_cast<uint32_t>(kWarps * kRing * rows *
+                                 (kLanes * 16 + 32 * (fmt == 1 ? 2 : 1)));
+}
+
+// How a ring stage orders itself after the work before it.
+//  * StreamSync -- a launch of its own: programmatic dependent launch.  The
+//    weight prologue runs while the previous kernel in the stream finishes;
+//    x is read after griddepcontrol.wait.
+//  * GridSync -- one stage of a persistent sweep: when every warp of the CTA
+//    is done with the previous stage, the CTA arrives on that stage's counter
+//    and issues this stage's weight prologue, then waits (bounded) until all
+//    CTAs have arrived before it reads x, which the previous stage may have
+//    written.
+struct StreamSync {
+    __device__ __forceinline__ void before_prologue() {}
+    __device__ __forceinline__ bool wait_input() {
+        griddep_wait();
+        return true;
+    }
+    __device__ __forceinline__ void input_staged() { griddep_launch_dependents(); }
+};
+
+struct GridSync {
+    unsigned int* prev;  // arrival counter of the previous stage, or nullptr
+    int* go;             // shared: the outcome of thread 0's wait
+    // (the sweep kernel has synchronized the CTA: every warp is done with the
+    // previous stage's outputs, x and rings)
+    __device__ __forceinline__ void before_prologue() {
+        if (prev && threadIdx.x == 0) {
+            __threadfence();
+            atomicAdd(prev, 1u);
+        }
+    }
+    __device__ __forceinline__ bool wait_input() {
+        if (threadIdx.x == 0)
+            *go = (prev == nullptr || wait_counter_bounded(prev, gridDim.x)) ? 1 : 0;
+        __syncthreads();
+        return *go != 0;
+    }
+    __device__ __forceinline__ void input_staged() {}
+};
+
+// One weight (or gate/up pair) streamed through per-lane shared-memory rings:
+// every lane copies the 16-byte code vectors it will consume with cp.async
+// into its own ring slots, kRing-1 steps ahead; a few lanes copy each step's
+// scales (and biases) as 16-byte pieces, read by the warp after a __syncwarp.
+// Bytes in flight cost no registers: 3 steps x RG rows x 16 B per lane stay
+// outstanding.  Requires a multiple of 8 scales per row (16-byte pieces).
+// Returns false, with its copies drained, if the wait for x gave up.
+template <int FMT, int NMAT, int RG, int EPI, class SYNC>
+__device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem, SYNC& sync,
+                                           float* red_v, int* red_i) {
     using F = Fmt<FMT>;
     using RL = RingLayout<FMT, NMAT>;
     constexpr int ROWS = NMAT * RG;
     constexpr int kStepBytes = kLanes * 16;
     constexpr int kStepSides = kStepBytes * (FMT == 0 ? 1 : 2) / F::kBlock;  // 16
     constexpr int kSideLanes = 2 * ROWS * (F::kBias ? 2 : 1);  // lanes that copy side data
-    extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ float red_v[kWarps];
-    __shared__ int red_i[kWarps];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t N = p.n, K = p.k;
@@ -522,9 +569,9 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) 
     const int64_t side_per_row = K / F::kBlock;  // a multiple of 8 (16-byte pieces)
     const uint64_t pol = l2_policy_evict_first();
 
-    // shared memory: [ring of this CTA's warps][x fp32][hsum]
+    // shared memory: [rings of this CTA's warps][x fp32][hsum]
     const uint32_t ring = smem_u32(smem) + warp * (kRing * ROWS * RL::kPerRow);
-    float* xs = reinterpret_cast<float*>(smem + kWarps * kRing * ROWS * RL::kPerRow);
+    float* xs = reinterpret_cast<float*>(smem + ring_bytes(FMT, ROWS));
     float* hsum = xs + p.x_floats;
     auto slot_codes = [&](int s, int j) -> uint32_t {  // this lane's code vector
         return ring + (s * ROWS + j) * RL::kPerRow + lane * 16;
@@ -585,7 +632,8 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) 
         }
     };
 
-    // 1) weight prologue (independent of the previous kernel)
+    // 1) weight prologue (independent of the work before this stage)
+    sync.before_prologue();
     if (my_items > 0) set_item(0);
 #pragma unroll
     for (int d = 0; d < kRing - 1; ++d) {
@@ -594,11 +642,14 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) 
     }
     if (lane == 0) prefetch_items<FMT, NMAT, RG>(p, wg, tw, 1, p.prefetch_items - 1, my_items);
 
-    // 2) x from the previous kernel
-    griddep_wait();
+    // 2) x, which the work before this stage may have written
+    if (!sync.wait_input()) {
+        cp_async_wait<0>();
+        return false;
+    }
     stage_x<FMT>(p.x, xs, hsum, granules);
     __syncthreads();
-    griddep_launch_dependents();
+    sync.input_staged();
 
     // 3) stream: issue step t + kRing - 1, wait for step t, compute it
     const float4* xs4 = reinterpret_cast<const float4*>(xs);
@@ -645,6 +696,16 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) 
     }
     cp_async_wait<0>();
     if (EPI == kEpiHead) head_finish(p, best_v, best_i, warp, lane, red_v, red_i, kWarps);
+    return true;
+}
+
+template <int FMT, int NMAT, int RG, int EPI>
+__global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ float red_v[kWarps];
+    __shared__ int red_i[kWarps];
+    StreamSync sync;
+    ring_stage<FMT, NMAT, RG, EPI>(p, smem, sync, red_v, red_i);
 }
 
 size_t x_smem_bytes(int fmt, const Params& p) {
@@ -655,7 +716,7 @@ size_t x_smem_bytes(int fmt, const Params& p) {
 
 template <int FMT, int NMAT, int RG>
 constexpr size_t ring_smem_bytes() {
-    return static_cast<size_t>(kWarps) * kRing * NMAT * RG * RingLayout<FMT, NMAT>::kPerRow;
+    return ring_bytes(FMT, NMAT * RG);
 }
 
 // Per-CTA shared memory that still lets two CTAs share an SM.
@@ -734,12 +795,133 @@ qg_status dispatch_fmt(const GemvLaunch& L, const Params& p, const DeviceInfo& d
     return launch_pick<FMT, 1, 1, kEpiPlain>(p, dev, stream);
 }
 
-}  // namespace
+// ----------------------------------------------------------------------- //
+// Persistent sweep: every stage of a decode step in one launch.            //
+// ----------------------------------------------------------------------- //
+// A stage's variant within the kernel that runs its plan.  Each kernel holds
+// only as many ring variants as fit its 128 registers per thread without
+// spilling: kernel 0 runs int8 plans (every epilogue, 1/2/4 rows per warp
+// item), kernel 1 runs int4 plans (int4 projections at 1-2 rows, SwiGLU at
+// 1 row, and the int8 head the pages pair with an int4 body).
+enum : int32_t {
+    kVarPlain1, kVarPlain2, kVarPlain4, kVarSwiglu1, kVarSwiglu2,
+    kVarHead1, kVarHead2, kVarHead4
+};
+enum : int32_t { kI4Plain1, kI4Plain2, kI4Swiglu1, kI4Head8x1, kI4Head8x2, kI4Head8x4 };
 
-qg_status launch_gemv_s1(const GemvLaunch& L, cudaStream_t stream) {
-    DeviceInfo dev;
-    qg_status st = device_info(&dev);
-    if (st != QG_OK) return st;
+constexpr uint32_t kSweepMagic = 0x57534751u;  // "QGSW"
+
+struct SweepHeader {
+    uint32_t magic;
+    int32_t n_stages;
+    int32_t kernel;
+    uint32_t reserved[61];
+};
+static_assert(sizeof(SweepHeader) == 256, "header is 256 bytes");
+
+struct SweepStage {
+    Params p;
+    int32_t variant;
+    int32_t reserved;
+};
+
+__host__ __device__ constexpr size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Workspace: [header][arrival counters: one per stage + one exit counter]
+//            [16 bytes of argmax scratch per stage][stage descriptors]
+__host__ __device__ constexpr size_t sweep_counters_offset() { return sizeof(SweepHeader); }
+__host__ __device__ constexpr size_t sweep_scratch_offset(int n) {
+    return sweep_counters_offset() + align256(static_cast<size_t>(n + 1) * 4);
+}
+__host__ __device__ constexpr size_t sweep_stages_offset(int n) {
+    return sweep_scratch_offset(n) + align256(static_cast<size_t>(n) * 16);
+}
+
+// The stage's parameters are read from shared memory where they are needed
+// (per item, not per step), as a launch of its own reads its constant bank.
+template <int FMT, int NMAT, int RG, int EPI>
+__device__ __forceinline__ bool sweep_stage(const SweepStage* st, unsigned char* smem,
+                                            unsigned int* prev, int* go, float* red_v, int* red_i) {
+    GridSync sync{prev, go};
+    return ring_stage<FMT, NMAT, RG, EPI>(st->p, smem, sync, red_v, red_i);
+}
+
+template <int KERNEL>
+__device__ __forceinline__ bool sweep_dispatch(int v, const SweepStage* st, unsigned char* smem,
+                                               unsigned int* prev, int* go, float* red_v,
+                                               int* red_i) {
+#define QG_STAGE(F, M, R, E) return sweep_stage<F, M, R, E>(st, smem, prev, go, red_v, red_i)
+    if (KERNEL == 0) {
+        switch (v) {
+            case kVarPlain1: QG_STAGE(0, 1, 1, kEpiPlain);
+            case kVarPlain2: QG_STAGE(0, 1, 2, kEpiPlain);
+            case kVarPlain4: QG_STAGE(0, 1, 4, kEpiPlain);
+            case kVarSwiglu1: QG_STAGE(0, 2, 1, kEpiSwiglu);
+            case kVarSwiglu2: QG_STAGE(0, 2, 2, kEpiSwiglu);
+            case kVarHead1: QG_STAGE(0, 1, 1, kEpiHead);
+            case kVarHead2: QG_STAGE(0, 1, 2, kEpiHead);
+            default: QG_STAGE(0, 1, 4, kEpiHead);
+        }
+    } else {
+        switch (v) {
+            case kI4Plain1: QG_STAGE(1, 1, 1, kEpiPlain);
+            case kI4Plain2: QG_STAGE(1, 1, 2, kEpiPlain);
+            case kI4Swiglu1: QG_STAGE(1, 2, 1, kEpiSwiglu);
+            case kI4Head8x1: QG_STAGE(0, 1, 1, kEpiHead);
+            case kI4Head8x2: QG_STAGE(0, 1, 2, kEpiHead);
+            default: QG_STAGE(0, 1, 4, kEpiHead);
+        }
+    }
+#undef QG_STAGE
+}
+
+// One CTA per (SM, slot) for the whole sweep.  Stage s + 1 streams its first
+// weights while the grid waits for the last CTAs of stage s; x of stage s + 1
+// is read only after every CTA has finished stage s, the order a stream of
+// separate launches gives.  Requires every CTA to be resident at once (a
+// cooperative launch).
+template <int KERNEL>
+__global__ void __launch_bounds__(kThreads, 2) sweep_kernel(unsigned char* ws, int n_stages) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ float red_v[kWarps];
+    __shared__ int red_i[kWarps];
+    __shared__ int go;
+    __shared__ __align__(16) SweepStage cur;
+    const SweepHeader* hdr = reinterpret_cast<const SweepHeader*>(ws);
+    if (hdr->magic != kSweepMagic || hdr->n_stages != n_stages || hdr->kernel != KERNEL) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(&g_gemv_err, kGemvErrBadPlan);
+        return;
+    }
+    unsigned int* ctr = reinterpret_cast<unsigned int*>(ws + sweep_counters_offset());
+    const SweepStage* stages = reinterpret_cast<const SweepStage*>(ws + sweep_stages_offset(n_stages));
+    static_assert(sizeof(SweepStage) % 16 == 0, "stage descriptors copy as 16-byte pieces");
+    constexpr int kPieces = static_cast<int>(sizeof(SweepStage) / 16);
+    for (int s = 0; s < n_stages; ++s) {
+        __syncthreads();  // every warp is done with the previous stage
+        if (threadIdx.x < kPieces)
+            reinterpret_cast<uint4*>(&cur)[threadIdx.x] =
+                ldg_nc_v4(reinterpret_cast<const uint4*>(stages + s) + threadIdx.x);
+        __syncthreads();
+        unsigned int* prev = s > 0 ? ctr + (s - 1) : nullptr;
+        const bool ok = sweep_dispatch<KERNEL>(cur.variant, &cur, smem, prev, &go, red_v, red_i);
+        if (!ok) {
+            if (threadIdx.x == 0) atomicOr(&g_gemv_err, kGemvErrTimeout);
+            return;
+        }
+    }
+    // The last CTA to finish re-zeroes every counter for the next run (no CTA
+    // reads a counter after it has arrived here).
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(ctr + n_stages, 1u) == gridDim.x - 1) {
+            for (int s = 0; s <= n_stages; ++s) ctr[s] = 0u;
+            __threadfence();
+        }
+    }
+}
+
+Params make_params(const GemvLaunch& L) {
     Params p = {};
     for (int m = 0; m < 2; ++m) {
         const int src = m < L.nmat ? m : 0;
@@ -762,6 +944,125 @@ qg_status launch_gemv_s1(const GemvLaunch& L, cudaStream_t stream) {
     const int cpl = L.fmt == QG_FMT_I8_B32 ? Fmt<0>::kCodesPerLane : Fmt<1>::kCodesPerLane;
     const int granules = static_cast<int>(L.k / cpl);
     p.x_floats = align_up(granules, 8) * cpl;
+    return p;
+}
+
+// The variant of a sweep stage in kernel `kernel`: the standalone launch's
+// choice of rows per item, lowered to what the kernel holds and until the
+// stage's rings and x fit the per-CTA budget.  Returns -1 (with *status set)
+// if the kernel has no variant for the stage.
+int sweep_variant(int kernel, const GemvLaunch& L, const Params& p, int total_warps, int* rg_out,
+                  qg_status* status) {
+    const int block = L.fmt == QG_FMT_I8_B32 ? 32 : 64;
+    *status = QG_ERR_SHAPE;
+    if ((L.k / block) % 8 != 0) return -1;
+    const bool swiglu = L.epilogue == kEpiSwiglu, head = L.epilogue == kEpiHead;
+    int max_rg = swiglu ? 2 : 4;
+    if (kernel == 1) {
+        if (head ? L.fmt != QG_FMT_I8_B32 : L.fmt != QG_FMT_I4_G64) {
+            *status = QG_ERR_FORMAT;
+            return -1;
+        }
+        if (!head) max_rg = swiglu ? 1 : 2;
+    }
+    const size_t xb = x_smem_bytes(L.fmt, p);
+    const int nmat = swiglu ? 2 : 1;
+    for (int rg = pick_rg(L.n, max_rg, total_warps); rg >= 1; rg /= 2) {
+        if (xb + ring_bytes(L.fmt, nmat * rg) > kSmemPerCtaBudget) continue;
+        *rg_out = rg;
+        *status = QG_OK;
+        if (kernel == 0) {
+            if (swiglu) return rg == 2 ? kVarSwiglu2 : kVarSwiglu1;
+            if (head) return rg == 4 ? kVarHead4 : (rg == 2 ? kVarHead2 : kVarHead1);
+            return rg == 4 ? kVarPlain4 : (rg == 2 ? kVarPlain2 : kVarPlain1);
+        }
+        if (swiglu) return kI4Swiglu1;
+        if (head) return rg == 4 ? kI4Head8x4 : (rg == 2 ? kI4Head8x2 : kI4Head8x1);
+        return rg == 2 ? kI4Plain2 : kI4Plain1;
+    }
+    return -1;
+}
+
+}  // namespace
+
+size_t sweep_workspace_bytes(int n_stages) {
+    return sweep_stages_offset(n_stages) + static_cast<size_t>(n_stages) * sizeof(SweepStage);
+}
+
+qg_status plan_sweep(const GemvLaunch* L, int n_stages, void* ws, size_t ws_bytes,
+                     int* kernel_out) {
+    DeviceInfo dev;
+    qg_status st = device_info(&dev);
+    if (st != QG_OK) return st;
+    const size_t bytes = sweep_workspace_bytes(n_stages);
+    if (ws_bytes < bytes) return QG_ERR_WORKSPACE;
+    int kernel = 0;
+    for (int i = 0; i < n_stages; ++i)
+        if (L[i].fmt == QG_FMT_I4_G64) kernel = 1;
+    std::vector<unsigned char> host(bytes, 0);
+    SweepHeader* hdr = reinterpret_cast<SweepHeader*>(host.data());
+    hdr->magic = kSweepMagic;
+    hdr->n_stages = n_stages;
+    hdr->kernel = kernel;
+    SweepStage* stages = reinterpret_cast<SweepStage*>(host.data() + sweep_stages_offset(n_stages));
+    unsigned char* dev_base = static_cast<unsigned char*>(ws);
+    const int total_warps = dev.num_sms * kCtasPerSm * kWarps;
+    for (int i = 0; i < n_stages; ++i) {
+        GemvLaunch Li = L[i];
+        if (Li.epilogue == kEpiHead) Li.workspace = dev_base + sweep_scratch_offset(n_stages) + 16 * i;
+        Params p = make_params(Li);
+        int rg = 1;
+        const int v = sweep_variant(kernel, Li, p, total_warps, &rg, &st);
+        if (v < 0) return st;
+        const int nmat = Li.epilogue == kEpiSwiglu ? 2 : 1;
+        const int64_t item_bytes = static_cast<int64_t>(nmat) * rg * (Li.fmt == 0 ? Li.k : Li.k / 2);
+        p.prefetch_items = static_cast<int>(kPrefetchBytesPerWarp / item_bytes);
+        if (p.prefetch_items < 1) p.prefetch_items = 1;
+        stages[i].p = p;
+        stages[i].variant = v;
+    }
+    st = cuda_status(cudaMemcpy(ws, host.data(), bytes, cudaMemcpyHostToDevice));
+    if (st == QG_OK) *kernel_out = kernel;
+    return st;
+}
+
+qg_status launch_sweep(int kernel, void* ws, int n_stages, cudaStream_t stream) {
+    DeviceInfo dev;
+    qg_status st = device_info(&dev);
+    if (st != QG_OK) return st;
+    if (kernel != 0 && kernel != 1) return QG_ERR_PLAN;
+    auto kern = kernel == 0 ? sweep_kernel<0> : sweep_kernel<1>;
+    static bool attr_set[2][64] = {{false}};
+    if (dev.device >= 64 || !attr_set[kernel][dev.device]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kSmemPerCtaBudget));
+        if (e != cudaSuccess) return cuda_status(e);
+        if (dev.device < 64) attr_set[kernel][dev.device] = true;
+    }
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads,
+                                                                  kSmemPerCtaBudget);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (per_sm < 1) return QG_ERR_SHAPE;
+    if (per_sm > kCtasPerSm) per_sm = kCtasPerSm;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(dev.num_sms * per_sm));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemPerCtaBudget;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, static_cast<unsigned char*>(ws), n_stages));
+}
+
+qg_status launch_gemv_s1(const GemvLaunch& L, cudaStream_t stream) {
+    DeviceInfo dev;
+    qg_status st = device_info(&dev);
+    if (st != QG_OK) return st;
+    const Params p = make_params(L);
     if (L.fmt == QG_FMT_I8_B32) return dispatch_fmt<0>(L, p, dev, stream);
     return dispatch_fmt<1>(L, p, dev, stream);
 }

@@ -43,6 +43,19 @@ struct GemvLaunch {
     void* workspace;      // head: zeroed scratch (key + ticket)
 };
 qg_status launch_gemv_s1(const GemvLaunch& L, cudaStream_t stream);
+
+// Persistent sweep: n S=1 stages (validated GemvLaunch descriptions, head
+// workspaces ignored) planned into a device workspace, then run as one
+// cooperative launch.
+size_t sweep_workspace_bytes(int n_stages);
+qg_status plan_sweep(const GemvLaunch* L, int n_stages, void* ws, size_t ws_bytes, int* kernel);
+qg_status launch_sweep(int kernel, void* ws, int n_stages, cudaStream_t stream);
+
+// Device error bits of the S=1 kernels (read and cleared by qg_stream_check):
+// bit 0 a bounded wait gave up, bit 1 a sweep ran on a workspace that holds
+// no plan of that many stages.
+constexpr unsigned int kGemvErrTimeout = 1u;
+constexpr unsigned int kGemvErrBadPlan = 2u;
 unsigned int gemv_read_and_clear_error();
 
 // Quantizers.

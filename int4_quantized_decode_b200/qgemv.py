@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_PKG, "libqgemv.so")
 QG_OK = 0
 STATUS_NAMES = {0: "QG_OK", 1: "QG_ERR_NULL", 2: "QG_ERR_SHAPE", 3: "QG_ERR_ALIGN",
                 4: "QG_ERR_FORMAT", 5: "QG_ERR_WORKSPACE", 6: "QG_ERR_CUDA",
-                7: "QG_ERR_TIMEOUT"}
+                7: "QG_ERR_TIMEOUT", 8: "QG_ERR_PLAN"}
 FMT_I8_B32 = 0
 FMT_I4_G64 = 1
 
@@ -29,7 +29,9 @@ FMT_I4_G64 = 1
 ABI_SYMBOLS = ("qg_quantize_block32", "qg_quantize_int4_g64", "qg_gemv_s1",
                "qg_gemm_s16", "qg_gate_up_swiglu", "qg_head_argmax_workspace_bytes",
                "qg_head_argmax", "qg_stream_check", "qg_status_string", "qg_abi_version",
-               "qg_last_cuda_error", "qg_head_argmax_noalloc")
+               "qg_last_cuda_error", "qg_head_argmax_noalloc", "qg_sweep_workspace_bytes",
+               "qg_sweep_plan", "qg_sweep_run")
+STAGE_GEMV, STAGE_SWIGLU, STAGE_HEAD_ARGMAX = 0, 1, 2
 
 
 class QgError(RuntimeError):
@@ -46,6 +48,18 @@ class CWeight(ctypes.Structure):
                 ("n", ctypes.c_int64), ("k", ctypes.c_int64),
                 ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("biases", ctypes.c_void_p)]
+
+
+class CStage(ctypes.Structure):
+    _fields_ = [("op", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("w", CWeight), ("w_up", CWeight), ("x", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("y16", ctypes.c_void_p), ("h", ctypes.c_void_p),
+                ("logits", ctypes.c_void_p), ("idx", ctypes.c_void_p)]
+
+
+class CSweep(ctypes.Structure):
+    _fields_ = [("n_stages", ctypes.c_int32), ("kernel", ctypes.c_int32),
+                ("reserved", ctypes.c_int64 * 3)]
 
 
 _lib = None
@@ -71,6 +85,11 @@ def lib() -> ctypes.CDLL:
         L.qg_head_argmax_workspace_bytes.restype = ctypes.c_size_t
         L.qg_head_argmax.argtypes = [W, P, P, P, P, ctypes.c_size_t, P]
         L.qg_head_argmax_noalloc.argtypes = [W, P, P, P, P]
+        L.qg_sweep_workspace_bytes.argtypes = [I]
+        L.qg_sweep_workspace_bytes.restype = ctypes.c_size_t
+        L.qg_sweep_plan.argtypes = [ctypes.POINTER(CStage), I, P, ctypes.c_size_t,
+                                    ctypes.POINTER(CSweep)]
+        L.qg_sweep_run.argtypes = [ctypes.POINTER(CSweep), P, P]
         L.qg_stream_check.argtypes = [P]
         L.qg_status_string.argtypes = [I]
         L.qg_status_string.restype = ctypes.c_char_p
@@ -79,7 +98,7 @@ def lib() -> ctypes.CDLL:
         L.qg_last_cuda_error.restype = ctypes.c_char_p
         for name in ABI_SYMBOLS:
             if name not in ("qg_head_argmax_workspace_bytes", "qg_status_string",
-                            "qg_last_cuda_error", "qg_head_argmax_noalloc"):
+                            "qg_last_cuda_error", "qg_sweep_workspace_bytes"):
                 getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -251,3 +270,73 @@ def qg_head_argmax_noalloc(W: QWeight, x: torch.Tensor, idx: torch.Tensor,
 
 def qg_stream_check(stream=None) -> None:
     _check("qg_stream_check", lib().qg_stream_check(_stream(stream)))
+
+
+# ----------------------------------------------------------------- sweeps --
+def stage_gemv(W: QWeight, x: torch.Tensor, y: Optional[torch.Tensor] = None,
+               y16: Optional[torch.Tensor] = None) -> CStage:
+    """A sweep stage equal to qg_gemv_s1(W, x, y, y16)."""
+    _cuda(x, torch.float16, "x")
+    if y is not None:
+        _cuda(y, torch.float32, "y")
+    if y16 is not None:
+        _cuda(y16, torch.float16, "y16")
+    return CStage(STAGE_GEMV, 0, W.c(), CWeight(), _ptr(x), _ptr(y), _ptr(y16), None, None,
+                  None)
+
+
+def stage_swiglu(Wg: QWeight, Wu: QWeight, x: torch.Tensor, h: torch.Tensor) -> CStage:
+    """A sweep stage equal to qg_gate_up_swiglu(Wg, Wu, x, h) with S = 1."""
+    _cuda(x, torch.float16, "x")
+    _cuda(h, torch.float16, "h")
+    return CStage(STAGE_SWIGLU, 0, Wg.c(), Wu.c(), _ptr(x), None, None, _ptr(h), None, None)
+
+
+def stage_head(W: QWeight, x: torch.Tensor, idx: torch.Tensor,
+               logits: Optional[torch.Tensor] = None) -> CStage:
+    """A sweep stage equal to qg_head_argmax(W, x, idx, ..., logits)."""
+    _cuda(x, torch.float16, "x")
+    _cuda(idx, torch.int32, "idx")
+    if logits is not None:
+        _cuda(logits, torch.float32, "logits")
+    return CStage(STAGE_HEAD_ARGMAX, 0, W.c(), CWeight(), _ptr(x), None, None, None,
+                  _ptr(logits), _ptr(idx))
+
+
+def qg_sweep_workspace_bytes(n_stages: int) -> int:
+    return int(lib().qg_sweep_workspace_bytes(int(n_stages)))
+
+
+def qg_sweep_plan(stages, workspace: torch.Tensor) -> CSweep:
+    """Plan `stages` (a list of CStage) into `workspace` (a uint8 CUDA tensor,
+    256-byte aligned, of at least qg_sweep_workspace_bytes(len(stages))
+    bytes).  Synchronous."""
+    _cuda(workspace, torch.uint8, "workspace")
+    arr = (CStage * len(stages))(*stages)
+    sw = CSweep()
+    _check("qg_sweep_plan", lib().qg_sweep_plan(arr, len(stages), _ptr(workspace),
+                                                workspace.numel(), ctypes.byref(sw)))
+    return sw
+
+
+def qg_sweep_run(sweep: CSweep, workspace: torch.Tensor, stream=None) -> None:
+    _check("qg_sweep_run", lib().qg_sweep_run(ctypes.byref(sweep), _ptr(workspace),
+                                              _stream(stream)))
+
+
+class SweepPlan:
+    """A planned sweep: its workspace, its host descriptor, and the tensors
+    its stages point to (kept alive as long as the plan)."""
+
+    def __init__(self, stages, tensors, device="cuda"):
+        n = len(stages)
+        nbytes = qg_sweep_workspace_bytes(n)
+        self._buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        off = (-self._buf.data_ptr()) % 256                # a 256-byte aligned view
+        self.workspace = self._buf[off:off + nbytes]
+        self.n_stages = n
+        self.tensors = list(tensors)
+        self.sweep = qg_sweep_plan(stages, self.workspace)
+
+    def run(self, stream=None) -> None:
+        qg_sweep_run(self.sweep, self.workspace, stream)

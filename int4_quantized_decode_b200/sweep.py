@@ -15,6 +15,11 @@ output.  With S = 16 (chunked prefill) every projection runs on the tensor-core
 path with a [16, K] chunk, o reads a fresh seeded chunk, and the head reads the
 chunk's last row.
 
+At S = 1 the sweep runs either as 4 launches per layer + 1 (one per call, with
+programmatic dependent launch between them) or as ONE persistent launch that
+runs the same stages in the same order (qg_sweep_plan / qg_sweep_run); the two
+give bit-identical results.
+
 All work is enqueued through the C ABI on the current stream; this module only
 allocates buffers, draws the seeded weights, and replays the graph.
 """
@@ -55,6 +60,7 @@ class DecodeSweep:
         self.head = self._quantized("head", -1, dec.vocab, dec.hidden, head_fmt)
         self._make_buffers(keep_logits)
         self.graph: Optional[torch.cuda.CUDAGraph] = None
+        self.plan: Optional[qg.SweepPlan] = None
 
     # ------------------------------------------------------------ weights --
     def _quantized(self, proj: str, layer: int, n: int, k: int, fmt: int,
@@ -118,9 +124,8 @@ class DecodeSweep:
                 for L in self.layers)
         return b + self.head.nbytes
 
-    @property
-    def launches_per_sweep(self) -> int:
-        return 4 * self.dec.layers + 1
+    def launches_per_sweep(self, persistent: bool = False) -> int:
+        return 1 if persistent else 4 * self.dec.layers + 1
 
     def inputs(self) -> List[torch.Tensor]:
         """The per-step activation tensors (contiguous), in a fixed order."""
@@ -146,24 +151,48 @@ class DecodeSweep:
     def run_head(self, stream=None) -> None:
         qg.qg_head_argmax(self.head, self.head_input(), self.idx, self.ws, self.logits, stream)
 
-    def step(self, stream=None) -> None:
+    def stages(self) -> List[qg.CStage]:
+        """The S = 1 sweep as persistent-launch stages, in run_layer's order."""
+        assert self.S == 1, "the persistent sweep runs S = 1 stages"
+        d, st = self.dec, []
+        for l, L in enumerate(self.layers):
+            st.append(qg.stage_gemv(L.qkv, self.x[l], self.y_qkv[0], self.y16_qkv))
+            st.append(qg.stage_gemv(L.o, self.y16_qkv[: d.q_dim], self.y_o[0]))
+            st.append(qg.stage_swiglu(L.gate, L.up, self.x[l], self.h[0]))
+            st.append(qg.stage_gemv(L.down, self.h[0], self.y_down[0]))
+        st.append(qg.stage_head(self.head, self.head_input(), self.idx, self.logits))
+        return st
+
+    def make_plan(self) -> qg.SweepPlan:
+        """Plan the persistent sweep (synchronous; outside stream capture)."""
+        if self.plan is None:
+            self.plan = qg.SweepPlan(self.stages(), [], self.device)
+        return self.plan
+
+    def step(self, stream=None, persistent: bool = False) -> None:
         """Enqueue one sweep on `stream` (default: the current stream)."""
+        if persistent:
+            self.make_plan().run(stream)
+            return
         for l in range(self.dec.layers):
             self.run_layer(l, stream)
         self.run_head(stream)
 
-    def capture(self, sweeps_per_graph: int = 1) -> torch.cuda.CUDAGraph:
+    def capture(self, sweeps_per_graph: int = 1,
+                persistent: bool = False) -> torch.cuda.CUDAGraph:
         """Capture `sweeps_per_graph` back-to-back sweeps into one CUDA graph."""
+        if persistent:
+            self.make_plan()
         s = torch.cuda.Stream(device=self.device)
         s.wait_stream(torch.cuda.current_stream(self.device))
         with torch.cuda.stream(s):
-            self.step()  # warm the launch paths (function attributes) outside capture
+            self.step(persistent=persistent)  # warm the launch paths outside capture
         torch.cuda.current_stream(self.device).wait_stream(s)
         torch.cuda.synchronize(self.device)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=s):
             for _ in range(sweeps_per_graph):
-                self.step()
+                self.step(persistent=persistent)
         self.graph = g
         self.sweeps_per_graph = sweeps_per_graph
         return g

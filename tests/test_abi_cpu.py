@@ -45,7 +45,7 @@ def test_status_strings_and_version(L):
     for code, name in qg.STATUS_NAMES.items():
         assert qg.status_string(code).startswith(name)
     assert qg.status_string(99) == "QG_ERR_UNKNOWN"
-    assert L.qg_abi_version() == 100
+    assert L.qg_abi_version() == 101
     assert L.qg_head_argmax_workspace_bytes(151936) >= 16
 
 
@@ -101,3 +101,50 @@ def test_head_and_quantize_validation(L):
     assert L.qg_quantize_block32(0x1004, 4, 64, 0x1000, 0x2000, None) == 3
     assert L.qg_quantize_int4_g64(0x1000, 4, 64, 0x1000, 0x2000, None, None) == 1
     assert L.qg_quantize_int4_g64(0x1000, 4, 96, 0x1000, 0x2000, 0x3000, None) == 2
+
+
+def stage(op=0, w=None, w_up=None, x=0x4000, y=0x5000, y16=None, h=None, logits=None, idx=None):
+    return qg.CStage(op, 0, w if w is not None else W(), w_up if w_up is not None else qg.CWeight(),
+                     x, y, y16, h, logits, idx)
+
+
+def plan(L, stages, ws=0x10000, nbytes=None, sweep=True):
+    arr = (qg.CStage * max(1, len(stages)))(*stages)
+    n = len(stages)
+    if nbytes is None:
+        nbytes = L.qg_sweep_workspace_bytes(max(n, 1))
+    out = qg.CSweep()
+    return L.qg_sweep_plan(arr if stages else None, n, ws, nbytes,
+                           ctypes.byref(out) if sweep else None)
+
+
+def test_sweep_validation(L):
+    assert L.qg_sweep_workspace_bytes(0) == 0
+    assert L.qg_sweep_workspace_bytes(1) > 0
+    assert L.qg_sweep_workspace_bytes(113) > L.qg_sweep_workspace_bytes(1)
+    assert plan(L, []) == 1                                    # NULL stages
+    assert plan(L, [stage()], sweep=False) == 1                # NULL descriptor
+    arr = (qg.CStage * 1)(stage())
+    out = qg.CSweep()
+    assert L.qg_sweep_plan(arr, 0, 0x10000, 1 << 20, ctypes.byref(out)) == 2
+    assert plan(L, [stage()], nbytes=64) == 5                  # workspace too small
+    assert plan(L, [stage()], ws=None) == 5
+    assert plan(L, [stage()], ws=0x10010) == 3                 # 256-byte alignment
+    assert plan(L, [stage(op=9)]) == 4                         # unknown op
+    assert plan(L, [stage(w=W(fmt=7))]) == 4
+    assert plan(L, [stage(x=None)]) == 1
+    assert plan(L, [stage(x=0x4008)]) == 3
+    assert plan(L, [stage(y=None)]) == 1                       # GEMV needs an output
+    assert plan(L, [stage(op=1, y=None)]) == 1                 # SwiGLU: no w_up
+    assert plan(L, [stage(op=1, w_up=W(fmt=1, k=128), y=None, h=0x6000)]) == 4
+    assert plan(L, [stage(op=1, w_up=W(n=16), y=None, h=0x6000)]) == 2
+    assert plan(L, [stage(op=1, w_up=W(), y=None)]) == 1       # SwiGLU needs h
+    assert plan(L, [stage(op=2, y=None)]) == 1                 # head needs idx
+    assert plan(L, [stage(op=2, y=None, idx=0x7002)]) == 3
+    # a bad stage anywhere fails the whole plan
+    assert plan(L, [stage(), stage(), stage(x=None)]) == 1
+    sw = qg.CSweep(1, 0)
+    assert L.qg_sweep_run(ctypes.byref(sw), None, None) == 1
+    assert L.qg_sweep_run(None, 0x10000, None) == 1
+    assert L.qg_sweep_run(ctypes.byref(qg.CSweep(0, 0)), 0x10000, None) == 2
+    assert L.qg_sweep_run(ctypes.byref(sw), 0x10010, None) == 3
