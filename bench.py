@@ -2,13 +2,14 @@
 """Benchmark the decode weight sweep through libqgemv.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl ours|reference] [--path auto|persistent|launches]
+                    [--impl ours|reference] [--path launches|persistent]
 
 A step is one full sweep of the decoder's weights (every layer's q|k|v, o,
 gate/up + SwiGLU and down, then the LM head + argmax) replayed from a CUDA
-graph.  At S=1 the sweep runs by default as one persistent launch
-(qg_sweep_run); `--path launches` times the same stages as one launch per
-call instead (S=16 always runs that way).  The default workload is the Qwen3-VL-2B-shaped int8 block-32 S=1
+graph, one launch per call (chained with programmatic dependent launch).
+`--path persistent` times the same S=1 stages as one persistent launch
+(qg_sweep_run) instead; on B200 its grid-wide barrier between stages costs
+more than the launch chaining it replaces, so it is not the default.  The default workload is the Qwen3-VL-2B-shaped int8 block-32 S=1
 sweep (1.83 GB per sweep, far larger than the 126 MB L2, so no flush is
 needed between steps).  N > 1 runs one replica per GPU (launch with torchrun):
 decode sweeps are independent, so nothing is exchanged and the time is the
@@ -60,8 +61,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--path", default="auto", choices=["auto", "persistent", "launches"],
-                    help="S=1 sweep as one persistent launch (auto) or one launch per call")
+    ap.add_argument("--path", default="launches", choices=["launches", "persistent"],
+                    help="S=1 sweep as one launch per call (default) or one persistent launch")
     ap.add_argument("--graph-sweeps", type=int, default=1,
                     help="sweeps captured per CUDA graph (steps are rounded up to a multiple)")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0,
@@ -317,7 +318,7 @@ def run_ours(a):
     dname, body_fmt, head_fmt, S = WORKLOADS[a.workload]
     dec = getattr(wl, dname)
     sw = DecodeSweep(dec, body_fmt, head_fmt, S=S, device=dev)
-    persistent = S == 1 and a.path != "launches"
+    persistent = a.path == "persistent"
     if a.path == "persistent" and S != 1:
         raise SystemExit("--path persistent needs an S=1 workload")
     G = max(1, a.graph_sweeps)

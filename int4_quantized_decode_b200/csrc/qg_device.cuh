@@ -140,16 +140,22 @@ __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
     return v;
 }
 
-// Wait until *counter >= target (a counter other CTAs of this grid increment
-// after a __threadfence).  Gives up after kWaitLimitCycles; returns whether
-// the target was reached.
+// Add 1 to a grid-wide counter with release semantics at GPU scope: after a
+// __syncthreads, what every thread of the CTA wrote before it is visible to a
+// thread that acquires the counter's new value.
+__device__ __forceinline__ void red_release_gpu_inc(unsigned int* counter) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(counter) : "memory");
+}
+
+// Wait until *counter >= target (a counter other CTAs of this grid raise with
+// red_release_gpu_inc).  Gives up after kWaitLimitCycles; returns whether the
+// target was reached.
 __device__ __forceinline__ bool wait_counter_bounded(const unsigned int* counter,
                                                      unsigned int target) {
     if (ld_acquire_gpu(counter) >= target) return true;
     const long long t0 = clock64();
     while (ld_acquire_gpu(counter) < target) {
         if (clock64() - t0 > kWaitLimitCycles) return false;
-        __nanosleep(64);
     }
     return true;
 }

@@ -74,6 +74,7 @@ struct Params {
     unsigned int* ws_ticket;
     int x_floats;        // floats reserved for x in shared memory
     int prefetch_items;  // items per warp prefetched into L2 before the wait
+    int x_bulk;          // ring path: x arrives by one bulk copy into a raw buffer
 };
 
 __host__ __device__ constexpr int align_up(int v, int a) { return (v + a - 1) / a * a; }
@@ -185,10 +186,11 @@ struct Frag {
 
 // ------------------------------------------------------ shared kernel parts --
 // Stage x (fp16 in global memory, written by the previous kernel or by an
-// earlier stage of the same sweep, hence read through L2) into shared memory
-// as fp32 in the conflict-free piece layout; int4 also gets the sum of x over
-// each 32-code lane granule and the pair-permuted order dot32_i4 uses.
-template <int FMT>
+// earlier stage of the same sweep, hence read through L2; or already copied
+// raw into shared memory, FROM_SMEM) into shared memory as fp32 in the
+// conflict-free piece layout; int4 also gets the sum of x over each 32-code
+// lane granule and the pair-permuted order dot32_i4 uses.
+template <int FMT, bool FROM_SMEM = false>
 __device__ __forceinline__ void stage_x(const uint16_t* __restrict__ x, float* xs, float* hsum,
                                         int granules) {
     using F = Fmt<FMT>;
@@ -198,7 +200,8 @@ __device__ __forceinline__ void stage_x(const uint16_t* __restrict__ x, float* x
         float gsum = 0.f;
 #pragma unroll
         for (int c = 0; c < F::kCodesPerLane / 8; ++c) {
-            const uint4 v = ldg_cg_v4(xg + 8 * c);
+            const uint4 v = FROM_SMEM ? *reinterpret_cast<const uint4*>(xg + 8 * c)
+                                      : ldg_cg_v4(xg + 8 * c);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
             float a[8];
 #pragma unroll
@@ -520,17 +523,20 @@ struct StreamSync {
 };
 
 struct GridSync {
-    unsigned int* prev;  // arrival counter of the previous stage, or nullptr
-    int* go;             // shared: the outcome of thread 0's wait
+    unsigned int* prev;        // arrival counter of the previous stage, or nullptr
+    int* go;                   // shared: the outcome of thread 0's wait
+    const uint4* next_src;     // the next stage's descriptor (global), or nullptr
+    uint4* next_dst;           // where the CTA keeps it (shared)
+    int next_pieces;           // its 16-byte pieces
     // (the sweep kernel has synchronized the CTA: every warp is done with the
     // previous stage's outputs, x and rings)
     __device__ __forceinline__ void before_prologue() {
-        if (prev && threadIdx.x == 0) {
-            __threadfence();
-            atomicAdd(prev, 1u);
-        }
+        if (prev && threadIdx.x == 0) red_release_gpu_inc(prev);
     }
     __device__ __forceinline__ bool wait_input() {
+        // the next stage's descriptor is fetched while the grid waits
+        if (next_src && static_cast<int>(threadIdx.x) < next_pieces)
+            next_dst[threadIdx.x] = ldg_nc_v4(next_src + threadIdx.x);
         if (threadIdx.x == 0)
             *go = (prev == nullptr || wait_counter_bounded(prev, gridDim.x)) ? 1 : 0;
         __syncthreads();
@@ -569,10 +575,21 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
     const int64_t side_per_row = K / F::kBlock;  // a multiple of 8 (16-byte pieces)
     const uint64_t pol = l2_policy_evict_first();
 
-    // shared memory: [rings of this CTA's warps][x fp32][hsum]
+    // shared memory: [rings of this CTA's warps][x fp32][hsum][x fp16 raw]
     const uint32_t ring = smem_u32(smem) + warp * (kRing * ROWS * RL::kPerRow);
     float* xs = reinterpret_cast<float*>(smem + ring_bytes(FMT, ROWS));
     float* hsum = xs + p.x_floats;
+    uint16_t* xraw = reinterpret_cast<uint16_t*>(hsum + (FMT == 1 ? granules : 0));
+    // x by bulk copy: one 1-D copy of k fp16 values, completing on xbar (its
+    // requests do not queue behind the ring's 16-byte copies)
+    __shared__ __align__(8) uint64_t xbar;
+    if (p.x_bulk) {
+        if (threadIdx.x == 0) {
+            mbar_init(&xbar, 1);
+            fence_mbar_init();
+        }
+        __syncthreads();
+    }
     auto slot_codes = [&](int s, int j) -> uint32_t {  // this lane's code vector
         return ring + (s * ROWS + j) * RL::kPerRow + lane * 16;
     };
@@ -647,7 +664,22 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
         cp_async_wait<0>();
         return false;
     }
-    stage_x<FMT>(p.x, xs, hsum, granules);
+    if (p.x_bulk) {
+        if (threadIdx.x == 0) {
+            const uint32_t bytes = static_cast<uint32_t>(K * 2);
+            mbar_arrive_expect_tx(&xbar, bytes);
+            bulk_g2s(xraw, p.x, bytes, &xbar, l2_policy_evict_last());
+        }
+        if (!mbar_wait_bounded(&xbar, 0)) {
+            if (threadIdx.x == 0) atomicOr(&g_gemv_err, kGemvErrTimeout);
+            mbar_wait_bounded(&xbar, 0);  // the copy may still land: wait again, bounded
+            cp_async_wait<0>();
+            return false;
+        }
+        stage_x<FMT, true>(xraw, xs, hsum, granules);
+    } else {
+        stage_x<FMT>(p.x, xs, hsum, granules);
+    }
     __syncthreads();
     sync.input_staged();
 
@@ -708,9 +740,12 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) 
     ring_stage<FMT, NMAT, RG, EPI>(p, smem, sync, red_v, red_i);
 }
 
+// x's shared memory: fp32 x, the int4 sums, and the raw fp16 copy if x
+// arrives by bulk copy.
 size_t x_smem_bytes(int fmt, const Params& p) {
     size_t b = static_cast<size_t>(p.x_floats) * 4;
     if (fmt == QG_FMT_I4_G64) b += static_cast<size_t>(p.k / Fmt<1>::kCodesPerLane) * 4;
+    if (p.x_bulk) b += static_cast<size_t>(p.k) * 2;
     return b;
 }
 
@@ -765,13 +800,21 @@ int pick_rg(int64_t n, int max_rg, int total_warps) {
 }
 
 template <int FMT, int NMAT, int RG, int EPI>
-qg_status launch_pick(const Params& p, const DeviceInfo& dev, cudaStream_t stream) {
+qg_status launch_pick(const Params& p0, const DeviceInfo& dev, cudaStream_t stream) {
     // The ring kernel copies side data (scales, biases) as 16-byte pieces of 8:
     // a row's count must be a multiple of 8; its ring must fit beside x in the
-    // per-CTA budget.
+    // per-CTA budget, with x's raw bulk-copy buffer if there is room for it.
+    Params p = p0;
     const bool even_sides = (p.k / Fmt<FMT>::kBlock) % 8 == 0;
-    const bool fits = x_smem_bytes(FMT, p) + ring_smem_bytes<FMT, NMAT, RG>() <= kSmemPerCtaBudget;
-    if (even_sides && fits) return launch_t<FMT, NMAT, RG, EPI, true>(p, dev, stream);
+    if (even_sides) {
+        p.x_bulk = 1;
+        if (x_smem_bytes(FMT, p) + ring_smem_bytes<FMT, NMAT, RG>() <= kSmemPerCtaBudget)
+            return launch_t<FMT, NMAT, RG, EPI, true>(p, dev, stream);
+        p.x_bulk = 0;
+        if (x_smem_bytes(FMT, p) + ring_smem_bytes<FMT, NMAT, RG>() <= kSmemPerCtaBudget)
+            return launch_t<FMT, NMAT, RG, EPI, true>(p, dev, stream);
+    }
+    p.x_bulk = 0;
     return launch_t<FMT, NMAT, RG, EPI, false>(p, dev, stream);
 }
 
@@ -822,7 +865,7 @@ static_assert(sizeof(SweepHeader) == 256, "header is 256 bytes");
 struct SweepStage {
     Params p;
     int32_t variant;
-    int32_t reserved;
+    int32_t reserved[3];
 };
 
 __host__ __device__ constexpr size_t align256(size_t v) { return (v + 255) / 256 * 256; }
@@ -841,16 +884,14 @@ __host__ __device__ constexpr size_t sweep_stages_offset(int n) {
 // (per item, not per step), as a launch of its own reads its constant bank.
 template <int FMT, int NMAT, int RG, int EPI>
 __device__ __forceinline__ bool sweep_stage(const SweepStage* st, unsigned char* smem,
-                                            unsigned int* prev, int* go, float* red_v, int* red_i) {
-    GridSync sync{prev, go};
+                                            GridSync& sync, float* red_v, int* red_i) {
     return ring_stage<FMT, NMAT, RG, EPI>(st->p, smem, sync, red_v, red_i);
 }
 
 template <int KERNEL>
 __device__ __forceinline__ bool sweep_dispatch(int v, const SweepStage* st, unsigned char* smem,
-                                               unsigned int* prev, int* go, float* red_v,
-                                               int* red_i) {
-#define QG_STAGE(F, M, R, E) return sweep_stage<F, M, R, E>(st, smem, prev, go, red_v, red_i)
+                                               GridSync& sync, float* red_v, int* red_i) {
+#define QG_STAGE(F, M, R, E) return sweep_stage<F, M, R, E>(st, smem, sync, red_v, red_i)
     if (KERNEL == 0) {
         switch (v) {
             case kVarPlain1: QG_STAGE(0, 1, 1, kEpiPlain);
@@ -886,7 +927,7 @@ __global__ void __launch_bounds__(kThreads, 2) sweep_kernel(unsigned char* ws, i
     __shared__ float red_v[kWarps];
     __shared__ int red_i[kWarps];
     __shared__ int go;
-    __shared__ __align__(16) SweepStage cur;
+    __shared__ __align__(16) SweepStage desc[2];  // this stage's and the next one's
     const SweepHeader* hdr = reinterpret_cast<const SweepHeader*>(ws);
     if (hdr->magic != kSweepMagic || hdr->n_stages != n_stages || hdr->kernel != KERNEL) {
         if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(&g_gemv_err, kGemvErrBadPlan);
@@ -896,14 +937,16 @@ __global__ void __launch_bounds__(kThreads, 2) sweep_kernel(unsigned char* ws, i
     const SweepStage* stages = reinterpret_cast<const SweepStage*>(ws + sweep_stages_offset(n_stages));
     static_assert(sizeof(SweepStage) % 16 == 0, "stage descriptors copy as 16-byte pieces");
     constexpr int kPieces = static_cast<int>(sizeof(SweepStage) / 16);
+    if (threadIdx.x < kPieces)
+        reinterpret_cast<uint4*>(&desc[0])[threadIdx.x] =
+            ldg_nc_v4(reinterpret_cast<const uint4*>(stages) + threadIdx.x);
     for (int s = 0; s < n_stages; ++s) {
-        __syncthreads();  // every warp is done with the previous stage
-        if (threadIdx.x < kPieces)
-            reinterpret_cast<uint4*>(&cur)[threadIdx.x] =
-                ldg_nc_v4(reinterpret_cast<const uint4*>(stages + s) + threadIdx.x);
-        __syncthreads();
-        unsigned int* prev = s > 0 ? ctr + (s - 1) : nullptr;
-        const bool ok = sweep_dispatch<KERNEL>(cur.variant, &cur, smem, prev, &go, red_v, red_i);
+        __syncthreads();  // every warp is done with the previous stage; desc[s & 1] is in
+        const SweepStage* cur = &desc[s & 1];
+        GridSync sync{s > 0 ? ctr + (s - 1) : nullptr, &go,
+                      s + 1 < n_stages ? reinterpret_cast<const uint4*>(stages + s + 1) : nullptr,
+                      reinterpret_cast<uint4*>(&desc[(s + 1) & 1]), kPieces};
+        const bool ok = sweep_dispatch<KERNEL>(cur->variant, cur, smem, sync, red_v, red_i);
         if (!ok) {
             if (threadIdx.x == 0) atomicOr(&g_gemv_err, kGemvErrTimeout);
             return;
@@ -913,7 +956,6 @@ __global__ void __launch_bounds__(kThreads, 2) sweep_kernel(unsigned char* ws, i
     // reads a counter after it has arrived here).
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
         if (atomicAdd(ctr + n_stages, 1u) == gridDim.x - 1) {
             for (int s = 0; s <= n_stages; ++s) ctr[s] = 0u;
             __threadfence();
@@ -951,7 +993,7 @@ Params make_params(const GemvLaunch& L) {
 // choice of rows per item, lowered to what the kernel holds and until the
 // stage's rings and x fit the per-CTA budget.  Returns -1 (with *status set)
 // if the kernel has no variant for the stage.
-int sweep_variant(int kernel, const GemvLaunch& L, const Params& p, int total_warps, int* rg_out,
+int sweep_variant(int kernel, const GemvLaunch& L, Params* p, int total_warps, int* rg_out,
                   qg_status* status) {
     const int block = L.fmt == QG_FMT_I8_B32 ? 32 : 64;
     *status = QG_ERR_SHAPE;
@@ -965,10 +1007,12 @@ int sweep_variant(int kernel, const GemvLaunch& L, const Params& p, int total_wa
         }
         if (!head) max_rg = swiglu ? 1 : 2;
     }
-    const size_t xb = x_smem_bytes(L.fmt, p);
     const int nmat = swiglu ? 2 : 1;
     for (int rg = pick_rg(L.n, max_rg, total_warps); rg >= 1; rg /= 2) {
-        if (xb + ring_bytes(L.fmt, nmat * rg) > kSmemPerCtaBudget) continue;
+        p->x_bulk = 1;  // x by bulk copy if its raw buffer fits too
+        if (x_smem_bytes(L.fmt, *p) + ring_bytes(L.fmt, nmat * rg) > kSmemPerCtaBudget)
+            p->x_bulk = 0;
+        if (x_smem_bytes(L.fmt, *p) + ring_bytes(L.fmt, nmat * rg) > kSmemPerCtaBudget) continue;
         *rg_out = rg;
         *status = QG_OK;
         if (kernel == 0) {
@@ -1012,7 +1056,7 @@ qg_status plan_sweep(const GemvLaunch* L, int n_stages, void* ws, size_t ws_byte
         if (Li.epilogue == kEpiHead) Li.workspace = dev_base + sweep_scratch_offset(n_stages) + 16 * i;
         Params p = make_params(Li);
         int rg = 1;
-        const int v = sweep_variant(kernel, Li, p, total_warps, &rg, &st);
+        const int v = sweep_variant(kernel, Li, &p, total_warps, &rg, &st);
         if (v < 0) return st;
         const int nmat = Li.epilogue == kEpiSwiglu ? 2 : 1;
         const int64_t item_bytes = static_cast<int64_t>(nmat) * rg * (Li.fmt == 0 ? Li.k : Li.k / 2);
