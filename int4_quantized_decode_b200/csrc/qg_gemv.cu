@@ -14,16 +14,17 @@
 //    (On this GPU a plain 16-byte load stream reaches ~7.3 TB/s, while 1-D
 //    bulk copies need >= 16 KB per copy to get there: every bulk copy carries
 //    a fixed cost, and rows of 2-6 KB would pay it too often.)
-//  * x (fp16) is staged once per CTA into shared memory as fp32, in a layout
-//    where each 8-lane phase of a 16-byte read hits distinct banks; one x read
-//    serves all RG rows of the warp.
-//  * Dequantization happens in registers with no int->float conversion
-//    instruction: int8 codes are byte-permuted into the mantissa of 2^23 and
-//    the offset subtracted; int4 nibbles are masked in place into that
-//    mantissa.  Products accumulate in fp32 with the packed sm_100 f32x2 FMA;
-//    each block's fp16 scale is applied once per 16 (int8) or 32 (int4)
-//    codes; the int4 bias uses sum_k (q s + b) x = s sum q x + b sum x with the
-//    per-half-group sums of x computed once per CTA.
+//  * x (fp16) is staged once per CTA into shared memory, still fp16, in a
+//    layout where each 8-lane phase of a 16-byte read hits distinct banks,
+//    with a few sums of x per lane granule; one x read serves all RG rows.
+//  * Dequantization needs no int->float conversion: one byte permute (int8,
+//    two codes) or one mask-and-or (int4, two codes) builds a pair of fp16
+//    values 1024 + u, exact, and the sm_100 mixed-precision FMA
+//    (fma.rn.f32.f16) multiplies it by the fp16 x pair into an fp32
+//    accumulator, exactly.  The constant 1024 (+128 for int8's offset
+//    binary) comes out as a per-granule term 1024 sum x precomputed at
+//    staging.  Each block's fp16 scale is applied once per 16 (int8) or 32
+//    (int4) codes; the int4 bias uses sum_k (q s + b) x = s sum q x + b sum x.
 //  * Lanes split K within a row; a warp-shuffle reduction finishes each row.
 //  * Programmatic dependent launch: before waiting on the previous kernel in
 //    the stream, every warp asks L2 to prefetch (cp.async.bulk.prefetch.L2) the
@@ -55,7 +56,8 @@ template <int FMT>
 struct Fmt {
     static constexpr int kCodesPerLane = FMT == 0 ? 16 : 32;   // one 16-byte vector
     static constexpr int kBlock = FMT == 0 ? 32 : 64;
-    static constexpr int kPieces = kCodesPerLane / 4;           // float4 pieces of x per lane
+    static constexpr int kPieces = kCodesPerLane / 8;           // 16-byte fp16 x pieces per lane
+    static constexpr int kSums = FMT == 0 ? 1 : 2;              // floats of x sums per granule
     static constexpr bool kBias = FMT == 1;
 };
 
@@ -72,7 +74,7 @@ struct Params {
     int32_t* idx;
     unsigned long long* ws_key;
     unsigned int* ws_ticket;
-    int x_floats;        // floats reserved for x in shared memory
+    int x_words;         // 4-byte words reserved for the staged fp16 x in shared memory
     int prefetch_items;  // items per warp prefetched into L2 before the wait
     int x_bulk;          // ring path: x arrives by one bulk copy into a raw buffer
 };
@@ -103,58 +105,58 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
 }
 
 // ------------------------------------------------------------ dot products --
-// 16 int8 codes (one 16-byte vector) against 16 fp32 activations.
-__device__ __forceinline__ float dot16_i8(const uint4 c, const float4* xv) {
-    const float2 off = make_float2(-8388736.0f, -8388736.0f);  // -(2^23 + 128)
-    float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+// acc_a += lo(q2) * lo(x2), acc_b += hi(q2) * hi(x2): fp16 x fp16 -> fp32,
+// one rounding (the products of 11-bit significands are exact in fp32).
+__device__ __forceinline__ void fma_f16x2_f32(float& acc_a, float& acc_b, uint32_t q2,
+                                              uint32_t x2) {
+    asm("{\n\t.reg .f16 q0, q1, x0, x1;\n\t"
+        "mov.b32 {q0, q1}, %2;\n\t"
+        "mov.b32 {x0, x1}, %3;\n\t"
+        "fma.rn.f32.f16 %0, q0, x0, %0;\n\t"
+        "fma.rn.f32.f16 %1, q1, x1, %1;\n\t}"
+        : "+f"(acc_a), "+f"(acc_b)
+        : "r"(q2), "r"(x2));
+}
+
+// 16 int8 codes (one 16-byte vector) against their 16 fp16 x (two pieces, in
+// k order): returns sum_k (1152 + q_k) x_k.  The code byte q (two's
+// complement) is turned into offset binary u = q + 128 and permuted under
+// 0x64, the fp16 encoding of 1024 + u (exact for u < 1024).
+__device__ __forceinline__ float dot16_i8(const uint4 c, const uint4* xv) {
+    float a0 = 0.f, a1 = 0.f;
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    const uint32_t x[8] = {xv[0].x, xv[0].y, xv[0].z, xv[0].w,
+                           xv[1].x, xv[1].y, xv[1].z, xv[1].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t u = w[i] ^ 0x80808080u;
+        fma_f16x2_f32(a0, a1, __byte_perm(u, 0x64646464u, 0x4140), x[2 * i]);
+        fma_f16x2_f32(a0, a1, __byte_perm(u, 0x64646464u, 0x4342), x[2 * i + 1]);
+    }
+    return a0 + a1;
+}
+
+// 32 int4 codes (one 16-byte vector, even k in the low nibble) against their
+// 32 fp16 x, staged per 8-code word as the pairs (x0,x4) (x1,x5) (x2,x6)
+// (x3,x7).  One mask-and-or per pair puts nibbles 0/4 and 2/6 (after a shift
+// by 8) in the low bits of the fp16 mantissa (1024 + q) and nibbles 1/5 and
+// 3/7 four bits higher (1024 + 16 q).  Returns
+//   sum_even (1024 + q) x + sum_odd (1024 + 16 q) x / 16.
+__device__ __forceinline__ float dot32_i4(const uint4 c, const uint4* xv) {
+    float l0 = 0.f, l1 = 0.f, h0 = 0.f, h1 = 0.f;
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t u = w[i] ^ 0x80808080u;  // two's complement -> q + 128
-        const float f0 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7440));
-        const float f1 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7441));
-        const float f2 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7442));
-        const float f3 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7443));
-        const float2 q01 = __fadd2_rn(make_float2(f0, f1), off);  // exact q
-        const float2 q23 = __fadd2_rn(make_float2(f2, f3), off);
-        a0 = __ffma2_rn(q01, make_float2(xv[i].x, xv[i].y), a0);
-        a1 = __ffma2_rn(q23, make_float2(xv[i].z, xv[i].w), a1);
+        const uint32_t v = w[i], v8 = v >> 8;
+        fma_f16x2_f32(l0, l1, (v & 0x000F000Fu) | 0x64006400u, xv[i].x);
+        fma_f16x2_f32(h0, h1, (v & 0x00F000F0u) | 0x64006400u, xv[i].y);
+        fma_f16x2_f32(l0, l1, (v8 & 0x000F000Fu) | 0x64006400u, xv[i].z);
+        fma_f16x2_f32(h0, h1, (v8 & 0x00F000F0u) | 0x64006400u, xv[i].w);
     }
-    return (a0.x + a0.y) + (a1.x + a1.y);
+    return (l0 + l1) + (h0 + h1) * 0.0625f;
 }
 
-// 32 int4 codes (one 16-byte vector) against 32 activations that the staging
-// step stored per 8-code word as (x0, x5, x1, x6, x2, x7, x3, x4/16): nibble j
-// is masked in place into the mantissa of 2^23, giving 2^23 + n_j 16^e_j, and
-// the accumulators are kept per power of 16 and rescaled exactly at the end.
-__device__ __forceinline__ float dot32_i4(const uint4 c, const float4* xv) {
-    const float2 off = make_float2(-8388608.0f, -8388608.0f);  // -2^23
-    const uint32_t M = 0x4B000000u;
-    float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
-    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t v = w[i];
-        const uint32_t s = v >> 20;
-        const float n0 = __uint_as_float((v & 0x0000000Fu) | M);   // n0
-        const float n1 = __uint_as_float((v & 0x000000F0u) | M);   // 16 n1
-        const float n2 = __uint_as_float((v & 0x00000F00u) | M);   // 256 n2
-        const float n3 = __uint_as_float((v & 0x0000F000u) | M);   // 4096 n3
-        const float n4 = __uint_as_float((v & 0x000F0000u) | M);   // 65536 n4
-        const float n5 = __uint_as_float((s & 0x0000000Fu) | M);   // n5
-        const float n6 = __uint_as_float((s & 0x000000F0u) | M);   // 16 n6
-        const float n7 = __uint_as_float((s & 0x00000F00u) | M);   // 256 n7
-        const float4 xa = xv[2 * i], xb = xv[2 * i + 1];
-        a0 = __ffma2_rn(__fadd2_rn(make_float2(n0, n5), off), make_float2(xa.x, xa.y), a0);
-        a1 = __ffma2_rn(__fadd2_rn(make_float2(n1, n6), off), make_float2(xa.z, xa.w), a1);
-        a2 = __ffma2_rn(__fadd2_rn(make_float2(n2, n7), off), make_float2(xb.x, xb.y), a2);
-        a3 = __ffma2_rn(__fadd2_rn(make_float2(n3, n4), off), make_float2(xb.z, xb.w), a3);
-    }
-    return ((a0.x + a0.y) + (a1.x + a1.y) * 0.0625f) +
-           ((a2.x + a2.y) * 0.00390625f + (a3.x + a3.y) * 0.000244140625f);
-}
-
-// float4 index of piece `i` of lane-granule `g` in the staged x: the eight
+// 16-byte index of piece `i` of lane-granule `g` in the staged x: the eight
 // granules read by one 8-lane phase of a 16-byte shared load are adjacent.
 template <int FMT>
 __device__ __forceinline__ int x_piece(int g, int i) {
@@ -187,40 +189,43 @@ struct Frag {
 // ------------------------------------------------------ shared kernel parts --
 // Stage x (fp16 in global memory, written by the previous kernel or by an
 // earlier stage of the same sweep, hence read through L2; or already copied
-// raw into shared memory, FROM_SMEM) into shared memory as fp32 in the
-// conflict-free piece layout; int4 also gets the sum of x over each 32-code
-// lane granule and the pair-permuted order dot32_i4 uses.
+// raw into shared memory, FROM_SMEM) into shared memory, still fp16, in the
+// conflict-free piece layout (int4: each 8-code word as the pairs the dot
+// product wants), and per lane granule the sums that remove the dot
+// products' constant terms:
+//   int8: sums[g] = 1152 sum x;
+//   int4: sums[2g] = 1024 sum_even x + 64 sum_odd x, sums[2g+1] = sum x.
 template <int FMT, bool FROM_SMEM = false>
-__device__ __forceinline__ void stage_x(const uint16_t* __restrict__ x, float* xs, float* hsum,
+__device__ __forceinline__ void stage_x(const uint16_t* __restrict__ x, uint4* xs, float* sums,
                                         int granules) {
     using F = Fmt<FMT>;
-    float4* xs4 = reinterpret_cast<float4*>(xs);
     for (int g = threadIdx.x; g < granules; g += blockDim.x) {
         const uint16_t* xg = x + static_cast<int64_t>(g) * F::kCodesPerLane;
-        float gsum = 0.f;
+        float se = 0.f, so = 0.f;  // sums over even and odd k
 #pragma unroll
-        for (int c = 0; c < F::kCodesPerLane / 8; ++c) {
+        for (int c = 0; c < F::kPieces; ++c) {
             const uint4 v = FROM_SMEM ? *reinterpret_cast<const uint4*>(xg + 8 * c)
                                       : ldg_cg_v4(xg + 8 * c);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            float a[8];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                a[2 * e] = h2f(static_cast<uint16_t>(w[e] & 0xFFFFu));
-                a[2 * e + 1] = h2f(static_cast<uint16_t>(w[e] >> 16));
+                se += h2f(static_cast<uint16_t>(w[e] & 0xFFFFu));
+                so += h2f(static_cast<uint16_t>(w[e] >> 16));
             }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) gsum += a[e];
             if (FMT == 0) {
-                xs4[x_piece<FMT>(g, 2 * c)] = make_float4(a[0], a[1], a[2], a[3]);
-                xs4[x_piece<FMT>(g, 2 * c + 1)] = make_float4(a[4], a[5], a[6], a[7]);
-            } else {
-                // one 8-code word: (x0, x5, x1, x6) (x2, x7, x3, x4/16)
-                xs4[x_piece<FMT>(g, 2 * c)] = make_float4(a[0], a[5], a[1], a[6]);
-                xs4[x_piece<FMT>(g, 2 * c + 1)] = make_float4(a[2], a[7], a[3], a[4] * 0.0625f);
+                xs[x_piece<FMT>(g, c)] = v;
+            } else {  // (x0,x1)(x2,x3)(x4,x5)(x6,x7) -> (x0,x4)(x1,x5)(x2,x6)(x3,x7)
+                xs[x_piece<FMT>(g, c)] =
+                    make_uint4(__byte_perm(w[0], w[2], 0x5410), __byte_perm(w[0], w[2], 0x7632),
+                               __byte_perm(w[1], w[3], 0x5410), __byte_perm(w[1], w[3], 0x7632));
             }
         }
-        if (FMT == 1) hsum[g] = gsum;
+        if (FMT == 0) {
+            sums[g] = 1152.0f * (se + so);
+        } else {
+            sums[2 * g] = 1024.0f * se + 64.0f * so;
+            sums[2 * g + 1] = se + so;
+        }
     }
 }
 
@@ -338,8 +343,8 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
     constexpr int kStepBytes = kLanes * 16;  // code bytes of one warp step along a row
     constexpr int kStepSides = kStepBytes * (FMT == 0 ? 1 : 2) / F::kBlock;  // scales per step
     extern __shared__ __align__(128) unsigned char smem[];
-    float* xs = reinterpret_cast<float*>(smem);
-    float* hsum = xs + p.x_floats;
+    uint4* xs = reinterpret_cast<uint4*>(smem);
+    float* sums = reinterpret_cast<float*>(smem) + p.x_words;
     __shared__ float red_v[kWarps];
     __shared__ int red_i[kWarps];
 
@@ -410,12 +415,11 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
 
     // 2) x from the previous kernel
     griddep_wait();
-    stage_x<FMT>(p.x, xs, hsum, granules);
+    stage_x<FMT>(p.x, xs, sums, granules);
     __syncthreads();
     griddep_launch_dependents();
 
     // 3) stream
-    const float4* xs4 = reinterpret_cast<const float4*>(xs);
     const int x_lane = ((lane >> 3) * F::kPieces) * 8 + (lane & 7);  // x_piece(lane, 0)
     constexpr int kXStep = 4 * F::kPieces * 8;                      // per 32 granules
     float acc[ROWS];
@@ -427,17 +431,19 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
     auto consume = [&](const Frag<ROWS>& f) {
         const int g = cu_st * kLanes + lane;
         if (g < granules) {
-            float4 xv[F::kPieces];
-            const float4* xp = xs4 + x_lane + cu_st * kXStep;
+            uint4 xv[F::kPieces];
+            const uint4* xp = xs + x_lane + cu_st * kXStep;
 #pragma unroll
             for (int i = 0; i < F::kPieces; ++i) xv[i] = xp[i * 8];
-            const float hs = FMT == 1 ? hsum[g] : 0.f;
+            const float c0 = sums[F::kSums * g];
+            const float c1 = FMT == 1 ? sums[2 * g + 1] : 0.f;
 #pragma unroll
             for (int j = 0; j < ROWS; ++j) {
                 if (FMT == 0)
-                    acc[j] = fmaf(h2f(f.s[j]), dot16_i8(f.c[j], xv), acc[j]);
+                    acc[j] = fmaf(h2f(f.s[j]), dot16_i8(f.c[j], xv) - c0, acc[j]);
                 else
-                    acc[j] = fmaf(h2f(f.s[j]), dot32_i4(f.c[j], xv), fmaf(h2f(f.b[j]), hs, acc[j]));
+                    acc[j] = fmaf(h2f(f.s[j]), dot32_i4(f.c[j], xv) - c0,
+                                  fmaf(h2f(f.b[j]), c1, acc[j]));
             }
         }
         if (++cu_st == nst) {
@@ -575,11 +581,11 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
     const int64_t side_per_row = K / F::kBlock;  // a multiple of 8 (16-byte pieces)
     const uint64_t pol = l2_policy_evict_first();
 
-    // shared memory: [rings of this CTA's warps][x fp32][hsum][x fp16 raw]
+    // shared memory: [rings of this CTA's warps][x fp16][x sums][x fp16 raw]
     const uint32_t ring = smem_u32(smem) + warp * (kRing * ROWS * RL::kPerRow);
-    float* xs = reinterpret_cast<float*>(smem + ring_bytes(FMT, ROWS));
-    float* hsum = xs + p.x_floats;
-    uint16_t* xraw = reinterpret_cast<uint16_t*>(hsum + (FMT == 1 ? granules : 0));
+    uint4* xs = reinterpret_cast<uint4*>(smem + ring_bytes(FMT, ROWS));
+    float* sums = reinterpret_cast<float*>(xs) + p.x_words;
+    uint16_t* xraw = reinterpret_cast<uint16_t*>(sums + align_up(F::kSums * granules, 4));
     // x by bulk copy: one 1-D copy of k fp16 values, completing on xbar (its
     // requests do not queue behind the ring's 16-byte copies)
     __shared__ __align__(8) uint64_t xbar;
@@ -676,17 +682,16 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
             cp_async_wait<0>();
             return false;
         }
-        stage_x<FMT, true>(xraw, xs, hsum, granules);
+        stage_x<FMT, true>(xraw, xs, sums, granules);
     } else {
-        stage_x<FMT>(p.x, xs, hsum, granules);
+        stage_x<FMT>(p.x, xs, sums, granules);
     }
     __syncthreads();
     sync.input_staged();
 
     // 3) stream: issue step t + kRing - 1, wait for step t, compute it
-    const float4* xs4 = reinterpret_cast<const float4*>(xs);
-    const int x_lane = ((lane >> 3) * F::kPieces) * 8 + (lane & 7);
-    constexpr int kXStep = 4 * F::kPieces * 8;
+    const int x_lane = ((lane >> 3) * F::kPieces) * 8 + (lane & 7);  // x_piece(lane, 0)
+    constexpr int kXStep = 4 * F::kPieces * 8;                      // per 32 granules
     const int side_off = (lane >> 1) * 2;  // this lane's scale (bias) inside the step's 16
     float acc[ROWS];
 #pragma unroll
@@ -701,20 +706,21 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
         __syncwarp();  // side pieces copied by other lanes are now visible
         const int g = cu_st * kLanes + lane;
         if (g < granules) {
-            float4 xv[F::kPieces];
-            const float4* xp = xs4 + x_lane + cu_st * kXStep;
+            uint4 xv[F::kPieces];
+            const uint4* xp = xs + x_lane + cu_st * kXStep;
 #pragma unroll
             for (int i = 0; i < F::kPieces; ++i) xv[i] = xp[i * 8];
-            const float hs = FMT == 1 ? hsum[g] : 0.f;
+            const float c0 = sums[F::kSums * g];
+            const float c1 = FMT == 1 ? sums[2 * g + 1] : 0.f;
 #pragma unroll
             for (int j = 0; j < ROWS; ++j) {
                 const uint4 c = lds128(slot_codes(cu_slot, j));
                 const float sc = h2f(lds16(slot_side(cu_slot, j, 0) + side_off));
                 if (FMT == 0) {
-                    acc[j] = fmaf(sc, dot16_i8(c, xv), acc[j]);
+                    acc[j] = fmaf(sc, dot16_i8(c, xv) - c0, acc[j]);
                 } else {
                     const float bi = h2f(lds16(slot_side(cu_slot, j, 1) + side_off));
-                    acc[j] = fmaf(sc, dot32_i4(c, xv), fmaf(bi, hs, acc[j]));
+                    acc[j] = fmaf(sc, dot32_i4(c, xv) - c0, fmaf(bi, c1, acc[j]));
                 }
             }
         }
@@ -740,11 +746,13 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) 
     ring_stage<FMT, NMAT, RG, EPI>(p, smem, sync, red_v, red_i);
 }
 
-// x's shared memory: fp32 x, the int4 sums, and the raw fp16 copy if x
-// arrives by bulk copy.
+// x's shared memory: the staged fp16 x, its per-granule sums, and the raw
+// fp16 copy if x arrives by bulk copy.
 size_t x_smem_bytes(int fmt, const Params& p) {
-    size_t b = static_cast<size_t>(p.x_floats) * 4;
-    if (fmt == QG_FMT_I4_G64) b += static_cast<size_t>(p.k / Fmt<1>::kCodesPerLane) * 4;
+    const int granules = static_cast<int>(
+        p.k / (fmt == QG_FMT_I8_B32 ? Fmt<0>::kCodesPerLane : Fmt<1>::kCodesPerLane));
+    const int nsums = (fmt == QG_FMT_I8_B32 ? Fmt<0>::kSums : Fmt<1>::kSums) * granules;
+    size_t b = static_cast<size_t>(p.x_words) * 4 + static_cast<size_t>(align_up(nsums, 4)) * 4;
     if (p.x_bulk) b += static_cast<size_t>(p.k) * 2;
     return b;
 }
@@ -985,7 +993,7 @@ Params make_params(const GemvLaunch& L) {
                       : nullptr;
     const int cpl = L.fmt == QG_FMT_I8_B32 ? Fmt<0>::kCodesPerLane : Fmt<1>::kCodesPerLane;
     const int granules = static_cast<int>(L.k / cpl);
-    p.x_floats = align_up(granules, 8) * cpl;
+    p.x_words = align_up(granules, 8) * cpl / 2;  // fp16 x, padded to whole 8-granule phases
     return p;
 }
 
