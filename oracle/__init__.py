@@ -27,6 +27,7 @@ GCC_FLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
 
 FMT_I8_B32 = 0
 FMT_I4_G64 = 1
+FMT_F16 = 2  # plain fp16 weights (the tied fp16 head of the int8lin bundle)
 
 
 def build(force: bool = False) -> str:
@@ -171,9 +172,17 @@ def matvec(fmt: int, codes, scales, biases, x_bits):
     """fp64 dequantize-then-matvec: returns (y [n], mag [n]) with
     y[r] = sum_k w_dq[r,k] x[k] and mag[r] = sum_k |w_dq[r,k] x[k]|."""
     codes = np.ascontiguousarray(codes)
-    scales = np.ascontiguousarray(scales, dtype=np.uint16)
     x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
     n = codes.shape[0]
+    if fmt == FMT_F16:  # plain fp16 weights: codes are the fp16 bits [n, k]
+        assert codes.dtype == np.uint16
+        k = codes.shape[1]
+        assert x_bits.shape == (k,)
+        y = np.empty(n, dtype=np.float64)
+        mag = np.empty(n, dtype=np.float64)
+        lib().orc_matvec(fmt, _p(codes), None, None, n, k, _p(x_bits), _p(y), _p(mag))
+        return y, mag
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
     if fmt == FMT_I8_B32:
         assert codes.dtype == np.int8
         k = codes.shape[1]

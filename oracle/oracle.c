@@ -199,11 +199,11 @@ void orc_matvec(int fmt, const void* codes, const uint16_t* scales,
     double* xd = (double*)malloc(sizeof(double) * (size_t)k);
     for (int64_t j = 0; j < k; ++j) xd[j] = orc_f16_to_f64(x[j]);
     const int64_t blk = fmt == 0 ? 32 : 64;
-    const int64_t nb = k / blk;
+    const int64_t nb = fmt == 2 ? 0 : k / blk;
 #pragma omp parallel
     {
-        double* sd = (double*)malloc(sizeof(double) * (size_t)nb);
-        double* bd = (double*)malloc(sizeof(double) * (size_t)nb);
+        double* sd = (double*)malloc(sizeof(double) * (size_t)(nb > 0 ? nb : 1));
+        double* bd = (double*)malloc(sizeof(double) * (size_t)(nb > 0 ? nb : 1));
 #pragma omp for schedule(static)
         for (int64_t r = 0; r < n; ++r) {
             for (int64_t b = 0; b < nb; ++b) {
@@ -213,7 +213,10 @@ void orc_matvec(int fmt, const void* codes, const uint16_t* scales,
             double acc = 0.0, am = 0.0;
             for (int64_t j = 0; j < k; ++j) {
                 double wdq;
-                if (fmt == 0) {
+                if (fmt == 2) {
+                    const uint16_t* c = (const uint16_t*)codes;
+                    wdq = orc_f16_to_f64(c[r * k + j]);
+                } else if (fmt == 0) {
                     const int8_t* c = (const int8_t*)codes;
                     wdq = (double)c[r * k + j] * sd[j / 32];
                 } else {

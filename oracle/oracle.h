@@ -71,7 +71,11 @@ void orc_dequant_row_i4(const uint8_t* codes, const uint16_t* scales,
  *   y[r]   = sum_k w_dq[r,k] * x[k]       (index order, fp64)
  *   mag[r] = sum_k |w_dq[r,k] * x[k]|     (for the error bound)
  * x is fp16 bits [k].  fmt: 0 = int8 block-32, 1 = int4 group-64
- * (biases ignored for fmt 0).  Either output may be NULL. */
+ * (biases ignored for fmt 0), 2 = plain fp16 weights (codes are fp16 bits
+ * [n,k], w_dq is their exact value; scales and biases ignored): the tied
+ * fp16 head of the pages' "int8lin" bundle ("Qwen3-VL (2B / 4B / 8B) --
+ * Core AI", Measured table: 2B int8lin with a tied fp16 head, 2.0 GB).
+ * Either output may be NULL. */
 void orc_matvec(int fmt, const void* codes, const uint16_t* scales,
                 const uint16_t* biases, int64_t n, int64_t k,
                 const uint16_t* x, double* y, double* mag);

@@ -300,6 +300,36 @@ def test_tied_head_is_embedding_times_x():
     np.testing.assert_allclose(logits, ref, rtol=1e-12, atol=1e-15)
 
 
+def test_matvec_fp16_weights_tied_head():
+    """Plain fp16 weights (the int8lin bundle's tied fp16 head): w_dq is the
+    fp16 value itself.  Exact rational sums, the ones / one-hot closed forms,
+    and logits = x E^T against numpy's own fp16 decode on a non-square table."""
+    rng = np.random.default_rng(31)
+    V, H = 72, 160
+    E = np_f16_bits(rng.normal(0, 0.02, (V, H)))
+    ef = f16_np(E)
+    xb = np_f16_bits(rng.normal(0, 1, H))
+    xs = f16_np(xb)
+    y, mag = oracle.matvec(oracle.FMT_F16, E, None, None, xb)
+    np.testing.assert_allclose(y, ef.astype(np.float64) @ xs.astype(np.float64),
+                               rtol=1e-12, atol=1e-15)
+    for r in (0, 37, V - 1):
+        exact = sum(Fraction(float(ef[r, j])) * Fraction(float(xs[j])) for j in range(H))
+        exact_mag = sum(abs(Fraction(float(ef[r, j])) * Fraction(float(xs[j]))) for j in range(H))
+        assert abs(Fraction(float(y[r])) - exact) <= Fraction(H) * Fraction(2) ** -53 * exact_mag
+        assert abs(Fraction(float(mag[r])) - exact_mag) <= Fraction(H) * Fraction(2) ** -53 * exact_mag
+    ones = np.full(H, 0x3C00, dtype=np.uint16)
+    y1, _ = oracle.matvec(oracle.FMT_F16, E, None, None, ones)
+    for r in range(V):
+        assert abs(Fraction(float(y1[r])) - sum(Fraction(float(v)) for v in ef[r])) <= \
+            Fraction(H) * Fraction(2) ** -53 * sum(abs(Fraction(float(v))) for v in ef[r])
+    for j in (0, 1, 77, H - 1):
+        e = np.zeros(H, dtype=np.uint16)
+        e[j] = 0x3C00
+        yj, _ = oracle.matvec(oracle.FMT_F16, E, None, None, e)
+        assert np.array_equal(yj, ef[:, j].astype(np.float64))
+
+
 # --------------------------------------------------------- SwiGLU ---------
 
 def test_silu_and_grad():
