@@ -44,6 +44,7 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 # name -> (decoder, body format, head format, S)
 WORKLOADS = {
     "qwen3vl-2b": ("QWEN3VL_2B", 0, 0, 1),
+    "qwen3vl-2b-f16head": ("QWEN3VL_2B", 0, 2, 1),
     "qwen3vl-4b": ("QWEN3VL_4B", 0, 0, 1),
     "qwen3vl-4b-int4": ("QWEN3VL_4B", 1, 0, 1),
     "qwen3vl-8b": ("QWEN3VL_8B", 0, 0, 1),
@@ -51,7 +52,7 @@ WORKLOADS = {
     "dense-27b": ("DENSE_27B", 0, 0, 1),
 }
 DEFAULT_WORKLOAD = "qwen3vl-2b"
-FMT_NAME = {0: "int8 block-32", 1: "int4 group-64"}
+FMT_NAME = {0: "int8 block-32", 1: "int4 group-64", 2: "fp16"}
 
 
 def parse_args(argv=None):
@@ -274,7 +275,7 @@ def run_reference(a):
 
 
 def _sweep_bytes(dec, body_fmt, head_fmt):
-    bpw = {0: 1.0625, 1: 0.5625}
+    bpw = {0: 1.0625, 1: 0.5625, 2: 2.0}
     return int(dec.weight_count(include_head=False) * bpw[body_fmt] +
                dec.vocab * dec.hidden * bpw[head_fmt])
 

@@ -63,15 +63,23 @@ typedef enum {
     QG_FMT_I8_B32 = 0,
     /* int4 codes (two per byte, even k in the low nibble), one fp16 scale and
      * one fp16 bias per 64 consecutive k:  w ~= q * s + b */
-    QG_FMT_I4_G64 = 1
+    QG_FMT_I4_G64 = 1,
+    /* plain fp16 weights, no scales: the tied fp16 LM head of the pages'
+     * "int8lin" bundle ("Qwen3-VL (2B / 4B / 8B, vision-language) -- Core AI",
+     * Measured table: 2B int8lin, tied fp16 head, 2.0 GB), where the head is
+     * the fp16 embedding table itself.  Accepted by qg_gemv_s1 (and
+     * qg_gemm_s16 with S == 1) and qg_head_argmax; QG_ERR_FORMAT elsewhere. */
+    QG_FMT_F16 = 2
 } qg_format;
 
 /* A quantized weight matrix [n, k].
  *   fmt    : a qg_format value.
- *   codes  : QG_FMT_I8_B32: int8 [n, k]; QG_FMT_I4_G64: uint8 [n, k/2].
- *            16-byte aligned.  k % 32 == 0 (int8) or k % 64 == 0 (int4).
- *   scales : fp16 [n, k/32] (int8) or [n, k/64] (int4); 16-byte aligned.
- *   biases : fp16 [n, k/64] for int4, 16-byte aligned; ignored for int8. */
+ *   codes  : QG_FMT_I8_B32: int8 [n, k]; QG_FMT_I4_G64: uint8 [n, k/2];
+ *            QG_FMT_F16: fp16 [n, k].  16-byte aligned.  k % 32 == 0
+ *            (int8), k % 64 == 0 (int4) or k % 8 == 0 (fp16).
+ *   scales : fp16 [n, k/32] (int8) or [n, k/64] (int4); 16-byte aligned;
+ *            ignored for fp16 weights.
+ *   biases : fp16 [n, k/64] for int4, 16-byte aligned; ignored otherwise. */
 typedef struct {
     int32_t fmt;
     int32_t reserved;
@@ -120,7 +128,7 @@ QG_API qg_status qg_quantize_int4_g64(const float* w, int64_t n, int64_t k,
  * qg_gemv_s1 -- one-token (S=1) quantized GEMV, the decode weight stream
  * ("Qwen3-VL 4B -- Core AI (.aimodel)", Measured: decode is bandwidth-bound).
  *   y[r] = sum_k w_dq[r, k] * x[k]     (fp32 accumulation)
- * W   : the weight (int8 block-32 or int4 group-64).
+ * W   : the weight (int8 block-32, int4 group-64 or plain fp16).
  * x   : fp16 [k], 16-byte aligned.
  * y   : fp32 [n] out (4-byte aligned), or NULL.
  * y16 : fp16 [n] out = fp16_rne(y) (2-byte aligned), or NULL.
@@ -165,7 +173,8 @@ QG_API qg_status qg_gate_up_swiglu(const qg_weight* Wg, const qg_weight* Wu,
  * ("Qwen3.8-27B ... -- Core AI", Verified: absmax int8 head, greedy
  * teacher-forced argmax).
  *   logits[v] = sum_k w_dq[v, k] x[k];   idx = the smallest v of the max
- * W         : the head weight [vocab, hidden] (int8 or int4).
+ * W         : the head weight [vocab, hidden] (int8, int4, or the tied fp16
+ *             embedding table itself).
  * x         : fp16 [k], 16-byte aligned.
  * logits    : fp32 [n] out (4-byte aligned) or NULL.
  * idx       : int32 [1] out, device memory.
@@ -238,7 +247,8 @@ QG_API qg_status qg_head_argmax_noalloc(const qg_weight* W, const uint16_t* x, f
  *
  * Formats: a plan is either all int8, or the int4 run's layout -- every
  *   GEMV and SwiGLU stage int4 and every head int8 (the pages pair an int4
- *   body with an absmax int8 head); other mixes give QG_ERR_FORMAT.
+ *   body with an absmax int8 head); other mixes, and fp16 weights, give
+ *   QG_ERR_FORMAT.
  *
  * qg_sweep_workspace_bytes(n) -- device bytes a plan of n stages needs.
  * qg_sweep_plan -- validates every stage (the same checks, with the same

@@ -54,6 +54,13 @@ int64_t block_of(int fmt) { return fmt == QG_FMT_I8_B32 ? 32 : 64; }
 // Shape, format and alignment of one weight descriptor.
 qg_status check_weight(const qg_weight* W) {
     if (!W) return QG_ERR_NULL;
+    if (W->fmt == QG_FMT_F16) {  // plain fp16 weights: rows of whole 16-byte vectors
+        if (!W->codes) return QG_ERR_NULL;
+        if (W->n < 1 || W->k < 8 || W->k % 8 != 0) return QG_ERR_SHAPE;
+        if (W->n > (int64_t(1) << 31) - 1) return QG_ERR_SHAPE;
+        if (!aligned(W->codes, 16)) return QG_ERR_ALIGN;
+        return QG_OK;
+    }
     if (W->fmt != QG_FMT_I8_B32 && W->fmt != QG_FMT_I4_G64) return QG_ERR_FORMAT;
     if (!W->codes || !W->scales) return QG_ERR_NULL;
     if (W->fmt == QG_FMT_I4_G64 && !W->biases) return QG_ERR_NULL;
@@ -206,7 +213,7 @@ qg_status qg_gate_up_swiglu(const qg_weight* Wg, const qg_weight* Wu, const uint
     if (st != QG_OK) return st;
     st = check_weight(Wu);
     if (st != QG_OK) return st;
-    if (Wg->fmt != Wu->fmt) return QG_ERR_FORMAT;
+    if (Wg->fmt != Wu->fmt || Wg->fmt == QG_FMT_F16) return QG_ERR_FORMAT;
     if (Wg->n != Wu->n || Wg->k != Wu->k) return QG_ERR_SHAPE;
     if (!X || !H) return QG_ERR_NULL;
     if (S < 1 || S > 16) return QG_ERR_SHAPE;

@@ -52,12 +52,14 @@ constexpr int kThreads = kWarps * kLanes;
 constexpr int kCtasPerSm = 2;
 constexpr int kPrefetchBytesPerWarp = 12 * 1024;
 
+// FMT: 0 int8 block-32, 1 int4 group-64, 2 plain fp16 weights (no scales).
 template <int FMT>
 struct Fmt {
-    static constexpr int kCodesPerLane = FMT == 0 ? 16 : 32;   // one 16-byte vector
-    static constexpr int kBlock = FMT == 0 ? 32 : 64;
+    static constexpr int kCodesPerLane = FMT == 0 ? 16 : (FMT == 1 ? 32 : 8);  // one 16-byte vector
+    static constexpr bool kScales = FMT != 2;
+    static constexpr int kBlock = FMT == 0 ? 32 : 64;           // codes per scale (FMT 0 and 1)
     static constexpr int kPieces = kCodesPerLane / 8;           // 16-byte fp16 x pieces per lane
-    static constexpr int kSums = FMT == 0 ? 1 : 2;              // floats of x sums per granule
+    static constexpr int kSums = FMT == 1 ? 2 : 1;              // floats of x sums per granule
     static constexpr bool kBias = FMT == 1;
 };
 
@@ -133,6 +135,16 @@ __device__ __forceinline__ float dot16_i8(const uint4 c, const uint4* xv) {
         fma_f16x2_f32(a0, a1, __byte_perm(u, 0x64646464u, 0x4140), x[2 * i]);
         fma_f16x2_f32(a0, a1, __byte_perm(u, 0x64646464u, 0x4342), x[2 * i + 1]);
     }
+    return a0 + a1;
+}
+
+// 8 fp16 weights (one 16-byte vector) against their 8 fp16 x: sum_k w_k x_k.
+__device__ __forceinline__ float dot8_f16(const uint4 c, const uint4* xv) {
+    float a0 = 0.f, a1 = 0.f;
+    fma_f16x2_f32(a0, a1, c.x, xv[0].x);
+    fma_f16x2_f32(a0, a1, c.y, xv[0].y);
+    fma_f16x2_f32(a0, a1, c.z, xv[0].z);
+    fma_f16x2_f32(a0, a1, c.w, xv[0].w);
     return a0 + a1;
 }
 
@@ -212,7 +224,7 @@ __device__ __forceinline__ void stage_x(const uint16_t* __restrict__ x, uint4* x
                 se += h2f(static_cast<uint16_t>(w[e] & 0xFFFFu));
                 so += h2f(static_cast<uint16_t>(w[e] >> 16));
             }
-            if (FMT == 0) {
+            if (FMT != 1) {
                 xs[x_piece<FMT>(g, c)] = v;
             } else {  // (x0,x1)(x2,x3)(x4,x5)(x6,x7) -> (x0,x4)(x1,x5)(x2,x6)(x3,x7)
                 xs[x_piece<FMT>(g, c)] =
@@ -222,6 +234,8 @@ __device__ __forceinline__ void stage_x(const uint16_t* __restrict__ x, uint4* x
         }
         if (FMT == 0) {
             sums[g] = 1152.0f * (se + so);
+        } else if (FMT == 2) {
+            sums[g] = 0.f;  // fp16 weights have no constant term
         } else {
             sums[2 * g] = 1024.0f * se + 64.0f * so;
             sums[2 * g + 1] = se + so;
@@ -309,8 +323,8 @@ __device__ __forceinline__ void prefetch_items(const Params& p, int64_t wg, int6
                                                int first, int count, int my_items) {
     using F = Fmt<FMT>;
     const int64_t N = p.n, K = p.k;
-    const int64_t row_bytes = FMT == 0 ? K : K / 2;
-    const int64_t side_per_row = K / F::kBlock;
+    const int64_t row_bytes = FMT == 0 ? K : (FMT == 1 ? K / 2 : K * 2);
+    const int64_t side_per_row = F::kScales ? K / F::kBlock : 0;
     for (int i = first; i < first + count && i < my_items; ++i) {
         const int64_t r0 = (wg + i * tw) * RG;
         const int64_t rows = N - r0 < RG ? N - r0 : RG;
@@ -321,7 +335,7 @@ __device__ __forceinline__ void prefetch_items(const Params& p, int64_t wg, int6
             const uintptr_t sa = reinterpret_cast<uintptr_t>(
                 (m == 0 ? p.scales[0] : p.scales[1]) + r0 * side_per_row);
             const uint32_t sbytes = static_cast<uint32_t>(rows * side_per_row * 2);
-            if (sa % 16 == 0 && sbytes % 16 == 0) {
+            if (F::kScales && sa % 16 == 0 && sbytes % 16 == 0) {
                 prefetch_l2(reinterpret_cast<const void*>(sa), sbytes);
                 if (F::kBias)
                     prefetch_l2((m == 0 ? p.biases[0] : p.biases[1]) + r0 * side_per_row, sbytes);
@@ -501,13 +515,13 @@ struct RingLayout {
     // fp16 scales (and 16 biases for int4)
     static constexpr int kCodes = kLanes * 16;
     static constexpr int kSide = 32;
-    static constexpr int kPerRow = kCodes + kSide * (FMT == 1 ? 2 : 1);
+    static constexpr int kPerRow = kCodes + kSide * (FMT == 1 ? 2 : (FMT == 0 ? 1 : 0));
 };
 
 // Shared memory of one CTA's rings; x (and the int4 sums) follow it.
 __host__ __device__ constexpr uint32_t ring_bytes(int fmt, int rows) {
     return static_cast<uint32_t>(kWarps * kRing * rows *
-                                 (kLanes * 16 + 32 * (fmt == 1 ? 2 : 1)));
+                                 (kLanes * 16 + 32 * (fmt == 1 ? 2 : (fmt == 0 ? 1 : 0))));
 }
 
 // How a ring stage orders itself after the work before it.
@@ -565,8 +579,8 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
     using RL = RingLayout<FMT, NMAT>;
     constexpr int ROWS = NMAT * RG;
     constexpr int kStepBytes = kLanes * 16;
-    constexpr int kStepSides = kStepBytes * (FMT == 0 ? 1 : 2) / F::kBlock;  // 16
-    constexpr int kSideLanes = 2 * ROWS * (F::kBias ? 2 : 1);  // lanes that copy side data
+    constexpr int kStepSides = F::kScales ? kStepBytes * (FMT == 0 ? 1 : 2) / F::kBlock : 0;  // 16
+    constexpr int kSideLanes = F::kScales ? 2 * ROWS * (F::kBias ? 2 : 1) : 0;  // side-data copiers
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t N = p.n, K = p.k;
@@ -577,8 +591,8 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
     const int64_t tw = static_cast<int64_t>(gridDim.x) * kWarps;
     const int my_items = wg < items ? static_cast<int>((items - wg + tw - 1) / tw) : 0;
     const int total = my_items * nst;
-    const int64_t row_bytes = FMT == 0 ? K : K / 2;
-    const int64_t side_per_row = K / F::kBlock;  // a multiple of 8 (16-byte pieces)
+    const int64_t row_bytes = FMT == 0 ? K : (FMT == 1 ? K / 2 : K * 2);
+    const int64_t side_per_row = F::kScales ? K / F::kBlock : 0;  // a multiple of 8 (16-byte pieces)
     const uint64_t pol = l2_policy_evict_first();
 
     // shared memory: [rings of this CTA's warps][x fp16][x sums][x fp16 raw]
@@ -715,6 +729,10 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
 #pragma unroll
             for (int j = 0; j < ROWS; ++j) {
                 const uint4 c = lds128(slot_codes(cu_slot, j));
+                if (FMT == 2) {
+                    acc[j] += dot8_f16(c, xv);
+                    continue;
+                }
                 const float sc = h2f(lds16(slot_side(cu_slot, j, 0) + side_off));
                 if (FMT == 0) {
                     acc[j] = fmaf(sc, dot16_i8(c, xv) - c0, acc[j]);
@@ -749,9 +767,10 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) 
 // x's shared memory: the staged fp16 x, its per-granule sums, and the raw
 // fp16 copy if x arrives by bulk copy.
 size_t x_smem_bytes(int fmt, const Params& p) {
-    const int granules = static_cast<int>(
-        p.k / (fmt == QG_FMT_I8_B32 ? Fmt<0>::kCodesPerLane : Fmt<1>::kCodesPerLane));
-    const int nsums = (fmt == QG_FMT_I8_B32 ? Fmt<0>::kSums : Fmt<1>::kSums) * granules;
+    const int cpl = fmt == QG_FMT_I8_B32 ? Fmt<0>::kCodesPerLane
+                    : (fmt == QG_FMT_I4_G64 ? Fmt<1>::kCodesPerLane : Fmt<2>::kCodesPerLane);
+    const int granules = static_cast<int>(p.k / cpl);
+    const int nsums = (fmt == QG_FMT_I4_G64 ? Fmt<1>::kSums : Fmt<0>::kSums) * granules;
     size_t b = static_cast<size_t>(p.x_words) * 4 + static_cast<size_t>(align_up(nsums, 4)) * 4;
     if (p.x_bulk) b += static_cast<size_t>(p.k) * 2;
     return b;
@@ -783,7 +802,8 @@ qg_status launch_t(Params p, const DeviceInfo& dev, cudaStream_t stream) {
     int64_t grid = (items + kWarps - 1) / kWarps;
     const int64_t max_grid = static_cast<int64_t>(dev.num_sms) * kCtasPerSm;
     if (grid > max_grid) grid = max_grid;
-    const int64_t item_bytes = static_cast<int64_t>(NMAT) * RG * (FMT == 0 ? p.k : p.k / 2);
+    const int64_t item_bytes =
+        static_cast<int64_t>(NMAT) * RG * (FMT == 0 ? p.k : (FMT == 1 ? p.k / 2 : p.k * 2));
     p.prefetch_items = static_cast<int>(kPrefetchBytesPerWarp / item_bytes);
     if (p.prefetch_items < 1) p.prefetch_items = 1;
 
@@ -813,7 +833,7 @@ qg_status launch_pick(const Params& p0, const DeviceInfo& dev, cudaStream_t stre
     // a row's count must be a multiple of 8; its ring must fit beside x in the
     // per-CTA budget, with x's raw bulk-copy buffer if there is room for it.
     Params p = p0;
-    const bool even_sides = (p.k / Fmt<FMT>::kBlock) % 8 == 0;
+    const bool even_sides = !Fmt<FMT>::kScales || (p.k / Fmt<FMT>::kBlock) % 8 == 0;
     if (even_sides) {
         p.x_bulk = 1;
         if (x_smem_bytes(FMT, p) + ring_smem_bytes<FMT, NMAT, RG>() <= kSmemPerCtaBudget)
@@ -823,7 +843,11 @@ qg_status launch_pick(const Params& p0, const DeviceInfo& dev, cudaStream_t stre
             return launch_t<FMT, NMAT, RG, EPI, true>(p, dev, stream);
     }
     p.x_bulk = 0;
-    return launch_t<FMT, NMAT, RG, EPI, false>(p, dev, stream);
+    if constexpr (Fmt<FMT>::kScales) {
+        return launch_t<FMT, NMAT, RG, EPI, false>(p, dev, stream);
+    } else {
+        return QG_ERR_SHAPE;  // fp16 weights run on the ring path only
+    }
 }
 
 template <int FMT>
@@ -831,9 +855,13 @@ qg_status dispatch_fmt(const GemvLaunch& L, const Params& p, const DeviceInfo& d
                        cudaStream_t stream) {
     const int tw = dev.num_sms * kCtasPerSm * kWarps;
     if (L.epilogue == kEpiSwiglu) {
-        const int rg = pick_rg(L.n, 2, tw);
-        if (rg == 2) return launch_pick<FMT, 2, 2, kEpiSwiglu>(p, dev, stream);
-        return launch_pick<FMT, 2, 1, kEpiSwiglu>(p, dev, stream);
+        if constexpr (FMT == 2) {
+            return QG_ERR_FORMAT;  // fp16 weights: GEMV and head only
+        } else {
+            const int rg = pick_rg(L.n, 2, tw);
+            if (rg == 2) return launch_pick<FMT, 2, 2, kEpiSwiglu>(p, dev, stream);
+            return launch_pick<FMT, 2, 1, kEpiSwiglu>(p, dev, stream);
+        }
     }
     const int rg = pick_rg(L.n, 4, tw);
     if (L.epilogue == kEpiHead) {
@@ -991,7 +1019,8 @@ Params make_params(const GemvLaunch& L) {
     p.ws_ticket = L.workspace
                       ? reinterpret_cast<unsigned int*>(static_cast<char*>(L.workspace) + 8)
                       : nullptr;
-    const int cpl = L.fmt == QG_FMT_I8_B32 ? Fmt<0>::kCodesPerLane : Fmt<1>::kCodesPerLane;
+    const int cpl = L.fmt == QG_FMT_I8_B32 ? Fmt<0>::kCodesPerLane
+                    : (L.fmt == QG_FMT_I4_G64 ? Fmt<1>::kCodesPerLane : Fmt<2>::kCodesPerLane);
     const int granules = static_cast<int>(L.k / cpl);
     p.x_words = align_up(granules, 8) * cpl / 2;  // fp16 x, padded to whole 8-granule phases
     return p;
@@ -1003,6 +1032,10 @@ Params make_params(const GemvLaunch& L) {
 // if the kernel has no variant for the stage.
 int sweep_variant(int kernel, const GemvLaunch& L, Params* p, int total_warps, int* rg_out,
                   qg_status* status) {
+    if (L.fmt == QG_FMT_F16) {  // the persistent kernels hold no fp16-weight variant
+        *status = QG_ERR_FORMAT;
+        return -1;
+    }
     const int block = L.fmt == QG_FMT_I8_B32 ? 32 : 64;
     *status = QG_ERR_SHAPE;
     if ((L.k / block) % 8 != 0) return -1;
@@ -1116,7 +1149,8 @@ qg_status launch_gemv_s1(const GemvLaunch& L, cudaStream_t stream) {
     if (st != QG_OK) return st;
     const Params p = make_params(L);
     if (L.fmt == QG_FMT_I8_B32) return dispatch_fmt<0>(L, p, dev, stream);
-    return dispatch_fmt<1>(L, p, dev, stream);
+    if (L.fmt == QG_FMT_I4_G64) return dispatch_fmt<1>(L, p, dev, stream);
+    return dispatch_fmt<2>(L, p, dev, stream);
 }
 
 unsigned int gemv_read_and_clear_error() {

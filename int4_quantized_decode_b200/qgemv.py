@@ -24,6 +24,7 @@ STATUS_NAMES = {0: "QG_OK", 1: "QG_ERR_NULL", 2: "QG_ERR_SHAPE", 3: "QG_ERR_ALIG
                 7: "QG_ERR_TIMEOUT", 8: "QG_ERR_PLAN"}
 FMT_I8_B32 = 0
 FMT_I4_G64 = 1
+FMT_F16 = 2  # plain fp16 weights (the tied fp16 head of the int8lin bundle)
 
 # every symbol include/qgemv.h declares
 ABI_SYMBOLS = ("qg_quantize_block32", "qg_quantize_int4_g64", "qg_gemv_s1",
@@ -138,9 +139,15 @@ class QWeight:
     fmt: int
     n: int
     k: int
-    codes: torch.Tensor            # int8 [n, k] or uint8 [n, k/2]
-    scales: torch.Tensor           # int16 (fp16 bits) [n, k/block]
+    codes: torch.Tensor            # int8 [n, k], uint8 [n, k/2] or fp16 [n, k]
+    scales: Optional[torch.Tensor]  # int16 (fp16 bits) [n, k/block]; None for fp16 weights
     biases: Optional[torch.Tensor] = None
+
+    @staticmethod
+    def fp16(w: torch.Tensor) -> "QWeight":
+        """Plain fp16 weights [n, k] (no quantization), e.g. a tied fp16 head."""
+        _cuda(w, torch.float16, "w")
+        return QWeight(FMT_F16, w.shape[0], w.shape[1], w, None)
 
     @staticmethod
     def empty(fmt: int, n: int, k: int, device="cuda") -> "QWeight":
@@ -153,20 +160,22 @@ class QWeight:
 
     def rows(self, r0: int, r1: int) -> "QWeight":
         """View of rows [r0, r1) (row ranges are valid weights on their own)."""
-        return QWeight(self.fmt, r1 - r0, self.k, self.codes[r0:r1], self.scales[r0:r1],
+        return QWeight(self.fmt, r1 - r0, self.k, self.codes[r0:r1],
+                       None if self.scales is None else self.scales[r0:r1],
                        None if self.biases is None else self.biases[r0:r1])
 
     @property
     def nbytes(self) -> int:
         b = self.codes.numel() * self.codes.element_size()
-        b += self.scales.numel() * 2
+        if self.scales is not None:
+            b += self.scales.numel() * 2
         if self.biases is not None:
             b += self.biases.numel() * 2
         return b
 
     def c(self) -> CWeight:
         return CWeight(self.fmt, 0, self.n, self.k, self.codes.data_ptr(),
-                       self.scales.data_ptr(),
+                       self.scales.data_ptr() if self.scales is not None else None,
                        self.biases.data_ptr() if self.biases is not None else None)
 
 

@@ -54,6 +54,7 @@ class DecodeSweep:
         self.body_fmt, self.head_fmt = body_fmt, head_fmt
         if S > 1:
             assert body_fmt == qg.FMT_I8_B32 and head_fmt == qg.FMT_I8_B32
+        assert body_fmt != qg.FMT_F16, "fp16 weights serve the head only"
         self.layers: List[LayerWeights] = []
         for l in range(dec.layers):
             self.layers.append(self._make_layer(l))
@@ -66,6 +67,8 @@ class DecodeSweep:
     def _quantized(self, proj: str, layer: int, n: int, k: int, fmt: int,
                    out: Optional[qg.QWeight] = None) -> qg.QWeight:
         w = wl.weight_fp32(n, k, self.dec.weight_seed(layer, proj), self.device)
+        if fmt == qg.FMT_F16:  # plain fp16 weights (the int8lin bundle's tied fp16 head)
+            return qg.QWeight.fp16(w.half())
         q = qg.quantize(w, fmt, out)
         del w
         return q

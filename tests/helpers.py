@@ -17,8 +17,11 @@ def host_weight(W, rows=None):
     b = W.biases
     if rows is not None:
         r = torch.as_tensor(rows, device=c.device)
-        c, s = c.index_select(0, r), s.index_select(0, r)
+        c = c.index_select(0, r)
+        s = s.index_select(0, r) if s is not None else None
         b = b.index_select(0, r) if b is not None else None
+    if W.fmt == 2:  # plain fp16 weights: the oracle takes their bit patterns
+        return bits(c), None, None
     c = c.cpu().numpy()
     return c, bits(s), (bits(b) if b is not None else None)
 

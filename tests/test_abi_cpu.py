@@ -148,3 +148,12 @@ def test_sweep_validation(L):
     assert L.qg_sweep_run(None, 0x10000, None) == 1
     assert L.qg_sweep_run(ctypes.byref(qg.CSweep(0, 0)), 0x10000, None) == 2
     assert L.qg_sweep_run(ctypes.byref(sw), 0x10010, None) == 3
+
+
+def test_fp16_weight_validation(L):
+    assert gemv(L, W(fmt=2, k=12, scales=0)) == 2              # rows of whole 16-byte vectors
+    assert gemv(L, W(fmt=2, codes=0x1008, scales=0)) == 3
+    assert gemv(L, W(fmt=2, codes=0, scales=0)) == 1
+    w = W(fmt=2, k=64, scales=0)
+    assert L.qg_gate_up_swiglu(ctypes.byref(w), ctypes.byref(w), 0x4000, 1, 0x6000, None) == 4
+    assert L.qg_gemm_s16(ctypes.byref(w), 0x4000, 4, 0x5000, None) == 4

@@ -173,3 +173,40 @@ def test_head_argmax_tied_embedding(cuda):
     yr, mag = oracle_gemv(W, x)
     np.testing.assert_allclose(yr, ref, rtol=1e-12, atol=1e-12)
     assert_within_bound(logits.cpu().numpy(), yr, mag)
+
+
+# ------------------------------------------------ plain fp16 weights -------
+@pytest.mark.parametrize("n,k", [(1, 8), (37, 264), (300, 2048), (4103, 2560), (151936, 2048),
+                                 (20011, 4096)])
+def test_fp16_weight_gemv_and_head(cuda, n, k):
+    """The int8lin bundle's tied fp16 head: GEMV and head argmax straight over
+    fp16 weights, vs the oracle's exact fp64 matvec of the same values."""
+    w = wl.weight_fp32(n, k, 700 + n % 31, cuda).half()
+    W = qg.QWeight.fp16(w)
+    x = wl.act_fp16(k, 701, cuda)
+    y = torch.full((n,), float("nan"), dtype=torch.float32, device=cuda)
+    y16 = torch.empty(n, dtype=torch.float16, device=cuda)
+    qg.qg_gemv_s1(W, x, y, y16)
+    idx = torch.full((1,), -1, dtype=torch.int32, device=cuda)
+    logits = torch.empty(n, dtype=torch.float32, device=cuda)
+    ws = qg.head_workspace(n, cuda)
+    qg.qg_head_argmax(W, x, idx, ws, logits)
+    qg.qg_stream_check()
+    rows = None if n <= 20011 else wl.sample_rows(n, 256, 3).tolist()
+    yr, mag = oracle_gemv(W, x, rows)
+    yd, ld = y.cpu().numpy(), logits.cpu().numpy()
+    assert_within_bound(yd if rows is None else yd[rows], yr, mag)
+    assert_within_bound(ld if rows is None else ld[rows], yr, mag)
+    assert np.array_equal(bits(y16), oracle.f32_to_f16_bits(yd))
+    full, _ = oracle_gemv(W, x) if rows is not None else (yr, mag)
+    assert oracle.argmax_ok(int(idx.item()), full)
+    assert int(ws.sum().item()) == 0
+
+
+def test_fp16_weights_rejected_where_unsupported(cuda):
+    W = qg.QWeight.fp16(wl.weight_fp32(64, 512, 1, cuda).half())
+    X = wl.act_fp16((4, 512), 2, cuda)
+    with pytest.raises(qg.QgError, match="QG_ERR_FORMAT"):
+        qg.qg_gemm_s16(W, X, torch.empty((4, 64), dtype=torch.float32, device=cuda))
+    with pytest.raises(qg.QgError, match="QG_ERR_FORMAT"):
+        qg.qg_gate_up_swiglu(W, W, X[0], torch.empty(64, dtype=torch.float16, device=cuda))

@@ -36,6 +36,10 @@ def _check_codes(sw, W, l, parts, rows):
         w = wl.weight_fp32(cnt, W.k, d.weight_seed(l, name), sw.device)
         wr = w.index_select(0, torch.as_tensor(sel, device=sw.device)).cpu().numpy()
         del w
+        if W.fmt == qg.FMT_F16:  # plain fp16 weights: the IEEE RNE of the draw
+            dc, _, _ = host_weight(W, [r for r in rows if off <= r < off + cnt])
+            assert np.array_equal(dc, oracle.f32_to_f16_bits(wr)), (name, l)
+            continue
         oc, os_, ob = oracle_quantize(W.fmt, wr)
         dc, ds, db = host_weight(W, [r for r in rows if off <= r < off + cnt])
         assert np.array_equal(dc, oc), (name, l)
@@ -139,6 +143,11 @@ def test_single_gemv_2048(cuda):
 
 def test_sweep_2b_int8(cuda):
     _check_sweep(wl.QWEN3VL_2B, I8, I8, 1, cuda)
+
+
+def test_sweep_2b_int8_tied_fp16_head(cuda):
+    """The int8lin bundle: int8 body, the fp16 embedding table as the head."""
+    _check_sweep(wl.QWEN3VL_2B, I8, qg.FMT_F16, 1, cuda)
 
 
 def test_sweep_4b_int8(cuda):
