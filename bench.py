@@ -48,8 +48,10 @@ WORKLOADS = {
     "qwen3vl-4b": ("QWEN3VL_4B", 0, 0, 1),
     "qwen3vl-4b-int4": ("QWEN3VL_4B", 1, 0, 1),
     "qwen3vl-8b": ("QWEN3VL_8B", 0, 0, 1),
+    "qwen3vl-8b-int4": ("QWEN3VL_8B", 1, 0, 1),
     "qwen3vl-8b-s16": ("QWEN3VL_8B", 0, 0, 16),
     "dense-27b": ("DENSE_27B", 0, 0, 1),
+    "dense-27b-int4": ("DENSE_27B", 1, 1, 1),
 }
 DEFAULT_WORKLOAD = "qwen3vl-2b"
 FMT_NAME = {0: "int8 block-32", 1: "int4 group-64", 2: "fp16"}

@@ -168,3 +168,12 @@ def test_sweep_8b_s16_chunk(cuda):
 
 def test_sweep_27b_int8(cuda):
     _check_sweep(wl.DENSE_27B, I8, I8, 1, cuda)
+
+
+def test_sweep_8b_int4_body(cuda):
+    _check_sweep(wl.QWEN3VL_8B, I4, I8, 1, cuda)
+
+
+def test_sweep_27b_int4_body_and_head(cuda):
+    """The 27B 'int4lin' option: every matrix int4 group-64, the head too."""
+    _check_sweep(wl.DENSE_27B, I4, I4, 1, cuda)
