@@ -80,6 +80,10 @@ def lib():
         L.orc_argmax.argtypes = [P, I64]
         L.orc_argmax.restype = I64
         L.orc_num_threads.argtypes = []
+        L.orc_f64_to_f16.argtypes = [D]
+        L.orc_f64_to_f16.restype = ctypes.c_uint16
+        L.orc_rmsnorm.argtypes = [P, P, I64, D, P, P]
+        L.orc_rmsnorm.restype = None
         L.orc_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -253,3 +257,25 @@ def argmax_ok(idx: int, logits_ref: np.ndarray, margin: float = ARGMAX_MARGIN) -
     if not (0 <= idx < logits_ref.shape[0]):
         return False
     return bool(logits_ref[idx] >= logits_ref[ref] - margin)
+
+
+# ------------------------------------------------- RMSNorm / fp64 -> fp16 ---
+
+def f64_to_f16_bits(x) -> np.ndarray:
+    """fp64 -> fp16 bit patterns, one IEEE round-to-nearest-even."""
+    a = np.asarray(x, dtype=np.float64)
+    f = lib().orc_f64_to_f16
+    return np.array([f(float(v)) for v in a.ravel()], dtype=np.uint16).reshape(a.shape)
+
+
+def rmsnorm(h, gamma_bits, eps: float):
+    """The decoder's pre-norm RMSNorm: (x fp16 bits [k], x before rounding fp64 [k])
+    for an fp32 hidden state h and fp16 gains."""
+    h = np.ascontiguousarray(h, dtype=np.float32)
+    g = np.ascontiguousarray(gamma_bits, dtype=np.uint16)
+    k = h.shape[0]
+    assert g.shape == (k,)
+    x = np.empty(k, dtype=np.uint16)
+    xe = np.empty(k, dtype=np.float64)
+    lib().orc_rmsnorm(_p(h), _p(g), k, float(eps), _p(x), _p(xe))
+    return x, xe

@@ -238,6 +238,44 @@ void orc_matvec(int fmt, const void* codes, const uint16_t* scales,
     free(xd);
 }
 
+/* ----------------------------------------------------- fp64 -> fp16 --- */
+
+uint16_t orc_f64_to_f16(double d) {
+    uint16_t sign = signbit(d) ? 0x8000u : 0u;
+    double a = fabs(d);
+    if (isnan(d)) return (uint16_t)(sign | 0x7E00u);
+    if (isinf(a)) return (uint16_t)(sign | 0x7C00u);
+    if (a == 0.0) return sign;
+    int e2;
+    frexp(a, &e2);       /* a = m * 2^e2, 0.5 <= m < 1, so 2^(e2-1) <= a < 2^e2 */
+    int E = e2 - 1;      /* unbiased exponent of a */
+    if (E < -14) E = -14; /* subnormal range: fixed quantum 2^-24 */
+    /* the significand in units of the quantum 2^(E-10) (exact power-of-two
+     * scaling), rounded half to even */
+    double q = nearbyint(ldexp(a, 10 - E));
+    if (q >= 2048.0) { /* rounded up to the next binade */
+        q /= 2.0;
+        E += 1;
+    }
+    if (E > 15) return (uint16_t)(sign | 0x7C00u);
+    if (q < 1024.0) return (uint16_t)(sign | (uint16_t)q); /* subnormal (E == -14) */
+    return (uint16_t)(sign | (uint16_t)((E + 15) << 10) | ((uint16_t)q & 0x3FFu));
+}
+
+/* ------------------------------------------------------------ RMSNorm --- */
+
+void orc_rmsnorm(const float* h, const uint16_t* gamma, int64_t k, double eps, uint16_t* x,
+                 double* x_exact) {
+    double ss = 0.0;
+    for (int64_t i = 0; i < k; ++i) ss += (double)h[i] * (double)h[i];
+    const double rms = sqrt(ss / (double)k + eps);
+    for (int64_t i = 0; i < k; ++i) {
+        const double v = (double)h[i] * orc_f16_to_f64(gamma[i]) / rms;
+        if (x_exact) x_exact[i] = v;
+        x[i] = orc_f64_to_f16(v);
+    }
+}
+
 /* ------------------------------------------------------------- SwiGLU --- */
 
 double orc_silu(double g) { return g / (1.0 + exp(-g)); }

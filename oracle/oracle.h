@@ -80,6 +80,21 @@ void orc_matvec(int fmt, const void* codes, const uint16_t* scales,
                 const uint16_t* biases, int64_t n, int64_t k,
                 const uint16_t* x, double* y, double* mag);
 
+/* fp64 -> fp16 bits, IEEE-754 binary16 round-to-nearest-even from the
+ * definition (one rounding of the fp64 value; subnormals kept, overflow ->
+ * +-Inf). */
+uint16_t orc_f64_to_f16(double d);
+
+/* The decoder's pre-norm RMSNorm of the fp32 residual stream, which feeds
+ * q|k|v, gate/up and the head (the pages' decoders are Qwen3-architecture
+ * models; the norm itself is not spelled out on the pages):
+ *   rms  = sqrt( sum_i h[i]^2 / k + eps )          (fp64, index order)
+ *   x[i] = fp16_rne( h[i] * gamma[i] / rms )       (fp64, one rounding)
+ * h fp32 [k], gamma fp16 bits [k]; out x fp16 bits [k], and optionally the
+ * fp64 values before the rounding (x_exact, or NULL). */
+void orc_rmsnorm(const float* h, const uint16_t* gamma, int64_t k, double eps,
+                 uint16_t* x, double* x_exact);
+
 /* silu(g) = g / (1 + exp(-g)) and its derivative, fp64. */
 double orc_silu(double g);
 double orc_silu_grad(double g);

@@ -436,3 +436,63 @@ def test_int4_signed_zero_group_gives_positive_zero_side_data():
     w2 = -np.zeros((1, 64), dtype=np.float32)
     codes, scales, biases = oracle.quantize_int4_g64(w2)
     assert scales[0, 0] == 0 and biases[0, 0] == 0
+
+
+# --------------------------------------------------------- RMSNorm --------
+
+def test_f64_to_f16_matches_ieee_library_conversion():
+    rng = np.random.default_rng(41)
+    vals = np.concatenate([
+        rng.normal(0, 1, 20000), rng.normal(0, 1e-5, 5000), rng.normal(0, 3e4, 5000),
+        np.ldexp(rng.uniform(1, 2, 5000), rng.integers(-30, 17, 5000)),
+        [0.0, -0.0, 65504.0, 65519.99, 65520.0, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26,
+         2.0 ** -14, 2.0 ** -14 - 2.0 ** -25, 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11]])
+    # midpoints between consecutive fp16 values and one fp64 ulp either side
+    f = np.arange(0x0000, 0x7BFF, 97, dtype=np.uint16).view(np.float16).astype(np.float64)
+    g = (np.arange(0x0000, 0x7BFF, 97, dtype=np.uint16) + 1).view(np.float16).astype(np.float64)
+    mid = (f + g) / 2
+    vals = np.concatenate([vals, mid, np.nextafter(mid, 0), np.nextafter(mid, np.inf), -mid])
+    ours = oracle.f64_to_f16_bits(vals)
+    ref = vals.astype(np.float16).view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_rmsnorm_closed_forms():
+    k = 64
+    rng = np.random.default_rng(43)
+    gam = np_f16_bits(rng.normal(1, 0.1, k))
+    # constant h = c, eps = 0: h / rms = sign(c) exactly, so x = +-gamma
+    for c in (0.75, -3.0, 1e-3):
+        x, _ = oracle.rmsnorm(np.full(k, c, np.float32), gam, 0.0)
+        assert np.array_equal(x, gam ^ (0x8000 if c < 0 else 0))
+    # scale invariance with eps = 0: h * 2^m gives the same bits
+    h = rng.normal(0, 1, k).astype(np.float32)
+    x0, _ = oracle.rmsnorm(h, gam, 0.0)
+    for m in (-7, 3, 20):
+        xm, _ = oracle.rmsnorm(h * np.float32(2.0 ** m), gam, 0.0)
+        assert np.array_equal(xm, x0)
+    # one-hot h = a e_j: rms = |a| / sqrt(k), so x_j = sign(a) sqrt(k) gamma_j = 8 gamma_j
+    for j, a in ((0, 2.5), (37, -0.125)):
+        e = np.zeros(k, np.float32)
+        e[j] = a
+        x, _ = oracle.rmsnorm(e, gam, 0.0)
+        want = np.zeros(k, np.uint16)
+        want[j] = oracle.f64_to_f16_bits(np.sign(a) * 8.0 * f16_np(gam[j:j + 1]).astype(np.float64))[0]
+        assert np.array_equal(x, want)
+    # eps only matters against a tiny mean square: h = 0 gives x = 0
+    x, _ = oracle.rmsnorm(np.zeros(k, np.float32), gam, 1e-6)
+    assert not np.any(x & 0x7FFF)
+
+
+def test_rmsnorm_matches_independent_numpy():
+    rng = np.random.default_rng(47)
+    for k in (128, 2048, 5120):
+        h = (rng.normal(0, 1, k) * rng.uniform(0.1, 30)).astype(np.float32)
+        gam = np_f16_bits(rng.normal(1, 0.2, k))
+        x, xe = oracle.rmsnorm(h, gam, 1e-6)
+        hd = h.astype(np.float64)
+        ref = hd * f16_np(gam).astype(np.float64) / np.sqrt(np.mean(hd * hd) + 1e-6)
+        np.testing.assert_allclose(xe, ref, rtol=1e-13, atol=0)
+        near_tie = np.abs(ref * 2.0 ** (10 - np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -14))))
+                          % 1 - 0.5) < 1e-9
+        assert np.array_equal(x[~near_tie], ref.astype(np.float16).view(np.uint16)[~near_tie])
