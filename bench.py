@@ -41,10 +41,11 @@ UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 
-# name -> (decoder, body format, head format, S)
+# name -> (decoder, body format, head format, S[, decode step])
 WORKLOADS = {
     "qwen3vl-2b": ("QWEN3VL_2B", 0, 0, 1),
     "qwen3vl-2b-f16head": ("QWEN3VL_2B", 0, 2, 1),
+    "qwen3vl-2b-decode": ("QWEN3VL_2B", 0, 0, 1, True),
     "qwen3vl-4b": ("QWEN3VL_4B", 0, 0, 1),
     "qwen3vl-4b-int4": ("QWEN3VL_4B", 1, 0, 1),
     "qwen3vl-8b": ("QWEN3VL_8B", 0, 0, 1),
@@ -252,7 +253,8 @@ def run_reference(a):
     if rank != 0:
         return 0
     from int4_quantized_decode_b200 import workloads as wl
-    dname, body_fmt, head_fmt, S = WORKLOADS[a.workload]
+    dname, body_fmt, head_fmt, S = WORKLOADS[a.workload][:4]
+    decode = len(WORKLOADS[a.workload]) > 4
     dec = getattr(wl, dname)
     sweep_bytes = _sweep_bytes(dec, body_fmt, head_fmt)
     oracle_sample(dec, body_fmt, S, 0, max_passes=a.warmup)
@@ -283,10 +285,13 @@ def _sweep_bytes(dec, body_fmt, head_fmt):
 
 
 def _config(a, dec, body_fmt, head_fmt, S, sweep_bytes):
+    decode = len(WORKLOADS[a.workload]) > 4
     return {
         "workload": (f"{dec.name}-shaped decode weight sweep, {FMT_NAME[body_fmt]} body + "
                      f"{FMT_NAME[head_fmt]} head{' (tied)' if dec.tied_head else ''}, "
-                     f"S={S}"),
+                     f"S={S}" + (", whole decode step minus attention (embedding gather, "
+                                 "RMSNorm and residual fused; the argmax feeds the next "
+                                 "step's gather)" if decode else "")),
         "layers": dec.layers, "hidden": dec.hidden, "inter": dec.inter,
         "vocab": dec.vocab, "S": S, "sweep_bytes": sweep_bytes,
         "parallelism": f"replicas x{a.gpus}",
@@ -318,9 +323,10 @@ def run_ours(a):
             import torch.distributed as dist
             dist.barrier(device_ids=[local])
 
-    dname, body_fmt, head_fmt, S = WORKLOADS[a.workload]
+    dname, body_fmt, head_fmt, S = WORKLOADS[a.workload][:4]
+    decode = len(WORKLOADS[a.workload]) > 4
     dec = getattr(wl, dname)
-    sw = DecodeSweep(dec, body_fmt, head_fmt, S=S, device=dev)
+    sw = DecodeSweep(dec, body_fmt, head_fmt, S=S, device=dev, decode_step=decode)
     persistent = a.path == "persistent"
     if a.path == "persistent" and S != 1:
         raise SystemExit("--path persistent needs an S=1 workload")
@@ -409,8 +415,11 @@ def _time_gate_up(sw, stream, dev, qg, torch):
     s.wait_stream(stream)
     with torch.cuda.graph(g, stream=s):
         for l, L in enumerate(sw.layers):
-            x = sw.x[l]
-            qg.qg_gate_up_swiglu(L.gate, L.up, x, sw.h if sw.S > 1 else sw.h[0])
+            if sw.decode_step:  # the decode step's variant: RMSNorm of the hidden state
+                qg.qg_rmsnorm_gate_up_swiglu(L.gate, L.up, sw.hstate, sw.gamma_mlp[l], sw.eps,
+                                             sw.h[0])
+            else:
+                qg.qg_gate_up_swiglu(L.gate, L.up, sw.x[l], sw.h if sw.S > 1 else sw.h[0])
     stream.wait_stream(s)
     reps = max(3, int(2e9 // (sw.layers[0].gate.nbytes * 2 * len(sw.layers))) + 3)
     for _ in range(3):

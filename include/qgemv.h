@@ -215,6 +215,48 @@ QG_API qg_status qg_head_argmax_noalloc(const qg_weight* W, const uint16_t* x, f
                                         int32_t* idx, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * The rest of a decode step around the weight stream, attention excluded:
+ * the embedding row of the chosen token and a decoder layer's pre-norm
+ * RMSNorm and residual adds, fused into the S=1 calls so that a chain of
+ * calls carries a real fp32 hidden state h from token to token.  The pages'
+ * engines gather fp16 embedding rows ("Qwen3.8-27B ... -- Core AI", The
+ * vision path: the host gathers text rows from the shipped fp16 embedding
+ * table); the norm belongs to the Qwen3-architecture decoders the pages
+ * port and is not spelled out there.
+ *   RMSNorm:  x[i] = fp16_rne( h[i] * gamma[i] / sqrt(sum_j h[j]^2 / k + eps) )
+ *             computed in fp32 inside every CTA that reads x (a fixed-order
+ *             reduction: results are deterministic).
+ * qg_embedding_gather       h[i] = table[*token][i] (fp16 -> fp32, exact).
+ *   table : fp16 [V, H], 2-byte aligned.  token : device int32 [1]; a value
+ *           outside [0, V) writes nothing and qg_stream_check reports
+ *           QG_ERR_SHAPE.  h : fp32 [H] out, 4-byte aligned.
+ * qg_rmsnorm_gemv_s1        qg_gemv_s1 with x = RMSNorm(h; gamma, eps).
+ * qg_rmsnorm_gate_up_swiglu qg_gate_up_swiglu (S = 1) with x = RMSNorm(h).
+ * qg_rmsnorm_head_argmax    qg_head_argmax with x = RMSNorm(h).
+ * qg_gemv_s1_residual       h[r] += (W x)[r] for every row r (the o and down
+ *                           projections adding into the residual stream);
+ *                           x must not overlap h.
+ *   h : fp32 [k] (the normed calls) or [n] (the residual call); gamma :
+ *       fp16 [k]; both 16-byte aligned.  0 <= eps <= 1 (QG_ERR_SHAPE).
+ * Accuracy: as the plain calls with x the fp64 RMSNorm rounded to fp16, plus
+ * one fp16 ulp of x per element (the device rounds x from fp32):
+ * |y - y_ref| <= (2e-3 + 2^-10) sum_k |w_dq x|.
+ * ------------------------------------------------------------------------- */
+QG_API qg_status qg_embedding_gather(const uint16_t* table, int64_t V, int64_t H,
+                                     const int32_t* token, float* h, cudaStream_t stream);
+QG_API qg_status qg_rmsnorm_gemv_s1(const qg_weight* W, const float* h, const uint16_t* gamma,
+                                    float eps, float* y, uint16_t* y16, cudaStream_t stream);
+QG_API qg_status qg_rmsnorm_gate_up_swiglu(const qg_weight* Wg, const qg_weight* Wu,
+                                           const float* h, const uint16_t* gamma, float eps,
+                                           uint16_t* H, cudaStream_t stream);
+QG_API qg_status qg_rmsnorm_head_argmax(const qg_weight* W, const float* h,
+                                        const uint16_t* gamma, float eps, float* logits,
+                                        int32_t* idx, void* workspace, size_t ws_bytes,
+                                        cudaStream_t stream);
+QG_API qg_status qg_gemv_s1_residual(const qg_weight* W, const uint16_t* x, float* h,
+                                     cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * qg_sweep_* -- a whole one-token decode step as ONE persistent launch.
  * A decode step reads every decoder weight once ("Qwen3-VL 4B -- Core AI
  * (.aimodel)", Measured), as an ordered chain of S=1 projections per layer
@@ -307,7 +349,8 @@ QG_API qg_status qg_sweep_run(const qg_sweep* sweep, void* workspace, cudaStream
 /* ---------------------------------------------------------------------------
  * qg_stream_check -- synchronize `stream` and report asynchronous failures:
  * QG_ERR_CUDA for a CUDA error, QG_ERR_PLAN if a sweep ran on a workspace
- * without its plan, QG_ERR_TIMEOUT if a kernel's bounded wait (on its own
+ * without its plan, QG_ERR_SHAPE if an embedding gather met a token id out
+ * of range, QG_ERR_TIMEOUT if a kernel's bounded wait (on its own
  * copies, or a sweep's wait between stages) expired since the last check
  * (the flags are then cleared).  Kernels never spin without a limit.
  * ------------------------------------------------------------------------- */

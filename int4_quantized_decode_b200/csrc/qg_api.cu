@@ -73,6 +73,29 @@ qg_status check_weight(const qg_weight* W) {
 
 constexpr int kMaxSweepStages = 65536;
 
+// The fp32 hidden state and fp16 gains of an RMSNorm input (read as 16-byte
+// vectors), and its epsilon.
+qg_status check_norm(const float* h, const uint16_t* gamma, float eps) {
+    if (!h || !gamma) return QG_ERR_NULL;
+    if (!(eps >= 0.0f) || eps > 1.0f) return QG_ERR_SHAPE;
+    if (!aligned(h, 16) || !aligned(gamma, 16)) return QG_ERR_ALIGN;
+    return QG_OK;
+}
+
+// The launch description of one weight with the plain epilogue.
+qg::GemvLaunch plain_launch(const qg_weight& W) {
+    qg::GemvLaunch L = {};
+    L.fmt = W.fmt;
+    L.epilogue = qg::kEpiPlain;
+    L.nmat = 1;
+    L.n = W.n;
+    L.k = W.k;
+    L.codes[0] = W.codes;
+    L.scales[0] = W.scales;
+    L.biases[0] = W.biases;
+    return L;
+}
+
 // One sweep stage -> the launch description of the S=1 call it stands for,
 // with that call's checks.
 qg_status stage_launch(const qg_stage& S, qg::GemvLaunch* out) {
@@ -129,7 +152,7 @@ qg_status stage_launch(const qg_stage& S, qg::GemvLaunch* out) {
 
 extern "C" {
 
-int qg_abi_version(void) { return 101; }
+int qg_abi_version(void) { return 102; }
 
 const char* qg_last_cuda_error(void) { return qg::last_cuda_error_name(); }
 
@@ -313,12 +336,100 @@ qg_status qg_sweep_run(const qg_sweep* sweep, void* workspace, cudaStream_t stre
     return qg::launch_sweep(sweep->kernel, workspace, sweep->n_stages, stream);
 }
 
+// ---------------------------------------------------- decode-step fusions ---
+
+qg_status qg_embedding_gather(const uint16_t* table, int64_t V, int64_t H, const int32_t* token,
+                              float* h, cudaStream_t stream) {
+    if (!table || !token || !h) return QG_ERR_NULL;
+    if (V < 1 || H < 1 || V > (int64_t(1) << 31) - 1) return QG_ERR_SHAPE;
+    if (!aligned(table, 2) || !aligned(token, 4) || !aligned(h, 4)) return QG_ERR_ALIGN;
+    return qg::launch_embedding_gather(table, V, H, token, h, stream);
+}
+
+qg_status qg_rmsnorm_gemv_s1(const qg_weight* W, const float* h, const uint16_t* gamma, float eps,
+                             float* y, uint16_t* y16, cudaStream_t stream) {
+    qg_status st = check_weight(W);
+    if (st != QG_OK) return st;
+    st = check_norm(h, gamma, eps);
+    if (st != QG_OK) return st;
+    if (!y && !y16) return QG_ERR_NULL;
+    if ((y && !aligned(y, 4)) || (y16 && !aligned(y16, 2))) return QG_ERR_ALIGN;
+    qg::GemvLaunch L = plain_launch(*W);
+    L.h_in = h;
+    L.gamma = gamma;
+    L.eps = eps;
+    L.y = y;
+    L.y16 = y16;
+    return qg::launch_gemv_s1(L, stream);
+}
+
+qg_status qg_gemv_s1_residual(const qg_weight* W, const uint16_t* x, float* h,
+                              cudaStream_t stream) {
+    qg_status st = check_weight(W);
+    if (st != QG_OK) return st;
+    if (!x || !h) return QG_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(h, 4)) return QG_ERR_ALIGN;
+    qg::GemvLaunch L = plain_launch(*W);
+    L.x = x;
+    L.h_res = h;
+    return qg::launch_gemv_s1(L, stream);
+}
+
+qg_status qg_rmsnorm_gate_up_swiglu(const qg_weight* Wg, const qg_weight* Wu, const float* h,
+                                    const uint16_t* gamma, float eps, uint16_t* H,
+                                    cudaStream_t stream) {
+    qg_status st = check_weight(Wg);
+    if (st != QG_OK) return st;
+    st = check_weight(Wu);
+    if (st != QG_OK) return st;
+    if (Wg->fmt != Wu->fmt || Wg->fmt == QG_FMT_F16) return QG_ERR_FORMAT;
+    if (Wg->n != Wu->n || Wg->k != Wu->k) return QG_ERR_SHAPE;
+    st = check_norm(h, gamma, eps);
+    if (st != QG_OK) return st;
+    if (!H) return QG_ERR_NULL;
+    if (!aligned(H, 2)) return QG_ERR_ALIGN;
+    qg::GemvLaunch L = plain_launch(*Wg);
+    L.epilogue = qg::kEpiSwiglu;
+    L.nmat = 2;
+    L.codes[1] = Wu->codes;
+    L.scales[1] = Wu->scales;
+    L.biases[1] = Wu->biases;
+    L.h_in = h;
+    L.gamma = gamma;
+    L.eps = eps;
+    L.h = H;
+    return qg::launch_gemv_s1(L, stream);
+}
+
+qg_status qg_rmsnorm_head_argmax(const qg_weight* W, const float* h, const uint16_t* gamma,
+                                 float eps, float* logits, int32_t* idx, void* workspace,
+                                 size_t ws_bytes, cudaStream_t stream) {
+    qg_status st = check_weight(W);
+    if (st != QG_OK) return st;
+    st = check_norm(h, gamma, eps);
+    if (st != QG_OK) return st;
+    if (!idx) return QG_ERR_NULL;
+    if (!workspace || ws_bytes < qg::kHeadWorkspaceBytes) return QG_ERR_WORKSPACE;
+    if ((logits && !aligned(logits, 4)) || !aligned(idx, 4) || !aligned(workspace, 16))
+        return QG_ERR_ALIGN;
+    qg::GemvLaunch L = plain_launch(*W);
+    L.epilogue = qg::kEpiHead;
+    L.h_in = h;
+    L.gamma = gamma;
+    L.eps = eps;
+    L.logits = logits;
+    L.idx = idx;
+    L.workspace = workspace;
+    return qg::launch_gemv_s1(L, stream);
+}
+
 qg_status qg_stream_check(cudaStream_t stream) {
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return qg::cuda_status(e);
     const unsigned int g = qg::gemv_read_and_clear_error();
     const unsigned int f = g | qg::gemm_s16_read_and_clear_error();
     if (g & qg::kGemvErrBadPlan) return QG_ERR_PLAN;
+    if (g & qg::kGemvErrToken) return QG_ERR_SHAPE;
     return f ? QG_ERR_TIMEOUT : QG_OK;
 }
 

@@ -79,6 +79,10 @@ struct Params {
     int x_words;         // 4-byte words reserved for the staged fp16 x in shared memory
     int prefetch_items;  // items per warp prefetched into L2 before the wait
     int x_bulk;          // ring path: x arrives by one bulk copy into a raw buffer
+    float eps;           // RMSNorm epsilon (with h_in)
+    const float* h_in;   // if set: x = RMSNorm(h_in; gamma, eps) instead of p.x
+    const uint16_t* gamma;
+    float* h_res;        // plain epilogue: if set, h_res[r] += y[r] (the residual stream)
 };
 
 __host__ __device__ constexpr int align_up(int v, int a) { return (v + a - 1) / a * a; }
@@ -201,23 +205,51 @@ struct Frag {
 // ------------------------------------------------------ shared kernel parts --
 // Stage x (fp16 in global memory, written by the previous kernel or by an
 // earlier stage of the same sweep, hence read through L2; or already copied
-// raw into shared memory, FROM_SMEM) into shared memory, still fp16, in the
+// raw into shared memory; or computed as an RMSNorm) into shared memory, still fp16, in the
 // conflict-free piece layout (int4: each 8-code word as the pairs the dot
 // product wants), and per lane granule the sums that remove the dot
 // products' constant terms:
 //   int8: sums[g] = 1152 sum x;
 //   int4: sums[2g] = 1024 sum_even x + 64 sum_odd x, sums[2g+1] = sum x.
-template <int FMT, bool FROM_SMEM = false>
+// Sources of x: kXGlobal (fp16 in global memory), kXShared (fp16 already in
+// shared memory), kXNorm (the RMSNorm of an fp32 hidden state: x = fp16(h *
+// rstd * gamma), rstd computed beforehand).
+enum XSource : int { kXGlobal = 0, kXShared = 1, kXNorm = 2 };
+
+__device__ __forceinline__ uint4 norm_piece(const float* h, const uint16_t* gamma, float rstd) {
+    // h: written by the previous kernel, which griddepcontrol.wait has made
+    // visible; read with plain (L1-cached) loads, hitting the lines that
+    // rmsnorm_rstd brought in.  (No stage of a persistent sweep takes an
+    // RMSNorm input, so no CTA of this grid writes h.)
+    const float4 a = *reinterpret_cast<const float4*>(h);
+    const float4 b = *reinterpret_cast<const float4*>(h + 4);
+    const uint4 gv = *reinterpret_cast<const uint4*>(gamma);
+    const float hv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float x0 = hv[2 * e] * rstd * h2f(static_cast<uint16_t>(gw[e] & 0xFFFFu));
+        const float x1 = hv[2 * e + 1] * rstd * h2f(static_cast<uint16_t>(gw[e] >> 16));
+        o[e] = static_cast<uint32_t>(f2h_rn(x0)) | (static_cast<uint32_t>(f2h_rn(x1)) << 16);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <int FMT, int SRC = kXGlobal>
 __device__ __forceinline__ void stage_x(const uint16_t* __restrict__ x, uint4* xs, float* sums,
-                                        int granules) {
+                                        int granules, const float* h = nullptr,
+                                        const uint16_t* gamma = nullptr, float rstd = 0.f) {
     using F = Fmt<FMT>;
     for (int g = threadIdx.x; g < granules; g += blockDim.x) {
-        const uint16_t* xg = x + static_cast<int64_t>(g) * F::kCodesPerLane;
+        const int64_t k0 = static_cast<int64_t>(g) * F::kCodesPerLane;
+        const uint16_t* xg = x + k0;
         float se = 0.f, so = 0.f;  // sums over even and odd k
 #pragma unroll
         for (int c = 0; c < F::kPieces; ++c) {
-            const uint4 v = FROM_SMEM ? *reinterpret_cast<const uint4*>(xg + 8 * c)
-                                      : ldg_cg_v4(xg + 8 * c);
+            const uint4 v = SRC == kXShared ? *reinterpret_cast<const uint4*>(xg + 8 * c)
+                          : SRC == kXGlobal ? ldg_cg_v4(xg + 8 * c)
+                                            : norm_piece(h + k0 + 8 * c, gamma + k0 + 8 * c, rstd);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -243,12 +275,47 @@ __device__ __forceinline__ void stage_x(const uint16_t* __restrict__ x, uint4* x
     }
 }
 
+// The residual stream's value at row r0 + lane, for lane < RG, read at the
+// start of an item so that its latency hides behind the item's steps.
+template <int RG, int EPI>
+__device__ __forceinline__ float residual_old(const Params& p, int64_t r0, int64_t N, int lane) {
+    if (EPI != kEpiPlain || p.h_res == nullptr || lane >= RG) return 0.f;
+    const int64_t r = r0 + lane < N ? r0 + lane : N - 1;
+    return p.h_res[r];
+}
+
+// The pre-norm RMSNorm's 1/rms of the fp32 hidden state h [k]: per-thread
+// sums of squares in index order, then the warp and the CTA in a fixed order;
+// every thread returns the same value.  red: kWarps floats of shared memory.
+__device__ __forceinline__ float rmsnorm_rstd(const float* h, const uint16_t* gamma, int64_t k,
+                                              float eps, float* red) {
+    float ss = 0.f;
+    for (int64_t i = threadIdx.x; i < k / 4; i += blockDim.x) {
+        const float4 v = *reinterpret_cast<const float4*>(h + 4 * i);
+        // bring the gains into L1 in the same round trip (the staging reads them)
+        if ((i & 1) == 0) asm volatile("prefetch.global.L1 [%0];" ::"l"(gamma + 4 * i));
+        ss = fmaf(v.x, v.x, ss);
+        ss = fmaf(v.y, v.y, ss);
+        ss = fmaf(v.z, v.z, ss);
+        ss = fmaf(v.w, v.w, ss);
+    }
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.f;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += red[w];
+    __syncthreads();  // red is free again
+    return __fdiv_rn(1.0f, __fsqrt_rn(__fdiv_rn(tot, static_cast<float>(k)) + eps));
+}
+
 // Finish the RG rows (x NMAT weights) of one warp item: reduce across lanes
-// and apply the epilogue; lane j writes row r0 + j.
+// and apply the epilogue; lane j writes row r0 + j.  h_old: lane j's value of
+// the residual stream at row r0 + j, read when the item started (no other
+// lane or CTA writes that row).
 template <int NMAT, int RG, int EPI>
 __device__ __forceinline__ void finish_item(float (&acc)[NMAT * RG], int64_t r0, int64_t N,
                                             const Params& p, int lane, float& best_v,
-                                            int& best_i) {
+                                            int& best_i, float h_old = 0.f) {
 #pragma unroll
     for (int j = 0; j < NMAT * RG; ++j) acc[j] = warp_sum(acc[j]);
     if (lane < RG && r0 + lane < N) {
@@ -263,6 +330,7 @@ __device__ __forceinline__ void finish_item(float (&acc)[NMAT * RG], int64_t r0,
         if (EPI == kEpiPlain) {
             if (p.y) p.y[r] = v0;
             if (p.y16) p.y16[r] = f2h_rn(v0);
+            if (p.h_res) p.h_res[r] = h_old + v0;  // residual stream (one lane owns the row)
         } else if (EPI == kEpiSwiglu) {
             p.h[r] = f2h_rn(v0 / (1.0f + expf(-v0)) * v1);
         } else {
@@ -429,7 +497,12 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
 
     // 2) x from the previous kernel
     griddep_wait();
-    stage_x<FMT>(p.x, xs, sums, granules);
+    if (p.h_in) {
+        const float rstd = rmsnorm_rstd(p.h_in, p.gamma, K, p.eps, red_v);
+        stage_x<FMT, kXNorm>(p.x, xs, sums, granules, p.h_in, p.gamma, rstd);
+    } else {
+        stage_x<FMT>(p.x, xs, sums, granules);
+    }
     __syncthreads();
     griddep_launch_dependents();
 
@@ -442,7 +515,9 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
     float best_v = -FLT_MAX;
     int best_i = INT_MAX;
     int cu_st = 0, cu_item = 0;
+    float h_old = 0.f;
     auto consume = [&](const Frag<ROWS>& f) {
+        if (cu_st == 0) h_old = residual_old<RG, EPI>(p, (wg + cu_item * tw) * RG, N, lane);
         const int g = cu_st * kLanes + lane;
         if (g < granules) {
             uint4 xv[F::kPieces];
@@ -461,7 +536,8 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
             }
         }
         if (++cu_st == nst) {
-            finish_item<NMAT, RG, EPI>(acc, (wg + cu_item * tw) * RG, N, p, lane, best_v, best_i);
+            finish_item<NMAT, RG, EPI>(acc, (wg + cu_item * tw) * RG, N, p, lane, best_v, best_i,
+                                       h_old);
             cu_st = 0;
             ++cu_item;
         }
@@ -696,7 +772,10 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
             cp_async_wait<0>();
             return false;
         }
-        stage_x<FMT, true>(xraw, xs, sums, granules);
+        stage_x<FMT, kXShared>(xraw, xs, sums, granules);
+    } else if (p.h_in) {
+        const float rstd = rmsnorm_rstd(p.h_in, p.gamma, K, p.eps, red_v);
+        stage_x<FMT, kXNorm>(p.x, xs, sums, granules, p.h_in, p.gamma, rstd);
     } else {
         stage_x<FMT>(p.x, xs, sums, granules);
     }
@@ -713,7 +792,9 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
     float best_v = -FLT_MAX;
     int best_i = INT_MAX;
     int cu_st = 0, cu_item = 0, cu_slot = 0;
+    float h_old = 0.f;
     for (int t = 0; t < total; ++t) {
+        if (cu_st == 0) h_old = residual_old<RG, EPI>(p, (wg + cu_item * tw) * RG, N, lane);
         if (t + kRing - 1 < total) issue();
         else cp_async_commit();
         cp_async_wait<kRing - 1>();
@@ -745,7 +826,8 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
         __syncwarp();  // every lane is done with this slot before it is refilled
         if (++cu_slot == kRing) cu_slot = 0;
         if (++cu_st == nst) {
-            finish_item<NMAT, RG, EPI>(acc, (wg + cu_item * tw) * RG, N, p, lane, best_v, best_i);
+            finish_item<NMAT, RG, EPI>(acc, (wg + cu_item * tw) * RG, N, p, lane, best_v, best_i,
+                                       h_old);
             cu_st = 0;
             ++cu_item;
         }
@@ -835,7 +917,7 @@ qg_status launch_pick(const Params& p0, const DeviceInfo& dev, cudaStream_t stre
     Params p = p0;
     const bool even_sides = !Fmt<FMT>::kScales || (p.k / Fmt<FMT>::kBlock) % 8 == 0;
     if (even_sides) {
-        p.x_bulk = 1;
+        p.x_bulk = p.h_in ? 0 : 1;  // an RMSNorm input is computed, not copied
         if (x_smem_bytes(FMT, p) + ring_smem_bytes<FMT, NMAT, RG>() <= kSmemPerCtaBudget)
             return launch_t<FMT, NMAT, RG, EPI, true>(p, dev, stream);
         p.x_bulk = 0;
@@ -901,7 +983,7 @@ static_assert(sizeof(SweepHeader) == 256, "header is 256 bytes");
 struct SweepStage {
     Params p;
     int32_t variant;
-    int32_t reserved[3];
+    int32_t reserved[5];
 };
 
 __host__ __device__ constexpr size_t align256(size_t v) { return (v + 255) / 256 * 256; }
@@ -1015,6 +1097,10 @@ Params make_params(const GemvLaunch& L) {
     p.h = L.h;
     p.logits = L.logits;
     p.idx = L.idx;
+    p.h_in = L.h_in;
+    p.gamma = L.gamma;
+    p.eps = L.eps;
+    p.h_res = L.h_res;
     p.ws_key = static_cast<unsigned long long*>(L.workspace);
     p.ws_ticket = L.workspace
                       ? reinterpret_cast<unsigned int*>(static_cast<char*>(L.workspace) + 8)
@@ -1050,7 +1136,7 @@ int sweep_variant(int kernel, const GemvLaunch& L, Params* p, int total_warps, i
     }
     const int nmat = swiglu ? 2 : 1;
     for (int rg = pick_rg(L.n, max_rg, total_warps); rg >= 1; rg /= 2) {
-        p->x_bulk = 1;  // x by bulk copy if its raw buffer fits too
+        p->x_bulk = p->h_in ? 0 : 1;  // x by bulk copy if its raw buffer fits too
         if (x_smem_bytes(L.fmt, *p) + ring_bytes(L.fmt, nmat * rg) > kSmemPerCtaBudget)
             p->x_bulk = 0;
         if (x_smem_bytes(L.fmt, *p) + ring_bytes(L.fmt, nmat * rg) > kSmemPerCtaBudget) continue;
@@ -1151,6 +1237,40 @@ qg_status launch_gemv_s1(const GemvLaunch& L, cudaStream_t stream) {
     if (L.fmt == QG_FMT_I8_B32) return dispatch_fmt<0>(L, p, dev, stream);
     if (L.fmt == QG_FMT_I4_G64) return dispatch_fmt<1>(L, p, dev, stream);
     return dispatch_fmt<2>(L, p, dev, stream);
+}
+
+// h[i] = fp32(table[token][i]): the embedding row of the token the previous
+// step chose ("Qwen3.8-27B ... -- Core AI", The vision path: the host gathers
+// text rows from the fp16 embedding table; here the row is gathered on the
+// device from the device-side argmax, so a decode loop never leaves the GPU).
+__global__ void __launch_bounds__(256) embedding_gather_kernel(const uint16_t* table, int64_t V,
+                                                               int64_t H, const int32_t* token,
+                                                               float* h) {
+    griddep_wait();  // the token may be the previous kernel's argmax
+    const int32_t t = *token;
+    if (t < 0 || t >= V) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(&g_gemv_err, kGemvErrToken);
+        return;
+    }
+    const uint16_t* row = table + static_cast<int64_t>(t) * H;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < H;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        h[i] = h2f(row[i]);
+    griddep_launch_dependents();
+}
+
+qg_status launch_embedding_gather(const uint16_t* table, int64_t V, int64_t H,
+                                  const int32_t* token, float* h, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((H + 1023) / 1024));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, embedding_gather_kernel, table, V, H, token, h));
 }
 
 unsigned int gemv_read_and_clear_error() {

@@ -41,6 +41,10 @@ struct GemvLaunch {
     float* logits;        // head: fp32 out or NULL
     int32_t* idx;         // head: argmax out
     void* workspace;      // head: zeroed scratch (key + ticket)
+    const float* h_in;    // if set: x = RMSNorm(h_in; gamma, eps) (x ignored)
+    const uint16_t* gamma;
+    float eps;
+    float* h_res;         // plain: if set, h_res += y (the residual stream)
 };
 qg_status launch_gemv_s1(const GemvLaunch& L, cudaStream_t stream);
 
@@ -56,7 +60,12 @@ qg_status launch_sweep(int kernel, void* ws, int n_stages, cudaStream_t stream);
 // no plan of that many stages.
 constexpr unsigned int kGemvErrTimeout = 1u;
 constexpr unsigned int kGemvErrBadPlan = 2u;
+constexpr unsigned int kGemvErrToken = 4u;  // embedding gather: token id out of range
 unsigned int gemv_read_and_clear_error();
+
+// h[i] = fp32(table[token][i]) for the device-side token id.
+qg_status launch_embedding_gather(const uint16_t* table, int64_t V, int64_t H,
+                                  const int32_t* token, float* h, cudaStream_t stream);
 
 // Quantizers.
 qg_status launch_quantize_block32(const float* w, int64_t n, int64_t k, int8_t* codes,

@@ -31,7 +31,8 @@ ABI_SYMBOLS = ("qg_quantize_block32", "qg_quantize_int4_g64", "qg_gemv_s1",
                "qg_gemm_s16", "qg_gate_up_swiglu", "qg_head_argmax_workspace_bytes",
                "qg_head_argmax", "qg_stream_check", "qg_status_string", "qg_abi_version",
                "qg_last_cuda_error", "qg_head_argmax_noalloc", "qg_sweep_workspace_bytes",
-               "qg_sweep_plan", "qg_sweep_run")
+               "qg_sweep_plan", "qg_sweep_run", "qg_embedding_gather", "qg_rmsnorm_gemv_s1",
+               "qg_rmsnorm_gate_up_swiglu", "qg_rmsnorm_head_argmax", "qg_gemv_s1_residual")
 STAGE_GEMV, STAGE_SWIGLU, STAGE_HEAD_ARGMAX = 0, 1, 2
 
 
@@ -91,6 +92,12 @@ def lib() -> ctypes.CDLL:
         L.qg_sweep_plan.argtypes = [ctypes.POINTER(CStage), I, P, ctypes.c_size_t,
                                     ctypes.POINTER(CSweep)]
         L.qg_sweep_run.argtypes = [ctypes.POINTER(CSweep), P, P]
+        F = ctypes.c_float
+        L.qg_embedding_gather.argtypes = [P, I64, I64, P, P, P]
+        L.qg_rmsnorm_gemv_s1.argtypes = [W, P, P, F, P, P, P]
+        L.qg_rmsnorm_gate_up_swiglu.argtypes = [W, W, P, P, F, P, P]
+        L.qg_rmsnorm_head_argmax.argtypes = [W, P, P, F, P, P, P, ctypes.c_size_t, P]
+        L.qg_gemv_s1_residual.argtypes = [W, P, P, P]
         L.qg_stream_check.argtypes = [P]
         L.qg_status_string.argtypes = [I]
         L.qg_status_string.restype = ctypes.c_char_p
@@ -349,3 +356,68 @@ class SweepPlan:
 
     def run(self, stream=None) -> None:
         qg_sweep_run(self.sweep, self.workspace, stream)
+
+
+# ------------------------------------------------------ decode-step fusions --
+def qg_embedding_gather(table: torch.Tensor, token: torch.Tensor, h: torch.Tensor,
+                        stream=None) -> None:
+    """h = fp32(table[token]) for the device-side token id (int32 [1])."""
+    _cuda(table, torch.float16, "table")
+    _cuda(token, torch.int32, "token")
+    _cuda(h, torch.float32, "h")
+    V, H = table.shape
+    _check("qg_embedding_gather", lib().qg_embedding_gather(_ptr(table), V, H, _ptr(token),
+                                                            _ptr(h), _stream(stream)))
+
+
+def _norm_args(h, gamma):
+    _cuda(h, torch.float32, "h")
+    _cuda(gamma, torch.float16, "gamma")
+
+
+def qg_rmsnorm_gemv_s1(W: QWeight, h: torch.Tensor, gamma: torch.Tensor, eps: float,
+                       y: Optional[torch.Tensor] = None, y16: Optional[torch.Tensor] = None,
+                       stream=None) -> None:
+    _norm_args(h, gamma)
+    if y is not None:
+        _cuda(y, torch.float32, "y")
+    if y16 is not None:
+        _cuda(y16, torch.float16, "y16")
+    cw = W.c()
+    _check("qg_rmsnorm_gemv_s1",
+           lib().qg_rmsnorm_gemv_s1(ctypes.byref(cw), _ptr(h), _ptr(gamma), float(eps), _ptr(y),
+                                    _ptr(y16), _stream(stream)))
+
+
+def qg_gemv_s1_residual(W: QWeight, x: torch.Tensor, h: torch.Tensor, stream=None) -> None:
+    """h += W x (the residual stream)."""
+    _cuda(x, torch.float16, "x")
+    _cuda(h, torch.float32, "h")
+    cw = W.c()
+    _check("qg_gemv_s1_residual",
+           lib().qg_gemv_s1_residual(ctypes.byref(cw), _ptr(x), _ptr(h), _stream(stream)))
+
+
+def qg_rmsnorm_gate_up_swiglu(Wg: QWeight, Wu: QWeight, h: torch.Tensor, gamma: torch.Tensor,
+                              eps: float, H: torch.Tensor, stream=None) -> None:
+    _norm_args(h, gamma)
+    _cuda(H, torch.float16, "H")
+    cg, cu = Wg.c(), Wu.c()
+    _check("qg_rmsnorm_gate_up_swiglu",
+           lib().qg_rmsnorm_gate_up_swiglu(ctypes.byref(cg), ctypes.byref(cu), _ptr(h),
+                                           _ptr(gamma), float(eps), _ptr(H), _stream(stream)))
+
+
+def qg_rmsnorm_head_argmax(W: QWeight, h: torch.Tensor, gamma: torch.Tensor, eps: float,
+                           idx: torch.Tensor, workspace: torch.Tensor,
+                           logits: Optional[torch.Tensor] = None, stream=None) -> None:
+    _norm_args(h, gamma)
+    _cuda(idx, torch.int32, "idx")
+    _cuda(workspace, torch.uint8, "workspace")
+    if logits is not None:
+        _cuda(logits, torch.float32, "logits")
+    cw = W.c()
+    _check("qg_rmsnorm_head_argmax",
+           lib().qg_rmsnorm_head_argmax(ctypes.byref(cw), _ptr(h), _ptr(gamma), float(eps),
+                                        _ptr(logits), _ptr(idx), _ptr(workspace),
+                                        workspace.numel(), _stream(stream)))

@@ -15,6 +15,18 @@ output.  With S = 16 (chunked prefill) every projection runs on the tensor-core
 path with a [16, K] chunk, o reads a fresh seeded chunk, and the head reads the
 chunk's last row.
 
+With decode_step=True (S = 1) the sweep is a whole decode step minus
+attention instead, carrying a real fp32 hidden state h from token to token:
+
+    h = E[token]                                     (embedding gather)
+    per layer:  qkv = W_qkv RMSNorm(h)               (y16 = fp16 q|k|v)
+                h  += W_o  fp16(q)                   (attention stand-in)
+                hh  = SwiGLU(W_g, W_u; RMSNorm(h))
+                h  += W_down hh
+    token = argmax( W_head RMSNorm(h) )               (the next step's token)
+
+so a graph of several sweeps is an autoregressive chain.
+
 At S = 1 the sweep runs either as 4 launches per layer + 1 (one per call, with
 programmatic dependent launch between them) or as ONE persistent launch that
 runs the same stages in the same order (qg_sweep_plan / qg_sweep_run); the two
@@ -48,18 +60,22 @@ class DecodeSweep:
 
     def __init__(self, dec: wl.Decoder, body_fmt: int = qg.FMT_I8_B32,
                  head_fmt: int = qg.FMT_I8_B32, S: int = 1, device="cuda",
-                 keep_logits: bool = False):
+                 keep_logits: bool = False, decode_step: bool = False, eps: float = 1e-6):
         assert 1 <= S <= 16
         self.dec, self.S, self.device = dec, S, torch.device(device)
         self.body_fmt, self.head_fmt = body_fmt, head_fmt
         if S > 1:
             assert body_fmt == qg.FMT_I8_B32 and head_fmt == qg.FMT_I8_B32
         assert body_fmt != qg.FMT_F16, "fp16 weights serve the head only"
+        assert not decode_step or S == 1, "the decode step runs S = 1"
+        self.decode_step, self.eps = decode_step, eps
         self.layers: List[LayerWeights] = []
         for l in range(dec.layers):
             self.layers.append(self._make_layer(l))
         self.head = self._quantized("head", -1, dec.vocab, dec.hidden, head_fmt)
         self._make_buffers(keep_logits)
+        if decode_step:
+            self._make_decode_state()
         self.graph: Optional[torch.cuda.CUDAGraph] = None
         self.plan: Optional[qg.SweepPlan] = None
 
@@ -119,6 +135,17 @@ class DecodeSweep:
         self.idx = torch.zeros(1, dtype=torch.int32, device=dev)
         self.ws = qg.head_workspace(d.vocab, dev)
 
+    def _make_decode_state(self) -> None:
+        d, dev = self.dec, self.device
+        # the fp16 embedding table (for a tied head the same draw the head
+        # was quantized from), the RMSNorm gains, the hidden state and token
+        self.embed = wl.weight_fp32(d.vocab, d.hidden, d.weight_seed(-1, "embed"), dev).half()
+        self.gamma_attn = [wl.gamma_fp16(d.hidden, d.gamma_seed(l, 0), dev) for l in range(d.layers)]
+        self.gamma_mlp = [wl.gamma_fp16(d.hidden, d.gamma_seed(l, 1), dev) for l in range(d.layers)]
+        self.gamma_final = wl.gamma_fp16(d.hidden, d.gamma_seed(-1, 0), dev)
+        self.hstate = torch.zeros(d.hidden, dtype=torch.float32, device=dev)
+        self.idx.fill_(1)  # the first step's token
+
     # ------------------------------------------------------------- sweep --
     @property
     def weight_bytes(self) -> int:
@@ -128,10 +155,15 @@ class DecodeSweep:
         return b + self.head.nbytes
 
     def launches_per_sweep(self, persistent: bool = False) -> int:
-        return 1 if persistent else 4 * self.dec.layers + 1
+        if persistent:
+            return 1
+        return 4 * self.dec.layers + (2 if self.decode_step else 1)
 
     def inputs(self) -> List[torch.Tensor]:
-        """The per-step activation tensors (contiguous), in a fixed order."""
+        """The per-step input tensors (contiguous), in a fixed order: the
+        activations, or for the decode step the token it starts from."""
+        if self.decode_step:
+            return [self.idx]
         return [self.x_all] if self.x_o_all is None else [self.x_all, self.x_o_all]
 
     def head_input(self) -> torch.Tensor:
@@ -140,7 +172,15 @@ class DecodeSweep:
     def run_layer(self, l: int, stream=None) -> None:
         """Enqueue layer l's four launches on `stream` (default: current)."""
         d, L = self.dec, self.layers[l]
-        if self.S == 1:
+        if self.decode_step:
+            h = self.hstate
+            qg.qg_rmsnorm_gemv_s1(L.qkv, h, self.gamma_attn[l], self.eps, self.y_qkv[0],
+                                  self.y16_qkv, stream)
+            qg.qg_gemv_s1_residual(L.o, self.y16_qkv[: d.q_dim], h, stream)
+            qg.qg_rmsnorm_gate_up_swiglu(L.gate, L.up, h, self.gamma_mlp[l], self.eps, self.h[0],
+                                         stream)
+            qg.qg_gemv_s1_residual(L.down, self.h[0], h, stream)
+        elif self.S == 1:
             qg.qg_gemv_s1(L.qkv, self.x[l], self.y_qkv[0], self.y16_qkv, stream)
             qg.qg_gemv_s1(L.o, self.y16_qkv[: d.q_dim], self.y_o[0], None, stream)
             qg.qg_gate_up_swiglu(L.gate, L.up, self.x[l], self.h[0], stream)
@@ -152,11 +192,20 @@ class DecodeSweep:
             qg.qg_gemm_s16(L.down, self.h, self.y_down, stream)
 
     def run_head(self, stream=None) -> None:
+        if self.decode_step:
+            qg.qg_rmsnorm_head_argmax(self.head, self.hstate, self.gamma_final, self.eps, self.idx,
+                                      self.ws, self.logits, stream)
+            return
         qg.qg_head_argmax(self.head, self.head_input(), self.idx, self.ws, self.logits, stream)
+
+    def run_embed(self, stream=None) -> None:
+        """h = E[token], the token the previous step chose."""
+        qg.qg_embedding_gather(self.embed, self.idx, self.hstate, stream)
 
     def stages(self) -> List[qg.CStage]:
         """The S = 1 sweep as persistent-launch stages, in run_layer's order."""
         assert self.S == 1, "the persistent sweep runs S = 1 stages"
+        assert not self.decode_step, "the persistent sweep has no RMSNorm or residual stages"
         d, st = self.dec, []
         for l, L in enumerate(self.layers):
             st.append(qg.stage_gemv(L.qkv, self.x[l], self.y_qkv[0], self.y16_qkv))
@@ -177,6 +226,8 @@ class DecodeSweep:
         if persistent:
             self.make_plan().run(stream)
             return
+        if self.decode_step:
+            self.run_embed(stream)
         for l in range(self.dec.layers):
             self.run_layer(l, stream)
         self.run_head(stream)

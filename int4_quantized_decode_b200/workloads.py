@@ -32,7 +32,7 @@ W_STD = 0.02
 
 # proj ids used in weight seeds
 PROJ_ID = {"q": 0, "k": 1, "v": 2, "o": 3, "gate": 4, "up": 5, "down": 6,
-           "outgate": 7, "head": 15}
+           "outgate": 7, "embed": 14, "head": 15}
 
 
 @dataclass(frozen=True)
@@ -85,9 +85,16 @@ class Decoder:
 
     # --- seeds ------------------------------------------------------------
     def weight_seed(self, layer: int, proj: str) -> int:
-        if proj == "head":
-            return 1000 * self.seed_id + PROJ_ID["head"]
+        if proj == "head" or (proj == "embed" and self.tied_head):
+            return 1000 * self.seed_id + PROJ_ID["head"]  # a tied head is the embedding
+        if proj == "embed":
+            return 1000 * self.seed_id + PROJ_ID["embed"]
         return 1000 * self.seed_id + 16 * layer + PROJ_ID[proj]
+
+    def gamma_seed(self, layer: int, which: int) -> int:
+        """Seed of an RMSNorm gain vector: which 0 = before attention, 1 =
+        before the MLP; layer -1 = the final norm before the head."""
+        return 700000 + 1000 * self.seed_id + 2 * (layer if layer >= 0 else 499) + which
 
     def x_seed(self, layer: int) -> int:
         """Seed of the fresh fp16 activation of layer ``layer`` (-1: head)."""
@@ -149,3 +156,8 @@ def sample_rows(n: int, count: int, seed: int) -> torch.Tensor:
     idx = torch.randperm(n, generator=g)[: max(count - 2, 0)]
     idx = torch.cat([idx, torch.tensor([0, n - 1])])
     return torch.unique(idx).sort().values
+
+
+def gamma_fp16(k: int, seed: int, device="cuda") -> torch.Tensor:
+    """RMSNorm gains: fp16 = RNE(1 + 0.1 N(0, 1)) drawn like the activations."""
+    return (1.0 + 0.1 * act_fp16(k, seed, device).float()).half()

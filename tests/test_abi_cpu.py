@@ -45,7 +45,7 @@ def test_status_strings_and_version(L):
     for code, name in qg.STATUS_NAMES.items():
         assert qg.status_string(code).startswith(name)
     assert qg.status_string(99) == "QG_ERR_UNKNOWN"
-    assert L.qg_abi_version() == 101
+    assert L.qg_abi_version() == 102
     assert L.qg_head_argmax_workspace_bytes(151936) >= 16
 
 
@@ -157,3 +157,22 @@ def test_fp16_weight_validation(L):
     w = W(fmt=2, k=64, scales=0)
     assert L.qg_gate_up_swiglu(ctypes.byref(w), ctypes.byref(w), 0x4000, 1, 0x6000, None) == 4
     assert L.qg_gemm_s16(ctypes.byref(w), 0x4000, 4, 0x5000, None) == 4
+
+
+def test_decode_step_validation(L):
+    w = W()
+    h, g = 0x8000, 0x9000
+    assert L.qg_embedding_gather(None, 10, 64, 0x4000, h, None) == 1
+    assert L.qg_embedding_gather(0x1000, 0, 64, 0x4000, h, None) == 2
+    assert L.qg_embedding_gather(0x1001, 10, 64, 0x4000, h, None) == 3
+    assert L.qg_rmsnorm_gemv_s1(ctypes.byref(w), None, g, 1e-6, 0x5000, None, None) == 1
+    assert L.qg_rmsnorm_gemv_s1(ctypes.byref(w), h, g, -1.0, 0x5000, None, None) == 2
+    assert L.qg_rmsnorm_gemv_s1(ctypes.byref(w), h + 4, g, 1e-6, 0x5000, None, None) == 3
+    assert L.qg_rmsnorm_gemv_s1(ctypes.byref(w), h, g, 1e-6, None, None, None) == 1
+    assert L.qg_gemv_s1_residual(ctypes.byref(w), 0x4000, None, None) == 1
+    assert L.qg_gemv_s1_residual(ctypes.byref(w), 0x4008, h, None) == 3
+    wf = W(fmt=2, k=64, scales=0)
+    assert L.qg_rmsnorm_gate_up_swiglu(ctypes.byref(wf), ctypes.byref(wf), h, g, 1e-6, 0x6000,
+                                       None) == 4
+    assert L.qg_rmsnorm_head_argmax(ctypes.byref(w), h, g, 1e-6, None, 0x7000, 0x7100, 8,
+                                    None) == 5

@@ -1,0 +1,190 @@
+"""The decode step around the weight stream: embedding gather, RMSNorm fused
+into the S=1 calls, residual adds, vs the fp64 oracle (teacher-forced on the
+device's own hidden state)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import assert_within_bound, bits, oracle_gemv
+from int4_quantized_decode_b200 import qgemv as qg
+from int4_quantized_decode_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+I8, I4, F16 = qg.FMT_I8_B32, qg.FMT_I4_G64, qg.FMT_F16
+EPS = 1e-6
+TOL = oracle.GEMV_TOL + 2.0 ** -10  # plus one fp16 ulp of the device-rounded x
+
+
+def _weight(fmt, n, k, seed, dev):
+    w = wl.weight_fp32(n, k, seed, dev)
+    return qg.QWeight.fp16(w.half()) if fmt == F16 else qg.quantize(w, fmt)
+
+
+def _hidden(k, seed, dev, scale=3.0):
+    return (wl.weight_fp32(1, k, seed, dev)[0] * (scale / 0.02)).contiguous()
+
+
+def _gamma(k, seed, dev):
+    return (1.0 + 0.1 * wl.act_fp16(k, seed, dev).float()).half()
+
+
+def _x_ref(h, gamma, dev):
+    xb, _ = oracle.rmsnorm(h.cpu().numpy(), bits(gamma), EPS)
+    return torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.float16)
+
+
+@pytest.mark.parametrize("fmt,n,k", [(I8, 300, 2048), (I8, 4096, 2560), (I4, 1000, 2560),
+                                     (I8, 2048, 6144), (F16, 777, 4096), (I8, 20001, 5120)])
+def test_rmsnorm_gemv(cuda, fmt, n, k):
+    W = _weight(fmt, n, k, 800 + n % 7, cuda)
+    h, gam = _hidden(k, 801, cuda), _gamma(k, 802, cuda)
+    y = torch.full((n,), float("nan"), dtype=torch.float32, device=cuda)
+    y16 = torch.empty(n, dtype=torch.float16, device=cuda)
+    qg.qg_rmsnorm_gemv_s1(W, h, gam, EPS, y, y16)
+    qg.qg_stream_check()
+    yr, mag = oracle_gemv(W, _x_ref(h, gam, cuda))
+    yd = y.cpu().numpy()
+    assert_within_bound(yd, yr, mag, TOL)
+    assert np.array_equal(bits(y16), oracle.f32_to_f16_bits(yd))
+
+
+@pytest.mark.parametrize("fmt,n,k", [(I8, 2048, 2048), (I4, 2560, 9728), (I8, 5120, 17408)])
+def test_residual_add(cuda, fmt, n, k):
+    W = _weight(fmt, n, k, 810, cuda)
+    x = wl.act_fp16(k, 811, cuda)
+    h0 = _hidden(n, 812, cuda)
+    h = h0.clone()
+    qg.qg_gemv_s1_residual(W, x, h)
+    qg.qg_stream_check()
+    yr, mag = oracle_gemv(W, x)
+    hn, ho = h.cpu().numpy().astype(np.float64), h0.cpu().numpy().astype(np.float64)
+    err = np.abs(hn - (ho + yr))
+    assert np.all(err <= oracle.GEMV_TOL * mag + np.spacing(np.abs(hn).astype(np.float32)))
+
+
+@pytest.mark.parametrize("fmt,n,k", [(I8, 6144, 2048), (I4, 9728, 2560)])
+def test_rmsnorm_gate_up_swiglu(cuda, fmt, n, k):
+    Wg, Wu = _weight(fmt, n, k, 820, cuda), _weight(fmt, n, k, 821, cuda)
+    h, gam = _hidden(k, 822, cuda), _gamma(k, 823, cuda)
+    H = torch.empty(n, dtype=torch.float16, device=cuda)
+    qg.qg_rmsnorm_gate_up_swiglu(Wg, Wu, h, gam, EPS, H)
+    qg.qg_stream_check()
+    x = _x_ref(h, gam, cuda)
+    gr, mg = oracle_gemv(Wg, x)
+    ur, mu = oracle_gemv(Wu, x)
+    hr, hb = oracle.swiglu(gr, ur, mg, mu, TOL)
+    assert np.all(np.abs(H.cpu().numpy().astype(np.float64) - hr) <= hb)
+
+
+@pytest.mark.parametrize("fmt,V,k", [(I8, 151936, 2048), (F16, 151936, 2048), (I4, 20000, 2560)])
+def test_rmsnorm_head_argmax(cuda, fmt, V, k):
+    W = _weight(fmt, V, k, 830, cuda)
+    h, gam = _hidden(k, 831, cuda), _gamma(k, 832, cuda)
+    idx = torch.full((1,), -1, dtype=torch.int32, device=cuda)
+    logits = torch.empty(V, dtype=torch.float32, device=cuda)
+    ws = qg.head_workspace(V, cuda)
+    qg.qg_rmsnorm_head_argmax(W, h, gam, EPS, idx, ws, logits)
+    qg.qg_stream_check()
+    yr, mag = oracle_gemv(W, _x_ref(h, gam, cuda))
+    assert_within_bound(logits.cpu().numpy(), yr, mag, TOL)
+    assert oracle.argmax_ok(int(idx.item()), yr)
+    assert int(ws.sum().item()) == 0
+
+
+def test_embedding_gather_exact_and_out_of_range(cuda):
+    V, H = 151936, 2048
+    E = wl.weight_fp32(V, H, 840, cuda).half()
+    h = torch.full((H,), float("nan"), dtype=torch.float32, device=cuda)
+    for t in (0, 12345, V - 1):
+        tok = torch.tensor([t], dtype=torch.int32, device=cuda)
+        qg.qg_embedding_gather(E, tok, h)
+        qg.qg_stream_check()
+        assert torch.equal(h, E[t].float())
+    before = h.clone()
+    for bad in (V, -1):
+        qg.qg_embedding_gather(E, torch.tensor([bad], dtype=torch.int32, device=cuda), h)
+        with pytest.raises(qg.QgError, match="QG_ERR_SHAPE"):
+            qg.qg_stream_check()
+        assert torch.equal(h, before)
+
+
+def test_decode_step_chain_2b(cuda):
+    """The 2B-shaped decode step minus attention, teacher-forced op by op on the
+    device's own state: gather, every norm-fused projection of the first and
+    the last layer (sampled rows), the residual stream, the head's argmax; then
+    the graph of two chained steps equals two eager steps bit for bit, and the
+    second step starts from the first step's token."""
+    import gc
+    from int4_quantized_decode_b200.sweep import DecodeSweep
+    d = wl.QWEN3VL_2B
+    sw = DecodeSweep(d, I8, I8, S=1, device=cuda, keep_logits=True, decode_step=True)
+    try:
+        tok0 = int(sw.idx.item())
+        sw.run_embed()
+        qg.qg_stream_check()
+        assert torch.equal(sw.hstate, sw.embed[tok0].float())
+        rows = wl.sample_rows(d.hidden, 64, 5).tolist()
+        for l in range(d.layers):
+            L = sw.layers[l]
+            check = l in (0, d.layers - 1)
+            h0 = sw.hstate.clone()
+            qg.qg_rmsnorm_gemv_s1(L.qkv, sw.hstate, sw.gamma_attn[l], sw.eps, sw.y_qkv[0],
+                                  sw.y16_qkv)
+            if check:
+                x = _x_ref(h0, sw.gamma_attn[l], cuda)
+                r = wl.sample_rows(d.qkv_rows, 64, 6).tolist()
+                yr, mag = oracle_gemv(L.qkv, x, r)
+                assert_within_bound(sw.y_qkv[0].cpu().numpy()[r], yr, mag, TOL)
+            xo = sw.y16_qkv[: d.q_dim].clone()
+            qg.qg_gemv_s1_residual(L.o, sw.y16_qkv[: d.q_dim], sw.hstate)
+            if check:
+                yr, mag = oracle_gemv(L.o, xo, rows)
+                dh = (sw.hstate.cpu().numpy().astype(np.float64) - h0.cpu().numpy())[rows]
+                assert np.all(np.abs(dh - yr) <= oracle.GEMV_TOL * mag +
+                              np.spacing(np.abs(sw.hstate.cpu().numpy()[rows])))
+            h1 = sw.hstate.clone()
+            qg.qg_rmsnorm_gate_up_swiglu(L.gate, L.up, sw.hstate, sw.gamma_mlp[l], sw.eps,
+                                         sw.h[0])
+            if check:
+                x = _x_ref(h1, sw.gamma_mlp[l], cuda)
+                r = wl.sample_rows(d.inter, 64, 7).tolist()
+                gr, mg = oracle_gemv(L.gate, x, r)
+                ur, mu = oracle_gemv(L.up, x, r)
+                hr, hb = oracle.swiglu(gr, ur, mg, mu, TOL)
+                assert np.all(np.abs(sw.h[0].cpu().numpy().astype(np.float64)[r] - hr) <= hb)
+            hh = sw.h[0].clone()
+            qg.qg_gemv_s1_residual(L.down, sw.h[0], sw.hstate)
+            if check:
+                yr, mag = oracle_gemv(L.down, hh, rows)
+                dh = (sw.hstate.cpu().numpy().astype(np.float64) - h1.cpu().numpy())[rows]
+                assert np.all(np.abs(dh - yr) <= oracle.GEMV_TOL * mag +
+                              np.spacing(np.abs(sw.hstate.cpu().numpy()[rows])))
+        hf = sw.hstate.clone()
+        sw.run_head()
+        qg.qg_stream_check()
+        assert np.all(np.isfinite(hf.cpu().numpy()))
+        yr, mag = oracle_gemv(sw.head, _x_ref(hf, sw.gamma_final, cuda))
+        assert_within_bound(sw.logits.cpu().numpy(), yr, mag, TOL)
+        tok1 = int(sw.idx.item())
+        assert oracle.argmax_ok(tok1, yr)
+        # two chained steps in one graph == two eager steps from the same start
+        sw.idx.fill_(tok0)
+        sw.step()
+        sw.step()
+        qg.qg_stream_check()
+        eager = (int(sw.idx.item()), sw.hstate.clone(), sw.logits.clone())
+        g = sw.capture(sweeps_per_graph=2)
+        sw.idx.fill_(tok0)
+        g.replay()
+        qg.qg_stream_check()
+        assert int(sw.idx.item()) == eager[0]
+        assert torch.equal(sw.hstate, eager[1]) and torch.equal(sw.logits, eager[2])
+        sw.idx.fill_(tok0)
+        sw.step()
+        qg.qg_stream_check()
+        assert int(sw.idx.item()) == tok1  # the first step alone chooses tok1 again
+    finally:
+        del sw
+        gc.collect()
+        torch.cuda.empty_cache()
