@@ -143,8 +143,10 @@ QG_API qg_status qg_gemv_s1(const qg_weight* W, const uint16_t* x, float* y,
  * through the same weights ("Qwen3.8-27B ... -- Core AI", The vision path:
  * a static S=16 'prefill' chunk beside the S=1 'main' decode).
  *   Y[s, r] = sum_k X[s, k] * w_dq[r, k],   0 <= s < S
- * W : the weight (int8 block-32 only; QG_ERR_FORMAT for int4).  For S > 1,
- *     k % 512 == 0 (QG_ERR_SHAPE otherwise); S == 1 runs qg_gemv_s1.
+ * W : the weight (int8 block-32 only; QG_ERR_FORMAT for int4 and fp16
+ *     weights).  For S > 1, k % 512 == 0 (QG_ERR_SHAPE otherwise); S == 1
+ *     runs qg_gemv_s1.  For S > 1 each weight enters the tensor cores as
+ *     fp16(q * s), one rounding.
  * X : fp16 [S, k] row-major, 16-byte aligned.   1 <= S <= 16.
  * Y : fp32 [S, n] out, 4-byte aligned.
  * Accuracy: each row s obeys the qg_gemv_s1 bound for x = X[s].
@@ -160,7 +162,7 @@ QG_API qg_status qg_gemm_s16(const qg_weight* W, const uint16_t* X, int S, float
  *   silu(g) = g / (1 + exp(-g))
  * Wg, Wu : weights of identical format and shape [n = intermediate, k].
  *          S == 1 accepts int8 or int4; S > 1 (tensor cores) int8 only,
- *          with k % 512 == 0.
+ *          with k % 512 == 0 (fp16 weights: QG_ERR_FORMAT).
  * X      : fp16 [S, k], 16-byte aligned.   1 <= S <= 16.
  * H      : fp16 [S, n] out, 2-byte aligned.
  * ------------------------------------------------------------------------- */

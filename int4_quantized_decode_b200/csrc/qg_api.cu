@@ -426,7 +426,7 @@ qg_status qg_rmsnorm_head_argmax(const qg_weight* W, const float* h, const uint1
 qg_status qg_stream_check(cudaStream_t stream) {
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return qg::cuda_status(e);
-    const unsigned int g = qg::gemv_read_and_clear_error();
+    const unsigned int g = qg::gemv_read_and_clear_error() | qg::gemv_decode_read_and_clear_error();
     const unsigned int f = g | qg::gemm_s16_read_and_clear_error();
     if (g & qg::kGemvErrBadPlan) return QG_ERR_PLAN;
     if (g & qg::kGemvErrToken) return QG_ERR_SHAPE;

@@ -21,8 +21,12 @@ qg_status device_info(DeviceInfo* out);
 qg_status cuda_status(cudaError_t e);
 const char* last_cuda_error_name();
 
-// Epilogues of the S=1 streaming kernel.
-enum GemvEpilogue : int { kEpiPlain = 0, kEpiSwiglu = 1, kEpiHead = 2 };
+// Epilogues of the S=1 streaming kernel.  kEpiResidual (h_res += y) and the
+// flag kEpiNormIn (x = RMSNorm of an fp32 hidden state) are chosen by the
+// launcher from h_res / h_in; callers set one of the first three.
+enum GemvEpilogue : int { kEpiPlain = 0, kEpiSwiglu = 1, kEpiHead = 2, kEpiResidual = 3 };
+constexpr int kEpiNormIn = 8;
+__host__ __device__ constexpr int epi_kind(int epi) { return epi & 7; }
 
 // One S=1 streaming launch: NMAT (1 or 2) weights of identical format and
 // shape, one fp16 activation, one of three epilogues.
@@ -47,6 +51,8 @@ struct GemvLaunch {
     float* h_res;         // plain: if set, h_res += y (the residual stream)
 };
 qg_status launch_gemv_s1(const GemvLaunch& L, cudaStream_t stream);
+// The decode-step variants (h_in or h_res set), compiled on their own.
+qg_status launch_gemv_s1_decode(const GemvLaunch& L, cudaStream_t stream);
 
 // Persistent sweep: n S=1 stages (validated GemvLaunch descriptions, head
 // workspaces ignored) planned into a device workspace, then run as one
@@ -62,6 +68,7 @@ constexpr unsigned int kGemvErrTimeout = 1u;
 constexpr unsigned int kGemvErrBadPlan = 2u;
 constexpr unsigned int kGemvErrToken = 4u;  // embedding gather: token id out of range
 unsigned int gemv_read_and_clear_error();
+unsigned int gemv_decode_read_and_clear_error();
 
 // h[i] = fp32(table[token][i]) for the device-side token id.
 qg_status launch_embedding_gather(const uint16_t* table, int64_t V, int64_t H,
