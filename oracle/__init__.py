@@ -84,6 +84,10 @@ def lib():
         L.orc_f64_to_f16.restype = ctypes.c_uint16
         L.orc_rmsnorm.argtypes = [P, P, I64, D, P, P]
         L.orc_rmsnorm.restype = None
+        L.orc_rope.argtypes = [P, I64, I64, D, P]
+        L.orc_rope.restype = None
+        L.orc_decode_attention.argtypes = [P, I64, I64, I64, P, P, I64, I64, D, P, P, P, P]
+        L.orc_decode_attention.restype = None
         L.orc_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -279,3 +283,31 @@ def rmsnorm(h, gamma_bits, eps: float):
     xe = np.empty(k, dtype=np.float64)
     lib().orc_rmsnorm(_p(h), _p(g), k, float(eps), _p(x), _p(xe))
     return x, xe
+
+
+def rope(x, pos: int, theta: float):
+    """RoPE (rotate-half pairing) of one head vector at position pos, fp64."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty_like(x)
+    lib().orc_rope(_p(x), x.shape[0], int(pos), float(theta), _p(out))
+    return out
+
+
+def decode_attention(qkv, hq: int, hkv: int, d: int, kcache, vcache, pos: int, theta: float):
+    """One decode step's attention (see orc_decode_attention): returns
+    (o fp64 [hq*d], mag fp64 [hq*d], k_new fp16 bits [hkv*d], v_new fp16 bits [hkv*d]).
+    kcache / vcache: fp16 bits [hkv, l_max, d]; rows 0..pos-1 are read."""
+    qkv = np.ascontiguousarray(qkv, dtype=np.float32)
+    kc = np.ascontiguousarray(kcache, dtype=np.uint16)
+    vc = np.ascontiguousarray(vcache, dtype=np.uint16)
+    assert qkv.shape == ((hq + 2 * hkv) * d,) and hq % hkv == 0
+    assert kc.shape == vc.shape and kc.shape[0] == hkv and kc.shape[2] == d
+    l_max = kc.shape[1]
+    assert 0 <= pos < l_max
+    o = np.empty(hq * d, dtype=np.float64)
+    mag = np.empty(hq * d, dtype=np.float64)
+    k_new = np.empty(hkv * d, dtype=np.uint16)
+    v_new = np.empty(hkv * d, dtype=np.uint16)
+    lib().orc_decode_attention(_p(qkv), hq, hkv, d, _p(kc), _p(vc), l_max, int(pos),
+                               float(theta), _p(k_new), _p(v_new), _p(o), _p(mag))
+    return o, mag, k_new, v_new

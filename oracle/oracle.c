@@ -276,6 +276,76 @@ void orc_rmsnorm(const float* h, const uint16_t* gamma, int64_t k, double eps, u
     }
 }
 
+/* --------------------------------------------------- decode attention --- */
+
+void orc_rope(const double* x, int64_t d, int64_t pos, double theta, double* out) {
+    const int64_t half = d / 2;
+    for (int64_t i = 0; i < half; ++i) {
+        const double f = pow(theta, -2.0 * (double)i / (double)d);
+        const double a = (double)pos * f;
+        const double c = cos(a), s = sin(a);
+        out[i] = x[i] * c - x[i + half] * s;
+        out[i + half] = x[i + half] * c + x[i] * s;
+    }
+}
+
+void orc_decode_attention(const float* qkv, int64_t hq, int64_t hkv, int64_t d,
+                          const uint16_t* kcache, const uint16_t* vcache, int64_t l_max,
+                          int64_t pos, double theta, uint16_t* k_new, uint16_t* v_new,
+                          double* o, double* mag) {
+    const int64_t group = hq / hkv;
+    const double scale = 1.0 / sqrt((double)d);
+    double* xin = (double*)malloc((size_t)d * sizeof(double));
+    double* rot = (double*)malloc((size_t)d * sizeof(double));
+    double* kj = (double*)malloc((size_t)d * sizeof(double));
+    double* s = (double*)malloc((size_t)(pos + 1) * sizeof(double));
+    /* the appended rows */
+    for (int64_t g = 0; g < hkv; ++g) {
+        for (int64_t i = 0; i < d; ++i) xin[i] = (double)qkv[hq * d + g * d + i];
+        orc_rope(xin, d, pos, theta, rot);
+        for (int64_t i = 0; i < d; ++i) {
+            k_new[g * d + i] = orc_f64_to_f16(rot[i]);
+            v_new[g * d + i] = orc_f64_to_f16((double)qkv[hq * d + hkv * d + g * d + i]);
+        }
+    }
+    for (int64_t h = 0; h < hq; ++h) {
+        const int64_t g = h / group;
+        for (int64_t i = 0; i < d; ++i) xin[i] = (double)qkv[h * d + i];
+        orc_rope(xin, d, pos, theta, rot);
+        double m = -HUGE_VAL;
+        for (int64_t j = 0; j <= pos; ++j) {
+            for (int64_t i = 0; i < d; ++i)
+                kj[i] = orc_f16_to_f64(j == pos ? k_new[g * d + i]
+                                                : kcache[(g * l_max + j) * d + i]);
+            double dot = 0.0;
+            for (int64_t i = 0; i < d; ++i) dot += rot[i] * kj[i];
+            s[j] = dot * scale;
+            if (s[j] > m) m = s[j];
+        }
+        double z = 0.0;
+        for (int64_t j = 0; j <= pos; ++j) {
+            s[j] = exp(s[j] - m);
+            z += s[j];
+        }
+        for (int64_t i = 0; i < d; ++i) {
+            double acc = 0.0, mg = 0.0;
+            for (int64_t j = 0; j <= pos; ++j) {
+                const double v = orc_f16_to_f64(j == pos ? v_new[g * d + i]
+                                                         : vcache[(g * l_max + j) * d + i]);
+                const double p = s[j] / z;
+                acc += p * v;
+                mg += p * fabs(v);
+            }
+            o[h * d + i] = acc;
+            mag[h * d + i] = mg;
+        }
+    }
+    free(xin);
+    free(rot);
+    free(kj);
+    free(s);
+}
+
 /* ------------------------------------------------------------- SwiGLU --- */
 
 double orc_silu(double g) { return g / (1.0 + exp(-g)); }

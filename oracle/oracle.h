@@ -114,6 +114,38 @@ double orc_ulp_f16(double v);
 /* Greedy argmax: the smallest index holding the largest value. */
 int64_t orc_argmax(const double* v, int64_t n);
 
+/* ------------------------------------------------------ decode attention ---
+ * The attention core of one decode step of the pages' Qwen3-VL decoders
+ * ("Qwen3-VL (2B / 4B / 8B, vision-language) -- Core AI", architecture
+ * paragraph: pure attention, head_dim 128, 8 kv heads, rope theta 5e6;
+ * "Qwen3-VL 4B & 8B -- Core ML stateful", gotchas: for text positions the
+ * interleaved M-RoPE is exactly standard 1-D RoPE, and the rotary helper
+ * pairs the two halves of a head; "Qwen3-VL 2B -- Core AI", integration
+ * checklist: the KV cache is the engine's native K/V pair).  Readings where
+ * the pages are silent: no per-head q/k norm, softmax scale 1/sqrt(d).
+ *
+ * RoPE of one head x[d] at position pos (rotate-half pairing, fp64):
+ *   f_i = theta^(-2i/d),  a = pos * f_i,  for i < d/2:
+ *   out[i]       = x[i] cos a - x[i+d/2] sin a
+ *   out[i+d/2]   = x[i+d/2] cos a + x[i] sin a */
+void orc_rope(const double* x, int64_t d, int64_t pos, double theta, double* out);
+
+/* One decode step's attention for the token at position pos:
+ *   qkv    fp32 [hq*d | hkv*d | hkv*d]: q, k, v of the token (the q|k|v
+ *          projection's output);
+ *   kcache, vcache fp16 bits [hkv][l_max][d]: rows 0..pos-1 hold the
+ *          earlier tokens (already rotated keys); row pos is not read;
+ *   k_new, v_new out fp16 bits [hkv*d]: the rows this token appends,
+ *          fp16_rne(RoPE(k)) and fp16_rne(v), which also stand in for row pos;
+ *   o, mag out fp64 [hq*d]: o = sum_j p_j v_j and mag = sum_j p_j |v_j| with
+ *          p = softmax_j( RoPE(q_h) . k_j / sqrt(d) ), j = 0..pos, query head
+ *          h reading kv head h / (hq / hkv).
+ * All arithmetic fp64 in index order (the max is subtracted before exp). */
+void orc_decode_attention(const float* qkv, int64_t hq, int64_t hkv, int64_t d,
+                          const uint16_t* kcache, const uint16_t* vcache, int64_t l_max,
+                          int64_t pos, double theta, uint16_t* k_new, uint16_t* v_new,
+                          double* o, double* mag);
+
 /* Threads the parallel row loops use (OpenMP). */
 int orc_num_threads(void);
 

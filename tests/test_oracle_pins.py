@@ -496,3 +496,120 @@ def test_rmsnorm_matches_independent_numpy():
         near_tie = np.abs(ref * 2.0 ** (10 - np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -14))))
                           % 1 - 0.5) < 1e-9
         assert np.array_equal(x[~near_tie], ref.astype(np.float16).view(np.uint16)[~near_tie])
+
+
+# ------------------------------------------------------ decode attention ---
+THETA = 5e6   # rope theta of the pages' Qwen3-VL decoders
+
+
+def test_rope_closed_forms():
+    rng = np.random.default_rng(51)
+    x = rng.normal(0, 1, 128)
+    assert np.array_equal(oracle.rope(x, 0, THETA), x)              # position 0: identity
+    # d = 2: one pair at frequency theta^0 = 1, the textbook rotation by pos radians
+    for pos in (1, 7, 1000):
+        r = oracle.rope(np.array([0.6, -0.8]), pos, THETA)
+        c, s = math.cos(pos), math.sin(pos)
+        np.testing.assert_allclose(r, [0.6 * c + 0.8 * s, -0.8 * c + 0.6 * s], rtol=0, atol=1e-14)
+    # pairs are (i, i + d/2) and each rotation keeps its pair's length
+    r = oracle.rope(x, 12345, THETA)
+    np.testing.assert_allclose(r[:64] ** 2 + r[64:] ** 2, x[:64] ** 2 + x[64:] ** 2, rtol=1e-12)
+    # a unit vector on dimension 64 + i turns into dimension i with -sin
+    e = np.zeros(128)
+    e[64 + 5] = 1.0
+    r = oracle.rope(e, 3, THETA)
+    a = 3 * THETA ** (-2 * 5 / 128)
+    np.testing.assert_allclose([r[5], r[64 + 5]], [-math.sin(a), math.cos(a)], atol=1e-15)
+    assert np.count_nonzero(r) == 2
+
+
+def test_rope_scores_depend_on_relative_position_only():
+    rng = np.random.default_rng(52)
+    q, k = rng.normal(0, 1, 128), rng.normal(0, 1, 128)
+    s0 = oracle.rope(q, 40, THETA) @ oracle.rope(k, 15, THETA)
+    for shift in (1, 100, 5000):
+        s = oracle.rope(q, 40 + shift, THETA) @ oracle.rope(k, 15 + shift, THETA)
+        assert abs(s - s0) <= 1e-9 * (np.abs(q) @ np.abs(k))
+    # and not on the absolute one: moving only the key changes the score
+    assert abs(oracle.rope(q, 40, THETA) @ oracle.rope(k, 16, THETA) - s0) > 1e-6
+
+
+def _attn_inputs(rng, hq, hkv, d, l_max, pos):
+    qkv = rng.normal(0, 1, (hq + 2 * hkv) * d).astype(np.float32)
+    kc = np_f16_bits(rng.normal(0, 1, (hkv, l_max, d)))
+    vc = np_f16_bits(rng.normal(0, 1, (hkv, l_max, d)))
+    return qkv, kc, vc
+
+
+def test_attention_first_token_returns_its_value():
+    """pos = 0: one key, softmax weight 1, so every head returns its kv head's
+    (fp16) value row; the appended key is fp16(RoPE(k)) = fp16(k) at position 0."""
+    rng = np.random.default_rng(53)
+    hq, hkv, d = 16, 8, 128
+    qkv, kc, vc = _attn_inputs(rng, hq, hkv, d, 4, 0)
+    o, mag, kn, vn = oracle.decode_attention(qkv, hq, hkv, d, kc, vc, 0, THETA)
+    k = qkv[hq * d:(hq + hkv) * d]
+    v = qkv[(hq + hkv) * d:]
+    assert np.array_equal(kn, np_f16_bits(k.astype(np.float64)))
+    assert np.array_equal(vn, np_f16_bits(v.astype(np.float64)))
+    vrow = f16_np(vn).astype(np.float64).reshape(hkv, d)
+    np.testing.assert_array_equal(o.reshape(hq, d), np.repeat(vrow, hq // hkv, axis=0))
+    np.testing.assert_array_equal(mag.reshape(hq, d), np.abs(np.repeat(vrow, hq // hkv, axis=0)))
+
+
+def test_attention_zero_query_is_the_mean_and_pins_the_head_groups():
+    """q = 0: every score is 0, the weights uniform, so head h returns the
+    mean of its kv head's value rows (kv head h // (hq/hkv))."""
+    rng = np.random.default_rng(54)
+    hq, hkv, d, l_max, pos = 32, 8, 128, 12, 9
+    qkv, kc, vc = _attn_inputs(rng, hq, hkv, d, l_max, pos)
+    qkv[:hq * d] = 0.0
+    o, _, _, vn = oracle.decode_attention(qkv, hq, hkv, d, kc, vc, pos, THETA)
+    rows = f16_np(vc).astype(np.float64)[:, :pos, :]
+    allv = np.concatenate([rows, f16_np(vn).astype(np.float64).reshape(hkv, 1, d)], axis=1)
+    want = np.repeat(allv.mean(axis=1), hq // hkv, axis=0)
+    np.testing.assert_allclose(o.reshape(hq, d), want, rtol=0, atol=1e-14)
+
+
+def test_attention_matches_numpy_softmax_brute_force():
+    rng = np.random.default_rng(55)
+    for hq, hkv, d, l_max, pos in ((4, 2, 8, 9, 6), (16, 8, 128, 40, 33), (6, 3, 16, 5, 4)):
+        qkv, kc, vc = _attn_inputs(rng, hq, hkv, d, l_max, pos)
+        o, mag, kn, vn = oracle.decode_attention(qkv, hq, hkv, d, kc, vc, pos, THETA)
+        K = f16_np(kc).astype(np.float64).copy()
+        V = f16_np(vc).astype(np.float64).copy()
+        K[:, pos, :] = f16_np(kn).astype(np.float64).reshape(hkv, d)
+        V[:, pos, :] = f16_np(vn).astype(np.float64).reshape(hkv, d)
+        for h in range(hq):
+            g = h // (hq // hkv)
+            q = oracle.rope(qkv[h * d:(h + 1) * d].astype(np.float64), pos, THETA)
+            s = K[g, :pos + 1] @ q / math.sqrt(d)
+            p = np.exp(s - s.max())
+            p /= p.sum()
+            np.testing.assert_allclose(o[h * d:(h + 1) * d], p @ V[g, :pos + 1], rtol=1e-12,
+                                       atol=1e-13)
+            np.testing.assert_allclose(mag[h * d:(h + 1) * d], p @ np.abs(V[g, :pos + 1]),
+                                       rtol=1e-12, atol=1e-13)
+
+
+def test_attention_scale_and_dominant_key():
+    """Two positions with scores a and b give weights e^a / (e^a + e^b): with
+    q = c e_0 at position 0 (no rotation) and keys e_0, 0 the first weight is
+    1 / (1 + e^(-c/sqrt(d))), pinning the 1/sqrt(d) scale; a large c makes the
+    matching key dominate."""
+    hq, hkv, d, l_max = 2, 1, 128, 4
+    for c in (3.0, 1000.0):
+        qkv = np.zeros((hq + 2 * hkv) * d, np.float32)
+        qkv[0] = qkv[d] = c                           # both query heads: c e_0
+        qkv[(hq + hkv) * d:] = 0.25                   # the new token's value row
+        kc = np.zeros((hkv, l_max, d), np.uint16)
+        vc = np.zeros((hkv, l_max, d), np.uint16)
+        kc[0, 0, 0] = np_f16_bits(np.array([1.0]))[0]  # key of position 0: e_0
+        vc[0, 0, :] = np_f16_bits(np.array([-1.0]))[0]
+        # pos = 1: the new key is fp16(RoPE(0)) = 0, score 0; position 0 scores
+        # RoPE(c e_0, 1) . e_0 / sqrt(d) = c cos(1) / sqrt(d)
+        o, _, _, _ = oracle.decode_attention(qkv, hq, hkv, d, kc, vc, 1, THETA)
+        a = c * math.cos(1.0) / math.sqrt(d)
+        w0 = 1.0 / (1.0 + math.exp(-a))
+        np.testing.assert_allclose(o[:d], np.full(d, w0 * -1.0 + (1 - w0) * 0.25), rtol=1e-13)
+    assert abs(o[0] + 1.0) < 1e-15                    # c = 1000: position 0 dominates
