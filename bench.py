@@ -41,11 +41,13 @@ UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 
-# name -> (decoder, body format, head format, S[, decode step])
+# name -> (decoder, body format, head format, S[, decode step[, K/V cache rows]])
 WORKLOADS = {
     "qwen3vl-2b": ("QWEN3VL_2B", 0, 0, 1),
     "qwen3vl-2b-f16head": ("QWEN3VL_2B", 0, 2, 1),
     "qwen3vl-2b-decode": ("QWEN3VL_2B", 0, 0, 1, True),
+    "qwen3vl-2b-decode-attn4k": ("QWEN3VL_2B", 0, 0, 1, True, 4096),
+    "qwen3vl-8b-decode-attn4k": ("QWEN3VL_8B", 0, 0, 1, True, 4096),
     "qwen3vl-4b": ("QWEN3VL_4B", 0, 0, 1),
     "qwen3vl-4b-int4": ("QWEN3VL_4B", 1, 0, 1),
     "qwen3vl-8b": ("QWEN3VL_8B", 0, 0, 1),
@@ -284,14 +286,28 @@ def _sweep_bytes(dec, body_fmt, head_fmt):
                dec.vocab * dec.hidden * bpw[head_fmt])
 
 
+def _context(workload):
+    w = WORKLOADS[workload]
+    return w[5] if len(w) > 5 else 0
+
+
 def _config(a, dec, body_fmt, head_fmt, S, sweep_bytes):
     decode = len(WORKLOADS[a.workload]) > 4
+    ctx = _context(a.workload)
+    if ctx:
+        step = (f", whole decode step (embedding gather, RMSNorm and residual fused, "
+                f"RoPE + GQA attention over a {ctx}-row fp16 K/V cache per layer at its last "
+                f"row; the argmax feeds the next step's gather); value counts weight bytes "
+                f"only, the K/V rows read are kv_bytes")
+    elif decode:
+        step = (", whole decode step minus attention (embedding gather, RMSNorm and residual "
+                "fused; the argmax feeds the next step's gather)")
+    else:
+        step = ""
     return {
         "workload": (f"{dec.name}-shaped decode weight sweep, {FMT_NAME[body_fmt]} body + "
                      f"{FMT_NAME[head_fmt]} head{' (tied)' if dec.tied_head else ''}, "
-                     f"S={S}" + (", whole decode step minus attention (embedding gather, "
-                                 "RMSNorm and residual fused; the argmax feeds the next "
-                                 "step's gather)" if decode else "")),
+                     f"S={S}" + step),
         "layers": dec.layers, "hidden": dec.hidden, "inter": dec.inter,
         "vocab": dec.vocab, "S": S, "sweep_bytes": sweep_bytes,
         "parallelism": f"replicas x{a.gpus}",
@@ -326,7 +342,8 @@ def run_ours(a):
     dname, body_fmt, head_fmt, S = WORKLOADS[a.workload][:4]
     decode = len(WORKLOADS[a.workload]) > 4
     dec = getattr(wl, dname)
-    sw = DecodeSweep(dec, body_fmt, head_fmt, S=S, device=dev, decode_step=decode)
+    sw = DecodeSweep(dec, body_fmt, head_fmt, S=S, device=dev, decode_step=decode,
+                     context=_context(a.workload))
     persistent = a.path == "persistent"
     if a.path == "persistent" and S != 1:
         raise SystemExit("--path persistent needs an S=1 workload")
@@ -379,7 +396,10 @@ def run_ours(a):
         "data": "synthetic (seeded N(0,0.02) weights, N(0,1) fp16 activations)",
         "config": dict(_config(a, dec, body_fmt, head_fmt, S, sweep_bytes),
                        path="persistent (one launch per sweep)" if persistent
-                       else "one launch per call"),
+                       else "one launch per call",
+                       **({"kv_bytes": sw.kv_bytes,
+                           "gbs_incl_kv": round(value * (sweep_bytes + sw.kv_bytes) /
+                                                sweep_bytes, 2)} if sw.kv_bytes else {})),
         "sweeps_per_s": round(sweeps_s, 2),
         "tokens_per_s": round(sweeps_s * S, 2),
         "hbm_frac": round(value / world / peak, 4),

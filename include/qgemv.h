@@ -259,6 +259,42 @@ QG_API qg_status qg_gemv_s1_residual(const qg_weight* W, const uint16_t* x, floa
                                      cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * qg_decode_attention -- the attention core of one decode step over an fp16
+ * K/V cache, for the pages' Qwen3-VL decoders ("Qwen3-VL (2B / 4B / 8B,
+ * vision-language) -- Core AI", architecture paragraph: pure attention,
+ * head_dim 128, 8 kv heads, rope theta 5e6; "Qwen3-VL 4B & 8B -- Core ML
+ * stateful", gotchas: for text positions the interleaved M-RoPE is standard
+ * 1-D RoPE with the two halves of a head paired; "Qwen3-VL 2B -- Core AI",
+ * integration checklist: the KV cache is the native K/V pair).  Readings
+ * where the pages are silent: no per-head q/k norm, scale 1/sqrt(d).
+ *   RoPE(x, p)[i]       = x[i] cos(p f_i) - x[i+d/2] sin(p f_i)
+ *   RoPE(x, p)[i + d/2] = x[i+d/2] cos(p f_i) + x[i] sin(p f_i),  f_i = theta^(-2i/d)
+ *   the token at position p = *pos appends K[g][p] = fp16_rne(RoPE(k_g, p)),
+ *   V[g][p] = fp16_rne(v_g), then for every query head h (kv head g = h/(hq/hkv))
+ *   o_h = fp16_rne( sum_{j <= p} softmax_j( RoPE(q_h, p) . K[g][j] / sqrt(d) ) V[g][j] )
+ * qkv    : fp32 [hq*d | hkv*d | hkv*d], the q|k|v projection's output, 16-byte
+ *          aligned.
+ * kcache, vcache : fp16 [hkv][l_max][d], 16-byte aligned; rows 0..p-1 hold the
+ *          earlier tokens (rotated keys), row p is written by this call.
+ * pos    : device int32 [1]; outside [0, l_max) the call writes nothing and
+ *          qg_stream_check reports QG_ERR_SHAPE.
+ * o      : fp16 [hq*d] out, 16-byte aligned (the o projection's input).
+ * d == 128 and hq / hkv in {1, 2, 4} (QG_ERR_SHAPE otherwise); theta > 0.
+ * workspace : device memory of at least qg_decode_attention_workspace_bytes,
+ *          256-byte aligned, ZEROED ONCE before first use.  Its first 256
+ *          bytes hold per-kv-head counters that every call leaves zeroed again;
+ *          the rest is scratch for the split partials.  Calls sharing one
+ *          workspace must be serialized.
+ * Accuracy: |o - o_ref| <= 1e-3 * sum_j p_j |V[g][j]| + ulp_f16(o_ref) per
+ * element, o_ref the fp64 attention on the same fp16 cache.  Deterministic.
+ * ------------------------------------------------------------------------- */
+QG_API size_t qg_decode_attention_workspace_bytes(int hq, int hkv);
+QG_API qg_status qg_decode_attention(const float* qkv, int hq, int hkv, int d,
+                                     uint16_t* kcache, uint16_t* vcache, int64_t l_max,
+                                     const int32_t* pos, double theta, uint16_t* o,
+                                     void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * qg_sweep_* -- a whole one-token decode step as ONE persistent launch.
  * A decode step reads every decoder weight once ("Qwen3-VL 4B -- Core AI
  * (.aimodel)", Measured), as an ordered chain of S=1 projections per layer

@@ -152,7 +152,7 @@ qg_status stage_launch(const qg_stage& S, qg::GemvLaunch* out) {
 
 extern "C" {
 
-int qg_abi_version(void) { return 102; }
+int qg_abi_version(void) { return 103; }
 
 const char* qg_last_cuda_error(void) { return qg::last_cuda_error_name(); }
 
@@ -346,6 +346,40 @@ qg_status qg_embedding_gather(const uint16_t* table, int64_t V, int64_t H, const
     return qg::launch_embedding_gather(table, V, H, token, h, stream);
 }
 
+size_t qg_decode_attention_workspace_bytes(int hq, int hkv) {
+    if (hq < 1 || hkv < 1 || hq % hkv != 0) return 0;
+    return qg::decode_attention_workspace_bytes(hq, hkv);
+}
+
+qg_status qg_decode_attention(const float* qkv, int hq, int hkv, int d, uint16_t* kcache,
+                              uint16_t* vcache, int64_t l_max, const int32_t* pos, double theta,
+                              uint16_t* o, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (!qkv || !kcache || !vcache || !pos || !o || !workspace) return QG_ERR_NULL;
+    if (hkv < 1 || hq < hkv || hq % hkv != 0 || l_max < 1 || l_max > (int64_t(1) << 31) - 1)
+        return QG_ERR_SHAPE;
+    const int group = hq / hkv;
+    if (d != 128 || (group != 1 && group != 2 && group != 4)) return QG_ERR_SHAPE;
+    if (!(theta > 0.0)) return QG_ERR_SHAPE;
+    if (!aligned(qkv, 16) || !aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(pos, 4) ||
+        !aligned(o, 16) || !aligned(workspace, 256))
+        return QG_ERR_ALIGN;
+    if (ws_bytes < qg::decode_attention_workspace_bytes(hq, hkv)) return QG_ERR_WORKSPACE;
+    qg::AttentionLaunch L = {};
+    L.qkv = qkv;
+    L.kcache = kcache;
+    L.vcache = vcache;
+    L.l_max = l_max;
+    L.hq = hq;
+    L.hkv = hkv;
+    L.d = d;
+    L.pos = pos;
+    L.theta = theta;
+    L.o = o;
+    L.workspace = workspace;
+    L.ws_bytes = ws_bytes;
+    return qg::launch_decode_attention(L, stream);
+}
+
 qg_status qg_rmsnorm_gemv_s1(const qg_weight* W, const float* h, const uint16_t* gamma, float eps,
                              float* y, uint16_t* y16, cudaStream_t stream) {
     qg_status st = check_weight(W);
@@ -428,8 +462,9 @@ qg_status qg_stream_check(cudaStream_t stream) {
     if (e != cudaSuccess) return qg::cuda_status(e);
     const unsigned int g = qg::gemv_read_and_clear_error() | qg::gemv_decode_read_and_clear_error();
     const unsigned int f = g | qg::gemm_s16_read_and_clear_error();
+    const unsigned int a = qg::attention_read_and_clear_error();  // a position out of range
     if (g & qg::kGemvErrBadPlan) return QG_ERR_PLAN;
-    if (g & qg::kGemvErrToken) return QG_ERR_SHAPE;
+    if ((g & qg::kGemvErrToken) || a) return QG_ERR_SHAPE;
     return f ? QG_ERR_TIMEOUT : QG_OK;
 }
 

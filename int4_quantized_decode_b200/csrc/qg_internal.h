@@ -81,6 +81,23 @@ qg_status launch_quantize_int4_g64(const float* w, int64_t n, int64_t k, uint8_t
                                    uint16_t* scales, uint16_t* biases, cudaStream_t stream);
 
 // S <= 16 tensor-core path (int8 block-32): plain (Y fp32) or SwiGLU (H fp16).
+// One decode step's attention core (qg_attention.cu).
+struct AttentionLaunch {
+    const float* qkv;       // fp32 [hq*d | hkv*d | hkv*d]
+    uint16_t* kcache;       // fp16 [hkv][l_max][d]
+    uint16_t* vcache;
+    int64_t l_max;
+    int hq, hkv, d;
+    const int32_t* pos;     // device
+    double theta;
+    uint16_t* o;            // fp16 [hq*d]
+    void* workspace;
+    size_t ws_bytes;
+};
+size_t decode_attention_workspace_bytes(int hq, int hkv);
+qg_status launch_decode_attention(const AttentionLaunch& L, cudaStream_t stream);
+unsigned int attention_read_and_clear_error();  // bit 0: position outside [0, l_max)
+
 struct GemmS16Launch {
     int epilogue;  // kEpiPlain or kEpiSwiglu
     int S;

@@ -32,7 +32,9 @@ ABI_SYMBOLS = ("qg_quantize_block32", "qg_quantize_int4_g64", "qg_gemv_s1",
                "qg_head_argmax", "qg_stream_check", "qg_status_string", "qg_abi_version",
                "qg_last_cuda_error", "qg_head_argmax_noalloc", "qg_sweep_workspace_bytes",
                "qg_sweep_plan", "qg_sweep_run", "qg_embedding_gather", "qg_rmsnorm_gemv_s1",
-               "qg_rmsnorm_gate_up_swiglu", "qg_rmsnorm_head_argmax", "qg_gemv_s1_residual")
+               "qg_rmsnorm_gate_up_swiglu", "qg_rmsnorm_head_argmax", "qg_gemv_s1_residual",
+               "qg_decode_attention_workspace_bytes", "qg_decode_attention")
+ROPE_THETA = 5e6  # rope theta of the pages' Qwen3-VL decoders
 STAGE_GEMV, STAGE_SWIGLU, STAGE_HEAD_ARGMAX = 0, 1, 2
 
 
@@ -98,6 +100,10 @@ def lib() -> ctypes.CDLL:
         L.qg_rmsnorm_gate_up_swiglu.argtypes = [W, W, P, P, F, P, P]
         L.qg_rmsnorm_head_argmax.argtypes = [W, P, P, F, P, P, P, ctypes.c_size_t, P]
         L.qg_gemv_s1_residual.argtypes = [W, P, P, P]
+        L.qg_decode_attention_workspace_bytes.argtypes = [I, I]
+        L.qg_decode_attention_workspace_bytes.restype = ctypes.c_size_t
+        L.qg_decode_attention.argtypes = [P, I, I, I, P, P, I64, P, ctypes.c_double, P, P,
+                                          ctypes.c_size_t, P]
         L.qg_stream_check.argtypes = [P]
         L.qg_status_string.argtypes = [I]
         L.qg_status_string.restype = ctypes.c_char_p
@@ -106,7 +112,8 @@ def lib() -> ctypes.CDLL:
         L.qg_last_cuda_error.restype = ctypes.c_char_p
         for name in ABI_SYMBOLS:
             if name not in ("qg_head_argmax_workspace_bytes", "qg_status_string",
-                            "qg_last_cuda_error", "qg_sweep_workspace_bytes"):
+                            "qg_last_cuda_error", "qg_sweep_workspace_bytes",
+                            "qg_decode_attention_workspace_bytes"):
                 getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -421,3 +428,37 @@ def qg_rmsnorm_head_argmax(W: QWeight, h: torch.Tensor, gamma: torch.Tensor, eps
            lib().qg_rmsnorm_head_argmax(ctypes.byref(cw), _ptr(h), _ptr(gamma), float(eps),
                                         _ptr(logits), _ptr(idx), _ptr(workspace),
                                         workspace.numel(), _stream(stream)))
+
+
+# ------------------------------------------------------- decode attention --
+def attention_workspace(hq: int, hkv: int, device="cuda") -> torch.Tensor:
+    """A zeroed workspace for qg_decode_attention (its counters stay zeroed
+    between calls; the rest is scratch)."""
+    n = lib().qg_decode_attention_workspace_bytes(hq, hkv)
+    if n == 0:
+        raise QgError("qg_decode_attention_workspace_bytes", 2)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def qg_decode_attention(qkv: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor,
+                        pos: torch.Tensor, o: torch.Tensor, workspace: torch.Tensor,
+                        theta: float = ROPE_THETA, stream=None) -> None:
+    """One decode step's attention: appends the token's rotated key and value
+    at row *pos of the fp16 caches [hkv, l_max, d] and writes o (fp16 [hq*d])
+    from the fp32 q|k|v projection output."""
+    _cuda(qkv, torch.float32, "qkv")
+    _cuda(kcache, torch.float16, "kcache")
+    _cuda(vcache, torch.float16, "vcache")
+    _cuda(pos, torch.int32, "pos")
+    _cuda(o, torch.float16, "o")
+    if kcache.dim() != 3 or kcache.shape != vcache.shape:
+        raise ValueError("kcache and vcache must both be [hkv, l_max, d]")
+    hkv, l_max, d = kcache.shape
+    hq = o.numel() // d
+    if o.numel() != hq * d or qkv.numel() != (hq + 2 * hkv) * d:
+        raise ValueError("qkv must be [(hq + 2 hkv) d] and o [hq d]")
+    _check("qg_decode_attention",
+           lib().qg_decode_attention(_ptr(qkv), hq, hkv, d, _ptr(kcache), _ptr(vcache), l_max,
+                                     _ptr(pos), float(theta), _ptr(o), _ptr(workspace),
+                                     workspace.numel(), _stream(stream)))
+

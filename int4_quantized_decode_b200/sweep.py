@@ -60,7 +60,8 @@ class DecodeSweep:
 
     def __init__(self, dec: wl.Decoder, body_fmt: int = qg.FMT_I8_B32,
                  head_fmt: int = qg.FMT_I8_B32, S: int = 1, device="cuda",
-                 keep_logits: bool = False, decode_step: bool = False, eps: float = 1e-6):
+                 keep_logits: bool = False, decode_step: bool = False, eps: float = 1e-6,
+                 context: int = 0):
         assert 1 <= S <= 16
         self.dec, self.S, self.device = dec, S, torch.device(device)
         self.body_fmt, self.head_fmt = body_fmt, head_fmt
@@ -68,7 +69,8 @@ class DecodeSweep:
             assert body_fmt == qg.FMT_I8_B32 and head_fmt == qg.FMT_I8_B32
         assert body_fmt != qg.FMT_F16, "fp16 weights serve the head only"
         assert not decode_step or S == 1, "the decode step runs S = 1"
-        self.decode_step, self.eps = decode_step, eps
+        assert context == 0 or decode_step, "attention runs inside the decode step"
+        self.decode_step, self.eps, self.context = decode_step, eps, context
         self.layers: List[LayerWeights] = []
         for l in range(dec.layers):
             self.layers.append(self._make_layer(l))
@@ -145,6 +147,28 @@ class DecodeSweep:
         self.gamma_final = wl.gamma_fp16(d.hidden, d.gamma_seed(-1, 0), dev)
         self.hstate = torch.zeros(d.hidden, dtype=torch.float32, device=dev)
         self.idx.fill_(1)  # the first step's token
+        if self.context:
+            # Attention over a K/V cache of `context` rows per layer: the step
+            # decodes the token at the last row; rows before it are seeded
+            # history (rotated keys and values ~ N(0, 1) in fp16).
+            hd = d.head_dim
+            assert not d.out_gate and d.q_dim % hd == 0 and d.kv_dim % hd == 0
+            hkv = d.kv_dim // hd
+            self.kcache, self.vcache = [], []
+            for l in range(d.layers):
+                self.kcache.append(wl.act_fp16((hkv, self.context, hd), d.kv_seed(l, 0), dev))
+                self.vcache.append(wl.act_fp16((hkv, self.context, hd), d.kv_seed(l, 1), dev))
+            self.pos = torch.full((1,), self.context - 1, dtype=torch.int32, device=dev)
+            self.attn_out = torch.empty(d.q_dim, dtype=torch.float16, device=dev)
+            self.attn_ws = qg.attention_workspace(d.q_dim // hd, hkv, dev)
+
+    @property
+    def kv_bytes(self) -> int:
+        """K/V cache bytes one decode step's attention reads (every row up to
+        and including the current position, both caches, every layer)."""
+        if not self.context:
+            return 0
+        return self.dec.layers * 2 * self.dec.kv_dim * self.context * 2
 
     # ------------------------------------------------------------- sweep --
     @property
@@ -157,7 +181,8 @@ class DecodeSweep:
     def launches_per_sweep(self, persistent: bool = False) -> int:
         if persistent:
             return 1
-        return 4 * self.dec.layers + (2 if self.decode_step else 1)
+        per_layer = 5 if self.context else 4
+        return per_layer * self.dec.layers + (2 if self.decode_step else 1)
 
     def inputs(self) -> List[torch.Tensor]:
         """The per-step input tensors (contiguous), in a fixed order: the
@@ -170,13 +195,19 @@ class DecodeSweep:
         return self.x_head if self.S == 1 else self.x_head[self.S - 1]
 
     def run_layer(self, l: int, stream=None) -> None:
-        """Enqueue layer l's four launches on `stream` (default: current)."""
+        """Enqueue layer l's launches on `stream` (default: current): four, five with
+        the attention of a decode step over a K/V cache."""
         d, L = self.dec, self.layers[l]
         if self.decode_step:
             h = self.hstate
             qg.qg_rmsnorm_gemv_s1(L.qkv, h, self.gamma_attn[l], self.eps, self.y_qkv[0],
                                   self.y16_qkv, stream)
-            qg.qg_gemv_s1_residual(L.o, self.y16_qkv[: d.q_dim], h, stream)
+            if self.context:
+                qg.qg_decode_attention(self.y_qkv[0], self.kcache[l], self.vcache[l], self.pos,
+                                       self.attn_out, self.attn_ws, stream=stream)
+                qg.qg_gemv_s1_residual(L.o, self.attn_out, h, stream)
+            else:
+                qg.qg_gemv_s1_residual(L.o, self.y16_qkv[: d.q_dim], h, stream)
             qg.qg_rmsnorm_gate_up_swiglu(L.gate, L.up, h, self.gamma_mlp[l], self.eps, self.h[0],
                                          stream)
             qg.qg_gemv_s1_residual(L.down, self.h[0], h, stream)

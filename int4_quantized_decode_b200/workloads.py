@@ -100,6 +100,15 @@ class Decoder:
         """Seed of the fresh fp16 activation of layer ``layer`` (-1: head)."""
         return 500000 + 1000 * self.seed_id + (layer if layer >= 0 else 999)
 
+    def kv_seed(self, layer: int, which: int) -> int:
+        """Seed of layer ``layer``'s synthetic K (which 0) or V (which 1)
+        cache history: the rows earlier decode steps would have written."""
+        return 800000 + 1000 * self.seed_id + 2 * layer + which
+
+    @property
+    def head_dim(self) -> int:
+        return 128  # the pages' Qwen3-VL decoders
+
     def chunk_seed(self, layer: int) -> int:
         """Seed of the S=16 activation chunk of layer ``layer`` (-1: head)."""
         return 600000 + 1000 * self.seed_id + (layer if layer >= 0 else 999)

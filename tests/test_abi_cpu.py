@@ -45,7 +45,7 @@ def test_status_strings_and_version(L):
     for code, name in qg.STATUS_NAMES.items():
         assert qg.status_string(code).startswith(name)
     assert qg.status_string(99) == "QG_ERR_UNKNOWN"
-    assert L.qg_abi_version() == 102
+    assert L.qg_abi_version() == 103
     assert L.qg_head_argmax_workspace_bytes(151936) >= 16
 
 
@@ -179,3 +179,30 @@ def test_decode_step_validation(L):
                                        None) == 4
     assert L.qg_rmsnorm_head_argmax(ctypes.byref(w), h, g, 1e-6, None, 0x7000, 0x7100, 8,
                                     None) == 5
+
+
+def test_decode_attention_validation(L):
+    ws_n = L.qg_decode_attention_workspace_bytes(16, 8)
+    assert ws_n >= 8 * 4 + 8 * 2 * 130 * 4
+    assert L.qg_decode_attention_workspace_bytes(16, 5) == 0          # hq % hkv != 0
+    qkv, kc, vc, pos, o, ws = 0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x60000
+
+    def call(**kw):
+        a = dict(qkv=qkv, hq=16, hkv=8, d=128, kc=kc, vc=vc, l_max=64, pos=pos, theta=5e6,
+                 o=o, ws=ws, ws_n=ws_n)
+        a.update(kw)
+        return L.qg_decode_attention(a["qkv"], a["hq"], a["hkv"], a["d"], a["kc"], a["vc"],
+                                     a["l_max"], a["pos"], a["theta"], a["o"], a["ws"],
+                                     a["ws_n"], None)
+    assert call(qkv=None) == 1
+    assert call(pos=None) == 1
+    assert call(ws=None) == 1
+    assert call(d=64) == 2                                 # head_dim 128 only
+    assert call(hq=24) == 2                                # hq / hkv = 3
+    assert call(hq=64) == 2                                # hq / hkv = 8
+    assert call(l_max=0) == 2
+    assert call(theta=0.0) == 2
+    assert call(kc=kc + 8) == 3
+    assert call(o=o + 2) == 3
+    assert call(ws=ws + 16) == 3
+    assert call(ws_n=ws_n - 1) == 5

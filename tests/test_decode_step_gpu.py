@@ -188,3 +188,80 @@ def test_decode_step_chain_2b(cuda):
         del sw
         gc.collect()
         torch.cuda.empty_cache()
+
+
+def _u16(t):
+    return t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("dec,ctx", [(wl.QWEN3VL_2B, 300), (wl.QWEN3VL_8B, 1025)])
+def test_decode_step_with_attention(cuda, dec, ctx):
+    """The whole decode step with RoPE + GQA attention over each layer's K/V
+    cache (2 and 4 query heads per kv head): the attention of the first two
+    layers, teacher-forced on the layer's own q|k|v output and the cache as it
+    stood, is within its bound and appends the oracle's rows; the next
+    projection reads the attention output; the step's argmax is the oracle's
+    on the final hidden state; a graph of the step equals the eager step."""
+    import gc
+    from int4_quantized_decode_b200.sweep import DecodeSweep
+    sw = DecodeSweep(dec, I8, I8, S=1, device=cuda, keep_logits=True, decode_step=True,
+                     context=ctx)
+    hd = dec.head_dim
+    hq, hkv, pos = dec.q_dim // hd, dec.kv_dim // hd, ctx - 1
+    try:
+        tok0 = int(sw.idx.item())
+        sw.run_embed()
+        for l in range(2):  # op by op, as run_layer enqueues them
+            L = sw.layers[l]
+            kc0, vc0 = _u16(sw.kcache[l]), _u16(sw.vcache[l])
+            qg.qg_rmsnorm_gemv_s1(L.qkv, sw.hstate, sw.gamma_attn[l], sw.eps, sw.y_qkv[0],
+                                  sw.y16_qkv)
+            qg.qg_decode_attention(sw.y_qkv[0], sw.kcache[l], sw.vcache[l], sw.pos,
+                                   sw.attn_out, sw.attn_ws)
+            qg.qg_stream_check()
+            o_ref, mag, kn, vn = oracle.decode_attention(
+                sw.y_qkv[0].cpu().numpy(), hq, hkv, hd, kc0, vc0, pos, qg.ROPE_THETA)
+            od = sw.attn_out.cpu().float().numpy().astype(np.float64)
+            ulp = np.array([oracle.ulp_f16(v) for v in o_ref])
+            assert np.all(np.abs(od - o_ref) <= 1e-3 * mag + ulp)
+            assert np.array_equal(_u16(sw.vcache[l])[:, pos, :].reshape(-1), vn)
+            kd = _u16(sw.kcache[l])[:, pos, :].reshape(-1).astype(np.int32)
+            assert np.all(np.abs(kd - kn.astype(np.int32)) <= 1)
+            assert np.array_equal(_u16(sw.kcache[l])[:, :pos], kc0[:, :pos])
+            # o adds W_o (attention output) into the residual stream
+            h0 = sw.hstate.clone()
+            qg.qg_gemv_s1_residual(L.o, sw.attn_out, sw.hstate)
+            qg.qg_stream_check()
+            rows = wl.sample_rows(dec.hidden, 32, l).tolist()
+            yr, ymag = oracle_gemv(L.o, sw.attn_out, rows)
+            hn = sw.hstate.cpu().numpy()
+            dh = (hn.astype(np.float64) - h0.cpu().numpy())[rows]
+            assert np.all(np.abs(dh - yr) <= oracle.GEMV_TOL * ymag + np.spacing(np.abs(hn[rows])))
+            qg.qg_rmsnorm_gate_up_swiglu(L.gate, L.up, sw.hstate, sw.gamma_mlp[l], sw.eps,
+                                         sw.h[0])
+            qg.qg_gemv_s1_residual(L.down, sw.h[0], sw.hstate)
+        for l in range(2, dec.layers):
+            sw.run_layer(l)
+        hf = sw.hstate.clone()
+        sw.run_head()
+        qg.qg_stream_check()
+        yr, mag = oracle_gemv(sw.head, _x_ref(hf, sw.gamma_final, cuda))
+        assert oracle.argmax_ok(int(sw.idx.item()), yr)
+        tok1 = int(sw.idx.item())
+        # the graph of one step equals the eager step from the same token
+        g = sw.capture(sweeps_per_graph=1)
+        sw.idx.fill_(tok0)
+        sw.step()
+        qg.qg_stream_check()
+        eager = (int(sw.idx.item()), sw.hstate.clone(), sw.logits.clone(), sw.attn_out.clone())
+        assert eager[0] == tok1
+        sw.idx.fill_(tok0)
+        g.replay()
+        qg.qg_stream_check()
+        assert int(sw.idx.item()) == eager[0]
+        assert torch.equal(sw.hstate, eager[1]) and torch.equal(sw.logits, eager[2])
+        assert torch.equal(sw.attn_out, eager[3])
+    finally:
+        del sw
+        gc.collect()
+        torch.cuda.empty_cache()
