@@ -14,11 +14,13 @@
 //  * grid = splits x kv heads; a CTA takes one contiguous chunk of the
 //    positions 0..pos of one kv head and all G query heads that read it, so
 //    each K/V row is read once per token;
-//  * inside a CTA, each group of 16 lanes streams its own subsequence of the
-//    chunk (one 16-byte load of K and of V per lane and row, 8 dims per lane,
-//    four rows in flight) with an online softmax per query head, rescaled
-//    once per four rows; groups, then warps, merge their (max, sum, acc)
-//    states;
+//  * one CTA of 8 warps per SM takes a long chunk, streamed through a
+//    three-stage cp.async ring of 64 rows of K and V (after an L2 prefetch of
+//    the chunk issued before the wait on the previous kernel);
+//  * inside a CTA, each group of 16 lanes takes four rows of every stage
+//    (8 dims per lane, 16-byte shared loads) with an online softmax per query
+//    head, rescaled once per stage; groups, then warps, merge their (max,
+//    sum, acc) states;
 //  * every CTA writes its partial state; the last CTA of a kv head (an atomic
 //    ticket, no CTA ever waits) merges the splits, writes o in fp16 and
 //    re-zeroes its ticket;
@@ -38,17 +40,18 @@ QG_DEFINE_ERROR_FLAG(g_attn_err);
 namespace {
 
 constexpr int kD = 128;            // head_dim of the pages' Qwen3-VL decoders
-constexpr int kWarpsA = 4;
+constexpr int kWarpsA = 8;
 constexpr int kThreadsA = kWarpsA * 32;
 constexpr int kGroupLanes = 16;    // lanes per subsequence: 16 x 8 dims = one row
-constexpr int kSubseq = kThreadsA / kGroupLanes;  // 8 subsequences per CTA
+constexpr int kSubseq = kThreadsA / kGroupLanes;  // 16 subsequences per CTA
 constexpr int kDimsPerLane = kD / kGroupLanes;    // 8: one 16-byte load per row
 constexpr int kUnroll = 4;                        // rows of a subsequence per stage
-constexpr int kStageRows = kSubseq * kUnroll;     // 32 rows of K and of V per stage
+constexpr int kStageRows = kSubseq * kUnroll;     // 64 rows of K and of V per stage
 constexpr int kStages = 3;                        // ring depth: two stages in flight
 constexpr int kRowBytes = kD * 2;
-constexpr int kStageBytes = 2 * kStageRows * kRowBytes;  // K rows, then V rows: 16 KB
+constexpr int kStageBytes = 2 * kStageRows * kRowBytes;  // K rows, then V rows: 32 KB
 constexpr int kRingBytesA = kStages * kStageBytes;
+constexpr int kMaxSplitsK = 32;                   // splits of one kv head's rows, at most
 
 struct AttnParams {
     const float* qkv;
@@ -117,7 +120,7 @@ __device__ __forceinline__ void merge_state(float& m, float& l, float* a, float 
 }
 
 template <int G>
-__global__ void __launch_bounds__(kThreadsA, 3) decode_attention_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(kThreadsA, 1) decode_attention_kernel(const AttnParams p) {
     __shared__ float q_s[G][kD];
     __shared__ float kn_s[kD];        // the new key, fp16-rounded, as fp32
     __shared__ float vn_s[kD];
@@ -126,7 +129,8 @@ __global__ void __launch_bounds__(kThreadsA, 3) decode_attention_kernel(const At
     __shared__ float cs_s[kD / 2][2];
     __shared__ float wst[kWarpsA][G][kD + 2];  // per-warp merged states
     __shared__ unsigned int last_s;
-    __shared__ float sm_m[kThreadsA], sm_l[kThreadsA];  // split maxima (then weights), sums
+    __shared__ float sm_m[kThreadsA / kD][kMaxSplitsK];  // split maxima (then weights)
+    __shared__ float sm_l[kThreadsA / kD][kMaxSplitsK];  // split sums
 
     const int split = blockIdx.x, g = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(kThreadsA, 3) decode_attention_kernel(const At
         kn_s[tid] = h2f(r0);
         kn_s[tid + kD / 2] = h2f(r1);
     }
-    {
+    if (tid < kD) {
         const float* vin = p.qkv + static_cast<int64_t>(p.hq + p.hkv) * kD + g * kD;
         const uint16_t v = f2h_rn(vin[tid]);
         vn_h[tid] = v;
@@ -224,7 +228,7 @@ __global__ void __launch_bounds__(kThreadsA, 3) decode_attention_kernel(const At
     griddep_launch_dependents();
 
     // the CTA whose chunk holds pos appends the new rows
-    if (pos >= j0 && pos < j1) {
+    if (pos >= j0 && pos < j1 && tid < kD) {
         const int64_t row = (static_cast<int64_t>(g) * p.l_max + pos) * kD;
         p.kc[row + tid] = kn_h[tid];
         p.vc[row + tid] = vn_h[tid];
@@ -338,17 +342,22 @@ __global__ void __launch_bounds__(kThreadsA, 3) decode_attention_kernel(const At
     }
     __syncthreads();
 
-    // ---- merge the warps: thread tid owns dim tid of every head; write the partial
+    // ---- merge the warps: thread tid owns dim tid % 128 of heads tid / 128,
+    // tid / 128 + 2, ...; write the partial
     float* part = p.part + (static_cast<int64_t>(g) * p.splits + split) * G * (kD + 2);
+    const int dim = tid & (kD - 1), hh = tid / kD;
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-        float mm = wst[0][h][0], ll = wst[0][h][1], aa = wst[0][h][2 + tid];
-        for (int w = 1; w < kWarpsA; ++w)
-            merge_state<1>(mm, ll, &aa, wst[w][h][0], wst[w][h][1], &wst[w][h][2 + tid]);
-        part[h * (kD + 2) + 2 + tid] = aa;
-        if (tid == 0) {
-            part[h * (kD + 2)] = mm;
-            part[h * (kD + 2) + 1] = ll;
+    for (int hb = 0; hb < G; hb += kThreadsA / kD) {
+        const int h = hb + hh;
+        if (h < G) {
+            float mm = wst[0][h][0], ll = wst[0][h][1], aa = wst[0][h][2 + dim];
+            for (int w = 1; w < kWarpsA; ++w)
+                merge_state<1>(mm, ll, &aa, wst[w][h][0], wst[w][h][1], &wst[w][h][2 + dim]);
+            part[h * (kD + 2) + 2 + dim] = aa;
+            if (dim == 0) {
+                part[h * (kD + 2)] = mm;
+                part[h * (kD + 2) + 1] = ll;
+            }
         }
     }
 
@@ -359,54 +368,56 @@ __global__ void __launch_bounds__(kThreadsA, 3) decode_attention_kernel(const At
     __syncthreads();
     if (!last_s) return;
     __threadfence();
-    // Merge the splits: thread s (< splits) fetches split s's max and sum, the
-    // CTA forms the weights e^(m_s - M) once, then thread tid sums dim tid over
-    // the splits with independent loads (none waits on the one before).
+    // Merge the splits, two heads at a time (threads 0-127 and 128-255):
+    // thread s (< splits) of a head's half fetches split s's max and sum and
+    // forms its weight e^(m_s - M); then every thread sums its dim over all
+    // splits with loads that are all in flight at once.
     const float* base = p.part + static_cast<int64_t>(g) * p.splits * G * (kD + 2);
+    const int64_t stride = static_cast<int64_t>(G) * (kD + 2);
+#pragma unroll 1
+    for (int hb = 0; hb < G; hb += kThreadsA / kD) {
+        const int h = hb + hh;
+        const bool act = h < G;
+        const float* col = base + static_cast<int64_t>(act ? h : 0) * (kD + 2);
+        float v[kMaxSplitsK];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-        if (tid < p.splits) {
-            const float* ps = base + (static_cast<int64_t>(tid) * G + h) * (kD + 2);
-            sm_m[tid] = __ldcg(ps);
-            sm_l[tid] = __ldcg(ps + 1);
+        for (int sidx = 0; sidx < kMaxSplitsK; ++sidx)
+            v[sidx] = act && sidx < p.splits ? __ldcg(col + sidx * stride + 2 + dim) : 0.f;
+        if (act && dim < p.splits) {
+            sm_m[hh][dim] = __ldcg(col + dim * stride);
+            sm_l[hh][dim] = __ldcg(col + dim * stride + 1);
         }
         __syncthreads();
         float mx = -INFINITY;
-        for (int sidx = 0; sidx < p.splits; ++sidx) mx = fmaxf(mx, sm_m[sidx]);
-        __syncthreads();  // every thread has read the maxima
-        if (tid < p.splits) sm_m[tid] = sm_m[tid] == -INFINITY ? 0.f : expf(sm_m[tid] - mx);
+        if (act)
+            for (int sidx = 0; sidx < p.splits; ++sidx) mx = fmaxf(mx, sm_m[hh][sidx]);
+        __syncthreads();  // every thread has the maximum
+        if (act && dim < p.splits)
+            sm_m[hh][dim] = sm_m[hh][dim] == -INFINITY ? 0.f : expf(sm_m[hh][dim] - mx);
         __syncthreads();
-        float ll = 0.f, aa = 0.f;
-        const float* col = base + static_cast<int64_t>(h) * (kD + 2) + 2 + tid;
-        const int64_t stride = static_cast<int64_t>(G) * (kD + 2);
-        int sidx = 0;
-        for (; sidx + 8 <= p.splits; sidx += 8) {
-            float v[8];
+        if (act) {
+            float ll = 0.f, aa = 0.f;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = __ldcg(col + (sidx + u) * stride);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                aa = fmaf(sm_m[sidx + u], v[u], aa);
-                ll = fmaf(sm_m[sidx + u], sm_l[sidx + u], ll);
+            for (int sidx = 0; sidx < kMaxSplitsK; ++sidx) {
+                if (sidx < p.splits) {
+                    ll = fmaf(sm_m[hh][sidx], sm_l[hh][sidx], ll);
+                    aa = fmaf(sm_m[hh][sidx], v[sidx], aa);
+                }
             }
+            p.o[static_cast<int64_t>(g * G + h) * kD + dim] = f2h_rn(aa / ll);
         }
-        for (; sidx < p.splits; ++sidx) {
-            aa = fmaf(sm_m[sidx], __ldcg(col + sidx * stride), aa);
-            ll = fmaf(sm_m[sidx], sm_l[sidx], ll);
-        }
-        p.o[static_cast<int64_t>(g * G + h) * kD + tid] = f2h_rn(aa / ll);
-        __syncthreads();  // sm_m / sm_l are refilled for the next head
+        __syncthreads();  // sm_m / sm_l are refilled for the next heads
     }
     if (tid == 0) p.ticket[g] = 0u;
 }
 
-constexpr int kMaxSplits = 128;
-static_assert(kMaxSplits <= kThreadsA, "the merge gives each split one thread");
+constexpr int kMaxSplits = kMaxSplitsK;
 
 int pick_splits(int hkv, int group, int64_t l_max, int num_sms) {
     (void)group;
-    const int per_sm = 3;  // resident CTAs per SM (registers, and 60 KB of shared memory each)
-    int s = (per_sm * num_sms + hkv - 1) / hkv;
+    // one CTA per SM (the kernel's shared memory allows no more), in one wave:
+    // long chunks keep the final merge of the splits short
+    int s = num_sms / hkv;
     if (s > kMaxSplits) s = kMaxSplits;
     if (s > l_max) s = static_cast<int>(l_max);
     return s < 1 ? 1 : s;
