@@ -1,6 +1,10 @@
 """Launch one libqgemv kernel case a few times, for profilers.
 
     python -m int4_quantized_decode_b200.profile_case --op swiglu --n 6144 --k 2048
+    python -m int4_quantized_decode_b200.profile_case --op attention --n 16 --k 16384
+
+For --op attention, n is the number of query heads (8 kv heads, head_dim 128)
+and k the K/V cache rows; the token sits at the last row.
 
 Builds one seeded weight (two for swiglu), quantizes it, and launches the op
 `--launches` times on the current device, then synchronizes.  It prints
@@ -16,7 +20,7 @@ import torch
 from . import qgemv as qg
 from . import workloads as wl
 
-OPS = ("gemv", "swiglu", "head", "s16", "s16swiglu", "quantize")
+OPS = ("gemv", "swiglu", "head", "s16", "s16swiglu", "quantize", "attention")
 
 
 def main(argv=None) -> int:
@@ -29,6 +33,20 @@ def main(argv=None) -> int:
     ap.add_argument("--launches", type=int, default=3)
     a = ap.parse_args(argv)
     dev = torch.device("cuda:0")
+    if a.op == "attention":
+        hkv, hd = 8, 128
+        kc = wl.act_fp16((hkv, a.k, hd), 11, dev)
+        vc = wl.act_fp16((hkv, a.k, hd), 12, dev)
+        qkv = wl.act_fp16((a.n + 2 * hkv) * hd, 13, dev).float()
+        o = torch.empty(a.n * hd, dtype=torch.float16, device=dev)
+        ws = qg.attention_workspace(a.n, hkv, dev)
+        pos = torch.full((1,), a.k - 1, dtype=torch.int32, device=dev)
+        torch.cuda.synchronize()
+        for _ in range(a.launches):
+            qg.qg_decode_attention(qkv, kc, vc, pos, o, ws)
+        qg.qg_stream_check()
+        print(f"attention hq={a.n} hkv={hkv} rows={a.k} x{a.launches}")
+        return 0
     w = wl.weight_fp32(a.n, a.k, 7, dev)
     if a.op == "quantize":
         out = qg.QWeight.empty(a.fmt, a.n, a.k, dev)
