@@ -52,6 +52,7 @@ constexpr int kRowBytes = kD * 2;
 constexpr int kStageBytes = 2 * kStageRows * kRowBytes;  // K rows, then V rows: 32 KB
 constexpr int kRingBytesA = kStages * kStageBytes;
 constexpr int kMaxSplitsK = 32;                   // splits of one kv head's rows, at most
+constexpr int kPrefetchRows = 256;                // rows of a chunk prefetched into L2
 
 struct AttnParams {
     const float* qkv;
@@ -138,14 +139,16 @@ __global__ void __launch_bounds__(kThreadsA, 1) decode_attention_kernel(const At
     extern __shared__ __align__(128) unsigned char ring[];
     const uint32_t ring0 = smem_u32(ring);
 
-    // Before the wait on the previous kernel: ask L2 for this CTA's rows.  A
-    // prefetch is only a hint (L2 stays coherent with whatever the previous
-    // kernel writes), and the position is read again after the wait.
+    // Before the wait on the previous kernel: ask L2 for the first rows of
+    // this CTA's chunk (at most kPrefetchRows, so that long caches do not
+    // overflow L2).  A prefetch is only a hint (L2 stays coherent with whatever
+    // the previous kernel writes), and the position is read again after the wait.
     if (lane == 0) {
         const int32_t pg = *reinterpret_cast<const volatile int32_t*>(p.pos);
         if (pg >= 0 && pg < p.l_max) {
             int64_t a0, a1;
             chunk_of(pg, p.splits, split, a0, a1);
+            if (a1 > a0 + kPrefetchRows) a1 = a0 + kPrefetchRows;
             // warp w prefetches its quarter of the chunk, in pieces of <= 16 KB
             const int64_t q0 = a0 + (a1 - a0) * warp / kWarpsA;
             const int64_t q1 = a0 + (a1 - a0) * (warp + 1) / kWarpsA;
