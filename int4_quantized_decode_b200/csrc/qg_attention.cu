@@ -127,11 +127,10 @@ __global__ void __launch_bounds__(kThreadsA, 1) decode_attention_kernel(const At
     __shared__ float vn_s[kD];
     __shared__ __align__(16) uint16_t kn_h[kD];
     __shared__ __align__(16) uint16_t vn_h[kD];
-    __shared__ float cs_s[kD / 2][2];
     __shared__ float wst[kWarpsA][G][kD + 2];  // per-warp merged states
     __shared__ unsigned int last_s;
-    __shared__ float sm_m[kThreadsA / kD][kMaxSplitsK];  // split maxima (then weights)
-    __shared__ float sm_l[kThreadsA / kD][kMaxSplitsK];  // split sums
+    __shared__ float sm_m[G][kMaxSplitsK];  // split maxima (then weights)
+    __shared__ float sm_l[G][kMaxSplitsK];  // split sums
 
     const int split = blockIdx.x, g = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -143,8 +142,16 @@ __global__ void __launch_bounds__(kThreadsA, 1) decode_attention_kernel(const At
     // this CTA's chunk (at most kPrefetchRows, so that long caches do not
     // overflow L2).  A prefetch is only a hint (L2 stays coherent with whatever
     // the previous kernel writes), and the position is read again after the wait.
+    const int32_t pg = *reinterpret_cast<const volatile int32_t*>(p.pos);
+    // RoPE angles a_i = pos * theta^(-2i/d) in fp64 for that early read of the
+    // position (thread i < d/2 keeps pair i's cos and sin in registers)
+    double rc = 1.0, rs = 0.0;
+    auto angles = [&](int32_t at) {
+        const double f = pow(p.theta, -2.0 * static_cast<double>(tid) / kD);
+        sincos(static_cast<double>(at) * f, &rs, &rc);
+    };
+    if (tid < kD / 2 && pg >= 0 && pg < p.l_max) angles(pg);
     if (lane == 0) {
-        const int32_t pg = *reinterpret_cast<const volatile int32_t*>(p.pos);
         if (pg >= 0 && pg < p.l_max) {
             int64_t a0, a1;
             chunk_of(pg, p.splits, split, a0, a1);
@@ -193,39 +200,37 @@ __global__ void __launch_bounds__(kThreadsA, 1) decode_attention_kernel(const At
         cp_async_commit_a();
     }
 
-    // RoPE angles in fp64: a_i = pos * theta^(-2i/d)
+    // Thread i < d/2 rotates pair i of the new key (fp64, rounded once to
+    // fp16) and of every query head that reads this kv head; its loads of the
+    // key and query pairs go out together.
     if (tid < kD / 2) {
-        const double f = pow(p.theta, -2.0 * static_cast<double>(tid) / kD);
-        double s, c;
-        sincos(static_cast<double>(pos) * f, &s, &c);
-        cs_s[tid][0] = static_cast<float>(c);
-        cs_s[tid][1] = static_cast<float>(s);
-        // the new key: rotated in fp64 from the fp64 cos/sin, rounded once
+        if (pos != pg) angles(pos);  // the position changed after the early read
         const float* kin = p.qkv + static_cast<int64_t>(p.hq) * kD + g * kD;
-        const double x0 = kin[tid], x1 = kin[tid + kD / 2];
-        const uint16_t r0 = __half_as_ushort(__double2half(x0 * c - x1 * s));
-        const uint16_t r1 = __half_as_ushort(__double2half(x1 * c + x0 * s));
+        const double k0 = kin[tid], k1 = kin[tid + kD / 2];
+        double q0[G], q1[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float* qin = p.qkv + static_cast<int64_t>(g * G + h) * kD;
+            q0[h] = qin[tid];
+            q1[h] = qin[tid + kD / 2];
+        }
+        const uint16_t r0 = __half_as_ushort(__double2half(k0 * rc - k1 * rs));
+        const uint16_t r1 = __half_as_ushort(__double2half(k1 * rc + k0 * rs));
         kn_h[tid] = r0;
         kn_h[tid + kD / 2] = r1;
         kn_s[tid] = h2f(r0);
         kn_s[tid + kD / 2] = h2f(r1);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            q_s[h][tid] = static_cast<float>(q0[h] * rc - q1[h] * rs);
+            q_s[h][tid + kD / 2] = static_cast<float>(q1[h] * rc + q0[h] * rs);
+        }
     }
     if (tid < kD) {
         const float* vin = p.qkv + static_cast<int64_t>(p.hq + p.hkv) * kD + g * kD;
         const uint16_t v = f2h_rn(vin[tid]);
         vn_h[tid] = v;
         vn_s[tid] = h2f(v);
-    }
-    __syncthreads();
-    if (tid < kD / 2) {
-        const double c = cs_s[tid][0], s = cs_s[tid][1];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            const float* qin = p.qkv + static_cast<int64_t>(g * G + h) * kD;
-            const double x0 = qin[tid], x1 = qin[tid + kD / 2];
-            q_s[h][tid] = static_cast<float>(x0 * c - x1 * s);
-            q_s[h][tid + kD / 2] = static_cast<float>(x1 * c + x0 * s);
-        }
     }
     __syncthreads();
     griddep_launch_dependents();
@@ -371,45 +376,58 @@ __global__ void __launch_bounds__(kThreadsA, 1) decode_attention_kernel(const At
     __syncthreads();
     if (!last_s) return;
     __threadfence();
-    // Merge the splits, two heads at a time (threads 0-127 and 128-255):
-    // thread s (< splits) of a head's half fetches split s's max and sum and
-    // forms its weight e^(m_s - M); then every thread sums its dim over all
-    // splits with loads that are all in flight at once.
+    // Merge the splits of every head in one pass (threads 0-127 take heads
+    // 0, 2, ..., threads 128-255 heads 1, 3, ...): thread s (< splits) of a
+    // head fetches split s's max and sum and forms its weight e^(m_s - M);
+    // every thread sums its dim over all splits with loads that are all in
+    // flight at once.
     const float* base = p.part + static_cast<int64_t>(g) * p.splits * G * (kD + 2);
     const int64_t stride = static_cast<int64_t>(G) * (kD + 2);
-#pragma unroll 1
-    for (int hb = 0; hb < G; hb += kThreadsA / kD) {
-        const int h = hb + hh;
-        const bool act = h < G;
-        const float* col = base + static_cast<int64_t>(act ? h : 0) * (kD + 2);
-        float v[kMaxSplitsK];
+    constexpr int kHalves = kThreadsA / kD;                // 2: threads 0-127 and 128-255
+    constexpr int kHpt = (G + kHalves - 1) / kHalves;      // heads per thread
+    float v[kHpt][kMaxSplitsK];
+#pragma unroll
+    for (int e = 0; e < kHpt; ++e) {
+        const int h = hh + kHalves * e;
+        const float* col = base + static_cast<int64_t>(h < G ? h : 0) * (kD + 2);
 #pragma unroll
         for (int sidx = 0; sidx < kMaxSplitsK; ++sidx)
-            v[sidx] = act && sidx < p.splits ? __ldcg(col + sidx * stride + 2 + dim) : 0.f;
-        if (act && dim < p.splits) {
-            sm_m[hh][dim] = __ldcg(col + dim * stride);
-            sm_l[hh][dim] = __ldcg(col + dim * stride + 1);
+            v[e][sidx] = h < G && sidx < p.splits ? __ldcg(col + sidx * stride + 2 + dim) : 0.f;
+        if (h < G && dim < p.splits) {
+            sm_m[h][dim] = __ldcg(col + dim * stride);
+            sm_l[h][dim] = __ldcg(col + dim * stride + 1);
         }
-        __syncthreads();
-        float mx = -INFINITY;
-        if (act)
-            for (int sidx = 0; sidx < p.splits; ++sidx) mx = fmaxf(mx, sm_m[hh][sidx]);
-        __syncthreads();  // every thread has the maximum
-        if (act && dim < p.splits)
-            sm_m[hh][dim] = sm_m[hh][dim] == -INFINITY ? 0.f : expf(sm_m[hh][dim] - mx);
-        __syncthreads();
-        if (act) {
-            float ll = 0.f, aa = 0.f;
+    }
+    __syncthreads();
+    float mx[kHpt];
 #pragma unroll
-            for (int sidx = 0; sidx < kMaxSplitsK; ++sidx) {
-                if (sidx < p.splits) {
-                    ll = fmaf(sm_m[hh][sidx], sm_l[hh][sidx], ll);
-                    aa = fmaf(sm_m[hh][sidx], v[sidx], aa);
-                }
+    for (int e = 0; e < kHpt; ++e) {
+        const int h = hh + kHalves * e;
+        mx[e] = -INFINITY;
+        if (h < G)
+            for (int sidx = 0; sidx < p.splits; ++sidx) mx[e] = fmaxf(mx[e], sm_m[h][sidx]);
+    }
+    __syncthreads();  // every thread has its maxima
+#pragma unroll
+    for (int e = 0; e < kHpt; ++e) {
+        const int h = hh + kHalves * e;
+        if (h < G && dim < p.splits)
+            sm_m[h][dim] = sm_m[h][dim] == -INFINITY ? 0.f : expf(sm_m[h][dim] - mx[e]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < kHpt; ++e) {
+        const int h = hh + kHalves * e;
+        if (h >= G) continue;
+        float ll = 0.f, aa = 0.f;
+#pragma unroll
+        for (int sidx = 0; sidx < kMaxSplitsK; ++sidx) {
+            if (sidx < p.splits) {
+                ll = fmaf(sm_m[h][sidx], sm_l[h][sidx], ll);
+                aa = fmaf(sm_m[h][sidx], v[e][sidx], aa);
             }
-            p.o[static_cast<int64_t>(g * G + h) * kD + dim] = f2h_rn(aa / ll);
         }
-        __syncthreads();  // sm_m / sm_l are refilled for the next heads
+        p.o[static_cast<int64_t>(g * G + h) * kD + dim] = f2h_rn(aa / ll);
     }
     if (tid == 0) p.ticket[g] = 0u;
 }
