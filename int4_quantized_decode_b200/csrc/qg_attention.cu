@@ -89,7 +89,7 @@ __device__ __forceinline__ uint4 lds128_a(uint32_t a) {
     return v;
 }
 
-// Rows [j0, j1) of the split that holds `split` when the token is at pos.
+// Rows [j0, j1) of split `split` when the token is at pos (empty past the end).
 __device__ __forceinline__ void chunk_of(int64_t pos, int splits, int split, int64_t& j0,
                                          int64_t& j1) {
     const int64_t n = pos + 1;
@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(kThreadsA, 1) decode_attention_kernel(const At
     int64_t j0, j1;
     chunk_of(pos, p.splits, split, j0, j1);
     const int nstages = static_cast<int>((j1 - j0 + kStageRows - 1) / kStageRows);
-    // Stage st of the chunk -> ring slot st % kStages: rows j0 + 32 st ..., K
+    // Stage st of the chunk -> ring slot st % kStages: rows j0 + 64 st ..., K
     // then V, 16 pieces of 16 bytes per row; row pos (not written yet) is
     // skipped, its values come from shared memory below.
     auto issue = [&](int st) {
@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(kThreadsA, 1) decode_attention_kernel(const At
     }
 
     // ---- stream: in each stage, subsequence sq = tid / 16 takes rows sq,
-    // sq + 8, sq + 16, sq + 24 (one rescale per stage)
+    // sq + 16, sq + 32, sq + 48 (one rescale per stage)
     const int sq = tid / kGroupLanes, gl = tid % kGroupLanes;
     const int d0 = gl * kDimsPerLane;
     float qr[G][kDimsPerLane];
