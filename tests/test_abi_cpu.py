@@ -66,6 +66,8 @@ def test_gemv_validation(L):
     assert gemv(L, W(k=48)) == 2                               # k % 32
     assert gemv(L, W(fmt=1, k=96)) == 2                        # k % 64
     assert gemv(L, W(n=0)) == 2
+    assert gemv(L, W(k=0)) == 2                                # empty rows
+    assert gemv(L, W(n=-1)) == 2
     assert gemv(L, W(codes=0x1008)) == 3                       # 16-byte codes
     assert gemv(L, W(scales=0x2002)) == 3
     assert gemv(L, W(), x=0) == 1
@@ -101,6 +103,8 @@ def test_head_and_quantize_validation(L):
     assert L.qg_head_argmax(ctypes.byref(w), 0x4000, None, 0x5000, 0x7008, 256, None) == 3
     assert L.qg_quantize_block32(None, 4, 64, 0x1000, 0x2000, None) == 1
     assert L.qg_quantize_block32(0x1000, 4, 40, 0x1000, 0x2000, None) == 2
+    assert L.qg_quantize_block32(0x1000, 0, 64, 0x1000, 0x2000, None) == 2   # no rows
+    assert L.qg_quantize_int4_g64(0x1000, 0, 64, 0x1000, 0x2000, 0x3000, None) == 2
     assert L.qg_quantize_block32(0x1004, 4, 64, 0x1000, 0x2000, None) == 3
     assert L.qg_quantize_int4_g64(0x1000, 4, 64, 0x1000, 0x2000, None, None) == 1
     assert L.qg_quantize_int4_g64(0x1000, 4, 96, 0x1000, 0x2000, 0x3000, None) == 2
