@@ -57,6 +57,7 @@ WORKLOADS = {
     "dense-27b-int4": ("DENSE_27B", 1, 1, 1),
 }
 DEFAULT_WORKLOAD = "qwen3vl-2b"
+SINGLE_GEMV = "gemv-2048"  # the single 2048x2048 int8 GEMV (fits in L2: rotated copies)
 FMT_NAME = {0: "int8 block-32", 1: "int4 group-64", 2: "fp16"}
 
 
@@ -65,7 +66,8 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(WORKLOADS) + [SINGLE_GEMV])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--path", default="launches", choices=["launches", "persistent"],
                     help="S=1 sweep as one launch per call (default) or one persistent launch")
@@ -494,8 +496,169 @@ def _time_e2e(sw, graph, G, steps, warmup, stream, dev, world, torch, persistent
             "steps": n}
 
 
+def run_single_gemv(a):
+    """The single 2048 x 2048 int8 block-32 GEMV.  Its 4.46 MB fit in L2, so
+    the HBM figure rotates through R distinct quantized copies (R x 4.46 MB,
+    at least 4x the 126 MB L2), one launch per copy inside a CUDA graph; the
+    same graph over one copy gives the labelled L2-hot figure."""
+    import torch
+
+    from int4_quantized_decode_b200 import qgemv as qg
+    from int4_quantized_decode_b200 import workloads as wl
+
+    rank, local, world = dist_env()
+    if world != 1:
+        raise SystemExit(f"--workload {SINGLE_GEMV} runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = wl.GEMV_2048
+    n, k, R = cfg["n"], cfg["k"], 256
+    W0 = qg.quantize(wl.weight_fp32(n, k, cfg["w_seed"], dev), qg.FMT_I8_B32)
+    copies = [qg.QWeight(W0.fmt, n, k, W0.codes.clone(), W0.scales.clone(), None)
+              for _ in range(R)]
+    x = wl.act_fp16(k, cfg["x_seed"], dev)
+    y = torch.empty(n, dtype=torch.float32, device=dev)
+    nbytes = W0.nbytes
+    stream = torch.cuda.Stream(device=dev)
+
+    def graph_over(ws):
+        with torch.cuda.stream(stream):
+            for w in ws[:4]:
+                qg.qg_gemv_s1(w, x, y, None, stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for w in ws:
+                qg.qg_gemv_s1(w, x, y, None, stream)
+        return g
+
+    def timed(g, reps):
+        # a graph replays on the current stream: time it there
+        cur = torch.cuda.current_stream(dev)
+        for _ in range(max(3, a.warmup)):
+            g.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(cur)
+        for _ in range(reps):
+            g.replay()
+        e1.record(cur)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / 1e3
+
+    reps = max(1, (a.steps + R - 1) // R)
+    g_hbm = graph_over(copies)
+    clocks = ClockSampler(local).start()
+    el_s = timed(g_hbm, reps)
+    clk = clocks.stop()
+    g_hot = graph_over([copies[0]] * R)
+    el_hot = timed(g_hot, reps)
+    qg.qg_stream_check()
+    launches = reps * R
+    value = launches * nbytes / el_s / 1e9
+    hot = launches * nbytes / el_hot / 1e9
+
+    # end to end through the C ABI with host buffers: x in, y out, every call
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(n, dtype=torch.float32).pin_memory()
+    m = max(50, min(2000, a.steps // 4))
+    with torch.cuda.stream(stream):
+        for i in range(m + 10):
+            if i == 10:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            x.copy_(x_host, non_blocking=True)
+            qg.qg_gemv_s1(copies[i % R], x, y, None, stream)
+            y_host.copy_(y, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e = m * nbytes / (e0.elapsed_time(e1) / 1e3) / 1e9
+
+    peak, peak_kind = hbm_peak()
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": 1,
+        "steps": launches, "warmup": a.warmup, "ms_per_step": round(el_s * 1e3 / launches, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "i8 x f16 -> f32", "data": "synthetic (seeded N(0,0.02) weights, N(0,1) x)",
+        "config": {"workload": (f"single {n}x{k} int8 block-32 GEMV, S=1; a step is one launch; "
+                                f"HBM figure over {R} rotating copies "
+                                f"({R * nbytes / 1e9:.2f} GB), one launch per copy in a graph"),
+                   "n": n, "k": k, "copies": R, "bytes_per_launch": nbytes,
+                   "l2_hot_gbs": round(hot, 2),
+                   "l2": "rotating copies totalling >= 4x L2 (no flush needed)"},
+        "roofline": {"bound": "hbm", "kernel": "gemv_ring_kernel (single GEMV)",
+                     "achieved": round(value, 1), "peak": peak,
+                     "peak_kind": f"{peak_kind} hbm_gbs (copy, MEASURED_PEAKS.json)"
+                     if peak_kind == "measured" else "fallback 6650 GB/s",
+                     "unit": "GB/s", "frac": round(value / peak, 4), "traffic": None,
+                     "algorithmic_bytes_per_launch": nbytes,
+                     "launch_us": round(el_s * 1e6 / launches, 3), "launches": launches},
+        "e2e": {"value": round(e2e, 2), "unit": UNIT, "h2d_bytes_per_step": k * 2,
+                "d2h_bytes_per_step": n * 4, "steps": m},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if not a.no_cpu_baseline:
+        import numpy as np
+
+        import oracle
+        w = wl.weight_fp32(n, k, cfg["w_seed"], "cpu").numpy()
+        c, sc = oracle.quantize_block32(w)
+        xb = x.cpu().numpy().view(np.uint16)
+        passes, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < min(a.cpu_budget_s, 5.0):
+            oracle.matvec(0, c, sc, None, xb)
+            passes += 1
+        el = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": round(passes * nbytes / el / 1e9, 3), "unit": UNIT,
+                                "cores": oracle.num_threads(), "kind": "oracle",
+                                "sample": f"the same GEMV x {passes} passes, fp64, {el:.1f} s"}
+    print(json.dumps(line))
+    return 0
+
+
+def run_reference_single_gemv(a):
+    """The reference arm on the single 2048 x 2048 GEMV: the oracle (fp64
+    dequantize-then-matvec on the host cores), each step one call."""
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    import numpy as np
+
+    import oracle
+    from int4_quantized_decode_b200 import workloads as wl
+    cfg = wl.GEMV_2048
+    n, k = cfg["n"], cfg["k"]
+    w = wl.weight_fp32(n, k, cfg["w_seed"], "cpu").numpy()
+    c, sc = oracle.quantize_block32(w)
+    xb = wl.act_fp16(k, cfg["x_seed"], "cpu").numpy().view(np.uint16)
+    nbytes = c.nbytes + sc.nbytes
+    for _ in range(a.warmup):
+        oracle.matvec(0, c, sc, None, xb)
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        oracle.matvec(0, c, sc, None, xb)
+    el = time.perf_counter() - t0
+    v = round(a.steps * nbytes / el / 1e9, 4)
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(el * 1e3 / a.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"single {n}x{k} int8 block-32 GEMV, S=1; a step is one call",
+                   "n": n, "k": k, "bytes_per_launch": nbytes},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": f"{a.steps} calls, fp64, {el:.2f} s"},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+    return 0
+
+
 def main(argv=None):
     a = parse_args(argv)
+    if a.workload == SINGLE_GEMV:
+        if a.impl == "reference":
+            return run_reference_single_gemv(a)
+        return run_single_gemv(a)
     if a.impl == "reference":
         return run_reference(a)
     return run_ours(a)
