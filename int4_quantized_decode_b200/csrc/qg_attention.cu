@@ -123,8 +123,6 @@ __device__ __forceinline__ void merge_state(float& m, float& l, float* a, float 
 template <int G>
 __global__ void __launch_bounds__(kThreadsA, 1) decode_attention_kernel(const AttnParams p) {
     __shared__ float q_s[G][kD];
-    __shared__ float kn_s[kD];        // the new key, fp16-rounded, as fp32
-    __shared__ float vn_s[kD];
     __shared__ __align__(16) uint16_t kn_h[kD];
     __shared__ __align__(16) uint16_t vn_h[kD];
     __shared__ float wst[kWarpsA][G][kD + 2];  // per-warp merged states
@@ -218,8 +216,6 @@ __global__ void __launch_bounds__(kThreadsA, 1) decode_attention_kernel(const At
         const uint16_t r1 = __half_as_ushort(__double2half(k1 * rc + k0 * rs));
         kn_h[tid] = r0;
         kn_h[tid + kD / 2] = r1;
-        kn_s[tid] = h2f(r0);
-        kn_s[tid + kD / 2] = h2f(r1);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             q_s[h][tid] = static_cast<float>(q0[h] * rc - q1[h] * rs);
@@ -230,7 +226,6 @@ __global__ void __launch_bounds__(kThreadsA, 1) decode_attention_kernel(const At
         const float* vin = p.qkv + static_cast<int64_t>(p.hq + p.hkv) * kD + g * kD;
         const uint16_t v = f2h_rn(vin[tid]);
         vn_h[tid] = v;
-        vn_s[tid] = h2f(v);
     }
     __syncthreads();
     griddep_launch_dependents();
