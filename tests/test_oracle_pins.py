@@ -354,6 +354,56 @@ def test_swiglu_closed_forms_and_bound():
     assert (bound >= 0.5 * 2.0**-24).all()
 
 
+def _swiglu_first_order(g, u, mg, mu, tol):
+    """The largest first-order change of silu(g) u over the box |dg| <= tol mg,
+    |du| <= tol mu, found by evaluating the function itself at the box's four
+    corners with a tolerance small enough that second-order terms vanish
+    (brute force: no formula of the bound is retyped)."""
+    h0 = oracle.silu(g) * u
+    worst = 0.0
+    for sg in (-1.0, 1.0):
+        for su in (-1.0, 1.0):
+            worst = max(worst, abs(oracle.silu(g + sg * tol * mg) * (u + su * tol * mu) - h0))
+    return worst
+
+
+def test_swiglu_bound_pinned_by_perturbation():
+    """The SwiGLU bound's propagated part is the worst case of silu(g) u over
+    the box of gate and up errors allowed by the GEMV bound: checked against
+    the function perturbed at the box corners, term by term and mixed.  A
+    dropped term, silu in place of its derivative, or a missing |u| fails."""
+    rng = np.random.default_rng(17)
+    tiny = 1e-7
+    cases = [(0.0, 2.5, 3.0, 0.0), (0.0, -1.5, 0.0, 4.0), (1.3, 0.7, 2.0, 0.0),
+             (-2.2, 1.1, 0.0, 5.0), (4.0, -3.0, 1.0, 2.0), (-0.4, 0.0, 3.0, 1.5)]
+    cases += [(float(rng.normal(0, 3)), float(rng.normal(0, 2)), float(rng.uniform(0, 5)),
+               float(rng.uniform(0, 5))) for _ in range(200)]
+    for g, u, mg, mu in cases:
+        h, b = oracle.swiglu(np.array([g]), np.array([u]), np.array([mg]), np.array([mu]), tiny)
+        e = b[0] - 0.5 * oracle.ulp_f16(abs(h[0]) + (b[0] - 0.5 * oracle.ulp_f16(abs(h[0]))))
+        ref = _swiglu_first_order(g, u, mg, mu, tiny)
+        assert e == pytest.approx(ref, rel=1e-5, abs=1e-18), (g, u, mg, mu)
+
+
+def test_swiglu_bound_closed_forms():
+    """g = 0: silu = 0 and silu' = 1/2, so the propagated part is tol mg |u| / 2
+    (the up error cannot move h); with no GEMV error at all (mg = mu = 0) the
+    bound is half an fp16 ulp of h (the output rounding alone), numpy's
+    spacing; large g: silu' -> 1 and silu(g) -> g."""
+    tol = 2e-3
+    h, b = oracle.swiglu(np.array([0.0]), np.array([3.0]), np.array([5.0]), np.array([7.0]), tol)
+    assert h[0] == 0.0
+    assert b[0] == pytest.approx(tol * 0.5 * 5.0 * 3.0 + 0.5 * float(np.spacing(np.float16(
+        tol * 0.5 * 5.0 * 3.0))), rel=1e-12)
+    for g, u in [(0.7, -2.0), (-3.0, 0.25), (6.0, 1.0)]:
+        h, b = oracle.swiglu(np.array([g]), np.array([u]), np.zeros(1), np.zeros(1), tol)
+        assert b[0] == 0.5 * float(np.spacing(np.float16(abs(h[0]))))
+    g, u, mg, mu = 60.0, 2.0, 1.0, 1.0
+    h, b = oracle.swiglu(np.array([g]), np.array([u]), np.array([mg]), np.array([mu]), tol)
+    e = tol * (mg * abs(u) + abs(g) * mu)
+    assert b[0] == pytest.approx(e + 0.5 * float(np.spacing(np.float16(abs(h[0]) + e))), rel=1e-9)
+
+
 def test_ulp_f16_matches_library_spacing():
     for v in [2.0**-24, 1e-5, 2.0**-14, 0.1, 0.5, 1.0, 1.5, 1000.0, 40000.0]:
         assert oracle.ulp_f16(v) == float(np.spacing(np.float16(v))), v
