@@ -16,15 +16,18 @@
 //    a fixed cost, and rows of 2-6 KB would pay it too often.)
 //  * x (fp16) is staged once per CTA into shared memory, still fp16, in a
 //    layout where each 8-lane phase of a 16-byte read hits distinct banks,
-//    with a few sums of x per lane granule; one x read serves all RG rows.
+//    with (int4) the sum of x per lane granule; one x read serves all RG rows.
 //  * Dequantization needs no int->float conversion: one byte permute (int8,
 //    two codes) or one mask-and-or (int4, two codes) builds a pair of fp16
-//    values 1024 + u, exact, and the sm_100 mixed-precision FMA
-//    (fma.rn.f32.f16) multiplies it by the fp16 x pair into an fp32
-//    accumulator, exactly.  The constant 1024 (+128 for int8's offset
-//    binary) comes out as a per-granule term 1024 sum x precomputed at
-//    staging.  Each block's fp16 scale is applied once per 16 (int8) or 32
-//    (int4) codes; the int4 bias uses sum_k (q s + b) x = s sum q x + b sum x.
+//    values 1024 + u, exact, and one packed fp16 subtraction of the constant
+//    turns it into the code itself (q, or 16 q for int4's odd nibbles),
+//    still exact.  The sm_100 mixed-precision FMA (fma.rn.f32.f16) then
+//    multiplies it by the fp16 x pair into an fp32 accumulator with an exact
+//    product, so the accumulated terms are q x themselves: the rounding error
+//    scales with sum |q x|, never with sum |x| (no large offset cancels).
+//    Each block's fp16 scale is applied once per 16 (int8) or 32 (int4)
+//    codes; the int4 bias uses sum_k (q s + b) x = s sum (q - q0) x + b' sum x
+//    around the group's zero point q0 (see i4_zero_point).
 //  * Lanes split K within a row; a warp-shuffle reduction finishes each row.
 //  * Programmatic dependent launch: before waiting on the previous kernel in
 //    the stream, every warp asks L2 to prefetch (cp.async.bulk.prefetch.L2) the
@@ -63,7 +66,7 @@ struct Fmt {
     static constexpr bool kScales = FMT != 2;
     static constexpr int kBlock = FMT == 0 ? 32 : 64;           // codes per scale (FMT 0 and 1)
     static constexpr int kPieces = kCodesPerLane / 8;           // 16-byte fp16 x pieces per lane
-    static constexpr int kSums = FMT == 1 ? 2 : 1;              // floats of x sums per granule
+    static constexpr int kSums = FMT == 1 ? 1 : 0;              // floats of x sums per granule
     static constexpr bool kBias = FMT == 1;
 };
 
@@ -128,10 +131,19 @@ __device__ __forceinline__ void fma_f16x2_f32(float& acc_a, float& acc_b, uint32
         : "r"(q2), "r"(x2));
 }
 
+// (a - b) on two packed fp16 values; exact whenever the differences are
+// integers of magnitude < 2048 (as for every use below).
+__device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 // 16 int8 codes (one 16-byte vector) against their 16 fp16 x (two pieces, in
-// k order): returns sum_k (1152 + q_k) x_k.  The code byte q (two's
-// complement) is turned into offset binary u = q + 128 and permuted under
-// 0x64, the fp16 encoding of 1024 + u (exact for u < 1024).
+// k order): returns sum_k q_k x_k.  The code byte q (two's complement) is
+// turned into offset binary u = q + 128 and permuted under 0x64, the fp16
+// encoding of 1024 + u (exact for u < 1024); subtracting 1152 (fp16 0x6480)
+// leaves q exactly, so every product q x is exact in fp32.
 __device__ __forceinline__ float dot16_i8(const uint4 c, const uint4* xv) {
     float a0 = 0.f, a1 = 0.f;
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
@@ -140,8 +152,10 @@ __device__ __forceinline__ float dot16_i8(const uint4 c, const uint4* xv) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const uint32_t u = w[i] ^ 0x80808080u;
-        fma_f16x2_f32(a0, a1, __byte_perm(u, 0x64646464u, 0x4140), x[2 * i]);
-        fma_f16x2_f32(a0, a1, __byte_perm(u, 0x64646464u, 0x4342), x[2 * i + 1]);
+        fma_f16x2_f32(a0, a1, hsub2_u32(__byte_perm(u, 0x64646464u, 0x4140), 0x64806480u),
+                      x[2 * i]);
+        fma_f16x2_f32(a0, a1, hsub2_u32(__byte_perm(u, 0x64646464u, 0x4342), 0x64806480u),
+                      x[2 * i + 1]);
     }
     return a0 + a1;
 }
@@ -156,24 +170,56 @@ __device__ __forceinline__ float dot8_f16(const uint4 c, const uint4* xv) {
     return a0 + a1;
 }
 
+// The zero point of an int4 group: q0 = clamp(rint(-b / s), 0, 15), the code
+// whose dequantized value lies nearest 0, as the packed fp16 constants
+// (1024 + q0, 1024 + q0) and (1024 + 16 q0, 1024 + 16 q0) that dot32_i4
+// subtracts, and the shifted bias b' = b + q0 s (exact in fp32 whenever the
+// two terms nearly cancel).  With it, w = q s + b = (q - q0) s + b', and a
+// term (q - q0) s is never larger than |w| + |b'| <= 2 |w| unless q = q0, in
+// which case w = b' itself: no term of the sum is much larger than the
+// weight it stands for, so s sum (q - q0) x + b' sum x does not cancel
+// catastrophically when w is near 0 (an affine group that straddles 0).
+// q0 only has to be near the zero crossing; any value in [0, 15] is exact.
+struct I4Zero {
+    uint32_t lo, hi;
+    float bias;
+};
+__device__ __forceinline__ I4Zero i4_zero_point(float s, float b) {
+    int q0 = 0;
+    if (s > 0.f) q0 = min(15, max(0, __float2int_rn(__fdividef(-b, s))));
+    const uint32_t lo = 0x6400u + static_cast<uint32_t>(q0);
+    const uint32_t hi = 0x6400u + (static_cast<uint32_t>(q0) << 4);
+    return {lo | (lo << 16), hi | (hi << 16), fmaf(static_cast<float>(q0), s, b)};
+}
+
 // 32 int4 codes (one 16-byte vector, even k in the low nibble) against their
 // 32 fp16 x, staged per 8-code word as the pairs (x0,x4) (x1,x5) (x2,x6)
 // (x3,x7).  One mask-and-or per pair puts nibbles 0/4 and 2/6 (after a shift
 // by 8) in the low bits of the fp16 mantissa (1024 + q) and nibbles 1/5 and
-// 3/7 four bits higher (1024 + 16 q).  Returns
-//   sum_even (1024 + q) x + sum_odd (1024 + 16 q) x / 16.
-__device__ __forceinline__ float dot32_i4(const uint4 c, const uint4* xv) {
+// 3/7 four bits higher (1024 + 16 q); subtracting the zero point's constants
+// leaves q - q0 and 16 (q - q0) exactly.  Returns sum_k (q_k - q0) x_k (every
+// product exact in fp32).
+__device__ __forceinline__ float dot32_i4(const uint4 c, const uint4* xv, const I4Zero& z) {
     float l0 = 0.f, l1 = 0.f, h0 = 0.f, h1 = 0.f;
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    constexpr uint32_t k1024 = 0x64006400u;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const uint32_t v = w[i], v8 = v >> 8;
-        fma_f16x2_f32(l0, l1, (v & 0x000F000Fu) | 0x64006400u, xv[i].x);
-        fma_f16x2_f32(h0, h1, (v & 0x00F000F0u) | 0x64006400u, xv[i].y);
-        fma_f16x2_f32(l0, l1, (v8 & 0x000F000Fu) | 0x64006400u, xv[i].z);
-        fma_f16x2_f32(h0, h1, (v8 & 0x00F000F0u) | 0x64006400u, xv[i].w);
+        fma_f16x2_f32(l0, l1, hsub2_u32((v & 0x000F000Fu) | k1024, z.lo), xv[i].x);
+        fma_f16x2_f32(h0, h1, hsub2_u32((v & 0x00F000F0u) | k1024, z.hi), xv[i].y);
+        fma_f16x2_f32(l0, l1, hsub2_u32((v8 & 0x000F000Fu) | k1024, z.lo), xv[i].z);
+        fma_f16x2_f32(h0, h1, hsub2_u32((v8 & 0x00F000F0u) | k1024, z.hi), xv[i].w);
     }
     return (l0 + l1) + (h0 + h1) * 0.0625f;
+}
+
+// acc += sum over one lane's 32 int4 codes of (q s + b) x, given the scale,
+// the bias and sx = the sum of those 32 x.
+__device__ __forceinline__ float i4_accumulate(float acc, float s, float b, const uint4 c,
+                                               const uint4* xv, float sx) {
+    const I4Zero z = i4_zero_point(s, b);
+    return fmaf(s, dot32_i4(c, xv, z), fmaf(z.bias, sx, acc));
 }
 
 // 16-byte index of piece `i` of lane-granule `g` in the staged x: the eight
@@ -211,10 +257,8 @@ struct Frag {
 // earlier stage of the same sweep, hence read through L2; or already copied
 // raw into shared memory; or computed as an RMSNorm) into shared memory, still fp16, in the
 // conflict-free piece layout (int4: each 8-code word as the pairs the dot
-// product wants), and per lane granule the sums that remove the dot
-// products' constant terms:
-//   int8: sums[g] = 1152 sum x;
-//   int4: sums[2g] = 1024 sum_even x + 64 sum_odd x, sums[2g+1] = sum x.
+// product wants), and for int4 per lane granule the sum the bias term
+// needs: sums[g] = sum x over the granule (int8 and fp16 weights need none).
 // Sources of x: kXGlobal (fp16 in global memory), kXShared (fp16 already in
 // shared memory), kXNorm (the RMSNorm of an fp32 hidden state: x = fp16(h *
 // rstd * gamma), rstd computed beforehand).
@@ -248,17 +292,19 @@ __device__ __forceinline__ void stage_x(const uint16_t* __restrict__ x, uint4* x
     for (int g = threadIdx.x; g < granules; g += blockDim.x) {
         const int64_t k0 = static_cast<int64_t>(g) * F::kCodesPerLane;
         const uint16_t* xg = x + k0;
-        float se = 0.f, so = 0.f;  // sums over even and odd k
+        float se = 0.f, so = 0.f;  // sums over even and odd k (int4 only)
 #pragma unroll
         for (int c = 0; c < F::kPieces; ++c) {
             const uint4 v = SRC == kXShared ? *reinterpret_cast<const uint4*>(xg + 8 * c)
                           : SRC == kXGlobal ? ldg_cg_v4(xg + 8 * c)
                                             : norm_piece(h + k0 + 8 * c, gamma + k0 + 8 * c, rstd);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            if (FMT == 1) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                se += h2f(static_cast<uint16_t>(w[e] & 0xFFFFu));
-                so += h2f(static_cast<uint16_t>(w[e] >> 16));
+                for (int e = 0; e < 4; ++e) {
+                    se += h2f(static_cast<uint16_t>(w[e] & 0xFFFFu));
+                    so += h2f(static_cast<uint16_t>(w[e] >> 16));
+                }
             }
             if (FMT != 1) {
                 xs[x_piece<FMT>(g, c)] = v;
@@ -268,14 +314,7 @@ __device__ __forceinline__ void stage_x(const uint16_t* __restrict__ x, uint4* x
                                __byte_perm(w[1], w[3], 0x5410), __byte_perm(w[1], w[3], 0x7632));
             }
         }
-        if (FMT == 0) {
-            sums[g] = 1152.0f * (se + so);
-        } else if (FMT == 2) {
-            sums[g] = 0.f;  // fp16 weights have no constant term
-        } else {
-            sums[2 * g] = 1024.0f * se + 64.0f * so;
-            sums[2 * g + 1] = se + so;
-        }
+        if (FMT == 1) sums[g] = se + so;
     }
 }
 
@@ -534,15 +573,13 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p) {
             const uint4* xp = xs + x_lane + cu_st * kXStep;
 #pragma unroll
             for (int i = 0; i < F::kPieces; ++i) xv[i] = xp[i * 8];
-            const float c0 = sums[F::kSums * g];
-            const float c1 = FMT == 1 ? sums[2 * g + 1] : 0.f;
+            const float c1 = FMT == 1 ? sums[g] : 0.f;
 #pragma unroll
             for (int j = 0; j < ROWS; ++j) {
                 if (FMT == 0)
-                    acc[j] = fmaf(h2f(f.s[j]), dot16_i8(f.c[j], xv) - c0, acc[j]);
+                    acc[j] = fmaf(h2f(f.s[j]), dot16_i8(f.c[j], xv), acc[j]);
                 else
-                    acc[j] = fmaf(h2f(f.s[j]), dot32_i4(f.c[j], xv) - c0,
-                                  fmaf(h2f(f.b[j]), c1, acc[j]));
+                    acc[j] = i4_accumulate(acc[j], h2f(f.s[j]), h2f(f.b[j]), f.c[j], xv, c1);
             }
         }
         if (++cu_st == nst) {
@@ -815,8 +852,7 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
             const uint4* xp = xs + x_lane + cu_st * kXStep;
 #pragma unroll
             for (int i = 0; i < F::kPieces; ++i) xv[i] = xp[i * 8];
-            const float c0 = sums[F::kSums * g];
-            const float c1 = FMT == 1 ? sums[2 * g + 1] : 0.f;
+            const float c1 = FMT == 1 ? sums[g] : 0.f;
 #pragma unroll
             for (int j = 0; j < ROWS; ++j) {
                 const uint4 c = lds128(slot_codes(cu_slot, j));
@@ -826,10 +862,10 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
                 }
                 const float sc = h2f(lds16(slot_side(cu_slot, j, 0) + side_off));
                 if (FMT == 0) {
-                    acc[j] = fmaf(sc, dot16_i8(c, xv) - c0, acc[j]);
+                    acc[j] = fmaf(sc, dot16_i8(c, xv), acc[j]);
                 } else {
                     const float bi = h2f(lds16(slot_side(cu_slot, j, 1) + side_off));
-                    acc[j] = fmaf(sc, dot32_i4(c, xv) - c0, fmaf(bi, c1, acc[j]));
+                    acc[j] = i4_accumulate(acc[j], sc, bi, c, xv, c1);
                 }
             }
         }
@@ -862,7 +898,7 @@ size_t x_smem_bytes(int fmt, const Params& p) {
     const int cpl = fmt == QG_FMT_I8_B32 ? Fmt<0>::kCodesPerLane
                     : (fmt == QG_FMT_I4_G64 ? Fmt<1>::kCodesPerLane : Fmt<2>::kCodesPerLane);
     const int granules = static_cast<int>(p.k / cpl);
-    const int nsums = (fmt == QG_FMT_I4_G64 ? Fmt<1>::kSums : Fmt<0>::kSums) * granules;
+    const int nsums = (fmt == QG_FMT_I4_G64 ? Fmt<1>::kSums : 0) * granules;
     size_t b = static_cast<size_t>(p.x_words) * 4 + static_cast<size_t>(align_up(nsums, 4)) * 4;
     if (p.x_bulk) b += static_cast<size_t>(p.k) * 2;
     return b;

@@ -170,3 +170,66 @@ def sample_rows(n: int, count: int, seed: int) -> torch.Tensor:
 def gamma_fp16(k: int, seed: int, device="cuda") -> torch.Tensor:
     """RMSNorm gains: fp16 = RNE(1 + 0.1 N(0, 1)) drawn like the activations."""
     return (1.0 + 0.1 * act_fp16(k, seed, device).float()).half()
+
+
+# ------------------------------------------------ adversarial structure ----
+# Inputs shaped to stress the S=1 arithmetic rather than to look like a
+# trained model: quantization blocks dominated by one outlier (their other
+# codes round to 0 or +-1), columns whose weights are exactly 0 in every row
+# while the activation there is huge, and affine int4 groups that straddle 0
+# with an exact zero level.  They are plain seeded draws with a fixed layout;
+# no quantization arithmetic happens here.
+
+def quiet_columns(k: int, seed: int, group: int, frac: float = 0.25) -> torch.Tensor:
+    """A bool mask [k] (CPU) of columns that carry an exact-zero weight in
+    every row: about `frac` of each group of `group` columns, never the
+    group's first two columns (the int4 layout below keeps its extremes
+    there)."""
+    g = _gen(seed, "cpu")
+    m = torch.rand(k, generator=g) < frac
+    m.view(-1, group)[:, :2] = False
+    return m
+
+
+def outlier_weight_fp32(n: int, k: int, seed: int, quiet: torch.Tensor,
+                        device="cpu") -> torch.Tensor:
+    """fp32 [n, k]: every block of 32 along k holds one entry of magnitude 1
+    (random sign, at a random position outside the quiet columns when it can)
+    and entries N(0, 1e-3) elsewhere, so int8 block-32 absmax codes are one
+    +-127 and mostly 0 or +-1; quiet columns are exactly 0 in every row."""
+    g = _gen(seed, "cpu")
+    w = torch.randn((n, k), generator=g, dtype=torch.float32).mul_(1e-3)
+    blocks = k // 32
+    qb = quiet.view(blocks, 32)
+    pos = torch.randint(0, 32, (n, blocks), generator=g)
+    # move an outlier that landed on a quiet column to the block's first column
+    pos = torch.where(qb[torch.arange(blocks), pos], torch.zeros_like(pos), pos)
+    sign = torch.randint(0, 2, (n, blocks), generator=g).float().mul_(2).sub_(1)
+    w.scatter_(1, torch.arange(blocks) * 32 + pos, sign)
+    w[:, quiet] = 0.0
+    return w.to(device)
+
+
+def affine_zero_weight_fp32(n: int, k: int, seed: int, quiet: torch.Tensor,
+                            device="cpu") -> torch.Tensor:
+    """fp32 [n, k] for int4 group-64: every group holds -1 at its first column
+    and 0.875 at its second (so its affine scale is 1.875/15 = 0.125 and its
+    bias -1, both exact in fp16, and the level q = 8 dequantizes to exactly
+    0), quiet columns exactly 0 (code 8), and U(-1, 0.875) elsewhere."""
+    g = _gen(seed, "cpu")
+    w = torch.rand((n, k), generator=g, dtype=torch.float32).mul_(1.875).sub_(1.0)
+    wg = w.view(n, k // 64, 64)
+    wg[:, :, 0] = -1.0
+    wg[:, :, 1] = 0.875
+    w[:, quiet] = 0.0
+    return w.to(device)
+
+
+def spiky_act_fp16(k: int, seed: int, quiet: torch.Tensor, big: float = 30000.0,
+                   device="cpu") -> torch.Tensor:
+    """fp16 [k]: N(0, 1) with +-`big` (random sign) at the quiet columns."""
+    g = _gen(seed, "cpu")
+    x = torch.randn(k, generator=g, dtype=torch.float32)
+    sign = torch.randint(0, 2, (k,), generator=g).float().mul_(2).sub_(1)
+    x = torch.where(quiet, sign * big, x)
+    return x.to(torch.float16).to(device)

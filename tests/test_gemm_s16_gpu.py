@@ -70,17 +70,26 @@ def test_swiglu_s16(cuda, n, k, S):
 
 
 def test_chunk_head_argmax_matches_s1(cuda):
-    """The head argmax of the chunk's last row equals the S=1 decode's."""
+    """The greedy token of a 16-token prefill chunk equals the one-token
+    decode's: the head logits of the chunk's last row, computed by the S=16
+    tensor-core path, are within the bound of the oracle, their argmax passes
+    the margin rule, and so does the S=1 fused head argmax of the same row;
+    when the oracle's top-2 gap exceeds both rows' bounds the two indices are
+    the same."""
     V, H, S = 151936, 4096, 16
     Wh = qg.quantize(wl.weight_fp32(V, H, wl.QWEN3VL_8B.weight_seed(-1, "head"), cuda), I8)
     X = wl.act_fp16((S, H), 71, cuda)
-    ws = qg.head_workspace(V, cuda)
-    i16 = torch.zeros(1, dtype=torch.int32, device=cuda)
-    qg.qg_head_argmax(Wh, X[S - 1], i16, ws)
-    x1 = X[S - 1].clone()                                   # the same token decoded alone
+    Y = torch.empty((S, V), dtype=torch.float32, device=cuda)
+    qg.qg_gemm_s16(Wh, X, Y)                                # the chunk, S = 16
     i1 = torch.zeros(1, dtype=torch.int32, device=cuda)
-    qg.qg_head_argmax(Wh, x1, i1, ws)
+    qg.qg_head_argmax(Wh, X[S - 1], i1, qg.head_workspace(V, cuda))  # the same token, S = 1
     qg.qg_stream_check()
-    assert int(i16.item()) == int(i1.item())
-    yr, _ = oracle_gemv(Wh, X[S - 1])
-    assert oracle.argmax_ok(int(i16.item()), yr)
+    yr, mag = oracle_gemv(Wh, X[S - 1])
+    last = Y[S - 1].cpu().numpy()
+    assert_within_bound(last, yr, mag)
+    i16 = int(np.argmax(last))
+    assert oracle.argmax_ok(i16, yr)
+    assert oracle.argmax_ok(int(i1.item()), yr)
+    top = np.argsort(yr)[::-1][:2]
+    if yr[top[0]] - yr[top[1]] > 2 * oracle.GEMV_TOL * (mag[top[0]] + mag[top[1]]):
+        assert i16 == int(i1.item()) == int(top[0])
