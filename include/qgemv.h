@@ -143,10 +143,11 @@ QG_API qg_status qg_gemv_s1(const qg_weight* W, const uint16_t* x, float* y,
  * through the same weights ("Qwen3.8-27B ... -- Core AI", The vision path:
  * a static S=16 'prefill' chunk beside the S=1 'main' decode).
  *   Y[s, r] = sum_k X[s, k] * w_dq[r, k],   0 <= s < S
- * W : the weight (int8 block-32 only; QG_ERR_FORMAT for int4 and fp16
- *     weights).  For S > 1, k % 512 == 0 (QG_ERR_SHAPE otherwise); S == 1
- *     runs qg_gemv_s1.  For S > 1 each weight enters the tensor cores as
- *     fp16(q * s), one rounding.
+ * W : the weight, int8 block-32 or int4 group-64 (QG_ERR_FORMAT for fp16
+ *     weights at S > 1).  For S > 1, k % 512 == 0 (QG_ERR_SHAPE otherwise);
+ *     S == 1 runs qg_gemv_s1.  For S > 1 each weight enters the tensor cores
+ *     (tcgen05.mma, fp32 accumulation) as fp16(q * s) (int8) or
+ *     fp16(q * s + b) (int4), one rounding each.
  * X : fp16 [S, k] row-major, 16-byte aligned.   1 <= S <= 16.
  * Y : fp32 [S, n] out, 4-byte aligned.
  * Accuracy: each row s obeys the qg_gemv_s1 bound for x = X[s].
@@ -160,9 +161,9 @@ QG_API qg_status qg_gemm_s16(const qg_weight* W, const uint16_t* X, int S, float
  * SwiGLU MLP):
  *   g = W_g x,  u = W_u x,  H[s, i] = fp16_rne( silu(g_i) * u_i ),
  *   silu(g) = g / (1 + exp(-g))
- * Wg, Wu : weights of identical format and shape [n = intermediate, k].
- *          S == 1 accepts int8 or int4; S > 1 (tensor cores) int8 only,
- *          with k % 512 == 0 (fp16 weights: QG_ERR_FORMAT).
+ * Wg, Wu : weights of identical format and shape [n = intermediate, k],
+ *          int8 or int4 (fp16 weights: QG_ERR_FORMAT); S > 1 (tensor cores)
+ *          needs k % 512 == 0.
  * X      : fp16 [S, k], 16-byte aligned.   1 <= S <= 16.
  * H      : fp16 [S, n] out, 2-byte aligned.
  * ------------------------------------------------------------------------- */
@@ -203,7 +204,10 @@ QG_API qg_status qg_head_argmax(const qg_weight* W, const uint16_t* x, float* lo
  * nothing (no cudaMalloc, no cudaFree, no allocating library routine).
  *   - The first call on each device looks up that array's device address
  *     (cudaGetSymbolAddress, with the device current); make that first call
- *     before capturing any stream into a CUDA graph.
+ *     before capturing any stream into a CUDA graph.  The address is kept
+ *     for the life of the process: after cudaDeviceReset (or anything else
+ *     that destroys the device's primary context) the library may hold a
+ *     stale address, so do not call this entry point on that device again.
  *   - Each call clears the scratch on `stream` before the kernel runs (an
  *     asynchronous memset of 256 bytes), because the array keeps what the
  *     previous call left there.
@@ -211,7 +215,9 @@ QG_API qg_status qg_head_argmax(const qg_weight* W, const uint16_t* x, float* lo
  *     GPU (different streams without ordering between them) race and give
  *     wrong indices.  Serialize them.
  *   - A weight whose argmax would need more scratch than the 256 bytes is
- *     refused with QG_ERR_WORKSPACE (today every n needs 16 bytes).
+ *     refused with QG_ERR_WORKSPACE.  Today qg_head_argmax_workspace_bytes
+ *     reports 256 bytes for every n (of which the kernel uses 16), so the
+ *     refusal only guards future layouts that need more.
  * ------------------------------------------------------------------------- */
 QG_API qg_status qg_head_argmax_noalloc(const qg_weight* W, const uint16_t* x, float* logits,
                                         int32_t* idx, cudaStream_t stream);

@@ -217,17 +217,19 @@ qg_status qg_gemm_s16(const qg_weight* W, const uint16_t* X, int S, float* Y,
     if (S < 1 || S > 16) return QG_ERR_SHAPE;
     if (!aligned(X, 16) || !aligned(Y, 4)) return QG_ERR_ALIGN;
     if (S == 1) return qg_gemv_s1(W, X, Y, nullptr, stream);
-    if (W->fmt != QG_FMT_I8_B32) return QG_ERR_FORMAT;
+    if (W->fmt == QG_FMT_F16) return QG_ERR_FORMAT;
     qg::GemmS16Launch L = {};
+    L.fmt = W->fmt;
     L.epilogue = qg::kEpiPlain;
     L.S = S;
     L.n = W->n;
     L.k = W->k;
-    L.codes[0] = L.codes[1] = static_cast<const int8_t*>(W->codes);
+    L.codes[0] = L.codes[1] = W->codes;
     L.scales[0] = L.scales[1] = W->scales;
+    L.biases[0] = L.biases[1] = W->biases;
     L.X = X;
     L.Y = Y;
-    return qg::launch_gemm_s16(L, stream);
+    return qg::launch_gemm_tc(L, stream);
 }
 
 qg_status qg_gate_up_swiglu(const qg_weight* Wg, const qg_weight* Wu, const uint16_t* X, int S,
@@ -258,19 +260,21 @@ qg_status qg_gate_up_swiglu(const qg_weight* Wg, const qg_weight* Wu, const uint
         L.h = H;
         return qg::launch_gemv_s1(L, stream);
     }
-    if (Wg->fmt != QG_FMT_I8_B32) return QG_ERR_FORMAT;
     qg::GemmS16Launch L = {};
+    L.fmt = Wg->fmt;
     L.epilogue = qg::kEpiSwiglu;
     L.S = S;
     L.n = Wg->n;
     L.k = Wg->k;
-    L.codes[0] = static_cast<const int8_t*>(Wg->codes);
+    L.codes[0] = Wg->codes;
     L.scales[0] = Wg->scales;
-    L.codes[1] = static_cast<const int8_t*>(Wu->codes);
+    L.biases[0] = Wg->biases;
+    L.codes[1] = Wu->codes;
     L.scales[1] = Wu->scales;
+    L.biases[1] = Wu->biases;
     L.X = X;
     L.H = H;
-    return qg::launch_gemm_s16(L, stream);
+    return qg::launch_gemm_tc(L, stream);
 }
 
 size_t qg_head_argmax_workspace_bytes(int64_t n) {
@@ -319,11 +323,11 @@ qg_status qg_sweep_plan(const qg_stage* stages, int n_stages, void* workspace, s
         qg_status st = stage_launch(stages[i], &L[i]);
         if (st != QG_OK) return st;
     }
+    qg_sweep out = {};
+    out.n_stages = n_stages;
     int kernel = -1;
     qg_status st = qg::plan_sweep(L.data(), n_stages, workspace, ws_bytes, &kernel);
     if (st != QG_OK) return st;
-    qg_sweep out = {};
-    out.n_stages = n_stages;
     out.kernel = kernel;
     *sweep = out;
     return QG_OK;
@@ -461,7 +465,7 @@ qg_status qg_stream_check(cudaStream_t stream) {
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return qg::cuda_status(e);
     const unsigned int g = qg::gemv_read_and_clear_error() | qg::gemv_decode_read_and_clear_error();
-    const unsigned int f = g | qg::gemm_s16_read_and_clear_error();
+    const unsigned int f = g | qg::gemm_tc_read_and_clear_error();
     const unsigned int a = qg::attention_read_and_clear_error();  // a position out of range
     if (g & qg::kGemvErrBadPlan) return QG_ERR_PLAN;
     if ((g & qg::kGemvErrToken) || a) return QG_ERR_SHAPE;

@@ -80,7 +80,6 @@ qg_status launch_quantize_block32(const float* w, int64_t n, int64_t k, int8_t* 
 qg_status launch_quantize_int4_g64(const float* w, int64_t n, int64_t k, uint8_t* codes,
                                    uint16_t* scales, uint16_t* biases, cudaStream_t stream);
 
-// S <= 16 tensor-core path (int8 block-32): plain (Y fp32) or SwiGLU (H fp16).
 // One decode step's attention core (qg_attention.cu).
 struct AttentionLaunch {
     const float* qkv;       // fp32 [hq*d | hkv*d | hkv*d]
@@ -98,18 +97,22 @@ size_t decode_attention_workspace_bytes(int hq, int hkv);
 qg_status launch_decode_attention(const AttentionLaunch& L, cudaStream_t stream);
 unsigned int attention_read_and_clear_error();  // bit 0: position outside [0, l_max)
 
+// S <= 16 tokens on the tensor cores (qg_gemm_tc.cu): int8 block-32 or int4
+// group-64 weights, plain (Y fp32) or SwiGLU (H fp16).
 struct GemmS16Launch {
+    int fmt;       // QG_FMT_I8_B32 or QG_FMT_I4_G64
     int epilogue;  // kEpiPlain or kEpiSwiglu
-    int S;
+    int S;         // 2..16
     int64_t n, k;
-    const int8_t* codes[2];
+    const void* codes[2];
     const uint16_t* scales[2];
+    const uint16_t* biases[2];  // int4 only
     const uint16_t* X;
     float* Y;
     uint16_t* H;
 };
-qg_status launch_gemm_s16(const GemmS16Launch& L, cudaStream_t stream);
-unsigned int gemm_s16_read_and_clear_error();
+qg_status launch_gemm_tc(const GemmS16Launch& L, cudaStream_t stream);
+unsigned int gemm_tc_read_and_clear_error();
 
 // Head-argmax workspace layout (bytes).
 constexpr size_t kHeadWorkspaceBytes = 256;

@@ -81,13 +81,13 @@ def test_gemm_s16_and_swiglu_validation(L):
     assert L.qg_gemm_s16(ctypes.byref(w), 0x4000, 0, 0x5000, None) == 2
     assert L.qg_gemm_s16(ctypes.byref(w), 0x4000, 17, 0x5000, None) == 2
     assert L.qg_gemm_s16(ctypes.byref(w), None, 4, 0x5000, None) == 1
-    w4 = W(fmt=1, k=512)                                       # S > 1: int8 only
-    assert L.qg_gemm_s16(ctypes.byref(w4), 0x4000, 4, 0x5000, None) == 4
     wf = W(fmt=2, k=512)                                       # fp16 weights: S == 1 only
     assert L.qg_gemm_s16(ctypes.byref(wf), 0x4000, 4, 0x5000, None) == 4
-    assert L.qg_gate_up_swiglu(ctypes.byref(w4), ctypes.byref(w4), 0x4000, 4, 0x6000, None) == 4
     w256 = W(k=256)                                            # S > 1 needs k % 512 == 0
     assert L.qg_gemm_s16(ctypes.byref(w256), 0x4000, 4, 0x5000, None) == 2
+    w4 = W(fmt=1, k=256)                                       # int4 too (S > 1)
+    assert L.qg_gemm_s16(ctypes.byref(w4), 0x4000, 4, 0x5000, None) == 2
+    assert L.qg_gate_up_swiglu(ctypes.byref(w4), ctypes.byref(w4), 0x4000, 4, 0x6000, None) == 2
     wg, wu = W(), W(fmt=1, k=64)
     assert L.qg_gate_up_swiglu(ctypes.byref(wg), ctypes.byref(wu), 0x4000, 1, 0x6000, None) == 4
     wu2 = W(n=16)
