@@ -148,42 +148,29 @@ def profiled_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """nvidia-smi clocks and throttle reasons: a sampler every 200 ms while a
+    region runs, and one-shot queries right before and after it (a timed
+    region shorter than the sampling period still gets a record)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.out = None
 
-    def start(self):
-        try:
-            self.out = tempfile.NamedTemporaryFile("w+", delete=False, suffix=".csv")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", str(self.gpu)], stdout=self.out, stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
-        return self
+    def _cmd(self, loop: bool):
+        c = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+             "-i", str(self.gpu)]
+        return c + (["-lms", "200"] if loop else [])
 
-    def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.out.flush()
-        self.out.seek(0)
-        rows = [r.strip().split(", ") for r in self.out.read().splitlines() if r.strip()]
-        self.out.close()
-        os.unlink(self.out.name)
+    @classmethod
+    def _parse(cls, text: str):
         sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
+        for line in text.splitlines():
+            r = line.strip().split(", ")
             if len(r) < 9:
                 continue
             try:
@@ -191,68 +178,167 @@ class ClockSampler:
                 mx = float(r[2])
             except ValueError:
                 continue
-            for n, v in zip(names, r[5:9]):
+            for n, v in zip(cls.REASONS, r[5:9]):
                 if v.strip().lower() == "active":
                     reasons.add(n)
+        return sm, mx, reasons
+
+    def query_once(self):
+        try:
+            out = subprocess.run(self._cmd(False), capture_output=True, text=True,
+                                 timeout=10).stdout
+        except (OSError, subprocess.TimeoutExpired):
+            return None
+        sm, mx, reasons = self._parse(out)
+        if not sm:
+            return None
+        return {"sm_mhz": sm[0], "sm_max_mhz": mx, "reasons": sorted(reasons)}
+
+    def start(self):
+        try:
+            self.out = tempfile.NamedTemporaryFile("w+", delete=False, suffix=".csv")
+            self.proc = subprocess.Popen(self._cmd(True), stdout=self.out,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def stop(self, before=None, after=None, soak_s=0.0):
+        """The record: median SM clock and the union of active reasons over
+        the sampler's rows and the one-shot queries `before` and `after`."""
+        sm, mx, reasons = [], None, set()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.out.flush()
+            self.out.seek(0)
+            sm, mx, reasons = self._parse(self.out.read())
+            self.out.close()
+            os.unlink(self.out.name)
+        for q in (before, after):
+            if q:
+                sm.append(q["sm_mhz"])
+                mx = q["sm_max_mhz"]
+                reasons |= set(q["reasons"])
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "samples": len(sm),
-                "reasons": sorted(reasons)}
+                "reasons": sorted(reasons), "before": before, "after": after,
+                "soak_s": round(soak_s, 3)}
 
 
 # ----------------------------------------------------------- CPU oracle ----
 
-def oracle_sample(dec, body_fmt, S, budget_s, max_passes=None):
-    """Time the CPU oracle (test infrastructure) on a bounded sample of the
-    workload: one decoder layer's projections, quantized by the oracle from
-    CPU-drawn weights, run as fp64 dequantize-then-matvec (+ SwiGLU) for S
-    tokens, repeated until `budget_s` (or `max_passes`).  Returns
-    (passes, seconds, bytes per pass, threads)."""
-    import numpy as np
+# Weights the host quantizes for an oracle sweep: a sweep up to this size is
+# run whole (every layer and the head); a larger decoder runs the head and as
+# many of its first layers as fit, and says so.
+ORACLE_MAX_WEIGHTS = 2.5e9
 
-    import oracle
-    from int4_quantized_decode_b200 import workloads as wl
 
-    fmt = body_fmt
-    qz = oracle.quantize_block32 if fmt == 0 else oracle.quantize_int4_g64
-    mats = {}
-    for name, n, k in dec.layer_matrices():
-        w = wl.weight_fp32(n, k, dec.weight_seed(0, name), "cpu").numpy()
-        q = qz(w)
-        mats[name] = (q[0], q[1], q[2] if fmt == 1 else None, k)
-    nbytes = sum(c.nbytes + s.nbytes + (b.nbytes if b is not None else 0)
-                 for c, s, b, _ in mats.values())
-    xs = [wl.act_fp16(dec.hidden, dec.x_seed(0) + s, "cpu").numpy().view(np.uint16)
-          for s in range(S)]
-    passes, t0 = 0, time.perf_counter()
+class OracleSweep:
+    """The CPU oracle (test infrastructure) over a decode weight sweep: the
+    same matrices, shapes and data flow as the GPU sweep, drawn on the host
+    from the same seeded distributions and quantized by the oracle.  One run
+    is per layer q|k|v(|gate) -> o (on fp16 q) -> gate/up + SwiGLU -> down (on
+    fp16 h), then the head + argmax, each an fp64 dequantize-then-matvec, for
+    every one of the S tokens."""
+
+    def __init__(self, dec, body_fmt, head_fmt, S):
+        import numpy as np
+
+        import oracle
+        from int4_quantized_decode_b200 import workloads as wl
+        self.np, self.oracle, self.dec, self.S = np, oracle, dec, S
+        self.body_fmt, self.head_fmt = body_fmt, head_fmt
+        per_layer = dec.weight_count(include_head=False) // dec.layers
+        room = ORACLE_MAX_WEIGHTS - dec.vocab * dec.hidden
+        self.layers = max(1, min(dec.layers, int(room // per_layer)))
+        self.mats = []
+        for l in range(self.layers):
+            m = {name: self._quantized(dec.weight_seed(l, name), n, k, body_fmt)
+                 for name, n, k in dec.layer_matrices()}
+            self.mats.append(m)
+        self.head = self._quantized(dec.weight_seed(-1, "head"), dec.vocab, dec.hidden, head_fmt)
+        self.bytes = sum(self._nbytes(m) for L in self.mats for m in L.values()) + \
+            self._nbytes(self.head)
+        self.xs = [[wl.act_fp16(dec.hidden, dec.x_seed(l) + 7919 * t, "cpu").numpy()
+                    .view(np.uint16) for t in range(S)] for l in range(self.layers + 1)]
+
+    @staticmethod
+    def _nbytes(m):
+        return sum(a.nbytes for a in m[:3] if a is not None)
+
+    def _quantized(self, seed, n, k, fmt):
+        from int4_quantized_decode_b200 import workloads as wl
+        w = wl.weight_fp32(n, k, seed, "cpu").numpy()
+        if fmt == 2:
+            return (w.astype(self.np.float16).view(self.np.uint16), None, None)
+        if fmt == 0:
+            c, sc = self.oracle.quantize_block32(w)
+            return (c, sc, None)
+        return self.oracle.quantize_int4_g64(w)
+
+    def run(self):
+        np, orc, dec = self.np, self.oracle, self.dec
+        qkv = [name for name, _ in dec.qkv_parts()]
+        idx = -1
+        for t in range(self.S):
+            for l, m in enumerate(self.mats):
+                x = self.xs[l][t]
+                q, _ = orc.matvec(self.body_fmt, *m[qkv[0]], x)
+                for name in qkv[1:]:
+                    orc.matvec(self.body_fmt, *m[name], x)
+                orc.matvec(self.body_fmt, *m["o"], q.astype(np.float16).view(np.uint16))
+                g, mg = orc.matvec(self.body_fmt, *m["gate"], x)
+                u, mu = orc.matvec(self.body_fmt, *m["up"], x)
+                h, _ = orc.swiglu(g, u, mg, mu, orc.GEMV_TOL)
+                orc.matvec(self.body_fmt, *m["down"], h.astype(np.float16).view(np.uint16))
+            logits, _ = orc.matvec(self.head_fmt, *self.head, self.xs[self.layers][t])
+            idx = orc.argmax(logits)
+        return idx
+
+    def describe(self):
+        whole = self.layers == self.dec.layers
+        what = (f"one whole sweep of the {self.dec.name} workload" if whole else
+                f"the head and the first {self.layers} of {self.dec.layers} layers of the "
+                f"{self.dec.name} sweep (a whole sweep would quantize more than "
+                f"{ORACLE_MAX_WEIGHTS / 1e9:.1f}e9 weights on the host)")
+        return (f"{what}: {self.bytes / 1e9:.3f} GB of {FMT_NAME[self.body_fmt]} body + "
+                f"{FMT_NAME[self.head_fmt]} head codes+scales, S={self.S}, fp64 "
+                f"dequantize-then-matvec + SwiGLU + argmax, host-drawn weights of the same "
+                f"seeded distribution quantized by the oracle")
+
+
+def time_oracle(osw, threads, min_s=0.0, max_runs=1):
+    """Seconds per oracle sweep on `threads` host threads: at least one run,
+    repeated up to `max_runs` while under `min_s` seconds in total."""
+    osw.oracle.set_num_threads(threads)
+    runs, t0 = 0, time.perf_counter()
     while True:
-        for x in xs:
-            for name in ("q", "k", "v") + (("outgate",) if dec.out_gate else ()):
-                c, s, b, _ = mats[name]
-                y, _ = oracle.matvec(fmt, c, s, b, x)
-            c, s, b, _ = mats["o"]
-            oracle.matvec(fmt, c, s, b, xs[0] if dec.q_dim == dec.hidden else
-                          np.resize(x, dec.q_dim))
-            g, mg = oracle.matvec(fmt, *mats["gate"][:3], x)
-            u, mu = oracle.matvec(fmt, *mats["up"][:3], x)
-            h, _ = oracle.swiglu(g, u, mg, mu, oracle.GEMV_TOL)
-            h16 = h.astype(np.float16).view(np.uint16)
-            oracle.matvec(fmt, *mats["down"][:3], h16)
-        passes += 1
+        osw.run()
+        runs += 1
         el = time.perf_counter() - t0
-        if (max_passes is not None and passes >= max_passes) or \
-                (max_passes is None and el >= budget_s):
-            return passes, el, nbytes, oracle.num_threads()
+        if runs >= max_runs or el >= min_s:
+            return el / runs, runs
 
 
-def cpu_baseline(dec, body_fmt, S, budget_s, sweep_bytes):
-    passes, el, nbytes, threads = oracle_sample(dec, body_fmt, S, budget_s)
-    gbs = passes * nbytes / el / 1e9
-    return {"value": round(gbs, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
+def cpu_baseline(dec, body_fmt, head_fmt, S, sweep_bytes):
+    import oracle
+    cores = os.cpu_count() or 1
+    osw = OracleSweep(dec, body_fmt, head_fmt, S)
+    t1, _ = time_oracle(osw, 1)
+    tn, runs = time_oracle(osw, cores, min_s=2.0, max_runs=8)
+    oracle.set_num_threads(cores)
+    gbs = osw.bytes / tn / 1e9
+    return {"value": round(gbs, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
             "sweeps_per_s": round(gbs * 1e9 / sweep_bytes, 4),
-            "sample": (f"layer 0 of the {dec.name} sweep ({nbytes / 1e6:.1f} MB of "
-                       f"{FMT_NAME[body_fmt]} codes+scales, S={S}) x {passes} passes, "
-                       f"fp64 dequantize-then-matvec + SwiGLU, {el:.1f} s")}
+            "single_thread": {"value": round(osw.bytes / t1 / 1e9, 3), "unit": UNIT,
+                              "cores": 1, "s_per_sweep": round(t1, 3)},
+            "s_per_sweep": round(tn, 4),
+            "sample": osw.describe() + f"; all-core figure the mean of {runs} runs"}
 
 
 # ------------------------------------------------------------ reference ----
@@ -261,25 +347,30 @@ def run_reference(a):
     rank, _, world = dist_env()
     if rank != 0:
         return 0
+    import oracle
     from int4_quantized_decode_b200 import workloads as wl
     dname, body_fmt, head_fmt, S = WORKLOADS[a.workload][:4]
-    decode = len(WORKLOADS[a.workload]) > 4
     dec = getattr(wl, dname)
     sweep_bytes = _sweep_bytes(dec, body_fmt, head_fmt)
-    oracle_sample(dec, body_fmt, S, 0, max_passes=a.warmup)
-    passes, el, nbytes, threads = oracle_sample(dec, body_fmt, S, 0, max_passes=a.steps)
-    gbs = passes * nbytes / el / 1e9
+    cores = os.cpu_count() or 1
+    osw = OracleSweep(dec, body_fmt, head_fmt, S)
+    oracle.set_num_threads(cores)
+    for _ in range(a.warmup):
+        osw.run()
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        osw.run()
+    el = time.perf_counter() - t0
+    gbs = a.steps * osw.bytes / el / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": UNIT,
         "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
-        "ms_per_step": round(el / passes * 1e3, 3), "higher_is_better": True,
+        "ms_per_step": round(el / a.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": _config(a, dec, body_fmt, head_fmt, S, sweep_bytes),
-        "sweeps_per_s": round(gbs * 1e9 / sweep_bytes, 5),
-        "cpu_baseline": {"value": round(gbs, 4), "unit": UNIT, "cores": threads,
-                         "kind": "oracle",
-                         "sample": (f"each step: layer 0 of the sweep ({nbytes / 1e6:.1f} MB "
-                                    f"quantized), fp64 dequantize-then-matvec + SwiGLU, S={S}")},
+        "sweeps_per_s": round(gbs * 1e9 / osw.bytes, 5),
+        "cpu_baseline": {"value": round(gbs, 4), "unit": UNIT, "cores": cores,
+                         "kind": "oracle", "sample": "each step: " + osw.describe()},
         "e2e": {"value": round(gbs, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -361,20 +452,37 @@ def run_ours(a):
     sweep_bytes = sw.weight_bytes
 
     # --- device-timed sweeps (inputs resident in HBM) ----------------------
+    w0 = time.perf_counter()
     for _ in range((a.warmup + G - 1) // G):
         graph.replay()
     qg.qg_stream_check()
+    per_replay = (time.perf_counter() - w0) / max(1, (a.warmup + G - 1) // G)
     barrier()
     torch.cuda.synchronize(dev)
     clocks = ClockSampler(local).start()
+    # A timed region shorter than the sampler's period gets a soak of the same
+    # replays first (untimed, about a second) so the record sees the clocks
+    # this load runs at; one-shot queries bracket the timed region itself.
+    soak = 0.0
+    if per_replay * (steps // G) < 1.0:
+        s0 = time.perf_counter()
+        while time.perf_counter() - s0 < 1.0:
+            for _ in range(max(1, int(0.05 / max(per_replay, 1e-6)))):
+                graph.replay()
+            torch.cuda.synchronize(dev)
+        soak = time.perf_counter() - s0
+    before = clocks.query_once()
+    barrier()
+    torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(steps // G):
         graph.replay()
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    after = clocks.query_once()
     barrier()
-    clk = clocks.stop()
+    clk = clocks.stop(before, after, soak)
     qg.qg_stream_check()
     el_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     el_s = el_ms / 1e3
@@ -423,7 +531,7 @@ def run_ours(a):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(dec, body_fmt, S, a.cpu_budget_s, sweep_bytes)
+        line["cpu_baseline"] = cpu_baseline(dec, body_fmt, head_fmt, S, sweep_bytes)
     if rank == 0:
         print(json.dumps(line))
     del graph, sw
@@ -554,8 +662,9 @@ def run_single_gemv(a):
     reps = max(1, (a.steps + R - 1) // R)
     g_hbm = graph_over(copies)
     clocks = ClockSampler(local).start()
+    before = clocks.query_once()
     el_s = timed(g_hbm, reps)
-    clk = clocks.stop()
+    clk = clocks.stop(before, clocks.query_once())
     g_hot = graph_over([copies[0]] * R)
     el_hot = timed(g_hot, reps)
     qg.qg_stream_check()

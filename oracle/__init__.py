@@ -80,6 +80,8 @@ def lib():
         L.orc_argmax.argtypes = [P, I64]
         L.orc_argmax.restype = I64
         L.orc_num_threads.argtypes = []
+        L.orc_set_num_threads.argtypes = [ctypes.c_int]
+        L.orc_set_num_threads.restype = None
         L.orc_f64_to_f16.argtypes = [D]
         L.orc_f64_to_f16.restype = ctypes.c_uint16
         L.orc_rmsnorm.argtypes = [P, P, I64, D, P, P]
@@ -236,6 +238,11 @@ def swiglu(g, u, mag_g, mag_u, tol: float):
 
 def num_threads() -> int:
     return int(lib().orc_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads the oracle's parallel loops use from now on."""
+    lib().orc_set_num_threads(int(n))
 
 
 def argmax(v) -> int:

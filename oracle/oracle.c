@@ -389,3 +389,7 @@ int64_t orc_argmax(const double* v, int64_t n) {
 /* ------------------------------------------------------------ threads --- */
 
 int orc_num_threads(void) { return omp_get_max_threads(); }
+
+/* Threads the parallel loops above use from now on (the baseline timing runs
+ * the oracle once on one thread and once on every core). */
+void orc_set_num_threads(int n) { omp_set_num_threads(n > 0 ? n : 1); }

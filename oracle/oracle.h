@@ -148,6 +148,7 @@ void orc_decode_attention(const float* qkv, int64_t hq, int64_t hkv, int64_t d,
 
 /* Threads the parallel row loops use (OpenMP). */
 int orc_num_threads(void);
+void orc_set_num_threads(int n);
 
 #ifdef __cplusplus
 }

@@ -2,8 +2,11 @@
 device memory (for example a plugin whose host framework owns every device
 allocation).  Called straight through the C ABI, it must give what
 qg_head_argmax gives with a caller-provided workspace, on two calls in a row
-(the built-in scratch keeps the previous call's contents, so the second call
-checks that it is cleared).  This file is collected last on purpose."""
+with different inputs: repeated calls that share the one built-in scratch
+array agree with the workspace call each time.  (A completed head call
+leaves its key and ticket at zero, so these calls find the array clean; the
+call's own clearing of it is there for a call that follows one that did not
+complete.)  This file is collected last on purpose."""
 import ctypes
 
 import numpy as np
