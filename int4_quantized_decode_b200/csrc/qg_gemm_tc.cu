@@ -63,7 +63,6 @@ constexpr int kCodeTileBytes = kTcRows * kCodeBox;  // 16 KB
 constexpr int kStages = 4;
 constexpr int kDqWarps = 8;
 constexpr int kThreadsTc = (2 + kDqWarps) * 32;
-constexpr uint32_t kTmemCols = 256;
 constexpr int kMaxClusterTc = 8;
 
 template <int FMT>
@@ -79,12 +78,19 @@ struct TcLayout {
     using F = TcFmt<FMT>;
     static constexpr int kStageBytes = NMAT * kCodeTileBytes + F::kXBoxes * kXBoxBytes;
     static constexpr int kSmem = kStages * kStageBytes;          // + 1 KB alignment slack
+    // Two single-weight CTAs fit on an SM (shared memory) and share its 512
+    // tensor-memory columns; a gate/up CTA is alone on its SM and takes all.
+    static constexpr uint32_t kTmemCols = NMAT == 1 ? 256 : 512;
     // tensor memory: D_m at columns [16 m, 16 m + 16); A slots after it, each
     // NMAT x 8 columns (16 fp16 of K per lane)
     static constexpr int kDCols = 16 * NMAT;
     static constexpr int kASlots = (static_cast<int>(kTmemCols) - kDCols) / (8 * NMAT) / 2 * 2;
-    static_assert(kASlots >= 4, "tensor memory holds too few A slots");
+    // a dequant warp writes all its A slots of a stage before it signals
+    // them, so the ring must hold a whole stage beyond the one being read
+    static_assert(kASlots >= F::kKSteps, "tensor memory holds too few A slots");
     static_assert(kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
+    static_assert(NMAT == 1 || kSmem > 116 * 1024, "a gate/up CTA must be alone on its SM");
+    static constexpr int kCtasPerSm = NMAT == 1 ? 2 : 1;
 };
 
 struct TcParams {
@@ -290,9 +296,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const uint32_t rank = P > 1 ? cluster_ctarank_tc() : 0u;
     const int64_t tile = blockIdx.x / P;
     const int64_t row0 = tile * kTcRows;
-    const int64_t kc = p.k / P;                       // this CTA's K range
-    const int64_t kbeg = static_cast<int64_t>(rank) * kc;
-    const int nstages = static_cast<int>(kc / F::kStageK);
+    // this CTA's K range: stages [st0, st1) of the row, split as evenly as the
+    // stage count allows
+    const int total_st = static_cast<int>(p.k / F::kStageK);
+    const int st0 = static_cast<int>(rank) * total_st / P;
+    const int st1 = (static_cast<int>(rank) + 1) * total_st / P;
+    const int64_t kbeg = static_cast<int64_t>(st0) * F::kStageK;
+    const int nstages = st1 - st0;
     const int nsteps = nstages * KSTEPS;
 
     if (threadIdx.x == 0) {
@@ -314,7 +324,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     if (warp == 1) {  // tensor memory for D and the A slots (whole warp)
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(&tmem_base_sh)),
-                     "r"(kTmemCols)
+                     "r"(L::kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -322,6 +332,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
+    // the next kernel in the stream may start its own prologue now (its reads
+    // of our outputs wait for our completion in griddepcontrol.wait)
+    griddep_launch_dependents();
 
     auto stage_codes = [&](int slot, int m) -> uint32_t {
         return sbase + slot * L::kStageBytes + m * kCodeTileBytes;
@@ -429,6 +442,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             if (st + 1 < nstages) load_sides(st + 1, sv_next, bv_next);
             if (!warp_wait_or_abort(&full_bar[slot], (st / kStages) & 1, &abort_sh)) break;
             bool ok = true;
+            // every A slot of this warp's steps of the stage is written, then
+            // one wait for the stores signals them all
             for (int kk = half; kk < KSTEPS; kk += 2) {
                 const int t = st * KSTEPS + kk;
                 const int a = t % NA;
@@ -461,13 +476,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                     }
                     tc_st8(tmem + lane_addr + a_col(a, m), av);
                 }
-                tc_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&afull_bar[a]);
             }
+            tc_wait_st();
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty_bar[slot]);  // this warp is done with the codes
+            if (lane == 0) {
+                if (ok)
+                    for (int kk = half; kk < KSTEPS; kk += 2)
+                        mbar_arrive(&afull_bar[(st * KSTEPS + kk) % NA]);
+                mbar_arrive(&empty_bar[slot]);  // this warp is done with the codes
+            }
             if (!ok) break;
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
@@ -499,7 +517,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     } else if (threadIdx.x == 32 && abort_sh) {
         mbar_wait_bounded(&done_bar, 0);  // MMAs in flight finish before the CTA exits
     }
-    griddep_launch_dependents();
 
     float* red = reinterpret_cast<float*>(sgen);  // stages are free: every copy landed and was read
     if (P > 1) {
@@ -513,9 +530,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         cluster_barrier();
         // rank r finishes rows [r * 128 / P, (r + 1) * 128 / P), summing the
         // ranks' partials in rank order
-        const int rows_per = kTcRows / P;
-        for (int e = threadIdx.x - 64; e >= 0 && e < rows_per * 16; e += kThreadsTc - 64) {
-            const int r = static_cast<int>(rank) * rows_per + e / 16, tok = e % 16;
+        const int r_lo = static_cast<int>(rank) * kTcRows / P;
+        const int r_hi = (static_cast<int>(rank) + 1) * kTcRows / P;
+        for (int e = threadIdx.x - 64; e >= 0 && e < (r_hi - r_lo) * 16; e += kThreadsTc - 64) {
+            const int r = r_lo + e / 16, tok = e % 16;
             float v[NMAT];
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
@@ -553,7 +571,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                     "r"(kTmemCols)
+                     "r"(L::kTmemCols)
                      : "memory");
     }
 }
@@ -627,19 +645,19 @@ qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream
     p.n = Lc.n;
     p.k = Lc.k;
     p.S = Lc.S;
-    // Split K over a cluster of P CTAs (P divides the stage count and 128):
-    // the P whose grid best fills one CTA per SM; ties go to the smaller P.
+    // Split K over a cluster of P CTAs (1..8, at most one per stage): every SM
+    // streams its CTAs' shares of the weight, so the time goes with the most
+    // CTAs any SM holds times the share of one, ceil(tiles P / SMs) / P; take
+    // the P that minimizes it, the smaller P on ties.
     const int64_t tiles = (Lc.n + kTcRows - 1) / kTcRows;
     const int64_t stages = Lc.k / F::kStageK;
     int P = 1;
-    double best = -1.0;
-    for (int c = 1; c <= kMaxClusterTc; c *= 2) {
-        if (stages % c != 0) break;
-        const int64_t ctas = tiles * c;
-        const int64_t waves = (ctas + dev.num_sms - 1) / dev.num_sms;
-        const double eff = static_cast<double>(ctas) / (waves * dev.num_sms);
-        if (eff > best + 1e-9) {
-            best = eff;
+    double best = 1e30;
+    for (int c = 1; c <= kMaxClusterTc && c <= stages; ++c) {
+        const int64_t per_sm = (tiles * c + dev.num_sms - 1) / dev.num_sms;
+        const double t = static_cast<double>(per_sm) / c;
+        if (t < best - 1e-9) {
+            best = t;
             P = c;
         }
     }

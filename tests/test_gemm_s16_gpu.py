@@ -1,4 +1,5 @@
-"""S <= 16 chunked-prefill GEMM (tensor cores) vs the fp64 oracle, and the
+"""S <= 16 chunked-prefill GEMM (tcgen05 tensor cores), int8 block-32 and int4
+group-64 weights, vs the fp64 oracle, and the
 chunk-consistency invariant: every row of the chunk agrees with the S=1 GEMV
 within the same bound, and the head argmax of the last row is the same
 ("Qwen3.8-27B ... -- Core AI", The vision path: chunked vs S=1 prefill must
@@ -13,15 +14,19 @@ from int4_quantized_decode_b200 import qgemv as qg
 from int4_quantized_decode_b200 import workloads as wl
 
 pytestmark = pytest.mark.gpu
-I8 = qg.FMT_I8_B32
+I8, I4 = qg.FMT_I8_B32, qg.FMT_I4_G64
 
 
-@pytest.mark.parametrize("n,k,S", [(1, 512, 16), (64, 512, 16), (100, 512, 3), (1000, 2048, 16),
-                                   (4096, 4096, 16), (6144, 4096, 7), (4096, 12288, 16),
-                                   (333, 1536, 2), (2050, 1024, 16), (130, 2560, 16)])
-def test_gemm_s16_parity(cuda, n, k, S):
+S16_SHAPES = [(1, 512, 16), (64, 512, 16), (100, 512, 3), (1000, 2048, 16), (4096, 4096, 16),
+              (6144, 4096, 7), (4096, 12288, 16), (333, 1536, 2), (2050, 1024, 16),
+              (130, 2560, 16)]
+
+
+@pytest.mark.parametrize("fmt,n,k,S", [(I8, n, k, S) for n, k, S in S16_SHAPES] +
+                         [(I4, n, k, S) for n, k, S in S16_SHAPES])
+def test_gemm_s16_parity(cuda, fmt, n, k, S):
     w = wl.weight_fp32(n, k, 300 + S, cuda)
-    W = qg.quantize(w, I8)
+    W = qg.quantize(w, fmt)
     X = wl.act_fp16((S, k), 400 + n % 13, cuda)
     Y = torch.full((S, n), float("nan"), dtype=torch.float32, device=cuda)
     qg.qg_gemm_s16(W, X, Y)
@@ -38,9 +43,10 @@ def test_gemm_s16_parity(cuda, n, k, S):
         assert_within_bound(y1.cpu().numpy(), yr, mag)
 
 
-def test_gemm_s16_deterministic(cuda):
+@pytest.mark.parametrize("fmt", [I8, I4])
+def test_gemm_s16_deterministic(cuda, fmt):
     n, k, S = 4096, 4096, 16
-    W = qg.quantize(wl.weight_fp32(n, k, 5, cuda), I8)
+    W = qg.quantize(wl.weight_fp32(n, k, 5, cuda), fmt)
     X = wl.act_fp16((S, k), 6, cuda)
     Y1 = torch.empty((S, n), dtype=torch.float32, device=cuda)
     Y2 = torch.empty_like(Y1)
@@ -50,10 +56,12 @@ def test_gemm_s16_deterministic(cuda):
     assert torch.equal(Y1, Y2)
 
 
-@pytest.mark.parametrize("n,k,S", [(12288, 4096, 16), (77, 512, 5), (1000, 2048, 16)])
-def test_swiglu_s16(cuda, n, k, S):
-    Wg = qg.quantize(wl.weight_fp32(n, k, 61, cuda), I8)
-    Wu = qg.quantize(wl.weight_fp32(n, k, 62, cuda), I8)
+@pytest.mark.parametrize("fmt,n,k,S", [(I8, 12288, 4096, 16), (I8, 77, 512, 5), (I8, 1000, 2048, 16),
+                                       (I4, 12288, 4096, 16), (I4, 77, 512, 5),
+                                       (I4, 1000, 2048, 16)])
+def test_swiglu_s16(cuda, fmt, n, k, S):
+    Wg = qg.quantize(wl.weight_fp32(n, k, 61, cuda), fmt)
+    Wu = qg.quantize(wl.weight_fp32(n, k, 62, cuda), fmt)
     X = wl.act_fp16((S, k), 63, cuda)
     H = torch.empty((S, n), dtype=torch.float16, device=cuda)
     qg.qg_gate_up_swiglu(Wg, Wu, X, H)
