@@ -246,9 +246,10 @@ QG_API qg_status qg_head_argmax_noalloc(const qg_weight* W, const uint16_t* x, f
  *                           x must not overlap h.
  *   h : fp32 [k] (the normed calls) or [n] (the residual call); gamma :
  *       fp16 [k]; both 16-byte aligned.  0 <= eps <= 1 (QG_ERR_SHAPE).
- * Accuracy: as the plain calls with x the fp64 RMSNorm rounded to fp16, plus
- * one fp16 ulp of x per element (the device rounds x from fp32):
- * |y - y_ref| <= (2e-3 + 2^-10) sum_k |w_dq x|.
+ * Accuracy: the device computes x in fp32 and rounds it to fp16, so x is
+ * within one fp16 ulp of the fp64 RMSNorm rounded to fp16; given that x (see
+ * qg_rmsnorm_f16), the outputs obey the plain calls' bound
+ * |y - y_ref(x)| <= 2e-3 sum_k |w_dq x|.
  * ------------------------------------------------------------------------- */
 QG_API qg_status qg_embedding_gather(const uint16_t* table, int64_t V, int64_t H,
                                      const int32_t* token, float* h, cudaStream_t stream);
@@ -263,6 +264,14 @@ QG_API qg_status qg_rmsnorm_head_argmax(const qg_weight* W, const float* h,
                                         cudaStream_t stream);
 QG_API qg_status qg_gemv_s1_residual(const qg_weight* W, const uint16_t* x, float* h,
                                      cudaStream_t stream);
+
+/* qg_rmsnorm_f16 -- x16 = fp16_rne(RMSNorm(h; gamma, eps)) for h fp32 [k],
+ * computed exactly as the RMSNorm-input calls above stage their x (the same
+ * fixed-order reduction and per-element arithmetic), so a caller can see the
+ * activation those calls multiply by.  h, gamma, x16 16-byte aligned (x16
+ * fp16 [k] out); k % 8 == 0; 0 <= eps <= 1 (QG_ERR_SHAPE otherwise). */
+QG_API qg_status qg_rmsnorm_f16(const float* h, const uint16_t* gamma, int64_t k, float eps,
+                                uint16_t* x16, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
  * qg_decode_attention -- the attention core of one decode step over an fp16

@@ -96,6 +96,12 @@ qg::GemvLaunch plain_launch(const qg_weight& W) {
     return L;
 }
 
+// Workspace of a sweep plan: room for either persistent kernel's layout.
+size_t sweep_ws_bytes(int n_stages) {
+    const size_t a = qg::sweep_workspace_bytes(n_stages), b = qg::stream_workspace_bytes(n_stages);
+    return a > b ? a : b;
+}
+
 // One sweep stage -> the launch description of the S=1 call it stands for,
 // with that call's checks.
 qg_status stage_launch(const qg_stage& S, qg::GemvLaunch* out) {
@@ -309,14 +315,14 @@ qg_status qg_head_argmax(const qg_weight* W, const uint16_t* x, float* logits, i
 
 size_t qg_sweep_workspace_bytes(int n_stages) {
     if (n_stages < 1 || n_stages > kMaxSweepStages) return 0;
-    return qg::sweep_workspace_bytes(n_stages);
+    return sweep_ws_bytes(n_stages);
 }
 
 qg_status qg_sweep_plan(const qg_stage* stages, int n_stages, void* workspace, size_t ws_bytes,
                         qg_sweep* sweep) {
     if (!stages || !sweep) return QG_ERR_NULL;
     if (n_stages < 1 || n_stages > kMaxSweepStages) return QG_ERR_SHAPE;
-    if (!workspace || ws_bytes < qg::sweep_workspace_bytes(n_stages)) return QG_ERR_WORKSPACE;
+    if (!workspace || ws_bytes < sweep_ws_bytes(n_stages)) return QG_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return QG_ERR_ALIGN;
     std::vector<qg::GemvLaunch> L(static_cast<size_t>(n_stages));
     for (int i = 0; i < n_stages; ++i) {
@@ -325,8 +331,20 @@ qg_status qg_sweep_plan(const qg_stage* stages, int n_stages, void* workspace, s
     }
     qg_sweep out = {};
     out.n_stages = n_stages;
+    // the stream sweep when the plan qualifies (all int8, rows of whole
+    // 512-code steps), else the general persistent kernels
+    int depth = 0, xmax = 0;
+    qg_status st = qg::plan_stream(L.data(), n_stages, workspace, ws_bytes, &depth, &xmax);
+    if (st == QG_OK) {
+        out.kernel = qg::kSweepKernelStream;
+        out.reserved[0] = depth;
+        out.reserved[1] = xmax;
+        *sweep = out;
+        return QG_OK;
+    }
+    if (st != QG_ERR_FORMAT && st != QG_ERR_SHAPE) return st;
     int kernel = -1;
-    qg_status st = qg::plan_sweep(L.data(), n_stages, workspace, ws_bytes, &kernel);
+    st = qg::plan_sweep(L.data(), n_stages, workspace, ws_bytes, &kernel);
     if (st != QG_OK) return st;
     out.kernel = kernel;
     *sweep = out;
@@ -337,6 +355,9 @@ qg_status qg_sweep_run(const qg_sweep* sweep, void* workspace, cudaStream_t stre
     if (!sweep || !workspace) return QG_ERR_NULL;
     if (sweep->n_stages < 1 || sweep->n_stages > kMaxSweepStages) return QG_ERR_SHAPE;
     if (!aligned(workspace, 256)) return QG_ERR_ALIGN;
+    if (sweep->kernel == qg::kSweepKernelStream)
+        return qg::launch_stream(workspace, sweep->n_stages, static_cast<int>(sweep->reserved[0]),
+                                 static_cast<int>(sweep->reserved[1]), stream);
     return qg::launch_sweep(sweep->kernel, workspace, sweep->n_stages, stream);
 }
 
@@ -399,6 +420,16 @@ qg_status qg_rmsnorm_gemv_s1(const qg_weight* W, const float* h, const uint16_t*
     L.y = y;
     L.y16 = y16;
     return qg::launch_gemv_s1(L, stream);
+}
+
+qg_status qg_rmsnorm_f16(const float* h, const uint16_t* gamma, int64_t k, float eps,
+                         uint16_t* x16, cudaStream_t stream) {
+    qg_status st = check_norm(h, gamma, eps);
+    if (st != QG_OK) return st;
+    if (!x16) return QG_ERR_NULL;
+    if (k < 8 || k % 8 != 0) return QG_ERR_SHAPE;
+    if (!aligned(x16, 16)) return QG_ERR_ALIGN;
+    return qg::launch_rmsnorm_f16(h, gamma, k, eps, x16, stream);
 }
 
 qg_status qg_gemv_s1_residual(const qg_weight* W, const uint16_t* x, float* h,
@@ -464,7 +495,8 @@ qg_status qg_rmsnorm_head_argmax(const qg_weight* W, const float* h, const uint1
 qg_status qg_stream_check(cudaStream_t stream) {
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return qg::cuda_status(e);
-    const unsigned int g = qg::gemv_read_and_clear_error() | qg::gemv_decode_read_and_clear_error();
+    const unsigned int g = qg::gemv_read_and_clear_error() | qg::gemv_decode_read_and_clear_error() |
+                           qg::stream_read_and_clear_error();
     const unsigned int f = g | qg::gemm_tc_read_and_clear_error();
     const unsigned int a = qg::attention_read_and_clear_error();  // a position out of range
     if (g & qg::kGemvErrBadPlan) return QG_ERR_PLAN;

@@ -34,6 +34,33 @@ qg_status launch_gemv_s1_decode(const GemvLaunch& L, cudaStream_t stream) {
     return dispatch_fmt<2, kEpiPlain, kEpiNormIn>(L, p, dev, stream);
 }
 
+// x = fp16(RMSNorm(h)) as the fused calls stage it: the same per-CTA
+// reduction (one 256-thread CTA, the same fixed order) and the same per-piece
+// arithmetic, so the values are the ones those calls multiply by.
+__global__ void __launch_bounds__(kThreads) rmsnorm_f16_kernel(const float* h, const uint16_t* gamma,
+                                                                int64_t k, float eps, uint16_t* x16) {
+    __shared__ float red[kWarps];
+    griddep_wait();
+    const float rstd = rmsnorm_rstd(h, gamma, k, eps, red);
+    for (int64_t i = threadIdx.x; i < k / 8; i += kThreads)
+        *reinterpret_cast<uint4*>(x16 + 8 * i) = norm_piece(h + 8 * i, gamma + 8 * i, rstd);
+    griddep_launch_dependents();
+}
+
+qg_status launch_rmsnorm_f16(const float* h, const uint16_t* gamma, int64_t k, float eps,
+                             uint16_t* x16, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, rmsnorm_f16_kernel, h, gamma, k, eps, x16));
+}
+
 unsigned int gemv_decode_read_and_clear_error() {
     unsigned int v = 0, zero = 0;
     if (cudaMemcpyFromSymbol(&v, g_gemv_err, sizeof v) != cudaSuccess) return 0;

@@ -53,6 +53,9 @@ struct GemvLaunch {
 qg_status launch_gemv_s1(const GemvLaunch& L, cudaStream_t stream);
 // The decode-step variants (h_in or h_res set), compiled on their own.
 qg_status launch_gemv_s1_decode(const GemvLaunch& L, cudaStream_t stream);
+// x16 = fp16(RMSNorm(h; gamma, eps)) exactly as the RMSNorm-input calls stage it.
+qg_status launch_rmsnorm_f16(const float* h, const uint16_t* gamma, int64_t k, float eps,
+                             uint16_t* x16, cudaStream_t stream);
 
 // Persistent sweep: n S=1 stages (validated GemvLaunch descriptions, head
 // workspaces ignored) planned into a device workspace, then run as one
@@ -60,6 +63,14 @@ qg_status launch_gemv_s1_decode(const GemvLaunch& L, cudaStream_t stream);
 size_t sweep_workspace_bytes(int n_stages);
 qg_status plan_sweep(const GemvLaunch* L, int n_stages, void* ws, size_t ws_bytes, int* kernel);
 qg_status launch_sweep(int kernel, void* ws, int n_stages, cudaStream_t stream);
+// The stream sweep (qg_stream.cu): all-int8 plans whose rows hold whole
+// 512-code steps run as one launch whose weight stream spans the stages.
+size_t stream_workspace_bytes(int n_stages);
+qg_status plan_stream(const GemvLaunch* L, int n, void* ws, size_t ws_bytes, int* depth,
+                      int* xmax);
+qg_status launch_stream(void* ws, int n, int depth, int xmax, cudaStream_t stream);
+unsigned int stream_read_and_clear_error();
+constexpr int kSweepKernelStream = 2;
 
 // Device error bits of the S=1 kernels (read and cleared by qg_stream_check):
 // bit 0 a bounded wait gave up, bit 1 a sweep ran on a workspace that holds

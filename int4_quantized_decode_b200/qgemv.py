@@ -33,6 +33,7 @@ ABI_SYMBOLS = ("qg_quantize_block32", "qg_quantize_int4_g64", "qg_gemv_s1",
                "qg_last_cuda_error", "qg_head_argmax_noalloc", "qg_sweep_workspace_bytes",
                "qg_sweep_plan", "qg_sweep_run", "qg_embedding_gather", "qg_rmsnorm_gemv_s1",
                "qg_rmsnorm_gate_up_swiglu", "qg_rmsnorm_head_argmax", "qg_gemv_s1_residual",
+               "qg_rmsnorm_f16",
                "qg_decode_attention_workspace_bytes", "qg_decode_attention")
 ROPE_THETA = 5e6  # rope theta of the pages' Qwen3-VL decoders
 STAGE_GEMV, STAGE_SWIGLU, STAGE_HEAD_ARGMAX = 0, 1, 2
@@ -100,6 +101,7 @@ def lib() -> ctypes.CDLL:
         L.qg_rmsnorm_gate_up_swiglu.argtypes = [W, W, P, P, F, P, P]
         L.qg_rmsnorm_head_argmax.argtypes = [W, P, P, F, P, P, P, ctypes.c_size_t, P]
         L.qg_gemv_s1_residual.argtypes = [W, P, P, P]
+        L.qg_rmsnorm_f16.argtypes = [P, P, I64, F, P, P]
         L.qg_decode_attention_workspace_bytes.argtypes = [I, I]
         L.qg_decode_attention_workspace_bytes.restype = ctypes.c_size_t
         L.qg_decode_attention.argtypes = [P, I, I, I, P, P, I64, P, ctypes.c_double, P, P,
@@ -394,6 +396,15 @@ def qg_rmsnorm_gemv_s1(W: QWeight, h: torch.Tensor, gamma: torch.Tensor, eps: fl
     _check("qg_rmsnorm_gemv_s1",
            lib().qg_rmsnorm_gemv_s1(ctypes.byref(cw), _ptr(h), _ptr(gamma), float(eps), _ptr(y),
                                     _ptr(y16), _stream(stream)))
+
+
+def qg_rmsnorm_f16(h: torch.Tensor, gamma: torch.Tensor, eps: float, x16: torch.Tensor,
+                   stream=None) -> None:
+    """x16 = fp16(RMSNorm(h; gamma, eps)) as the RMSNorm-input calls stage it."""
+    _norm_args(h, gamma)
+    _cuda(x16, torch.float16, "x16")
+    _check("qg_rmsnorm_f16", lib().qg_rmsnorm_f16(_ptr(h), _ptr(gamma), h.numel(), float(eps),
+                                                  _ptr(x16), _stream(stream)))
 
 
 def qg_gemv_s1_residual(W: QWeight, x: torch.Tensor, h: torch.Tensor, stream=None) -> None:

@@ -1,14 +1,17 @@
-"""The persistent sweep (qg_sweep_plan / qg_sweep_run) vs the single calls and
-the oracle.
+"""The persistent sweep (qg_sweep_plan / qg_sweep_run) vs the oracle and the
+single calls.
 
-A sweep is the chain of S=1 calls a decode step makes, run as one launch; its
-results must be bit-identical to the same calls enqueued one by one (the same
-arithmetic in the same order per row), and therefore within the oracle's bound.
-The chains below read earlier stages' outputs (o reads fp16 q, down reads the
-SwiGLU output, a head reads a GEMV's fp16 output), so a stage that read its x
-before the previous stage finished would differ.  Shapes cover every ring
-variant of both persistent kernels (1, 2 and 4 rows per warp item; ragged row
-counts)."""
+A sweep is the chain of S=1 calls a decode step makes, run as one launch.  An
+all-int8 plan whose rows hold whole 512-code steps runs on the stream kernel:
+its results are within the oracle's bound (teacher-forced on the x each stage
+actually read) and bit-identical from run to run (a fixed summation order per
+row), though not in the single calls' summation order.  Other plans run on
+the general persistent kernels, whose results are bit-identical to the same
+calls enqueued one by one.  The chains below read earlier stages' outputs (o
+reads fp16 q, down reads the SwiGLU output, a head reads a GEMV's fp16
+output), so a stage that read its x before the previous stage finished would
+differ.  Shapes cover ragged row counts and both item sizes of the stream
+kernel (one and two rows), and every ring variant of the general kernels."""
 import gc
 
 import numpy as np
@@ -131,23 +134,39 @@ def _equal(a, b):
                        b.view(torch.int32) if b.dtype == torch.float32 else b)
 
 
+STREAM = 2  # qg_sweep.kernel of the stream kernel
+
+
+def _counter_bytes(plan):
+    """Workspace bytes that hold the grid counters of the plan's kernel."""
+    n = plan.n_stages
+    return 4 * (n * 8 * 32 + 32) if plan.sweep.kernel == STREAM else 4 * (n + 1)
+
+
 @pytest.mark.parametrize("body", [I8, I4])
 def test_sweep_chain_bitwise_and_oracle(cuda, body):
     c = build_chain(cuda, body)
     ref = c.run_calls()
     outs = c._alloc()
     plan = qg.SweepPlan(c.stages(outs), [], cuda)
-    assert plan.sweep.kernel == (0 if body == I8 else 1)
+    assert plan.sweep.kernel == (STREAM if body == I8 else 1)
+    first = None
     for rep in range(3):                      # counters reset after every run
         for o in outs.values():
             for t in o:
                 t.fill_(0 if t.dtype != torch.float32 else float("nan"))
         plan.run()
         qg.qg_stream_check()
-        for kind, name, Ws, src, _ in c.ops:
-            for a, b in zip(outs[name], ref[name]):
-                assert _equal(a, b), (rep, name)
-        ctr = plan.workspace[256:256 + 4 * (plan.n_stages + 1)]
+        # the general kernels equal the single calls; the stream kernel equals
+        # itself from run to run
+        expect = ref if plan.sweep.kernel != STREAM else first
+        if expect is not None:
+            for kind, name, Ws, src, _ in c.ops:
+                for a, b in zip(outs[name], expect[name]):
+                    assert _equal(a, b), (rep, name)
+        if first is None:
+            first = {k: [t.clone() for t in v] for k, v in outs.items()}
+        ctr = plan.workspace[256:256 + _counter_bytes(plan)]
         assert int(ctr.sum().item()) == 0
     # every stage within the oracle's bound (teacher-forced on its actual x)
     for kind, name, Ws, src, _ in c.ops:
@@ -227,6 +246,9 @@ def test_sweep_wrong_plan_and_expired_wait_are_reported(cuda):
     c = build_chain(cuda, I8)
     outs = c._alloc()
     plan = qg.SweepPlan(c.stages(outs), [], cuda)
+    plan.run()
+    qg.qg_stream_check()
+    clean = {k: [t.clone() for t in v] for k, v in outs.items()}
     wrong = qg.CSweep(plan.sweep.n_stages, 1)
     qg.qg_sweep_run(wrong, plan.workspace)
     with pytest.raises(qg.QgError, match="QG_ERR_PLAN"):
@@ -239,25 +261,32 @@ def test_sweep_wrong_plan_and_expired_wait_are_reported(cuda):
     with pytest.raises(qg.QgError, match="QG_ERR_TIMEOUT"):
         qg.qg_stream_check()
     plan.sweep = qg.qg_sweep_plan(c.stages(outs), plan.workspace)   # plan again
+    for t in (t for v in outs.values() for t in v):
+        t.zero_()
     plan.run()
     qg.qg_stream_check()
-    ref = c.run_calls()
     for k, v in outs.items():
-        for a, b in zip(v, ref[k]):
+        for a, b in zip(v, clean[k]):
             assert _equal(a, b), k
 
 
 @pytest.mark.parametrize("dec,body", [(wl.QWEN3VL_2B, I8), (wl.QWEN3VL_4B, I4),
                                       (wl.DENSE_27B, I8)])
-def test_decode_sweep_persistent_equals_launches(cuda, dec, body):
-    """The full-size sweep bench.py times: the persistent launch leaves every
-    buffer (last layer's outputs, logits, token) bit-identical to the launch
-    path."""
+def test_decode_sweep_persistent(cuda, dec, body):
+    """The full-size sweep bench.py times: one persistent launch per sweep.
+    Two sweeps captured in a graph leave every buffer (last layer's outputs,
+    logits, token) bit-identical to one eager persistent sweep; the general
+    int4 kernel also equals the launch path bit for bit; and the last layer
+    and the head are within the oracle's bound on sampled rows, teacher-forced
+    on the x each stage read, with the token passing the margin rule."""
     sw = DecodeSweep(dec, body, I8, S=1, device=cuda, keep_logits=True)
     try:
+        bufs = [sw.y_qkv, sw.y16_qkv, sw.y_o, sw.h, sw.y_down, sw.logits, sw.idx]
         sw.step()
         qg.qg_stream_check()
-        bufs = [sw.y_qkv, sw.y16_qkv, sw.y_o, sw.h, sw.y_down, sw.logits, sw.idx]
+        launches = [b.clone() for b in bufs]
+        sw.step(persistent=True)
+        qg.qg_stream_check()
         ref = [b.clone() for b in bufs]
         for b in bufs:
             b.zero_()
@@ -266,7 +295,25 @@ def test_decode_sweep_persistent_equals_launches(cuda, dec, body):
         qg.qg_stream_check()
         for a, b in zip(bufs, ref):
             assert _equal(a, b)
+        if sw.make_plan().sweep.kernel != STREAM:
+            for a, b in zip(ref, launches):
+                assert _equal(a, b)
         assert int(sw.ws.sum().item()) == 0
+        L, d = sw.layers[-1], dec
+        x = sw.x[-1]
+        for W, xin, y in [(L.qkv, x, sw.y_qkv[0]), (L.o, sw.y16_qkv[: d.q_dim], sw.y_o[0]),
+                          (L.down, sw.h[0], sw.y_down[0])]:
+            rows = wl.sample_rows(W.n, SAMPLE, W.n).tolist()
+            yr, mag = oracle_gemv(W, xin, rows)
+            assert_within_bound(y.cpu().numpy()[rows], yr, mag)
+        rows = wl.sample_rows(L.gate.n, SAMPLE, 7).tolist()
+        gr, mg = oracle_gemv(L.gate, x, rows)
+        ur, mu = oracle_gemv(L.up, x, rows)
+        hr, hb = oracle.swiglu(gr, ur, mg, mu, oracle.GEMV_TOL)
+        assert np.all(np.abs(sw.h[0].cpu().numpy().astype(np.float64)[rows] - hr) <= hb)
+        full, mag = oracle_gemv(sw.head, sw.head_input())
+        assert_within_bound(sw.logits.cpu().numpy(), full, mag)
+        assert oracle.argmax_ok(int(sw.idx.item()), full)
     finally:
         del sw
         gc.collect()
