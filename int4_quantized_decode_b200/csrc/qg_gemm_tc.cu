@@ -60,9 +60,8 @@ constexpr int kCodeBox = 128;      // bytes of codes per tile row per stage (swi
 constexpr int kXBoxK = 64;         // k per X box (128 bytes of fp16)
 constexpr int kXBoxBytes = kTcTokens * kXBoxK * 2;  // 2 KB
 constexpr int kCodeTileBytes = kTcRows * kCodeBox;  // 16 KB
-constexpr int kStages = 4;
-constexpr int kDqWarps = 8;
-constexpr int kThreadsTc = (2 + kDqWarps) * 32;
+constexpr int kAcc = 4;            // accumulators per weight matrix: independent MMA chains
+constexpr int kGroupSteps = 8;     // 16-k steps per A group (one commit releases a group)
 constexpr int kMaxClusterTc = 8;
 
 template <int FMT>
@@ -77,20 +76,32 @@ template <int FMT, int NMAT>
 struct TcLayout {
     using F = TcFmt<FMT>;
     static constexpr int kStageBytes = NMAT * kCodeTileBytes + F::kXBoxes * kXBoxBytes;
+    // ring depth: a single-weight CTA keeps two per SM within shared memory;
+    // with one A group per stage (int8) the depth is even, so that each of
+    // the two dequantizing sets always takes the same slots and waits every
+    // phase of their barriers (a parity wait must not skip a phase)
+    static constexpr int kStages = NMAT == 1 ? 4 : (FMT == 0 ? 6 : 5);
     static constexpr int kSmem = kStages * kStageBytes;          // + 1 KB alignment slack
     // Two single-weight CTAs fit on an SM (shared memory) and share its 512
     // tensor-memory columns; a gate/up CTA is alone on its SM and takes all.
     static constexpr uint32_t kTmemCols = NMAT == 1 ? 256 : 512;
-    // tensor memory: D_m at columns [16 m, 16 m + 16); A slots after it, each
-    // NMAT x 8 columns (16 fp16 of K per lane)
-    static constexpr int kDCols = 16 * NMAT;
-    static constexpr int kASlots = (static_cast<int>(kTmemCols) - kDCols) / (8 * NMAT) / 2 * 2;
-    // a dequant warp writes all its A slots of a stage before it signals
-    // them, so the ring must hold a whole stage beyond the one being read
-    static_assert(kASlots >= F::kKSteps, "tensor memory holds too few A slots");
+    // tensor memory: accumulator c of matrix m at columns 16 (m kAcc + c);
+    // then the A groups, each kGroupSteps x NMAT x 8 columns (16 fp16 of K
+    // per lane and step)
+    static constexpr int kDCols = 16 * kAcc * NMAT;
+    static constexpr int kGroupCols = kGroupSteps * NMAT * 8;
+    static constexpr int kAGroups = (static_cast<int>(kTmemCols) - kDCols) / kGroupCols;
+    static constexpr int kGroupsPerStage = F::kKSteps / kGroupSteps;  // 1 or 2
+    // gate/up CTAs are alone on their SM: twice the dequantizing warps
+    static constexpr int kDqWarps = NMAT == 2 ? 16 : 8;
+    static constexpr int kThreads = (2 + kDqWarps) * 32;
+    static_assert(kAGroups >= 2, "tensor memory holds too few A groups to overlap");
+    static_assert(F::kKSteps % kGroupSteps == 0, "stages hold whole A groups");
+    static_assert(kGroupsPerStage != 1 || kStages % 2 == 0, "each set keeps its own slots");
+    static_assert(kGroupSteps % kAcc == 0, "every accumulator takes the same steps of a group");
     static_assert(kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
     static_assert(NMAT == 1 || kSmem > 116 * 1024, "a gate/up CTA must be alone on its SM");
-    static constexpr int kCtasPerSm = NMAT == 1 ? 2 : 1;
+    static_assert(NMAT == 2 || kSmem + 1024 <= 112 * 1024, "two single-weight CTAs per SM");
 };
 
 struct TcParams {
@@ -156,6 +167,16 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
             smem_u32(bar))
         : "memory");
+}
+// One lane of a converged warp (the same lane every time): the warp runs the
+// loop around an issuing instruction uniformly, so its operands stay
+// warp-uniform, and only the elected lane issues.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b32 r;\n\telect.sync r|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
 }
 __device__ __forceinline__ void tc_st8(uint32_t taddr, const uint32_t (&v)[8]) {
     asm volatile(
@@ -269,20 +290,27 @@ __device__ __forceinline__ bool warp_wait_or_abort(uint64_t* bar, uint32_t parit
 }
 
 template <int FMT, int NMAT, int EPI>
-__global__ void __launch_bounds__(kThreadsTc, 1)
+__global__ void __launch_bounds__(TcLayout<FMT, NMAT>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_codes0,
                    const __grid_constant__ CUtensorMap tm_codes1,
                    const __grid_constant__ CUtensorMap tm_x, const TcParams p) {
     using F = TcFmt<FMT>;
     using L = TcLayout<FMT, NMAT>;
-    constexpr int KSTEPS = F::kKSteps;
-    constexpr int NA = L::kASlots;
+    constexpr int NSTG = L::kStages;
+    constexpr int NG = L::kAGroups;
+    constexpr int GPS = L::kGroupsPerStage;
+    constexpr int NDQ = L::kDqWarps;
+    constexpr int SUB = NDQ / 4;  // dequantizing warps per tensor-memory lane quarter
+    constexpr int SETW = SUB / 2;  // of those, per set (the two sets take alternate A groups)
+    // a stage's codes are read by one set (int8: one group per stage) or by both
+    constexpr int kEmptyArrivals = (GPS == 1 ? NDQ / 2 : NDQ) + 1;
     extern __shared__ unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t full_bar[kStages];
-    __shared__ __align__(8) uint64_t empty_bar[kStages];
-    __shared__ __align__(8) uint64_t afull_bar[NA];
-    __shared__ __align__(8) uint64_t aempty_bar[NA];
+    __shared__ __align__(8) uint64_t full_bar[NSTG];
+    __shared__ __align__(8) uint64_t empty_bar[NSTG];
+    __shared__ __align__(8) uint64_t afull_bar[NG];
+    __shared__ __align__(8) uint64_t aempty_bar[NG];
     __shared__ __align__(8) uint64_t done_bar;
+    __shared__ __align__(8) uint64_t fin_bar;  // epilogue warps done with tensor memory
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
 
@@ -303,25 +331,26 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const int st1 = (static_cast<int>(rank) + 1) * total_st / P;
     const int64_t kbeg = static_cast<int64_t>(st0) * F::kStageK;
     const int nstages = st1 - st0;
-    const int nsteps = nstages * KSTEPS;
+    const int ngroups = nstages * GPS;
 
     if (threadIdx.x == 0) {
         abort_sh = 0;
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < NSTG; ++s) {
             mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], kDqWarps + 1);
+            mbar_init(&empty_bar[s], kEmptyArrivals);
         }
-        for (int j = 0; j < NA; ++j) {
-            mbar_init(&afull_bar[j], 4);
+        for (int j = 0; j < NG; ++j) {
+            mbar_init(&afull_bar[j], NDQ / 2);
             mbar_init(&aempty_bar[j], 1);
         }
         mbar_init(&done_bar, 1);
+        mbar_init(&fin_bar, 4);
         fence_mbar_init();
         prefetch_tmap(&tm_codes0);
         if (NMAT == 2) prefetch_tmap(&tm_codes1);
         prefetch_tmap(&tm_x);
     }
-    if (warp == 1) {  // tensor memory for D and the A slots (whole warp)
+    if (warp == 1) {  // tensor memory for D and the A groups (whole warp)
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(&tmem_base_sh)),
                      "r"(L::kTmemCols)
@@ -342,79 +371,104 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     auto stage_x = [&](int slot) -> uint32_t {
         return sbase + slot * L::kStageBytes + NMAT * kCodeTileBytes;
     };
-    auto a_col = [&](int slot, int m) -> uint32_t {
-        return static_cast<uint32_t>(L::kDCols + (slot * NMAT + m) * 8);
+    // accumulator c of matrix m; step j of A group g for matrix m
+    auto d_col = [](int m, int c) -> uint32_t { return static_cast<uint32_t>(16 * (m * kAcc + c)); };
+    auto a_col = [](int g, int j, int m) -> uint32_t {
+        return static_cast<uint32_t>(L::kDCols + g * L::kGroupCols + (j * NMAT + m) * 8);
     };
 
     if (warp == 0) {
         // ------------------------------------------------------- producer ---
-        if (lane == 0) {
-            const uint64_t pol_w = l2_policy_evict_first();
-            const uint64_t pol_x = l2_policy_evict_last();
-            const int code_bytes_per_k = FMT == 0 ? 1 : 0;  // int8: 1 byte per k; int4: 1/2
-            auto code_c0 = [&](int st) -> int {
-                const int64_t k0 = kbeg + static_cast<int64_t>(st) * F::kStageK;
-                return static_cast<int>(code_bytes_per_k ? k0 : k0 / 2);
-            };
-            auto issue_codes = [&](int st) {
-                const int slot = st % kStages;
-                mbar_arrive_expect_tx(&full_bar[slot], L::kStageBytes);
-                tma_load_2d(stage_codes(slot, 0), &tm_codes0, code_c0(st), static_cast<int>(row0),
+        // The whole warp runs the loop and waits; the elected lane issues.
+        const uint64_t pol_w = l2_policy_evict_first();
+        const uint64_t pol_x = l2_policy_evict_last();
+        const int code_bytes_per_k = FMT == 0 ? 1 : 0;  // int8: 1 byte per k; int4: 1/2
+        auto code_c0 = [&](int st) -> int {
+            const int64_t k0 = kbeg + static_cast<int64_t>(st) * F::kStageK;
+            return static_cast<int>(code_bytes_per_k ? k0 : k0 / 2);
+        };
+        auto issue_codes = [&](int st) {
+            const int slot = st % NSTG;
+            mbar_arrive_expect_tx(&full_bar[slot], L::kStageBytes);
+            tma_load_2d(stage_codes(slot, 0), &tm_codes0, code_c0(st), static_cast<int>(row0),
+                        &full_bar[slot], pol_w);
+            if (NMAT == 2)
+                tma_load_2d(stage_codes(slot, 1), &tm_codes1, code_c0(st), static_cast<int>(row0),
                             &full_bar[slot], pol_w);
-                if (NMAT == 2)
-                    tma_load_2d(stage_codes(slot, 1), &tm_codes1, code_c0(st),
-                                static_cast<int>(row0), &full_bar[slot], pol_w);
-            };
-            auto issue_x = [&](int st) {
-                const int slot = st % kStages;
-                const int64_t k0 = kbeg + static_cast<int64_t>(st) * F::kStageK;
+        };
+        auto issue_x = [&](int st) {
+            const int slot = st % NSTG;
+            const int64_t k0 = kbeg + static_cast<int64_t>(st) * F::kStageK;
 #pragma unroll
-                for (int b = 0; b < F::kXBoxes; ++b)
-                    tma_load_2d(stage_x(slot) + b * kXBoxBytes, &tm_x,
-                                static_cast<int>(k0 + b * kXBoxK), 0, &full_bar[slot], pol_x);
-            };
-            // codes of the first stages before the wait on the previous kernel
-            const int pre = nstages < kStages ? nstages : kStages;
+            for (int b = 0; b < F::kXBoxes; ++b)
+                tma_load_2d(stage_x(slot) + b * kXBoxBytes, &tm_x, static_cast<int>(k0 + b * kXBoxK),
+                            0, &full_bar[slot], pol_x);
+        };
+        // codes of the first stages before the wait on the previous kernel
+        const int pre = nstages < NSTG ? nstages : NSTG;
+        if (elect_one())
             for (int st = 0; st < pre; ++st) issue_codes(st);
-            griddep_wait();
+        __syncwarp();
+        griddep_wait();
+        if (elect_one())
             for (int st = 0; st < pre; ++st) issue_x(st);
-            for (int st = kStages; st < nstages; ++st) {
-                const int slot = st % kStages;
-                if (!wait_or_abort(&empty_bar[slot], ((st / kStages) - 1) & 1, &abort_sh)) break;
+        __syncwarp();
+        for (int st = NSTG; st < nstages; ++st) {
+            const int slot = st % NSTG;
+            if (!warp_wait_or_abort(&empty_bar[slot], ((st / NSTG) - 1) & 1, &abort_sh)) break;
+            if (elect_one()) {
                 issue_codes(st);
                 issue_x(st);
             }
-            // drain: every issued copy lands before the CTA may exit (bounded)
-            const int first = nstages > kStages ? nstages - kStages : 0;
-            for (int st = first; st < nstages; ++st)
-                mbar_wait_bounded(&full_bar[st % kStages], (st / kStages) & 1);
+            __syncwarp();
         }
+        // drain: every issued copy lands before the CTA may exit (bounded)
+        const int first = nstages > NSTG ? nstages - NSTG : 0;
+        for (int st = first; st < nstages; ++st)
+            mbar_wait_bounded(&full_bar[st % NSTG], (st / NSTG) & 1);
+        __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA ---
-        if (lane == 0) {
-            for (int t = 0; t < nsteps; ++t) {
-                const int st = t / KSTEPS, kk = t % KSTEPS;
-                const int slot = st % kStages;
-                const int a = t % NA;
-                if (kk == 0 && !wait_or_abort(&full_bar[slot], (st / kStages) & 1, &abort_sh)) break;
-                if (!wait_or_abort(&afull_bar[a], (t / NA) & 1, &abort_sh)) break;
-                tc_fence_after();
-                const uint64_t bdesc = sw128_kmajor_desc(stage_x(slot) + (kk / 4) * kXBoxBytes +
-                                                         (kk % 4) * (kKStep * 2));
+        // One A group (8 steps of 16 k) at a time, issued back to back: step j
+        // accumulates into accumulator j % kAcc, so consecutive MMAs do not
+        // wait for one another's result; one commit then releases the group.
+        // The whole warp runs the loop and waits; the elected lane issues the
+        // MMAs and their commits.
+        for (int g = 0; g < ngroups; ++g) {
+            const int st = g / GPS, gi = g % GPS;
+            const int slot = st % NSTG;
+            const int ag = g % NG;
+            if (gi == 0 && !warp_wait_or_abort(&full_bar[slot], (st / NSTG) & 1, &abort_sh)) break;
+            if (!warp_wait_or_abort(&afull_bar[ag], (g / NG) & 1, &abort_sh)) break;
+            tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
-                for (int m = 0; m < NMAT; ++m)
-                    tc_mma_ts(tmem + 16 * m, tmem + a_col(a, m), bdesc, kIdescF16M128N16,
-                              t > 0 ? 1u : 0u);
-                tc_commit(&aempty_bar[a]);                     // A slot free once read
-                if (kk == KSTEPS - 1) tc_commit(&empty_bar[slot]);  // X of this stage read
+                for (int j = 0; j < kGroupSteps; ++j) {
+                    const int kk = gi * kGroupSteps + j;  // 16-k step within the stage
+                    const uint64_t bdesc = sw128_kmajor_desc(stage_x(slot) + (kk / 4) * kXBoxBytes +
+                                                             (kk % 4) * (kKStep * 2));
+#pragma unroll
+                    for (int m = 0; m < NMAT; ++m)
+                        tc_mma_ts(tmem + d_col(m, j % kAcc), tmem + a_col(ag, j, m), bdesc,
+                                  kIdescF16M128N16, (g > 0 || j >= kAcc) ? 1u : 0u);
+                }
+                tc_commit(&aempty_bar[ag]);                     // A group free once read
+                if (gi == GPS - 1) tc_commit(&empty_bar[slot]);  // X of this stage read
             }
-            tc_commit(&done_bar);  // every MMA issued above has completed
+            __syncwarp();
         }
+        if (elect_one()) tc_commit(&done_bar);  // every MMA issued above has completed
+        __syncwarp();
     } else {
         // ---------------------------------------------------- dequantize ---
-        const int dq = warp - 2;              // 0..7
+        // Two sets of warps take alternate A groups, so that one set's group
+        // is dequantized while the other's stores drain; within a set, the
+        // SETW warps of a lane quarter split the group's steps.
+        const int dq = warp - 2;              // 0 .. NDQ - 1
         const int quarter = warp & 3;         // tensor-memory lanes 32*quarter .. +31
-        const int half = dq >> 2;             // this warp's parity of 16-k steps
+        const int sub = dq >> 2;              // 0 .. SUB - 1
+        const int set = sub / SETW;           // groups g = set (mod 2)
+        const int ssub = sub % SETW;          // steps j = ssub (mod SETW) of a group
         const int rl = quarter * 32 + lane;   // row within the tile
         const int64_t grow = row0 + rl < p.n ? row0 + rl : p.n - 1;  // tail rows: discard
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
@@ -435,23 +489,23 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             }
         };
         uint2 sv[NMAT], bv[NMAT], sv_next[NMAT], bv_next[NMAT];
-        if (nstages > 0) load_sides(0, sv, bv);
+        if (set < ngroups) load_sides(set / GPS, sv, bv);
         const int r7 = rl & 7;
-        for (int st = 0; st < nstages; ++st) {
-            const int slot = st % kStages;
-            if (st + 1 < nstages) load_sides(st + 1, sv_next, bv_next);
-            if (!warp_wait_or_abort(&full_bar[slot], (st / kStages) & 1, &abort_sh)) break;
-            bool ok = true;
-            // every A slot of this warp's steps of the stage is written, then
-            // one wait for the stores signals them all
-            for (int kk = half; kk < KSTEPS; kk += 2) {
-                const int t = st * KSTEPS + kk;
-                const int a = t % NA;
-                if (t >= NA && !warp_wait_or_abort(&aempty_bar[a], ((t / NA) - 1) & 1, &abort_sh)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
+        // every group a warp takes is its only group of that stage (int8: one
+        // group per stage; int4: two, one per set)
+        for (int g = set; g < ngroups; g += 2) {
+            const int st = g / GPS, gi = g % GPS;
+            const int slot = st % NSTG;
+            const int ag = g % NG;
+            if (g + 2 < ngroups) load_sides((g + 2) / GPS, sv_next, bv_next);
+            if (!warp_wait_or_abort(&full_bar[slot], (st / NSTG) & 1, &abort_sh)) break;
+            if (g >= NG && !warp_wait_or_abort(&aempty_bar[ag], ((g / NG) - 1) & 1, &abort_sh))
+                break;
+            tc_fence_after();
+#pragma unroll
+            for (int jj = 0; jj < kGroupSteps / SETW; ++jj) {
+                const int j = ssub + jj * SETW;
+                const int kk = gi * kGroupSteps + j;  // 16-k step within the stage
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m) {
                     uint32_t av[8];
@@ -467,26 +521,25 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                         // 16 codes = 8 bytes: half (kk & 1) of chunk kk / 2
                         const uint2 c = *reinterpret_cast<const uint2*>(
                             sgen + (tile_row - sbase) + ((((kk >> 1) ^ r7) << 4) | ((kk & 1) << 3)));
-                        const int g = kk >> 2;  // group of 64 within the stage
-                        const uint32_t sw = g < 2 ? sv[m].x : sv[m].y;
-                        const uint32_t bw = g < 2 ? bv[m].x : bv[m].y;
-                        const uint16_t s = static_cast<uint16_t>((g & 1) ? sw >> 16 : sw & 0xFFFFu);
-                        const uint16_t b = static_cast<uint16_t>((g & 1) ? bw >> 16 : bw & 0xFFFFu);
+                        const int q = kk >> 2;  // group of 64 within the stage
+                        const uint32_t sw = q < 2 ? sv[m].x : sv[m].y;
+                        const uint32_t bw = q < 2 ? bv[m].x : bv[m].y;
+                        const uint16_t s = static_cast<uint16_t>((q & 1) ? sw >> 16 : sw & 0xFFFFu);
+                        const uint16_t b = static_cast<uint16_t>((q & 1) ? bw >> 16 : bw & 0xFFFFu);
                         dequant16_i4(c, half2_bits(s), half2_bits(b), av);
                     }
-                    tc_st8(tmem + lane_addr + a_col(a, m), av);
+                    tc_st8(tmem + lane_addr + a_col(ag, j, m), av);
                 }
             }
+            // one wait for the group's stores, then the group and the codes
+            // are signalled
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                if (ok)
-                    for (int kk = half; kk < KSTEPS; kk += 2)
-                        mbar_arrive(&afull_bar[(st * KSTEPS + kk) % NA]);
-                mbar_arrive(&empty_bar[slot]);  // this warp is done with the codes
+                mbar_arrive(&afull_bar[ag]);
+                mbar_arrive(&empty_bar[slot]);  // done with the codes
             }
-            if (!ok) break;
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
                 sv[m] = sv_next[m];
@@ -507,17 +560,29 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         const bool done = wait_or_abort(&done_bar, 0, &abort_sh);
         tc_fence_after();
         __syncwarp();
+        // the kAcc partial sums of each matrix, added in accumulator order
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
-            tc_ld16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 16 * m, acc[m]);
+            const uint32_t base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+            tc_ld16(base + d_col(m, 0), acc[m]);
+#pragma unroll
+            for (int c = 1; c < kAcc; ++c) {
+                float v[16];
+                tc_ld16(base + d_col(m, c), v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[m][i] += v[i];
+            }
             if (!done)
 #pragma unroll
                 for (int i = 0; i < 16; ++i) acc[m][i] = 0.f;
         }
-    } else if (threadIdx.x == 32 && abort_sh) {
-        mbar_wait_bounded(&done_bar, 0);  // MMAs in flight finish before the CTA exits
+        // this warp's tensor-memory reads are complete (tcgen05.wait::ld)
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&fin_bar);
     }
 
+    // partials as [matrix][token][row]: consecutive rows in consecutive words
     float* red = reinterpret_cast<float*>(sgen);  // stages are free: every copy landed and was read
     if (P > 1) {
         __syncthreads();
@@ -525,21 +590,32 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-                for (int i = 0; i < 16; ++i) red[(rl * NMAT + m) * 16 + i] = acc[m][i];
+                for (int i = 0; i < 16; ++i) red[(m * 16 + i) * kTcRows + rl] = acc[m][i];
         }
         cluster_barrier();
-        // rank r finishes rows [r * 128 / P, (r + 1) * 128 / P), summing the
-        // ranks' partials in rank order
+        // rank r finishes rows [r * 128 / P, (r + 1) * 128 / P) of every
+        // token, summing the ranks' partials in rank order (all loads issued
+        // before the sums)
         const int r_lo = static_cast<int>(rank) * kTcRows / P;
         const int r_hi = (static_cast<int>(rank) + 1) * kTcRows / P;
-        for (int e = threadIdx.x - 64; e >= 0 && e < (r_hi - r_lo) * 16; e += kThreadsTc - 64) {
-            const int r = r_lo + e / 16, tok = e % 16;
+        const int R = r_hi - r_lo;
+        for (int e = threadIdx.x - 64; e >= 0 && e < R * 16; e += L::kThreads - 64) {
+            const int tok = e / R, r = r_lo + e % R;
+            float part[NMAT][kMaxClusterTc];
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m) {
+                const uint32_t addr = smem_u32(&red[(m * 16 + tok) * kTcRows + r]);
+#pragma unroll
+                for (int q = 0; q < kMaxClusterTc; ++q)
+                    if (q < P) part[m][q] = ld_dsmem(addr, static_cast<uint32_t>(q));
+            }
             float v[NMAT];
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
-                const uint32_t addr = smem_u32(&red[(r * NMAT + m) * 16 + tok]);
                 float s = 0.f;
-                for (int q = 0; q < P; ++q) s += ld_dsmem(addr, static_cast<uint32_t>(q));
+#pragma unroll
+                for (int q = 0; q < kMaxClusterTc; ++q)
+                    if (q < P) s += part[m][q];
                 v[m] = s;
             }
             const int64_t grow = row0 + r;
@@ -566,9 +642,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             }
         }
     }
-    tc_fence_before();
-    __syncthreads();
+    __syncwarp();
     if (warp == 1) {
+        // free tensor memory once no MMA is in flight and the epilogue warps
+        // have read their accumulators (bounded waits; the epilogue warps
+        // arrive even when the CTA gave up)
+        mbar_wait_bounded(&done_bar, 0);
+        mbar_wait_bounded(&fin_bar, 0);
+        __syncwarp();
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                      "r"(L::kTmemCols)
@@ -605,6 +686,32 @@ qg_status make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? QG_OK : QG_ERR_CUDA;
+}
+
+// Clusters of P CTAs the device holds at once for this kernel (cached per
+// device and P); 0 if the query fails.
+template <int FMT, int NMAT, int EPI>
+int clusters_per_wave(const DeviceInfo& dev, size_t smem, int P) {
+    static int cache[64][kMaxClusterTc + 1] = {{0}};
+    if (dev.device < 64 && cache[dev.device][P] != 0) return cache[dev.device][P];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(P * dev.num_sms));
+    cfg.blockDim = dim3(TcLayout<FMT, NMAT>::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(P);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<FMT, NMAT, EPI>, &cfg) != cudaSuccess) {
+        cudaGetLastError();  // clear the query's error
+        return 0;
+    }
+    if (dev.device < 64) cache[dev.device][P] = n > 0 ? n : -1;
+    return n;
 }
 
 template <int FMT, int NMAT, int EPI>
@@ -645,18 +752,28 @@ qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream
     p.n = Lc.n;
     p.k = Lc.k;
     p.S = Lc.S;
-    // Split K over a cluster of P CTAs (1..8, at most one per stage): every SM
-    // streams its CTAs' shares of the weight, so the time goes with the most
-    // CTAs any SM holds times the share of one, ceil(tiles P / SMs) / P; take
-    // the P that minimizes it, the smaller P on ties.
+    // Split K over a cluster of P CTAs (1..8, at most one per stage).  The
+    // clusters run in rounds of as many as the GPU holds at once (the
+    // occupancy query knows how clusters pack into the GPCs); within a round
+    // an SM's CTAs share its bandwidth.  A round costs (CTAs per SM) x (time
+    // of a tile's whole K on one SM) / P plus a fixed fill and epilogue; take
+    // the P that minimizes rounds x that, the smaller P on ties.
     const int64_t tiles = (Lc.n + kTcRows - 1) / kTcRows;
     const int64_t stages = Lc.k / F::kStageK;
+    const double bytes_per_k = FMT == 0 ? 1.0625 : 0.5625;
+    const double tile_us = kTcRows * static_cast<double>(Lc.k) * bytes_per_k * NMAT / 40e3;  // ~40 GB/s per SM
     int P = 1;
     double best = 1e30;
     for (int c = 1; c <= kMaxClusterTc && c <= stages; ++c) {
-        const int64_t per_sm = (tiles * c + dev.num_sms - 1) / dev.num_sms;
-        const double t = static_cast<double>(per_sm) / c;
-        if (t < best - 1e-9) {
+        const int cpw = clusters_per_wave<FMT, NMAT, EPI>(dev, smem, c);
+        if (cpw <= 0) continue;
+        const int64_t rounds = (tiles + cpw - 1) / cpw;
+        const int64_t per_round = (tiles + rounds - 1) / rounds;
+        const int64_t per_sm = (per_round * c + dev.num_sms - 1) / dev.num_sms;
+        const double fixed_us = c > 1 ? 4.0 : 3.0;
+        const double t = static_cast<double>(rounds) *
+                         (static_cast<double>(per_sm) * tile_us / c + fixed_us);
+        if (t < best * (1 - 1e-9)) {
             best = t;
             P = c;
         }
@@ -665,7 +782,7 @@ qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(tiles * P));
-    cfg.blockDim = dim3(kThreadsTc);
+    cfg.blockDim = dim3(L::kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
