@@ -42,6 +42,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "qg_device.cuh"
@@ -72,16 +73,21 @@ struct TcFmt {
     static constexpr int kGroup = FMT == 0 ? 32 : 64;      // k per scale (and bias)
 };
 
-template <int FMT, int NMAT>
+template <int FMT, int NMAT, bool SPLIT>
 struct TcLayout {
     using F = TcFmt<FMT>;
     static constexpr int kStageBytes = NMAT * kCodeTileBytes + F::kXBoxes * kXBoxBytes;
-    // ring depth: a single-weight CTA keeps two per SM within shared memory;
-    // with one A group per stage (int8) the depth is even, so that each of
-    // the two dequantizing sets always takes the same slots and waits every
-    // phase of their barriers (a parity wait must not skip a phase)
-    static constexpr int kStages = NMAT == 1 ? 4 : (FMT == 0 ? 6 : 5);
-    static constexpr int kSmem = kStages * kStageBytes;          // + 1 KB alignment slack
+    // ring depth: a single-weight CTA keeps two per SM within shared memory,
+    // a split gate/up CTA leaves room for the receive buffer; with one A
+    // group per stage (int8) the depth is even, so that each of the two
+    // dequantizing sets always takes the same slots and waits every phase of
+    // their barriers (a parity wait must not skip a phase)
+    static constexpr int kStages = (NMAT == 1 || SPLIT) ? 4 : (FMT == 0 ? 6 : 5);
+    // split K: the partials the CTAs of the cluster push for the rows this
+    // CTA finishes, [source rank][matrix][token][row], ceil(128 / P) rows
+    // per rank (P ceil(128 / P) < 128 + P)
+    static constexpr int kRecvBytes = SPLIT ? (kTcRows + kMaxClusterTc) * NMAT * 16 * 4 : 0;
+    static constexpr int kSmem = kStages * kStageBytes + kRecvBytes;  // + 1 KB alignment slack
     // Two single-weight CTAs fit on an SM (shared memory) and share its 512
     // tensor-memory columns; a gate/up CTA is alone on its SM and takes all.
     static constexpr uint32_t kTmemCols = NMAT == 1 ? 256 : 512;
@@ -101,7 +107,7 @@ struct TcLayout {
     static_assert(kGroupSteps % kAcc == 0, "every accumulator takes the same steps of a group");
     static_assert(kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
     static_assert(NMAT == 1 || kSmem > 116 * 1024, "a gate/up CTA must be alone on its SM");
-    static_assert(NMAT == 2 || kSmem + 1024 <= 112 * 1024, "two single-weight CTAs per SM");
+    static_assert(NMAT == 2 || kSmem + 2048 <= 113 * 1024, "two single-weight CTAs per SM");
 };
 
 struct TcParams {
@@ -125,14 +131,6 @@ __device__ __forceinline__ uint32_t cluster_ctarank_tc() {
 __device__ __forceinline__ void cluster_barrier() {
     asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
-__device__ __forceinline__ float ld_dsmem(uint32_t local_addr, uint32_t rank) {
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-    return v;
-}
-
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
                                             uint64_t* bar, uint64_t policy) {
     asm volatile(
@@ -289,13 +287,13 @@ __device__ __forceinline__ bool warp_wait_or_abort(uint64_t* bar, uint32_t parit
     return __all_sync(0xffffffffu, ok);
 }
 
-template <int FMT, int NMAT, int EPI>
-__global__ void __launch_bounds__(TcLayout<FMT, NMAT>::kThreads, 1)
+template <int FMT, int NMAT, int EPI, bool SPLIT>
+__global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_codes0,
                    const __grid_constant__ CUtensorMap tm_codes1,
                    const __grid_constant__ CUtensorMap tm_x, const TcParams p) {
     using F = TcFmt<FMT>;
-    using L = TcLayout<FMT, NMAT>;
+    using L = TcLayout<FMT, NMAT, SPLIT>;
     constexpr int NSTG = L::kStages;
     constexpr int NG = L::kAGroups;
     constexpr int GPS = L::kGroupsPerStage;
@@ -320,8 +318,8 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT>::kThreads, 1)
     unsigned char* sgen = smem_raw + (sbase - sraw);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int P = p.splits;
-    const uint32_t rank = P > 1 ? cluster_ctarank_tc() : 0u;
+    const int P = SPLIT ? p.splits : 1;
+    const uint32_t rank = SPLIT ? cluster_ctarank_tc() : 0u;
     const int64_t tile = blockIdx.x / P;
     const int64_t row0 = tile * kTcRows;
     // this CTA's K range: stages [st0, st1) of the row, split as evenly as the
@@ -582,43 +580,45 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT>::kThreads, 1)
         if (lane == 0) mbar_arrive(&fin_bar);
     }
 
-    // partials as [matrix][token][row]: consecutive rows in consecutive words
-    float* red = reinterpret_cast<float*>(sgen);  // stages are free: every copy landed and was read
-    if (P > 1) {
-        __syncthreads();
+    if (SPLIT) {
+        // Rank q finishes rows [q 128 / P, (q + 1) 128 / P).  Every CTA pushes
+        // its partial of each row into the finishing CTA's receive buffer
+        // (remote stores, no round trip); after one cluster barrier each CTA
+        // sums its rows' P partials in rank order from its own shared memory.
+        float* recv = reinterpret_cast<float*>(sgen + NSTG * L::kStageBytes);
+        const int rmax = (kTcRows + P - 1) / P;
         if (epi_warp) {
-#pragma unroll
-            for (int m = 0; m < NMAT; ++m)
-#pragma unroll
-                for (int i = 0; i < 16; ++i) red[(m * 16 + i) * kTcRows + rl] = acc[m][i];
-        }
-        cluster_barrier();
-        // rank r finishes rows [r * 128 / P, (r + 1) * 128 / P) of every
-        // token, summing the ranks' partials in rank order (all loads issued
-        // before the sums)
-        const int r_lo = static_cast<int>(rank) * kTcRows / P;
-        const int r_hi = (static_cast<int>(rank) + 1) * kTcRows / P;
-        const int R = r_hi - r_lo;
-        for (int e = threadIdx.x - 64; e >= 0 && e < R * 16; e += L::kThreads - 64) {
-            const int tok = e / R, r = r_lo + e % R;
-            float part[NMAT][kMaxClusterTc];
+            int owner = 0;
+            while (owner + 1 < P && (owner + 1) * kTcRows / P <= rl) ++owner;
+            const int r = rl - owner * kTcRows / P;
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
-                const uint32_t addr = smem_u32(&red[(m * 16 + tok) * kTcRows + r]);
+                const uint32_t base = smem_u32(
+                    &recv[((static_cast<int>(rank) * NMAT + m) * 16) * rmax + r]);
+                uint32_t remote;
+                asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+                             : "=r"(remote)
+                             : "r"(base), "r"(static_cast<uint32_t>(owner)));
 #pragma unroll
-                for (int q = 0; q < kMaxClusterTc; ++q)
-                    if (q < P) part[m][q] = ld_dsmem(addr, static_cast<uint32_t>(q));
+                for (int i = 0; i < 16; ++i)
+                    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote + i * rmax * 4),
+                                 "f"(acc[m][i])
+                                 : "memory");
             }
+        }
+        cluster_barrier();  // every push is visible; no remote access follows
+        const int r_lo = static_cast<int>(rank) * kTcRows / P;
+        const int R = (static_cast<int>(rank) + 1) * kTcRows / P - r_lo;
+        for (int e = threadIdx.x - 64; e >= 0 && e < R * 16; e += L::kThreads - 64) {
+            const int tok = e / R, r = e % R;
             float v[NMAT];
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
                 float s = 0.f;
-#pragma unroll
-                for (int q = 0; q < kMaxClusterTc; ++q)
-                    if (q < P) s += part[m][q];
+                for (int q = 0; q < P; ++q) s += recv[((q * NMAT + m) * 16 + tok) * rmax + r];
                 v[m] = s;
             }
-            const int64_t grow = row0 + r;
+            const int64_t grow = row0 + r_lo + r;
             if (tok < p.S && grow < p.n) {
                 if (EPI == kEpiPlain)
                     p.Y[static_cast<int64_t>(tok) * p.n + grow] = v[0];
@@ -627,7 +627,6 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT>::kThreads, 1)
                         f2h_rn(v[0] / (1.0f + expf(-v[0])) * v[NMAT - 1]);
             }
         }
-        cluster_barrier();  // peers keep their shared memory until it is read
     } else if (epi_warp) {
         const int64_t grow = row0 + rl;
         if (grow < p.n) {
@@ -688,15 +687,37 @@ qg_status make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int
     return r == CUDA_SUCCESS ? QG_OK : QG_ERR_CUDA;
 }
 
+// Shared memory of the kernel variant, and its attributes set once per device.
+template <int FMT, int NMAT, int EPI, bool SPLIT>
+qg_status prepare_tc(const DeviceInfo& dev, size_t* smem_out) {
+    using L = TcLayout<FMT, NMAT, SPLIT>;
+    auto kern = gemm_tc_kernel<FMT, NMAT, EPI, SPLIT>;
+    const size_t smem = L::kSmem + 1024;
+    if (smem + 2048 > static_cast<size_t>(dev.max_smem_optin)) return QG_ERR_SHAPE;
+    static bool attr_done[64] = {false};
+    if (dev.device >= 64 || !attr_done[dev.device]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return cuda_status(e);
+        // all of the unified L1 as shared memory: two single-weight CTAs per SM
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return cuda_status(e);
+        if (dev.device < 64) attr_done[dev.device] = true;
+    }
+    *smem_out = smem;
+    return QG_OK;
+}
+
 // Clusters of P CTAs the device holds at once for this kernel (cached per
 // device and P); 0 if the query fails.
-template <int FMT, int NMAT, int EPI>
+template <int FMT, int NMAT, int EPI, bool SPLIT>
 int clusters_per_wave(const DeviceInfo& dev, size_t smem, int P) {
     static int cache[64][kMaxClusterTc + 1] = {{0}};
     if (dev.device < 64 && cache[dev.device][P] != 0) return cache[dev.device][P];
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(P * dev.num_sms));
-    cfg.blockDim = dim3(TcLayout<FMT, NMAT>::kThreads);
+    cfg.blockDim = dim3(TcLayout<FMT, NMAT, SPLIT>::kThreads);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -706,7 +727,8 @@ int clusters_per_wave(const DeviceInfo& dev, size_t smem, int P) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<FMT, NMAT, EPI>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<FMT, NMAT, EPI, SPLIT>, &cfg) !=
+        cudaSuccess) {
         cudaGetLastError();  // clear the query's error
         return 0;
     }
@@ -717,28 +739,21 @@ int clusters_per_wave(const DeviceInfo& dev, size_t smem, int P) {
 template <int FMT, int NMAT, int EPI>
 qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream_t stream) {
     using F = TcFmt<FMT>;
-    using L = TcLayout<FMT, NMAT>;
-    auto kern = gemm_tc_kernel<FMT, NMAT, EPI>;
-    const size_t smem = L::kSmem + 1024;
-    if (smem + 2048 > static_cast<size_t>(dev.max_smem_optin)) return QG_ERR_SHAPE;
-    static bool attr_done[64] = {false};
-    if (dev.device >= 64 || !attr_done[dev.device]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return cuda_status(e);
-        if (dev.device < 64) attr_done[dev.device] = true;
-    }
+    size_t smem1 = 0, smemP = 0;
+    qg_status st = prepare_tc<FMT, NMAT, EPI, false>(dev, &smem1);
+    if (st != QG_OK) return st;
+    st = prepare_tc<FMT, NMAT, EPI, true>(dev, &smemP);
+    if (st != QG_OK) return st;
     CUtensorMap mc[2], mx;
     const uint64_t row_bytes = FMT == 0 ? static_cast<uint64_t>(Lc.k) : static_cast<uint64_t>(Lc.k) / 2;
     for (int m = 0; m < NMAT; ++m) {
-        qg_status st = make_map(&mc[m], Lc.codes[m], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_bytes,
-                                static_cast<uint64_t>(Lc.n), kCodeBox, kTcRows);
+        st = make_map(&mc[m], Lc.codes[m], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_bytes,
+                      static_cast<uint64_t>(Lc.n), kCodeBox, kTcRows);
         if (st != QG_OK) return st;
     }
     if (NMAT == 1) mc[1] = mc[0];
-    qg_status st = make_map(&mx, Lc.X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                            static_cast<uint64_t>(Lc.k), static_cast<uint64_t>(Lc.S), kXBoxK,
-                            kTcTokens);
+    st = make_map(&mx, Lc.X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, static_cast<uint64_t>(Lc.k),
+                  static_cast<uint64_t>(Lc.S), kXBoxK, kTcTokens);
     if (st != QG_OK) return st;
 
     TcParams p = {};
@@ -753,26 +768,36 @@ qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream
     p.k = Lc.k;
     p.S = Lc.S;
     // Split K over a cluster of P CTAs (1..8, at most one per stage).  The
-    // clusters run in rounds of as many as the GPU holds at once (the
-    // occupancy query knows how clusters pack into the GPCs); within a round
-    // an SM's CTAs share its bandwidth.  A round costs (CTAs per SM) x (time
-    // of a tile's whole K on one SM) / P plus a fixed fill and epilogue; take
-    // the P that minimizes rounds x that, the smaller P on ties.
+    // clusters run in rounds of as many as the GPU holds at once; a round
+    // costs the busiest SM's bytes over its rate plus a fixed cost (launch,
+    // pipeline fill, epilogue).  Rates and costs were measured on B200 by
+    // timing every P on the int8 and int4 projections of 2B-8B decoders: a
+    // single-weight CTA alone on its SM streams ~29 KB/us, an SM holding two
+    // ~54 KB/us, a gate/up CTA (alone by shared memory) ~45 KB/us; fixed cost
+    // ~4.4 us, ~6.8 us with the cluster reduction.  The occupancy query counts
+    // a kernel that allocates tensor memory as one CTA per SM although two
+    // single-weight CTAs co-reside, so their capacity is taken as twice the
+    // query's, and at least 90% of the slots for clusters of P (GPC packing).
+    // Take the P that minimizes rounds x round cost, the smaller P on ties.
     const int64_t tiles = (Lc.n + kTcRows - 1) / kTcRows;
     const int64_t stages = Lc.k / F::kStageK;
     const double bytes_per_k = FMT == 0 ? 1.0625 : 0.5625;
-    const double tile_us = kTcRows * static_cast<double>(Lc.k) * bytes_per_k * NMAT / 40e3;  // ~40 GB/s per SM
+    const double tile_kb = kTcRows * static_cast<double>(Lc.k) * bytes_per_k * NMAT / 1e3;
     int P = 1;
     double best = 1e30;
     for (int c = 1; c <= kMaxClusterTc && c <= stages; ++c) {
-        const int cpw = clusters_per_wave<FMT, NMAT, EPI>(dev, smem, c);
+        int cpw = c == 1 ? clusters_per_wave<FMT, NMAT, EPI, false>(dev, smem1, c)
+                         : clusters_per_wave<FMT, NMAT, EPI, true>(dev, smemP, c);
         if (cpw <= 0) continue;
+        if (NMAT == 1)
+            cpw = std::max(2 * cpw, static_cast<int>(0.9 * 2 * dev.num_sms / c));
         const int64_t rounds = (tiles + cpw - 1) / cpw;
         const int64_t per_round = (tiles + rounds - 1) / rounds;
         const int64_t per_sm = (per_round * c + dev.num_sms - 1) / dev.num_sms;
-        const double fixed_us = c > 1 ? 4.0 : 3.0;
+        const double rate = NMAT == 2 ? 45.0 : (per_sm >= 2 ? 54.0 : 29.0);
+        const double fixed_us = c > 1 ? 6.8 : 4.4;
         const double t = static_cast<double>(rounds) *
-                         (static_cast<double>(per_sm) * tile_us / c + fixed_us);
+                         (static_cast<double>(per_sm) * tile_kb / c / rate + fixed_us);
         if (t < best * (1 - 1e-9)) {
             best = t;
             P = c;
@@ -782,8 +807,8 @@ qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(tiles * P));
-    cfg.blockDim = dim3(L::kThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.blockDim = dim3(TcLayout<FMT, NMAT, false>::kThreads);
+    cfg.dynamicSmemBytes = P > 1 ? smemP : smem1;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     int na = 0;
@@ -797,7 +822,11 @@ qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream
     ++na;
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    return cuda_status(cudaLaunchKernelEx(&cfg, kern, mc[0], mc[1], mx, p));
+    if (P > 1)
+        return cuda_status(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<FMT, NMAT, EPI, true>, mc[0],
+                                              mc[1], mx, p));
+    return cuda_status(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<FMT, NMAT, EPI, false>, mc[0],
+                                          mc[1], mx, p));
 }
 
 }  // namespace
