@@ -496,8 +496,16 @@ def run_ours(a):
         dom = {"kernel": "sweep_kernel (persistent sweep)", "us": el_ms * 1e3 / steps,
                "gbs": sweep_bytes / (el_ms * 1e-3 / steps) / 1e9, "bytes": sweep_bytes,
                "launches": steps}
+        kinds = None
     else:
-        dom = _time_gate_up(sw, stream, dev, qg, torch)
+        # the dominant kernel is the kind of call with the largest share of
+        # the sweep's time
+        kinds = _time_kinds(sw, stream, dev, torch)
+        names = KERNEL_OF_KIND[(S == 1, decode)]
+        kd = max(kinds, key=lambda k: kinds[k]["share"])
+        dom = {"kernel": names[kd], "us": kinds[kd]["us"], "gbs": kinds[kd]["gbs"],
+               "bytes": kinds[kd]["bytes"], "launches": kinds[kd]["launches_per_sweep"] * steps,
+               "share": kinds[kd]["share"], "kind": kd}
 
     # --- end to end: pinned host inputs -> sweep -> greedy token to host ---
     e2e = _time_e2e(sw, graph, G, steps, a.warmup, stream, dev, world, torch, persistent)
@@ -525,7 +533,17 @@ def run_ours(a):
             "unit": "GB/s", "frac": round(dom["gbs"] / peak, 4),
             "traffic": profiled_traffic(dom["kernel"], a.workload),
             "algorithmic_bytes_per_launch": dom["bytes"],
-            "launch_us": round(dom["us"], 3), "launches": dom["launches"]},
+            "launch_us": round(dom["us"], 3), "launches": dom["launches"],
+            "time_share": round(dom.get("share", 1.0), 4),
+            "sweep_frac": round(value / world / peak, 4)},
+        **({"kernels": {k: {"kernel": KERNEL_OF_KIND[(S == 1, decode)][k],
+                            "us_per_launch": round(v["us"], 3),
+                            "launches_per_sweep": v["launches_per_sweep"],
+                            "bytes_per_launch": v["bytes"], "gbs": round(v["gbs"], 1),
+                            "frac": round(v["gbs"] / peak, 4), "time_share": round(v["share"], 4)}
+                        for k, v in kinds.items()},
+            "kernels_timing": "each kind alone: graph of its launches over all layers, L2 "
+                              "flushed before each replay"} if kinds else {}),
         "e2e": e2e,
         "gpu_launches": steps * sw.launches_per_sweep(persistent),
         "clocks": clk,
@@ -541,39 +559,71 @@ def run_ours(a):
     return 0
 
 
-def _time_gate_up(sw, stream, dev, qg, torch):
-    """Average duration of the fused gate/up SwiGLU launch, timed with CUDA
-    events on its stream over a graph of every layer's launch (the weights of
-    all layers together are far larger than L2)."""
-    g = torch.cuda.CUDAGraph()
+KERNEL_OF_KIND = {
+    # (S == 1, decode step) -> kind -> the kernel that runs it
+    (True, False): {"qkv": "gemv_ring_kernel", "o": "gemv_ring_kernel",
+                    "gate_up": "gemv_ring_kernel (fused gate/up + SwiGLU)",
+                    "down": "gemv_ring_kernel", "head": "gemv_ring_kernel (head + argmax)"},
+    (True, True): {"qkv": "gemv_ring_kernel (RMSNorm in)", "o": "gemv_ring_kernel (residual)",
+                   "attention": "decode_attention_kernel",
+                   "gate_up": "gemv_ring_kernel (RMSNorm in, fused gate/up + SwiGLU)",
+                   "down": "gemv_ring_kernel (residual)",
+                   "head": "gemv_ring_kernel (RMSNorm in, head + argmax)"},
+    (False, False): {"qkv": "gemm_tc_kernel", "o": "gemm_tc_kernel",
+                     "gate_up": "gemm_tc_kernel (fused gate/up + SwiGLU)",
+                     "down": "gemm_tc_kernel", "head": "gemv_ring_kernel (head + argmax)"},
+}
+
+
+def _time_kinds(sw, stream, dev, torch, reps=5):
+    """Average launch duration of every kind of call in the sweep (qkv, o,
+    gate/up, down, head, attention), each timed with CUDA events on its
+    stream over a graph of that kind's launches across all layers, with L2
+    flushed (a 256 MB write, more than the 126 MB L2) before every timed
+    replay.  Returns per kind: us per launch, bytes per launch, launches per
+    sweep, GB/s and the share of the summed time."""
+    by_kind = {}
+    for l in range(sw.dec.layers):
+        for kind, nbytes, _ in sw.layer_calls(l):
+            by_kind.setdefault(kind, []).append(nbytes)
+    by_kind["head"] = [sw.head.nbytes]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     s = torch.cuda.Stream(device=dev)
-    s.wait_stream(stream)
-    with torch.cuda.graph(g, stream=s):
-        for l, L in enumerate(sw.layers):
-            if sw.decode_step:  # the decode step's variant: RMSNorm of the hidden state
-                qg.qg_rmsnorm_gate_up_swiglu(L.gate, L.up, sw.hstate, sw.gamma_mlp[l], sw.eps,
-                                             sw.h[0])
+    out = {}
+    for kind in by_kind:
+        g = torch.cuda.CUDAGraph()
+        s.wait_stream(stream)
+        with torch.cuda.graph(g, stream=s):
+            if kind == "head":
+                sw.run_head(s)
             else:
-                qg.qg_gate_up_swiglu(L.gate, L.up, sw.x[l], sw.h if sw.S > 1 else sw.h[0])
-    stream.wait_stream(s)
-    reps = max(3, int(2e9 // (sw.layers[0].gate.nbytes * 2 * len(sw.layers))) + 3)
-    for _ in range(3):
-        g.replay()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        g.replay()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    launches = reps * len(sw.layers)
-    us = e0.elapsed_time(e1) * 1e3 / launches
-    nbytes = sw.layers[0].gate.nbytes + sw.layers[0].up.nbytes
-    del g
-    return {"kernel": ("gemv_ring_kernel (fused gate/up + SwiGLU)" if sw.S == 1
-                       else "gemm_s16_kernel (fused gate/up + SwiGLU)"),
-            "gbs": nbytes / (us * 1e-6) / 1e9, "us": us, "bytes": nbytes,
-            "launches": launches}
+                for l in range(sw.dec.layers):
+                    for k2, _, enqueue in sw.layer_calls(l, s):
+                        if k2 == kind:
+                            enqueue()
+        stream.wait_stream(s)
+        for _ in range(2):
+            g.replay()
+        total_ms = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            total_ms += e0.elapsed_time(e1)
+        n = len(by_kind[kind])
+        us = total_ms * 1e3 / (reps * n)
+        nbytes = sum(by_kind[kind]) / n
+        out[kind] = {"us": us, "bytes": int(nbytes), "launches_per_sweep": n,
+                     "gbs": nbytes / (us * 1e-6) / 1e9}
+        del g
+    del flush
+    tot = sum(v["us"] * v["launches_per_sweep"] for v in out.values())
+    for v in out.values():
+        v["share"] = v["us"] * v["launches_per_sweep"] / tot
+    return out
 
 
 def _time_e2e(sw, graph, G, steps, warmup, stream, dev, world, torch, persistent):

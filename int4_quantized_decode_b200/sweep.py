@@ -38,7 +38,7 @@ allocates buffers, draws the seeded weights, and replays the graph.
 from __future__ import annotations
 
 from dataclasses import dataclass
-from typing import List, Optional
+from typing import Callable, List, Optional, Tuple
 
 import torch
 
@@ -194,33 +194,56 @@ class DecodeSweep:
     def head_input(self) -> torch.Tensor:
         return self.x_head if self.S == 1 else self.x_head[self.S - 1]
 
+    def layer_calls(self, l: int, stream=None) -> List[Tuple[str, int, Callable[[], None]]]:
+        """Layer l's launches in run order as (kind, bytes, enqueue): kind is
+        one of qkv, attention, o, gate_up, down; bytes are the algorithmic
+        bytes the launch streams (weights; K/V rows for attention)."""
+        d, L = self.dec, self.layers[l]
+        calls: List[Tuple[str, int, Callable[[], None]]] = []
+        if self.decode_step:
+            h = self.hstate
+            calls.append(("qkv", L.qkv.nbytes, lambda: qg.qg_rmsnorm_gemv_s1(
+                L.qkv, h, self.gamma_attn[l], self.eps, self.y_qkv[0], self.y16_qkv, stream)))
+            if self.context:
+                calls.append(("attention", 2 * d.kv_dim * self.context * 2,
+                              lambda: qg.qg_decode_attention(
+                                  self.y_qkv[0], self.kcache[l], self.vcache[l], self.pos,
+                                  self.attn_out, self.attn_ws, stream=stream)))
+                calls.append(("o", L.o.nbytes,
+                              lambda: qg.qg_gemv_s1_residual(L.o, self.attn_out, h, stream)))
+            else:
+                calls.append(("o", L.o.nbytes, lambda: qg.qg_gemv_s1_residual(
+                    L.o, self.y16_qkv[: d.q_dim], h, stream)))
+            calls.append(("gate_up", L.gate.nbytes + L.up.nbytes,
+                          lambda: qg.qg_rmsnorm_gate_up_swiglu(
+                              L.gate, L.up, h, self.gamma_mlp[l], self.eps, self.h[0], stream)))
+            calls.append(("down", L.down.nbytes,
+                          lambda: qg.qg_gemv_s1_residual(L.down, self.h[0], h, stream)))
+        elif self.S == 1:
+            calls.append(("qkv", L.qkv.nbytes, lambda: qg.qg_gemv_s1(
+                L.qkv, self.x[l], self.y_qkv[0], self.y16_qkv, stream)))
+            calls.append(("o", L.o.nbytes, lambda: qg.qg_gemv_s1(
+                L.o, self.y16_qkv[: d.q_dim], self.y_o[0], None, stream)))
+            calls.append(("gate_up", L.gate.nbytes + L.up.nbytes, lambda: qg.qg_gate_up_swiglu(
+                L.gate, L.up, self.x[l], self.h[0], stream)))
+            calls.append(("down", L.down.nbytes, lambda: qg.qg_gemv_s1(
+                L.down, self.h[0], self.y_down[0], None, stream)))
+        else:
+            calls.append(("qkv", L.qkv.nbytes,
+                          lambda: qg.qg_gemm_s16(L.qkv, self.x[l], self.y_qkv, stream)))
+            calls.append(("o", L.o.nbytes,
+                          lambda: qg.qg_gemm_s16(L.o, self.x_o[l], self.y_o, stream)))
+            calls.append(("gate_up", L.gate.nbytes + L.up.nbytes, lambda: qg.qg_gate_up_swiglu(
+                L.gate, L.up, self.x[l], self.h, stream)))
+            calls.append(("down", L.down.nbytes,
+                          lambda: qg.qg_gemm_s16(L.down, self.h, self.y_down, stream)))
+        return calls
+
     def run_layer(self, l: int, stream=None) -> None:
         """Enqueue layer l's launches on `stream` (default: current): four, five with
         the attention of a decode step over a K/V cache."""
-        d, L = self.dec, self.layers[l]
-        if self.decode_step:
-            h = self.hstate
-            qg.qg_rmsnorm_gemv_s1(L.qkv, h, self.gamma_attn[l], self.eps, self.y_qkv[0],
-                                  self.y16_qkv, stream)
-            if self.context:
-                qg.qg_decode_attention(self.y_qkv[0], self.kcache[l], self.vcache[l], self.pos,
-                                       self.attn_out, self.attn_ws, stream=stream)
-                qg.qg_gemv_s1_residual(L.o, self.attn_out, h, stream)
-            else:
-                qg.qg_gemv_s1_residual(L.o, self.y16_qkv[: d.q_dim], h, stream)
-            qg.qg_rmsnorm_gate_up_swiglu(L.gate, L.up, h, self.gamma_mlp[l], self.eps, self.h[0],
-                                         stream)
-            qg.qg_gemv_s1_residual(L.down, self.h[0], h, stream)
-        elif self.S == 1:
-            qg.qg_gemv_s1(L.qkv, self.x[l], self.y_qkv[0], self.y16_qkv, stream)
-            qg.qg_gemv_s1(L.o, self.y16_qkv[: d.q_dim], self.y_o[0], None, stream)
-            qg.qg_gate_up_swiglu(L.gate, L.up, self.x[l], self.h[0], stream)
-            qg.qg_gemv_s1(L.down, self.h[0], self.y_down[0], None, stream)
-        else:
-            qg.qg_gemm_s16(L.qkv, self.x[l], self.y_qkv, stream)
-            qg.qg_gemm_s16(L.o, self.x_o[l], self.y_o, stream)
-            qg.qg_gate_up_swiglu(L.gate, L.up, self.x[l], self.h, stream)
-            qg.qg_gemm_s16(L.down, self.h, self.y_down, stream)
+        for _, _, enqueue in self.layer_calls(l, stream):
+            enqueue()
 
     def run_head(self, stream=None) -> None:
         if self.decode_step:
