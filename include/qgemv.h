@@ -202,12 +202,13 @@ QG_API qg_status qg_head_argmax(const qg_weight* W, const uint16_t* x, float* lo
  * the reduction scratch is a 256-byte array inside the library that every GPU
  * loading the library keeps until the process exits.  The call allocates
  * nothing (no cudaMalloc, no cudaFree, no allocating library routine).
- *   - The first call on each device looks up that array's device address
- *     (cudaGetSymbolAddress, with the device current); make that first call
- *     before capturing any stream into a CUDA graph.  The address is kept
- *     for the life of the process: after cudaDeviceReset (or anything else
- *     that destroys the device's primary context) the library may hold a
- *     stale address, so do not call this entry point on that device again.
+ *   - Every call whose stream is not being captured looks up that array's
+ *     device address (cudaGetSymbolAddress, with the device current), so a
+ *     call after cudaDeviceReset finds the reloaded array.  A call made
+ *     while `stream` is being captured into a CUDA graph uses the address
+ *     of the last uncaptured call on the device: make one uncaptured call
+ *     first (a first call during capture returns QG_ERR_CUDA), and capture
+ *     again after a device reset.
  *   - Each call clears the scratch on `stream` before the kernel runs (an
  *     asynchronous memset of 256 bytes), because the array keeps what the
  *     previous call left there.

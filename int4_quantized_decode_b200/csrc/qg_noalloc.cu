@@ -21,23 +21,32 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = 256;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch, looked up once per device.  In host
-// code the symbol's name is only a host-side handle, never a device address.
+// Device address of g_noalloc_scratch on each device.  In host code the
+// symbol's name is only a host-side handle, never a device address.  The
+// address is looked up again on every call whose stream is not being captured
+// (a reset context reloads the module and may move the array); a captured call
+// uses the address of the last uncaptured one, since a lookup during capture
+// may not be allowed.
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
 
-qg_status scratch_for_current_device(void** out) {
+qg_status scratch_for_current_device(cudaStream_t stream, void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_status(e);
     if (dev < 0 || dev >= kMaxDevices) return QG_ERR_CUDA;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(stream, &cap);
+    if (e != cudaSuccess) return cuda_status(e);
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (g_scratch_ptr[dev] == nullptr) {
+    if (cap == cudaStreamCaptureStatusNone) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return cuda_status(e);
         g_scratch_ptr[dev] = p;
+    } else if (g_scratch_ptr[dev] == nullptr) {
+        return QG_ERR_CUDA;  // first call on this device made during capture
     }
     *out = g_scratch_ptr[dev];
     return QG_OK;
@@ -53,7 +62,7 @@ extern "C" qg_status qg_head_argmax_noalloc(const qg_weight* W, const uint16_t* 
     // A request for more scratch than the built-in array holds is refused.
     if (qg_head_argmax_workspace_bytes(W->n) > qg::kNoAllocScratchBytes) return QG_ERR_WORKSPACE;
     void* scratch = nullptr;
-    qg_status st = qg::scratch_for_current_device(&scratch);
+    qg_status st = qg::scratch_for_current_device(stream, &scratch);
     if (st != QG_OK) return st;
     // The array keeps whatever the previous call left; the kernel needs its
     // key and ticket at zero, so clear them on this stream first.
