@@ -115,15 +115,16 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-# The sources of the S=1 streaming kernels whose DRAM traffic profiles/dram_traffic.txt
+# The sources of the S=1 and S<=16 kernels whose DRAM traffic profiles/dram_traffic.txt
 # records: a committed traffic figure is used only while these are unchanged.
-S1_KERNEL_SOURCES = ("qg_device.cuh", "qg_gemv.cu", "qg_gemv_impl.cuh", "qg_internal.h")
+KERNEL_SOURCES = ("qg_device.cuh", "qg_gemv.cu", "qg_gemv_impl.cuh", "qg_internal.h",
+                  "qg_gemm_tc.cu")
 
 
 def csrc_digest() -> str:
     h = hashlib.sha256()
     d = os.path.join(ROOT, "int4_quantized_decode_b200", "csrc")
-    for name in S1_KERNEL_SOURCES:
+    for name in KERNEL_SOURCES:
         with open(os.path.join(d, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
