@@ -64,6 +64,11 @@ constexpr int kCodeTileBytes = kTcRows * kCodeBox;  // 16 KB
 constexpr int kAcc = 4;            // accumulators per weight matrix: independent MMA chains
 constexpr int kGroupSteps = 8;     // 16-k steps per A group (one commit releases a group)
 constexpr int kMaxClusterTc = 8;
+// Gate/up as pair tiles: one 128-row MMA tile holds 64 gate rows (tensor-memory
+// lanes 0-63) and the same 64 rows of up (lanes 64-127), so a SwiGLU call runs
+// with single-weight resources (two CTAs per SM, twice the tiles).
+constexpr int kEpiPair = 100;
+constexpr int kPairRows = kTcRows / 2;
 
 template <int FMT>
 struct TcFmt {
@@ -86,7 +91,11 @@ struct TcLayout {
     // split K: the partials the CTAs of the cluster push for the rows this
     // CTA finishes, [source rank][matrix][token][row], ceil(128 / P) rows
     // per rank (P ceil(128 / P) < 128 + P)
-    static constexpr int kRecvBytes = SPLIT ? (kTcRows + kMaxClusterTc) * NMAT * 16 * 4 : 0;
+    // (pair tiles: [source rank][gate|up][token][pair row], ceil(64 / P) pair rows)
+    static constexpr int kRecvBytes =
+        !SPLIT ? 0
+               : (NMAT == 1 ? 2 * (kPairRows + kMaxClusterTc) * 16 * 4
+                            : (kTcRows + kMaxClusterTc) * NMAT * 16 * 4);
     static constexpr int kSmem = kStages * kStageBytes + kRecvBytes;  // + 1 KB alignment slack
     // Two single-weight CTAs fit on an SM (shared memory) and share its 512
     // tensor-memory columns; a gate/up CTA is alone on its SM and takes all.
@@ -320,8 +329,10 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = SPLIT ? p.splits : 1;
     const uint32_t rank = SPLIT ? cluster_ctarank_tc() : 0u;
+    constexpr bool PAIR = EPI == kEpiPair;
+    static_assert(!PAIR || NMAT == 1, "a pair tile holds both matrices in one MMA tile");
     const int64_t tile = blockIdx.x / P;
-    const int64_t row0 = tile * kTcRows;
+    const int64_t row0 = tile * (PAIR ? kPairRows : kTcRows);  // first output row
     // this CTA's K range: stages [st0, st1) of the row, split as evenly as the
     // stage count allows
     const int total_st = static_cast<int>(p.k / F::kStageK);
@@ -390,6 +401,9 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, 1)
             mbar_arrive_expect_tx(&full_bar[slot], L::kStageBytes);
             tma_load_2d(stage_codes(slot, 0), &tm_codes0, code_c0(st), static_cast<int>(row0),
                         &full_bar[slot], pol_w);
+            if (PAIR)  // up rows below the gate rows (64-row boxes)
+                tma_load_2d(stage_codes(slot, 0) + kPairRows * kCodeBox, &tm_codes1, code_c0(st),
+                            static_cast<int>(row0), &full_bar[slot], pol_w);
             if (NMAT == 2)
                 tma_load_2d(stage_codes(slot, 1), &tm_codes1, code_c0(st), static_cast<int>(row0),
                             &full_bar[slot], pol_w);
@@ -468,15 +482,21 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, 1)
         const int set = sub / SETW;           // groups g = set (mod 2)
         const int ssub = sub % SETW;          // steps j = ssub (mod SETW) of a group
         const int rl = quarter * 32 + lane;   // row within the tile
-        const int64_t grow = row0 + rl < p.n ? row0 + rl : p.n - 1;  // tail rows: discard
+        const int64_t grow_raw = PAIR ? row0 + (rl & (kPairRows - 1)) : row0 + rl;
+        const int64_t grow = grow_raw < p.n ? grow_raw : p.n - 1;  // tail rows: discard
+        const int msrc = PAIR ? rl / kPairRows : 0;                 // pair tile: gate or up
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
         const int64_t sides_per_row = p.k / F::kGroup;
         const uint16_t* srow[NMAT];
         const uint16_t* brow[NMAT];
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
-            srow[m] = p.scales[m] + grow * sides_per_row + kbeg / F::kGroup;
-            brow[m] = FMT == 1 ? p.biases[m] + grow * sides_per_row + kbeg / F::kGroup : nullptr;
+            // (a select, not an index: a parameter array indexed at run time
+            // would be copied to local memory)
+            const uint16_t* sbase = (m + msrc) == 0 ? p.scales[0] : p.scales[1];
+            const uint16_t* bbase = (m + msrc) == 0 ? p.biases[0] : p.biases[1];
+            srow[m] = sbase + grow * sides_per_row + kbeg / F::kGroup;
+            brow[m] = FMT == 1 ? bbase + grow * sides_per_row + kbeg / F::kGroup : nullptr;
         }
         // the row's 4 scales (and biases) of a stage: 8 bytes each
         auto load_sides = [&](int st, uint2 (&sv)[NMAT], uint2 (&bv)[NMAT]) {
@@ -580,7 +600,62 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, 1)
         if (lane == 0) mbar_arrive(&fin_bar);
     }
 
-    if (SPLIT) {
+    if (PAIR) {
+        // Pair tile: lane r holds gate row r, lane 64 + r the same row of up.
+        const int pr = rl & (kPairRows - 1), mm = rl / kPairRows;
+        if (SPLIT) {
+            // as below, by pair row: rank q finishes pair rows [q 64 / P, (q + 1) 64 / P)
+            // and receives both matrices' partials of them
+            float* recv = reinterpret_cast<float*>(sgen + NSTG * L::kStageBytes);
+            const int rmax = (kPairRows + P - 1) / P;
+            if (epi_warp) {
+                int owner = 0;
+                while (owner + 1 < P && (owner + 1) * kPairRows / P <= pr) ++owner;
+                const int r = pr - owner * kPairRows / P;
+                const uint32_t base =
+                    smem_u32(&recv[((static_cast<int>(rank) * 2 + mm) * 16) * rmax + r]);
+                uint32_t remote;
+                asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+                             : "=r"(remote)
+                             : "r"(base), "r"(static_cast<uint32_t>(owner)));
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote + i * rmax * 4),
+                                 "f"(acc[0][i])
+                                 : "memory");
+            }
+            cluster_barrier();  // every push is visible; no remote access follows
+            const int r_lo = static_cast<int>(rank) * kPairRows / P;
+            const int R = (static_cast<int>(rank) + 1) * kPairRows / P - r_lo;
+            for (int e = threadIdx.x - 64; e >= 0 && e < R * 16; e += L::kThreads - 64) {
+                const int tok = e / R, r = e % R;
+                float g = 0.f, u = 0.f;
+                for (int q = 0; q < P; ++q) {
+                    g += recv[((q * 2 + 0) * 16 + tok) * rmax + r];
+                    u += recv[((q * 2 + 1) * 16 + tok) * rmax + r];
+                }
+                const int64_t grow = row0 + r_lo + r;
+                if (tok < p.S && grow < p.n)
+                    p.H[static_cast<int64_t>(tok) * p.n + grow] = f2h_rn(g / (1.0f + expf(-g)) * u);
+            }
+        } else if (epi_warp) {
+            // the four epilogue warps exchange their rows through shared memory
+            // (the stages are free: every copy landed and was read)
+            float* xch = reinterpret_cast<float*>(sgen);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) xch[i * kTcRows + rl] = acc[0][i];
+            __syncwarp();
+            asm volatile("barrier.sync 1, 128;" ::: "memory");
+            for (int e = (warp - 2) * 32 + lane; e < kPairRows * 16; e += 128) {
+                const int tok = e / kPairRows, r = e % kPairRows;
+                const float g = xch[tok * kTcRows + r], u = xch[tok * kTcRows + kPairRows + r];
+                const int64_t grow = row0 + r;
+                if (tok < p.S && grow < p.n)
+                    p.H[static_cast<int64_t>(tok) * p.n + grow] = f2h_rn(g / (1.0f + expf(-g)) * u);
+            }
+        }
+        (void)mm;
+    } else if (SPLIT) {
         // Rank q finishes rows [q 128 / P, (q + 1) 128 / P).  Every CTA pushes
         // its partial of each row into the finishing CTA's receive buffer
         // (remote stores, no round trip); after one cluster barrier each CTA
@@ -736,37 +811,11 @@ int clusters_per_wave(const DeviceInfo& dev, size_t smem, int P) {
     return n;
 }
 
+// The split P of a launch and the time the model expects for it (us).
 template <int FMT, int NMAT, int EPI>
-qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream_t stream) {
+double choose_split(const GemmS16Launch& Lc, const DeviceInfo& dev, size_t smem1, size_t smemP,
+                    int* P_out) {
     using F = TcFmt<FMT>;
-    size_t smem1 = 0, smemP = 0;
-    qg_status st = prepare_tc<FMT, NMAT, EPI, false>(dev, &smem1);
-    if (st != QG_OK) return st;
-    st = prepare_tc<FMT, NMAT, EPI, true>(dev, &smemP);
-    if (st != QG_OK) return st;
-    CUtensorMap mc[2], mx;
-    const uint64_t row_bytes = FMT == 0 ? static_cast<uint64_t>(Lc.k) : static_cast<uint64_t>(Lc.k) / 2;
-    for (int m = 0; m < NMAT; ++m) {
-        st = make_map(&mc[m], Lc.codes[m], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_bytes,
-                      static_cast<uint64_t>(Lc.n), kCodeBox, kTcRows);
-        if (st != QG_OK) return st;
-    }
-    if (NMAT == 1) mc[1] = mc[0];
-    st = make_map(&mx, Lc.X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, static_cast<uint64_t>(Lc.k),
-                  static_cast<uint64_t>(Lc.S), kXBoxK, kTcTokens);
-    if (st != QG_OK) return st;
-
-    TcParams p = {};
-    for (int m = 0; m < 2; ++m) {
-        const int src = m < NMAT ? m : 0;
-        p.scales[m] = Lc.scales[src];
-        p.biases[m] = Lc.biases[src];
-    }
-    p.Y = Lc.Y;
-    p.H = Lc.H;
-    p.n = Lc.n;
-    p.k = Lc.k;
-    p.S = Lc.S;
     // Split K over a cluster of P CTAs (1..8, at most one per stage).  The
     // clusters run in rounds of as many as the GPU holds at once; a round
     // costs the busiest SM's bytes over its rate plus a fixed cost (launch,
@@ -779,9 +828,11 @@ qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream
     // single-weight CTAs co-reside, so their capacity is taken as twice the
     // query's, and at least 90% of the slots for clusters of P (GPC packing).
     // Take the P that minimizes rounds x round cost, the smaller P on ties.
-    const int64_t tiles = (Lc.n + kTcRows - 1) / kTcRows;
+    constexpr bool PAIR = EPI == kEpiPair;
+    const int64_t tiles = (Lc.n + (PAIR ? kPairRows : kTcRows) - 1) / (PAIR ? kPairRows : kTcRows);
     const int64_t stages = Lc.k / F::kStageK;
     const double bytes_per_k = FMT == 0 ? 1.0625 : 0.5625;
+    // a tile streams 128 weight rows per matrix (a pair tile: 64 of each)
     const double tile_kb = kTcRows * static_cast<double>(Lc.k) * bytes_per_k * NMAT / 1e3;
     int P = 1;
     double best = 1e30;
@@ -803,7 +854,48 @@ qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream
             P = c;
         }
     }
+    *P_out = P;
+    return best;
+}
+
+template <int FMT, int NMAT, int EPI>
+qg_status prepare_both(const DeviceInfo& dev, size_t* smem1, size_t* smemP) {
+    qg_status st = prepare_tc<FMT, NMAT, EPI, false>(dev, smem1);
+    if (st != QG_OK) return st;
+    return prepare_tc<FMT, NMAT, EPI, true>(dev, smemP);
+}
+
+template <int FMT, int NMAT, int EPI>
+qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream_t stream,
+                      int P, size_t smem1, size_t smemP) {
+    constexpr bool PAIR = EPI == kEpiPair;
+    constexpr int kMats = PAIR ? 2 : NMAT;
+    CUtensorMap mc[2], mx;
+    const uint64_t row_bytes = FMT == 0 ? static_cast<uint64_t>(Lc.k) : static_cast<uint64_t>(Lc.k) / 2;
+    for (int m = 0; m < kMats; ++m) {
+        qg_status st = make_map(&mc[m], Lc.codes[m], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_bytes,
+                                static_cast<uint64_t>(Lc.n), kCodeBox, PAIR ? kPairRows : kTcRows);
+        if (st != QG_OK) return st;
+    }
+    if (kMats == 1) mc[1] = mc[0];
+    qg_status st = make_map(&mx, Lc.X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                            static_cast<uint64_t>(Lc.k), static_cast<uint64_t>(Lc.S), kXBoxK,
+                            kTcTokens);
+    if (st != QG_OK) return st;
+
+    TcParams p = {};
+    for (int m = 0; m < 2; ++m) {
+        const int src = m < kMats ? m : 0;
+        p.scales[m] = Lc.scales[src];
+        p.biases[m] = Lc.biases[src];
+    }
+    p.Y = Lc.Y;
+    p.H = Lc.H;
+    p.n = Lc.n;
+    p.k = Lc.k;
+    p.S = Lc.S;
     p.splits = P;
+    const int64_t tiles = (Lc.n + (PAIR ? kPairRows : kTcRows) - 1) / (PAIR ? kPairRows : kTcRows);
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(tiles * P));
@@ -829,6 +921,30 @@ qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream
                                           mc[1], mx, p));
 }
 
+// One S <= 16 call: the split from the model; for gate/up, the two-matrix
+// tiles or the pair tiles, whichever the model expects to finish first.
+template <int FMT>
+qg_status launch_fmt(const GemmS16Launch& L, const DeviceInfo& dev, cudaStream_t stream) {
+    size_t s1 = 0, sP = 0;
+    int P = 1;
+    if (L.epilogue != kEpiSwiglu) {
+        qg_status st = prepare_both<FMT, 1, kEpiPlain>(dev, &s1, &sP);
+        if (st != QG_OK) return st;
+        choose_split<FMT, 1, kEpiPlain>(L, dev, s1, sP, &P);
+        return launch_tc_t<FMT, 1, kEpiPlain>(L, dev, stream, P, s1, sP);
+    }
+    size_t q1 = 0, qP = 0;
+    qg_status st = prepare_both<FMT, 2, kEpiSwiglu>(dev, &s1, &sP);
+    if (st != QG_OK) return st;
+    st = prepare_both<FMT, 1, kEpiPair>(dev, &q1, &qP);
+    if (st != QG_OK) return st;
+    int Pq = 1;
+    const double t2 = choose_split<FMT, 2, kEpiSwiglu>(L, dev, s1, sP, &P);
+    const double tq = choose_split<FMT, 1, kEpiPair>(L, dev, q1, qP, &Pq);
+    if (tq < t2) return launch_tc_t<FMT, 1, kEpiPair>(L, dev, stream, Pq, q1, qP);
+    return launch_tc_t<FMT, 2, kEpiSwiglu>(L, dev, stream, P, s1, sP);
+}
+
 }  // namespace
 
 qg_status launch_gemm_tc(const GemmS16Launch& L, cudaStream_t stream) {
@@ -838,13 +954,8 @@ qg_status launch_gemm_tc(const GemmS16Launch& L, cudaStream_t stream) {
     DeviceInfo dev;
     qg_status st = device_info(&dev);
     if (st != QG_OK) return st;
-    const bool swiglu = L.epilogue == kEpiSwiglu;
-    if (L.fmt == QG_FMT_I8_B32)
-        return swiglu ? launch_tc_t<0, 2, kEpiSwiglu>(L, dev, stream)
-                      : launch_tc_t<0, 1, kEpiPlain>(L, dev, stream);
-    if (L.fmt == QG_FMT_I4_G64)
-        return swiglu ? launch_tc_t<1, 2, kEpiSwiglu>(L, dev, stream)
-                      : launch_tc_t<1, 1, kEpiPlain>(L, dev, stream);
+    if (L.fmt == QG_FMT_I8_B32) return launch_fmt<0>(L, dev, stream);
+    if (L.fmt == QG_FMT_I4_G64) return launch_fmt<1>(L, dev, stream);
     return QG_ERR_FORMAT;
 }
 
