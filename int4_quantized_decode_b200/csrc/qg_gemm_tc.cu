@@ -12,28 +12,35 @@
 // 1.06 B of int8, per 0.56 B of int4), far below the tensor-core ridge.
 //
 // One CTA computes a 128-row weight tile (M = 128) for all 16 tokens (N = 16)
-// over a K range; the CTAs of a thread-block cluster split K and reduce their
-// fp32 partials through distributed shared memory in a fixed rank order
-// (deterministic, no global workspace).  Warp roles:
+// over a K range; gate/up runs as pair tiles (64 gate rows in tensor-memory
+// lanes 0-63, the same 64 rows of up in lanes 64-127), so every call runs with
+// the same single-weight resources, two CTAs per SM.  The CTAs of a thread-block
+// cluster split K; each pushes its fp32 partials into the shared memory of the
+// CTA that finishes those rows, which sums them in rank order after one
+// cluster barrier (deterministic, no global workspace).  Warp roles:
 //
-//  * warp 0, one thread -- producer: TMA (cp.async.bulk.tensor.2d, this GPU's
-//    memory only, no multicast) copies each stage's code tile (128 rows x 128
-//    bytes, 128-byte swizzle) and the X chunk (16 rows x 64 fp16 per box,
-//    128-byte swizzle, rows >= S filled with zeros by the copy) into a ring of
-//    shared-memory stages on one mbarrier each.  Codes do not depend on the
-//    previous kernel and are requested before griddepcontrol.wait; X after.
+//  * warp 0 -- producer (warp-uniform loop, the elected lane issues): TMA
+//    (cp.async.bulk.tensor.2d, this GPU's memory only, no multicast) copies
+//    each stage's code tile (128 rows x 128 bytes, 128-byte swizzle) and the
+//    X chunk (16 rows x 64 fp16 per box, rows >= S filled with zeros by the
+//    copy) into a ring of shared-memory stages on one mbarrier each.  Codes do
+//    not depend on the previous kernel and are requested before
+//    griddepcontrol.wait; X after.
 //  * warps 2..9 -- dequantize: thread = weight row (its warp's quarter of the
-//    tensor-memory lanes), two warps per quarter taking alternate 16-k steps.
-//    Each turns its row's 16 codes of a step into fp16(q s) (int8: byte
-//    permute into 1024 + u, exact subtraction, one rounding by the block
+//    tensor-memory lanes); two sets of four warps take alternate A groups of
+//    8 steps of 16 k, so one set dequantizes while the other's stores drain.
+//    Each thread turns its row's 16 codes of a step into fp16(q s) (int8:
+//    byte permute into 1024 + u, exact subtraction, one rounding by the block
 //    scale) or fp16(q s + b) (int4: one fused rounding) and stores them into
 //    tensor memory (tcgen05.st), where the MMA reads its A operand.
-//  * warp 1 -- allocates tensor memory; one thread issues tcgen05.mma
-//    kind::f16 (A from tensor memory, B = X from shared memory through a
-//    128-byte-swizzle K-major descriptor, fp32 accumulator D in tensor
-//    memory) and tcgen05.commit to release A slots and X stages.
-//  * epilogue: tcgen05.ld of D (thread = row, 16 columns = tokens), split-K
-//    reduction over the cluster, fp32 or SwiGLU fp16 store.
+//  * warp 1 -- allocates tensor memory; in a warp-uniform loop its elected
+//    lane issues tcgen05.mma kind::f16 (A from tensor memory, B = X from
+//    shared memory through a 128-byte-swizzle K-major descriptor, fp32 D in
+//    tensor memory, step j into accumulator j mod 4 so that consecutive MMAs
+//    never wait on each other) and one tcgen05.commit per A group.
+//  * epilogue (warps 2..5): tcgen05.ld of the four accumulators (thread =
+//    row, 16 columns = tokens), the split-K reduction, fp32 or SwiGLU fp16
+//    store; tensor memory is freed after they signal their reads are done.
 //
 // Every wait is bounded: a wait that gives up sets the CTA's abort flag and
 // the device error flag; the CTA then skips its remaining work, drains its
@@ -921,8 +928,11 @@ qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream
                                           mc[1], mx, p));
 }
 
-// One S <= 16 call: the split from the model; for gate/up, the two-matrix
-// tiles or the pair tiles, whichever the model expects to finish first.
+// One S <= 16 call, with the split from the model.  Gate/up runs as pair
+// tiles: on every shape of the 2B-27B decoders (and the test shapes) the model
+// expects them to finish before two-matrix tiles of 128 rows (one CTA per SM
+// by its 512 tensor-memory columns), and on the 8B gate/up they measured 24.4
+// against 27.2 us.
 template <int FMT>
 qg_status launch_fmt(const GemmS16Launch& L, const DeviceInfo& dev, cudaStream_t stream) {
     size_t s1 = 0, sP = 0;
@@ -933,16 +943,10 @@ qg_status launch_fmt(const GemmS16Launch& L, const DeviceInfo& dev, cudaStream_t
         choose_split<FMT, 1, kEpiPlain>(L, dev, s1, sP, &P);
         return launch_tc_t<FMT, 1, kEpiPlain>(L, dev, stream, P, s1, sP);
     }
-    size_t q1 = 0, qP = 0;
-    qg_status st = prepare_both<FMT, 2, kEpiSwiglu>(dev, &s1, &sP);
+    qg_status st = prepare_both<FMT, 1, kEpiPair>(dev, &s1, &sP);
     if (st != QG_OK) return st;
-    st = prepare_both<FMT, 1, kEpiPair>(dev, &q1, &qP);
-    if (st != QG_OK) return st;
-    int Pq = 1;
-    const double t2 = choose_split<FMT, 2, kEpiSwiglu>(L, dev, s1, sP, &P);
-    const double tq = choose_split<FMT, 1, kEpiPair>(L, dev, q1, qP, &Pq);
-    if (tq < t2) return launch_tc_t<FMT, 1, kEpiPair>(L, dev, stream, Pq, q1, qP);
-    return launch_tc_t<FMT, 2, kEpiSwiglu>(L, dev, stream, P, s1, sP);
+    choose_split<FMT, 1, kEpiPair>(L, dev, s1, sP, &P);
+    return launch_tc_t<FMT, 1, kEpiPair>(L, dev, stream, P, s1, sP);
 }
 
 }  // namespace
