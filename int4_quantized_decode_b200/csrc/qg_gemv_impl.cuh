@@ -184,12 +184,17 @@ struct I4Zero {
     uint32_t lo, hi;
     float bias;
 };
+// q0 comes from an approximate reciprocal (nearness is all it needs): with
+// s = 0 (a constant group) the product is +-inf or NaN, the conversion
+// saturates or gives 0, and any q0 is exact because every term (q - q0) s
+// is 0.
 __device__ __forceinline__ I4Zero i4_zero_point(float s, float b) {
-    int q0 = 0;
-    if (s > 0.f) q0 = min(15, max(0, __float2int_rn(__fdividef(-b, s))));
-    const uint32_t lo = 0x6400u + static_cast<uint32_t>(q0);
-    const uint32_t hi = 0x6400u + (static_cast<uint32_t>(q0) << 4);
-    return {lo | (lo << 16), hi | (hi << 16), fmaf(static_cast<float>(q0), s, b)};
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+    const int q0 = min(15, max(0, __float2int_rn(-b * r)));
+    const uint32_t u = static_cast<uint32_t>(q0);
+    return {0x64006400u + u * 0x00010001u, 0x64006400u + u * 0x00100010u,
+            fmaf(static_cast<float>(q0), s, b)};
 }
 
 // 32 int4 codes (one 16-byte vector, even k in the low nibble) against their
