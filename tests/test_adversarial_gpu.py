@@ -100,3 +100,39 @@ def test_gemm_s16_adversarial(cuda, n, k, S):
     for s in range(S):
         yr, mag = oracle_gemv(W, X[s])
         assert_within_bound(Y[s].cpu().numpy(), yr, mag)
+
+
+@pytest.mark.parametrize("n,k,S", [(300, 2560, 16), (77, 512, 3)])
+def test_gemm_s16_adversarial_int4(cuda, n, k, S):
+    """int4 at S <= 16 on the tensor cores: groups straddling 0 with an exact
+    zero level under quiet columns of +-30000 activations."""
+    quiet = wl.quiet_columns(k, 6000 + n, 64)
+    W = qg.quantize(wl.affine_zero_weight_fp32(n, k, 6001 + n, quiet, cuda), I4)
+    X = torch.stack([wl.spiky_act_fp16(k, 6100 + s, quiet, device=cuda) for s in range(S)])
+    Y = torch.empty((S, n), dtype=torch.float32, device=cuda)
+    qg.qg_gemm_s16(W, X, Y)
+    qg.qg_stream_check()
+    for s in range(S):
+        yr, mag = oracle_gemv(W, X[s])
+        assert_within_bound(Y[s].cpu().numpy(), yr, mag)
+
+
+@pytest.mark.parametrize("fmt,n,k,S", [(I8, 300, 2048, 16), (I8, 41, 512, 4), (I4, 300, 2560, 16),
+                                       (I4, 41, 512, 4)])
+def test_swiglu_s16_adversarial(cuda, fmt, n, k, S):
+    """The S <= 16 gate/up (pair tiles) on the same constructions."""
+    quiet = wl.quiet_columns(k, 7000 + n, 64)
+    make = wl.outlier_weight_fp32 if fmt == I8 else wl.affine_zero_weight_fp32
+    Wg = qg.quantize(make(n, k, 7001 + n, quiet, cuda), fmt)
+    Wu = qg.quantize(make(n, k, 7002 + n, quiet, cuda), fmt)
+    X = torch.stack([wl.spiky_act_fp16(k, 7100 + s, quiet, device=cuda) for s in range(S)])
+    H = torch.empty((S, n), dtype=torch.float16, device=cuda)
+    qg.qg_gate_up_swiglu(Wg, Wu, X, H)
+    qg.qg_stream_check()
+    Hd = H.cpu().numpy().astype(np.float64)
+    for s in range(S):
+        gr, mg = oracle_gemv(Wg, X[s])
+        ur, mu = oracle_gemv(Wu, X[s])
+        hr, hb = oracle.swiglu(gr, ur, mg, mu, oracle.GEMV_TOL)
+        err = np.abs(Hd[s] - hr)
+        assert np.all(err <= hb), f"token {s}: worst {np.max(err - hb)}"
