@@ -201,8 +201,8 @@ __device__ __forceinline__ void tc_st8(uint32_t taddr, const uint32_t (&v)[8]) {
 __device__ __forceinline__ void tc_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
-    uint32_t r[16];
+// 16 columns of this warp's 32 lanes, without waiting (tc_wait_ld completes it)
+__device__ __forceinline__ void tc_ld16_async(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
         "%14,%15}, [%16];"
@@ -211,9 +211,9 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
           "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr)
         : "memory");
+}
+__device__ __forceinline__ void tc_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // Instruction descriptor of kind::f16: fp16 A and B, both K-major, fp32 D,
@@ -304,7 +304,7 @@ __device__ __forceinline__ bool warp_wait_or_abort(uint64_t* bar, uint32_t parit
 }
 
 template <int FMT, int NMAT, int EPI, bool SPLIT>
-__global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, 1)
+__global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 1 ? 2 : 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_codes0,
                    const __grid_constant__ CUtensorMap tm_codes1,
                    const __grid_constant__ CUtensorMap tm_x, const TcParams p) {
@@ -589,13 +589,16 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, 1)
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
             const uint32_t base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-            tc_ld16(base + d_col(m, 0), acc[m]);
+            uint32_t r[kAcc][16];  // every accumulator's load in flight, one wait
 #pragma unroll
-            for (int c = 1; c < kAcc; ++c) {
-                float v[16];
-                tc_ld16(base + d_col(m, c), v);
+            for (int c = 0; c < kAcc; ++c) tc_ld16_async(base + d_col(m, c), r[c]);
+            tc_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) acc[m][i] += v[i];
+            for (int i = 0; i < 16; ++i) {
+                float v = __uint_as_float(r[0][i]);
+#pragma unroll
+                for (int c = 1; c < kAcc; ++c) v += __uint_as_float(r[c][i]);
+                acc[m][i] = v;
             }
             if (!done)
 #pragma unroll
