@@ -142,11 +142,30 @@ __device__ __forceinline__ uint32_t cluster_ctarank_tc() {
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
     return r;
 }
-// Every thread of the CTA arrives (release) and waits (acquire): the
-// non-.aligned form, safe whatever the warp's convergence.
-__device__ __forceinline__ void cluster_barrier() {
-    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+// The two halves of a cluster barrier, every thread of every CTA once each.
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
 }
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+// Copy `bytes` (a multiple of 16, both addresses 16-byte aligned) of this
+// CTA's shared memory into a peer's (dst and its mbarrier as shared::cluster
+// addresses); the bytes complete the peer's mbarrier transaction.
+__device__ __forceinline__ void bulk_s2peer(uint32_t dst, uint32_t src, uint32_t bytes,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+        "[%3];" ::"r"(dst),
+        "r"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
                                             uint64_t* bar, uint64_t policy) {
     asm volatile(
@@ -325,6 +344,7 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 
     __shared__ __align__(8) uint64_t aempty_bar[NG];
     __shared__ __align__(8) uint64_t done_bar;
     __shared__ __align__(8) uint64_t fin_bar;  // epilogue warps done with tensor memory
+    __shared__ __align__(8) uint64_t recv_bar; // split K: the peers' partials have landed
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
 
@@ -361,6 +381,7 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 
         }
         mbar_init(&done_bar, 1);
         mbar_init(&fin_bar, 4);
+        mbar_init(&recv_bar, 1);
         fence_mbar_init();
         prefetch_tmap(&tm_codes0);
         if (NMAT == 2) prefetch_tmap(&tm_codes1);
@@ -376,6 +397,9 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // split K: every CTA's receive barrier is initialized before any peer may
+    // copy into it (the matching wait comes just before the copies)
+    if (SPLIT) cluster_arrive();
     const uint32_t tmem = tmem_base_sh;
     // the next kernel in the stream may start its own prologue now (its reads
     // of our outputs wait for our completion in griddepcontrol.wait)
@@ -610,47 +634,85 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 
         if (lane == 0) mbar_arrive(&fin_bar);
     }
 
-    if (PAIR) {
-        // Pair tile: lane r holds gate row r, lane 64 + r the same row of up.
-        const int pr = rl & (kPairRows - 1), mm = rl / kPairRows;
-        if (SPLIT) {
-            // as below, by pair row: rank q finishes pair rows [q 64 / P, (q + 1) 64 / P)
-            // and receives both matrices' partials of them
-            float* recv = reinterpret_cast<float*>(sgen + NSTG * L::kStageBytes);
-            const int rmax = (kPairRows + P - 1) / P;
-            if (epi_warp) {
-                int owner = 0;
-                while (owner + 1 < P && (owner + 1) * kPairRows / P <= pr) ++owner;
-                const int r = pr - owner * kPairRows / P;
-                const uint32_t base =
-                    smem_u32(&recv[((static_cast<int>(rank) * 2 + mm) * 16) * rmax + r]);
-                uint32_t remote;
-                asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
-                             : "=r"(remote)
-                             : "r"(base), "r"(static_cast<uint32_t>(owner)));
+    if (SPLIT) {
+        // Split K.  Rank q finishes rows [q RT / P, (q + 1) RT / P) of the
+        // tile's RT rows (output rows; pair rows for a pair tile, each with
+        // the gate and up vectors).  Every CTA stages its partials in its own
+        // shared memory as [row][vector][token], then sends each finishing
+        // CTA its block with one bulk copy into that CTA's receive buffer
+        // ([source rank][row][vector][token]), completing on its receive
+        // barrier; each CTA sums its rows' partials in rank order.
+        constexpr int RT = PAIR ? kPairRows : kTcRows;
+        constexpr int VM = PAIR ? 2 : NMAT;
+        constexpr int kRowFloats = VM * 16;
+        float* stage = reinterpret_cast<float*>(sgen);  // the stages are free now
+        float* recv = reinterpret_cast<float*>(sgen + NSTG * L::kStageBytes);
+        auto lo_of = [&](int q) { return q * RT / P; };
+        if (epi_warp) {
+            const int ri = PAIR ? (rl & (kPairRows - 1)) : rl;
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote + i * rmax * 4),
-                                 "f"(acc[0][i])
-                                 : "memory");
+            for (int m = 0; m < NMAT; ++m) {
+                const int vm = PAIR ? rl / kPairRows : m;
+                float4* dst = reinterpret_cast<float4*>(stage + (ri * VM + vm) * 16);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_float4(acc[m][4 * i], acc[m][4 * i + 1], acc[m][4 * i + 2],
+                                         acc[m][4 * i + 3]);
             }
-            cluster_barrier();  // every push is visible; no remote access follows
-            const int r_lo = static_cast<int>(rank) * kPairRows / P;
-            const int R = (static_cast<int>(rank) + 1) * kPairRows / P - r_lo;
-            for (int e = threadIdx.x - 64; e >= 0 && e < R * 16; e += L::kThreads - 64) {
-                const int tok = e / R, r = e % R;
-                float g = 0.f, u = 0.f;
-                for (int q = 0; q < P; ++q) {
-                    g += recv[((q * 2 + 0) * 16 + tok) * rmax + r];
-                    u += recv[((q * 2 + 1) * 16 + tok) * rmax + r];
+            // the bulk copies (async proxy) read what these stores wrote
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        __syncwarp();
+        if (warp >= 2)  // warps 2.. : every staged row is visible to the senders and reducers
+            asm volatile("barrier.sync 2, %0;" ::"r"(L::kThreads - 64) : "memory");
+        const int r_lo = lo_of(static_cast<int>(rank));
+        const int R = lo_of(static_cast<int>(rank) + 1) - r_lo;
+        if (threadIdx.x == 64)
+            mbar_arrive_expect_tx(&recv_bar, static_cast<uint32_t>((P - 1) * R * kRowFloats * 4));
+        cluster_wait();  // every peer's receive barrier is initialized
+        if (warp == 2) {
+            if (lane < P && lane != static_cast<int>(rank)) {
+                const int q = lane, qlo = lo_of(q), qR = lo_of(q + 1) - qlo;
+                const uint32_t src = smem_u32(stage + qlo * kRowFloats);
+                const uint32_t dst = peer_addr(
+                    smem_u32(recv + static_cast<int>(rank) * qR * kRowFloats), static_cast<uint32_t>(q));
+                bulk_s2peer(dst, src, static_cast<uint32_t>(qR * kRowFloats * 4),
+                            peer_addr(smem_u32(&recv_bar), static_cast<uint32_t>(q)));
+            }
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+        if (threadIdx.x >= 64) {
+            if (!mbar_wait_bounded(&recv_bar, 0) && threadIdx.x == 64)
+                atomicOr(&g_tc_err, kGemvErrTimeout);
+            for (int e = threadIdx.x - 64; e < R * 16; e += L::kThreads - 64) {
+                const int r = e / 16, tok = e % 16;  // consecutive threads, consecutive words
+                float v[VM];
+#pragma unroll
+                for (int vm = 0; vm < VM; ++vm) {
+                    float sum = 0.f;
+                    for (int q = 0; q < P; ++q)
+                        sum += q == static_cast<int>(rank)
+                                   ? stage[((r_lo + r) * VM + vm) * 16 + tok]
+                                   : recv[((q * R + r) * VM + vm) * 16 + tok];
+                    v[vm] = sum;
                 }
                 const int64_t grow = row0 + r_lo + r;
-                if (tok < p.S && grow < p.n)
-                    p.H[static_cast<int64_t>(tok) * p.n + grow] = f2h_rn(g / (1.0f + expf(-g)) * u);
+                if (tok < p.S && grow < p.n) {
+                    if (EPI == kEpiPlain)
+                        p.Y[static_cast<int64_t>(tok) * p.n + grow] = v[0];
+                    else
+                        p.H[static_cast<int64_t>(tok) * p.n + grow] =
+                            f2h_rn(v[0] / (1.0f + expf(-v[0])) * v[VM - 1]);
+                }
             }
-        } else if (epi_warp) {
+        }
+        // this CTA's copies have read its staged partials before it may exit
+        if (warp == 2) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    } else if (PAIR) {
+        if (epi_warp) {
             // the four epilogue warps exchange their rows through shared memory
-            // (the stages are free: every copy landed and was read)
+            // (the stages are free: every copy landed and was read): lane r
+            // holds gate row r, lane 64 + r the same row of up
             float* xch = reinterpret_cast<float*>(sgen);
 #pragma unroll
             for (int i = 0; i < 16; ++i) xch[i * kTcRows + rl] = acc[0][i];
@@ -662,54 +724,6 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 
                 const int64_t grow = row0 + r;
                 if (tok < p.S && grow < p.n)
                     p.H[static_cast<int64_t>(tok) * p.n + grow] = f2h_rn(g / (1.0f + expf(-g)) * u);
-            }
-        }
-        (void)mm;
-    } else if (SPLIT) {
-        // Rank q finishes rows [q 128 / P, (q + 1) 128 / P).  Every CTA pushes
-        // its partial of each row into the finishing CTA's receive buffer
-        // (remote stores, no round trip); after one cluster barrier each CTA
-        // sums its rows' P partials in rank order from its own shared memory.
-        float* recv = reinterpret_cast<float*>(sgen + NSTG * L::kStageBytes);
-        const int rmax = (kTcRows + P - 1) / P;
-        if (epi_warp) {
-            int owner = 0;
-            while (owner + 1 < P && (owner + 1) * kTcRows / P <= rl) ++owner;
-            const int r = rl - owner * kTcRows / P;
-#pragma unroll
-            for (int m = 0; m < NMAT; ++m) {
-                const uint32_t base = smem_u32(
-                    &recv[((static_cast<int>(rank) * NMAT + m) * 16) * rmax + r]);
-                uint32_t remote;
-                asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
-                             : "=r"(remote)
-                             : "r"(base), "r"(static_cast<uint32_t>(owner)));
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote + i * rmax * 4),
-                                 "f"(acc[m][i])
-                                 : "memory");
-            }
-        }
-        cluster_barrier();  // every push is visible; no remote access follows
-        const int r_lo = static_cast<int>(rank) * kTcRows / P;
-        const int R = (static_cast<int>(rank) + 1) * kTcRows / P - r_lo;
-        for (int e = threadIdx.x - 64; e >= 0 && e < R * 16; e += L::kThreads - 64) {
-            const int tok = e / R, r = e % R;
-            float v[NMAT];
-#pragma unroll
-            for (int m = 0; m < NMAT; ++m) {
-                float s = 0.f;
-                for (int q = 0; q < P; ++q) s += recv[((q * NMAT + m) * 16 + tok) * rmax + r];
-                v[m] = s;
-            }
-            const int64_t grow = row0 + r_lo + r;
-            if (tok < p.S && grow < p.n) {
-                if (EPI == kEpiPlain)
-                    p.Y[static_cast<int64_t>(tok) * p.n + grow] = v[0];
-                else
-                    p.H[static_cast<int64_t>(tok) * p.n + grow] =
-                        f2h_rn(v[0] / (1.0f + expf(-v[0])) * v[NMAT - 1]);
             }
         }
     } else if (epi_warp) {
