@@ -844,10 +844,10 @@ double choose_split(const GemmS16Launch& Lc, const DeviceInfo& dev, size_t smem1
     // clusters run in rounds of as many as the GPU holds at once; a round
     // costs the busiest SM's bytes over its rate plus a fixed cost (launch,
     // pipeline fill, epilogue).  Rates and costs were measured on B200 by
-    // timing every P on the int8 and int4 projections of 2B-8B decoders: a
-    // single-weight CTA alone on its SM streams ~29 KB/us, an SM holding two
-    // ~54 KB/us, a gate/up CTA (alone by shared memory) ~45 KB/us; fixed cost
-    // ~4.4 us, ~6.8 us with the cluster reduction.  The occupancy query counts
+    // timing every P on the int8 and int4 projections of 2B-8B decoders: an
+    // int8 CTA alone on its SM streams ~29 KB/us, an SM holding two ~54 KB/us
+    // (int4, bound by its dequantization, about half of that); fixed cost
+    // ~4.4 us, ~4.6 us with the split's bulk-copy reduction.  The occupancy query counts
     // a kernel that allocates tensor memory as one CTA per SM although two
     // single-weight CTAs co-reside, so their capacity is taken as twice the
     // query's, and at least 90% of the slots for clusters of P (GPC packing).
@@ -869,8 +869,9 @@ double choose_split(const GemmS16Launch& Lc, const DeviceInfo& dev, size_t smem1
         const int64_t rounds = (tiles + cpw - 1) / cpw;
         const int64_t per_round = (tiles + rounds - 1) / rounds;
         const int64_t per_sm = (per_round * c + dev.num_sms - 1) / dev.num_sms;
-        const double rate = NMAT == 2 ? 45.0 : (per_sm >= 2 ? 54.0 : 29.0);
-        const double fixed_us = c > 1 ? 6.8 : 4.4;
+        const double fmt_rate = FMT == 0 ? 1.0 : 0.5;
+        const double rate = fmt_rate * (NMAT == 2 ? 45.0 : (per_sm >= 2 ? 54.0 : 29.0));
+        const double fixed_us = c > 1 ? 4.6 : 4.4;
         const double t = static_cast<double>(rounds) *
                          (static_cast<double>(per_sm) * tile_kb / c / rate + fixed_us);
         if (t < best * (1 - 1e-9)) {
