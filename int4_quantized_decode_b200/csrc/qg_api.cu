@@ -498,10 +498,10 @@ qg_status qg_stream_check(cudaStream_t stream) {
     const unsigned int g = qg::gemv_read_and_clear_error() | qg::gemv_decode_read_and_clear_error() |
                            qg::stream_read_and_clear_error();
     const unsigned int f = g | qg::gemm_tc_read_and_clear_error();
-    const unsigned int a = qg::attention_read_and_clear_error();  // a position out of range
+    const unsigned int a = qg::attention_read_and_clear_error();
     if (g & qg::kGemvErrBadPlan) return QG_ERR_PLAN;
-    if ((g & qg::kGemvErrToken) || a) return QG_ERR_SHAPE;
-    return f ? QG_ERR_TIMEOUT : QG_OK;
+    if ((g & qg::kGemvErrToken) || (a & 1u)) return QG_ERR_SHAPE;  // a position out of range
+    return (f || (a & 2u)) ? QG_ERR_TIMEOUT : QG_OK;
 }
 
 }  // extern "C"

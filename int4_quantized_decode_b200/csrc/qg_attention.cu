@@ -14,19 +14,24 @@
 //  * grid = splits x kv heads; a CTA takes one contiguous chunk of the
 //    positions 0..pos of one kv head and all G query heads that read it, so
 //    each K/V row is read once per token;
-//  * one CTA of 8 warps per SM takes a long chunk, streamed through a
-//    three-stage cp.async ring of 64 rows of K and V (after an L2 prefetch of
-//    the chunk issued before the wait on the previous kernel);
-//  * inside a CTA, each group of 16 lanes takes four rows of every stage
-//    (8 dims per lane, 16-byte shared loads) with an online softmax per query
-//    head, rescaled once per stage; groups, then warps, merge their (max,
-//    sum, acc) states;
+//  * one CTA per SM: a producer warp streams the chunk through a six-stage
+//    ring, 64 rows of K then 64 of V per stage, each stage two 1-D bulk copies
+//    completing on the stage's mbarrier (the rows of one kv head are
+//    contiguous), after an L2 prefetch of the chunk's first rows issued before
+//    the wait on the previous kernel;
+//  * eight compute warps take 8 rows of every stage each: 8 lanes per row
+//    (16 dims per lane, two 16-byte shared loads), a score per query head
+//    summed over the 8 lanes, softmax in base 2 (log2 e folded into q) with a
+//    running maximum per warp that is raised, and the state rescaled, only
+//    when a score exceeds it by more than 8 (so every weight stays <= 2^8);
+//    warps then merge their (max, sum, acc) states in shared memory;
 //  * every CTA writes its partial state; the last CTA of a kv head (an atomic
-//    ticket, no CTA ever waits) merges the splits, writes o in fp16 and
-//    re-zeroes its ticket;
+//    ticket, no CTA ever waits) merges the splits in one pass, writes o in fp16
+//    and re-zeroes its ticket;
 //  * the new token's key and value are computed by every CTA (RoPE angles in
-//    fp64, one fp16 rounding) and used for row pos, which no CTA reads from
-//    the cache; the CTA whose chunk holds pos writes them into the cache.
+//    fp64, one fp16 rounding) and stand in for row pos, which no CTA reads from
+//    the cache; the CTA whose chunk holds pos writes them into the cache once
+//    its own copies have landed.
 #include <cfloat>
 #include <cmath>
 
@@ -35,24 +40,29 @@
 
 namespace qg {
 
-QG_DEFINE_ERROR_FLAG(g_attn_err);
+QG_DEFINE_ERROR_FLAG(g_attn_err);  // bit 0: position out of range; bit 1: a wait expired
 
 namespace {
 
-constexpr int kD = 128;            // head_dim of the pages' Qwen3-VL decoders
-constexpr int kWarpsA = 8;
-constexpr int kThreadsA = kWarpsA * 32;
-constexpr int kGroupLanes = 16;    // lanes per subsequence: 16 x 8 dims = one row
-constexpr int kSubseq = kThreadsA / kGroupLanes;  // 16 subsequences per CTA
-constexpr int kDimsPerLane = kD / kGroupLanes;    // 8: one 16-byte load per row
-constexpr int kUnroll = 4;                        // rows of a subsequence per stage
-constexpr int kStageRows = kSubseq * kUnroll;     // 64 rows of K and of V per stage
-constexpr int kStages = 3;                        // ring depth: two stages in flight
-constexpr int kRowBytes = kD * 2;
-constexpr int kStageBytes = 2 * kStageRows * kRowBytes;  // K rows, then V rows: 32 KB
-constexpr int kRingBytesA = kStages * kStageBytes;
-constexpr int kMaxSplitsK = 32;                   // splits of one kv head's rows, at most
-constexpr int kPrefetchRows = 256;                // rows of a chunk prefetched into L2
+constexpr int kD = 128;               // head_dim of the pages' Qwen3-VL decoders
+constexpr int kRowBytes = kD * 2;     // one fp16 row of K or V
+constexpr int kLanesPerRow = 8;       // a row's 128 dims over 8 lanes
+constexpr int kRowGroups = 32 / kLanesPerRow;        // 4 rows in flight per warp
+constexpr int kComputeWarps = 8;
+constexpr int kComputeThreads = kComputeWarps * 32;
+constexpr int kThreadsA = kComputeThreads + 32;      // + the producer warp
+constexpr int kStageRows = 64;
+constexpr int kRowsPerWarp = kStageRows / kComputeWarps;   // 8
+constexpr int kRowsPerGroup = kRowsPerWarp / kRowGroups;   // 2 rows per lane group per stage
+constexpr int kStages = 6;
+constexpr int kStageBytes = 2 * kStageRows * kRowBytes;    // K rows, then V rows: 32 KB
+constexpr int kRingBytesA = kStages * kStageBytes;          // 192 KB
+constexpr int kMaxSplitsK = 32;       // splits of one kv head's rows, at most
+constexpr int kPrefetchRows = 256;    // rows of a chunk prefetched into L2
+constexpr float kLazyRescale = 8.f;   // base-2 headroom of the running maximum
+constexpr double kLog2e = 1.4426950408889634;
+constexpr int kComputeBar = 1;        // named barrier of the compute warps
+static_assert(kStageRows % (kComputeWarps * kRowGroups) == 0, "whole rows per lane group");
 
 struct AttnParams {
     const float* qkv;
@@ -60,24 +70,14 @@ struct AttnParams {
     uint16_t* vc;
     uint16_t* o;
     const int32_t* pos;
-    float* part;              // [hkv][splits][G][kD + 2]: m, l, acc
+    float* part;              // [hkv][splits][G][kD + 2]: m (base 2), l, acc
     unsigned int* ticket;     // [hkv]
     int64_t l_max;
     int hq, hkv, splits;
     double theta;
-    float scale;              // 1 / sqrt(d)
+    double qscale;            // log2(e) / sqrt(d): scores in base 2
 };
 
-__device__ __forceinline__ void cp_async16_a(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit_a() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait_a() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 __device__ __forceinline__ void prefetch_l2_a(const void* p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
@@ -87,6 +87,44 @@ __device__ __forceinline__ uint4 lds128_a(uint32_t a) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "r"(a));
     return v;
+}
+// 2^x (the hardware approximation; -inf gives +0)
+__device__ __forceinline__ float ex2_a(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// two fp32 lanes in one 64-bit register: the packed FMA does both products
+__device__ __forceinline__ uint64_t pack2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t r, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// The ticket: release orders this CTA's partial stores (seen by the calling
+// thread through the CTA barrier before it) ahead of the increment; acquire
+// orders the other CTAs' partials ahead of the reads that follow the barrier
+// after it.
+__device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int* p, unsigned int v) {
+    unsigned int old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+                 : "memory");
+    return old;
+}
+__device__ __forceinline__ void compute_bar() {
+    asm volatile("bar.sync %0, %1;" ::"n"(kComputeBar), "n"(kComputeThreads) : "memory");
 }
 
 // Rows [j0, j1) of split `split` when the token is at pos (empty past the end).
@@ -107,34 +145,30 @@ __device__ __forceinline__ void unpack8h(const uint4 a, float* out) {
     }
 }
 
-// Merge the online-softmax state (m2, l2, a2) into (m, l, a).
-template <int N>
-__device__ __forceinline__ void merge_state(float& m, float& l, float* a, float m2, float l2,
-                                            const float* a2) {
-    const float mn = fmaxf(m, m2);
-    const float c1 = m == -INFINITY ? 0.f : expf(m - mn);
-    const float c2 = m2 == -INFINITY ? 0.f : expf(m2 - mn);
-    l = l * c1 + l2 * c2;
-#pragma unroll
-    for (int i = 0; i < N; ++i) a[i] = a[i] * c1 + a2[i] * c2;
-    m = mn;
-}
-
 template <int G>
 __global__ void __launch_bounds__(kThreadsA, 1) decode_attention_kernel(const AttnParams p) {
     __shared__ float q_s[G][kD];
     __shared__ __align__(16) uint16_t kn_h[kD];
     __shared__ __align__(16) uint16_t vn_h[kD];
-    __shared__ float wst[kWarpsA][G][kD + 2];  // per-warp merged states
+    __shared__ float wst[kComputeWarps][G][kD + 2];  // per-warp states
+    __shared__ __align__(8) uint64_t full_bar[kStages];
+    __shared__ __align__(8) uint64_t empty_bar[kStages];
     __shared__ unsigned int last_s;
-    __shared__ float sm_m[G][kMaxSplitsK];  // split maxima (then weights)
-    __shared__ float sm_l[G][kMaxSplitsK];  // split sums
+    __shared__ float sm_m[kMaxSplitsK][G];  // split maxima (the last CTA)
+    __shared__ float sm_l[kMaxSplitsK][G];  // split sums
+    extern __shared__ __align__(128) unsigned char ring[];
 
     const int split = blockIdx.x, g = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    extern __shared__ __align__(128) unsigned char ring[];
-    const uint32_t ring0 = smem_u32(ring);
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], kComputeWarps);
+        }
+        fence_mbar_init();
+    }
 
     // Before the wait on the previous kernel: ask L2 for the first rows of
     // this CTA's chunk (at most kPrefetchRows, so that long caches do not
@@ -149,24 +183,39 @@ __global__ void __launch_bounds__(kThreadsA, 1) decode_attention_kernel(const At
         sincos(static_cast<double>(at) * f, &rs, &rc);
     };
     if (tid < kD / 2 && pg >= 0 && pg < p.l_max) angles(pg);
-    if (lane == 0) {
-        if (pg >= 0 && pg < p.l_max) {
-            int64_t a0, a1;
-            chunk_of(pg, p.splits, split, a0, a1);
-            if (a1 > a0 + kPrefetchRows) a1 = a0 + kPrefetchRows;
-            // warp w prefetches its quarter of the chunk, in pieces of <= 16 KB
-            const int64_t q0 = a0 + (a1 - a0) * warp / kWarpsA;
-            const int64_t q1 = a0 + (a1 - a0) * (warp + 1) / kWarpsA;
-            for (int64_t r = q0; r < q1; r += 64) {
-                const int64_t rows = q1 - r < 64 ? q1 - r : 64;
-                const int64_t off = (static_cast<int64_t>(g) * p.l_max + r) * kD;
-                prefetch_l2_a(p.kc + off, static_cast<uint32_t>(rows * kRowBytes));
-                prefetch_l2_a(p.vc + off, static_cast<uint32_t>(rows * kRowBytes));
-            }
+    if (lane == 0 && warp < kComputeWarps && pg >= 0 && pg < p.l_max) {
+        int64_t a0, a1;
+        chunk_of(pg, p.splits, split, a0, a1);
+        if (a1 > a0 + kPrefetchRows) a1 = a0 + kPrefetchRows;
+        // warp w prefetches its eighth of those rows, in pieces of <= 16 KB
+        const int64_t q0 = a0 + (a1 - a0) * warp / kComputeWarps;
+        const int64_t q1 = a0 + (a1 - a0) * (warp + 1) / kComputeWarps;
+        for (int64_t r = q0; r < q1; r += 64) {
+            const int64_t rows = q1 - r < 64 ? q1 - r : 64;
+            const int64_t off = (static_cast<int64_t>(g) * p.l_max + r) * kD;
+            prefetch_l2_a(p.kc + off, static_cast<uint32_t>(rows * kRowBytes));
+            prefetch_l2_a(p.vc + off, static_cast<uint32_t>(rows * kRowBytes));
         }
     }
-    griddep_wait();  // q|k|v come from the projection kernel before this one
+    __syncthreads();  // the barriers are initialised
+    griddep_wait();   // q|k|v come from the projection kernel before this one
     const int32_t pos = *p.pos;
+    // the new token's inputs, loaded together with the position
+    double k0 = 0.0, k1 = 0.0, q0[G], q1[G];
+    float vin = 0.f;
+    if (tid < kD / 2) {
+        const float* kin = p.qkv + static_cast<int64_t>(p.hq) * kD + g * kD;
+        k0 = kin[tid];
+        k1 = kin[tid + kD / 2];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float* qin = p.qkv + static_cast<int64_t>(g * G + h) * kD;
+            q0[h] = qin[tid];
+            q1[h] = qin[tid + kD / 2];
+        }
+    } else if (tid < kD / 2 + kD) {
+        vin = p.qkv[static_cast<int64_t>(p.hq + p.hkv) * kD + g * kD + (tid - kD / 2)];
+    }
     if (pos < 0 || pos >= p.l_max) {
         if (tid == 0 && split == 0 && g == 0) atomicOr(&g_attn_err, 1u);
         return;
@@ -174,255 +223,275 @@ __global__ void __launch_bounds__(kThreadsA, 1) decode_attention_kernel(const At
     int64_t j0, j1;
     chunk_of(pos, p.splits, split, j0, j1);
     const int nstages = static_cast<int>((j1 - j0 + kStageRows - 1) / kStageRows);
-    // Stage st of the chunk -> ring slot st % kStages: rows j0 + 64 st ..., K
-    // then V, 16 pieces of 16 bytes per row; row pos (not written yet) is
-    // skipped, its values come from shared memory below.
-    auto issue = [&](int st) {
-        const uint32_t slot = ring0 + (st % kStages) * kStageBytes;
-#pragma unroll
-        for (int k = 0; k < 2 * kStageRows * 16 / kThreadsA; ++k) {
-            const int i = tid + k * kThreadsA;
-            const int kv = i / (kStageRows * 16), rr = (i / 16) % kStageRows, col = i % 16;
-            const int64_t j = j0 + static_cast<int64_t>(st) * kStageRows + rr;
-            if (j < j1 && j != pos) {
-                const uint16_t* src = (kv == 0 ? p.kc : p.vc) +
-                                      (static_cast<int64_t>(g) * p.l_max + j) * kD + col * 8;
-                cp_async16_a(slot + (kv * kStageRows + rr) * kRowBytes + col * 16, src);
+
+    if (warp == kComputeWarps) {
+        // ---- producer: stage st -> slot st % kStages, rows j0 + 64 st ... of K
+        // then of V (row pos comes along with its old bytes and is never used)
+        griddep_launch_dependents();
+        if (lane == 0) {
+            const uint64_t pol = l2_policy_evict_first();
+            const uint16_t* kb = p.kc + (static_cast<int64_t>(g) * p.l_max + j0) * kD;
+            const uint16_t* vb = p.vc + (static_cast<int64_t>(g) * p.l_max + j0) * kD;
+            for (int st = 0; st < nstages; ++st) {
+                const int slot = st % kStages;
+                if (st >= kStages &&
+                    !mbar_wait_bounded(&empty_bar[slot], ((st / kStages) - 1) & 1)) {
+                    atomicOr(&g_attn_err, 2u);
+                    break;
+                }
+                const int64_t r0 = static_cast<int64_t>(st) * kStageRows;
+                const int64_t left = j1 - j0 - r0;
+                const uint32_t bytes =
+                    static_cast<uint32_t>(left < kStageRows ? left : kStageRows) * kRowBytes;
+                unsigned char* dst = ring + slot * kStageBytes;
+                mbar_arrive_expect_tx(&full_bar[slot], 2 * bytes);
+                bulk_g2s(dst, kb + r0 * kD, bytes, &full_bar[slot], pol);
+                bulk_g2s(dst + kStageRows * kRowBytes, vb + r0 * kD, bytes, &full_bar[slot], pol);
             }
         }
-    };
-    // the first stages stream while q, k and v are rotated
-#pragma unroll
-    for (int st = 0; st < kStages - 1; ++st) {
-        if (st < nstages) issue(st);
-        cp_async_commit_a();
+        return;
     }
 
-    // Thread i < d/2 rotates pair i of the new key (fp64, rounded once to
-    // fp16) and of every query head that reads this kv head; its loads of the
-    // key and query pairs go out together.
+    // ---- the new token: thread i < d/2 rotates pair i of the key (fp64,
+    // rounded once to fp16) and of every query head that reads this kv head
     if (tid < kD / 2) {
         if (pos != pg) angles(pos);  // the position changed after the early read
-        const float* kin = p.qkv + static_cast<int64_t>(p.hq) * kD + g * kD;
-        const double k0 = kin[tid], k1 = kin[tid + kD / 2];
-        double q0[G], q1[G];
+        kn_h[tid] = __half_as_ushort(__double2half(k0 * rc - k1 * rs));
+        kn_h[tid + kD / 2] = __half_as_ushort(__double2half(k1 * rc + k0 * rs));
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-            const float* qin = p.qkv + static_cast<int64_t>(g * G + h) * kD;
-            q0[h] = qin[tid];
-            q1[h] = qin[tid + kD / 2];
+            q_s[h][tid] = static_cast<float>((q0[h] * rc - q1[h] * rs) * p.qscale);
+            q_s[h][tid + kD / 2] = static_cast<float>((q1[h] * rc + q0[h] * rs) * p.qscale);
         }
-        const uint16_t r0 = __half_as_ushort(__double2half(k0 * rc - k1 * rs));
-        const uint16_t r1 = __half_as_ushort(__double2half(k1 * rc + k0 * rs));
-        kn_h[tid] = r0;
-        kn_h[tid + kD / 2] = r1;
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            q_s[h][tid] = static_cast<float>(q0[h] * rc - q1[h] * rs);
-            q_s[h][tid + kD / 2] = static_cast<float>(q1[h] * rc + q0[h] * rs);
-        }
+    } else if (tid < kD / 2 + kD) {
+        vn_h[tid - kD / 2] = f2h_rn(vin);
     }
-    if (tid < kD) {
-        const float* vin = p.qkv + static_cast<int64_t>(p.hq + p.hkv) * kD + g * kD;
-        const uint16_t v = f2h_rn(vin[tid]);
-        vn_h[tid] = v;
-    }
-    __syncthreads();
+    compute_bar();
     griddep_launch_dependents();
 
-    // the CTA whose chunk holds pos appends the new rows
+    // ---- stream: in each stage, warp w takes rows 8w .. 8w + 7; lane group
+    // rg = lane / 8 takes rows 8w + rg and 8w + 4 + rg, lane gl = lane % 8 of
+    // the group dims 8 gl .. 8 gl + 7 and 64 + 8 gl .. 64 + 8 gl + 7 (each
+    // group's two 16-byte loads cover 128 contiguous bytes: no bank conflict)
+    const int rg = lane / kLanesPerRow, gl = lane % kLanesPerRow;
+    // the lane's 16 dims as 8 pairs: pair i < 4 holds dims 8 gl + 2i, + 1;
+    // pair 4 + i dims 64 + 8 gl + 2i, + 1
+    uint64_t q2[G][8];
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            q2[h][i] = pack2(q_s[h][8 * gl + 2 * i], q_s[h][8 * gl + 2 * i + 1]);
+            q2[h][4 + i] =
+                pack2(q_s[h][kD / 2 + 8 * gl + 2 * i], q_s[h][kD / 2 + 8 * gl + 2 * i + 1]);
+        }
+    float m[G], l[G];
+    uint64_t acc2[G][8];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        m[h] = -INFINITY;
+        l[h] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc2[h][i] = 0ull;
+    }
+    const uint32_t ring0 = smem_u32(ring), kn_a = smem_u32(kn_h), vn_a = smem_u32(vn_h);
+    for (int st = 0; st < nstages; ++st) {
+        const int slot = st % kStages;
+        if (!mbar_wait_bounded(&full_bar[slot], (st / kStages) & 1)) {
+            if (lane == 0) atomicOr(&g_attn_err, 2u);
+            break;
+        }
+        const uint32_t kst = ring0 + slot * kStageBytes;
+        const uint32_t vst = kst + kStageRows * kRowBytes;
+        const int64_t jb = j0 + static_cast<int64_t>(st) * kStageRows;
+        float s[kRowsPerGroup][G];
+        bool valid[kRowsPerGroup];
+        uint32_t vaddr[kRowsPerGroup];
+#pragma unroll
+        for (int u = 0; u < kRowsPerGroup; ++u) {
+            const int rr = warp * kRowsPerWarp + u * kRowGroups + rg;
+            const int64_t j = jb + rr;
+            valid[u] = j < j1;
+            // row pos (and, with weight 0, rows past the chunk) read the new token
+            const bool fresh = !valid[u] || j == pos;
+            const uint32_t ka = fresh ? kn_a : kst + rr * kRowBytes;
+            vaddr[u] = fresh ? vn_a : vst + rr * kRowBytes;
+            float kf[16];
+            unpack8h(lds128_a(ka + 16 * gl), kf);
+            unpack8h(lds128_a(ka + kD + 16 * gl), kf + 8);
+            uint64_t k2[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) k2[i] = pack2(kf[2 * i], kf[2 * i + 1]);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                uint64_t a2 = fma2(q2[h][0], k2[0], 0ull);
+#pragma unroll
+                for (int i = 1; i < 8; ++i) a2 = fma2(q2[h][i], k2[i], a2);
+                float a0, a1;
+                unpack2(a2, a0, a1);
+                float a = a0 + a1;
+                a += __shfl_xor_sync(0xffffffffu, a, 1);
+                a += __shfl_xor_sync(0xffffffffu, a, 2);
+                a += __shfl_xor_sync(0xffffffffu, a, 4);
+                s[u][h] = a;
+            }
+        }
+        // the warp's running maximum (the same in every lane) is raised only
+        // when a score passes it by more than kLazyRescale
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int u = 0; u < kRowsPerGroup; ++u)
+                if (valid[u]) mx = fmaxf(mx, s[u][h]);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            if (mx > m[h] + kLazyRescale) {
+                const float c = ex2_a(m[h] - mx);  // 0 while m is -inf
+                const uint64_t c2 = pack2(c, c);
+                l[h] *= c;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc2[h][i] = mul2(acc2[h][i], c2);
+                m[h] = mx;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kRowsPerGroup; ++u) {
+            float vf[16];
+            unpack8h(lds128_a(vaddr[u] + 16 * gl), vf);
+            unpack8h(lds128_a(vaddr[u] + kD + 16 * gl), vf + 8);
+            uint64_t v2[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v2[i] = pack2(vf[2 * i], vf[2 * i + 1]);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float pj = valid[u] ? ex2_a(s[u][h] - m[h]) : 0.f;
+                const uint64_t p2 = pack2(pj, pj);
+                l[h] += pj;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc2[h][i] = fma2(p2, v2[i], acc2[h][i]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[slot]);  // this warp is done with the slot
+    }
+
+    // ---- the warp's four lane groups share its maximum: sum their states
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        float acc[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) unpack2(acc2[h][i], acc[2 * i], acc[2 * i + 1]);
+        l[h] += __shfl_xor_sync(0xffffffffu, l[h], 8);
+        l[h] += __shfl_xor_sync(0xffffffffu, l[h], 16);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 8);
+            acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 16);
+        }
+        if (rg == 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                wst[warp][h][2 + 8 * gl + i] = acc[i];
+                wst[warp][h][2 + kD / 2 + 8 * gl + i] = acc[8 + i];
+            }
+            if (gl == 0) {
+                wst[warp][h][0] = m[h];
+                wst[warp][h][1] = l[h];
+            }
+        }
+    }
+    compute_bar();
+
+    // ---- merge the warps (thread t: dim t % 128 of head t / 128, and of head
+    // t / 128 + 2 when G = 4) and write this split's partial
+    float* part = p.part + (static_cast<int64_t>(g) * p.splits + split) * G * (kD + 2);
+    for (int e = tid; e < G * kD; e += kComputeThreads) {
+        const int h = e / kD, dim = e % kD;
+        float mm = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kComputeWarps; ++w) mm = fmaxf(mm, wst[w][h][0]);
+        float ll = 0.f, aa = 0.f;
+#pragma unroll
+        for (int w = 0; w < kComputeWarps; ++w) {
+            const float mw = wst[w][h][0];
+            const float c = mw == -INFINITY ? 0.f : ex2_a(mw - mm);
+            ll = fmaf(c, wst[w][h][1], ll);
+            aa = fmaf(c, wst[w][h][2 + dim], aa);
+        }
+        part[h * (kD + 2) + 2 + dim] = aa;
+        if (dim == 0) {
+            part[h * (kD + 2)] = mm;
+            part[h * (kD + 2) + 1] = ll;
+        }
+    }
+    // the CTA whose chunk holds pos appends the new rows (its copies have landed)
     if (pos >= j0 && pos < j1 && tid < kD) {
         const int64_t row = (static_cast<int64_t>(g) * p.l_max + pos) * kD;
         p.kc[row + tid] = kn_h[tid];
         p.vc[row + tid] = vn_h[tid];
     }
 
-    // ---- stream: in each stage, subsequence sq = tid / 16 takes rows sq,
-    // sq + 16, sq + 32, sq + 48 (one rescale per stage)
-    const int sq = tid / kGroupLanes, gl = tid % kGroupLanes;
-    const int d0 = gl * kDimsPerLane;
-    float qr[G][kDimsPerLane];
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int i = 0; i < kDimsPerLane; ++i) qr[h][i] = q_s[h][d0 + i] * p.scale;
-    float m[G], l[G], acc[G][kDimsPerLane];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-        m[h] = -INFINITY;
-        l[h] = 0.f;
-#pragma unroll
-        for (int i = 0; i < kDimsPerLane; ++i) acc[h][i] = 0.f;
-    }
-    const uint4 kn4 = *reinterpret_cast<const uint4*>(kn_h + d0);
-    const uint4 vn4 = *reinterpret_cast<const uint4*>(vn_h + d0);
-    // Every thread runs every stage (the shuffles take the whole warp and the
-    // ring is refilled by the whole CTA); rows past the end are skipped.
-    for (int st = 0; st < nstages; ++st) {
-        if (st + kStages - 1 < nstages) issue(st + kStages - 1);
-        cp_async_commit_a();
-        cp_async_wait_a<kStages - 1>();
-        __syncthreads();  // every thread's copies of stage st have landed
-        const uint32_t slot = ring0 + (st % kStages) * kStageBytes;
-        uint4 kr[kUnroll], vr[kUnroll];
-        bool valid[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int rr = sq + u * kSubseq;
-            const int64_t j = j0 + static_cast<int64_t>(st) * kStageRows + rr;
-            valid[u] = j < j1;
-            if (valid[u] && j != pos) {
-                kr[u] = lds128_a(slot + rr * kRowBytes + d0 * 2);
-                vr[u] = lds128_a(slot + (kStageRows + rr) * kRowBytes + d0 * 2);
-            } else {
-                kr[u] = valid[u] ? kn4 : make_uint4(0u, 0u, 0u, 0u);
-                vr[u] = valid[u] ? vn4 : make_uint4(0u, 0u, 0u, 0u);
-            }
-        }
-        float kv[kUnroll][kDimsPerLane];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) unpack8h(kr[u], kv[u]);
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            float s[kUnroll];
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                float a = 0.f;
-#pragma unroll
-                for (int i = 0; i < kDimsPerLane; ++i) a = fmaf(qr[h][i], kv[u][i], a);
-                a += __shfl_xor_sync(0xffffffffu, a, 1);
-                a += __shfl_xor_sync(0xffffffffu, a, 2);
-                a += __shfl_xor_sync(0xffffffffu, a, 4);
-                a += __shfl_xor_sync(0xffffffffu, a, 8);
-                s[u] = a;
-            }
-            float mx = m[h];
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u)
-                if (valid[u]) mx = fmaxf(mx, s[u]);
-            if (mx == -INFINITY) continue;  // no valid row yet (uniform in the group)
-            const float corr = m[h] == -INFINITY ? 0.f : expf(m[h] - mx);
-            l[h] *= corr;
-#pragma unroll
-            for (int i = 0; i < kDimsPerLane; ++i) acc[h][i] *= corr;
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                if (!valid[u]) continue;
-                const float pj = expf(s[u] - mx);
-                float vv[kDimsPerLane];
-                unpack8h(vr[u], vv);
-                l[h] += pj;
-#pragma unroll
-                for (int i = 0; i < kDimsPerLane; ++i) acc[h][i] = fmaf(pj, vv[i], acc[h][i]);
-            }
-            m[h] = mx;
-        }
-        __syncthreads();  // the slot is consumed before it is refilled
-    }
-    cp_async_wait_a<0>();
-
-    // ---- merge the 2 subsequences of a warp (lanes 16 apart hold the same dims)
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-        {
-            const int off = kGroupLanes;
-            const float m2 = __shfl_xor_sync(0xffffffffu, m[h], off);
-            const float l2 = __shfl_xor_sync(0xffffffffu, l[h], off);
-            float a2[kDimsPerLane];
-#pragma unroll
-            for (int i = 0; i < kDimsPerLane; ++i)
-                a2[i] = __shfl_xor_sync(0xffffffffu, acc[h][i], off);
-            merge_state<kDimsPerLane>(m[h], l[h], acc[h], m2, l2, a2);
-        }
-        if (lane < kGroupLanes) {
-#pragma unroll
-            for (int i = 0; i < kDimsPerLane; ++i) wst[warp][h][2 + d0 + i] = acc[h][i];
-            if (lane == 0) {
-                wst[warp][h][0] = m[h];
-                wst[warp][h][1] = l[h];
-            }
-        }
-    }
-    __syncthreads();
-
-    // ---- merge the warps: thread tid owns dim tid % 128 of heads tid / 128,
-    // tid / 128 + 2, ...; write the partial
-    float* part = p.part + (static_cast<int64_t>(g) * p.splits + split) * G * (kD + 2);
-    const int dim = tid & (kD - 1), hh = tid / kD;
-#pragma unroll
-    for (int hb = 0; hb < G; hb += kThreadsA / kD) {
-        const int h = hb + hh;
-        if (h < G) {
-            float mm = wst[0][h][0], ll = wst[0][h][1], aa = wst[0][h][2 + dim];
-            for (int w = 1; w < kWarpsA; ++w)
-                merge_state<1>(mm, ll, &aa, wst[w][h][0], wst[w][h][1], &wst[w][h][2 + dim]);
-            part[h * (kD + 2) + 2 + dim] = aa;
-            if (dim == 0) {
-                part[h * (kD + 2)] = mm;
-                part[h * (kD + 2) + 1] = ll;
-            }
-        }
-    }
-
     // ---- the last CTA of this kv head merges the splits
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) last_s = atomicAdd(&p.ticket[g], 1u) == static_cast<unsigned int>(p.splits - 1);
-    __syncthreads();
+    compute_bar();  // every partial of this CTA is stored
+    if (tid == 0)
+        last_s = atom_add_acq_rel_gpu(&p.ticket[g], 1u) == static_cast<unsigned int>(p.splits - 1);
+    compute_bar();
     if (!last_s) return;
-    __threadfence();
-    // Merge the splits of every head in one pass (threads 0-127 take heads
-    // 0, 2, ..., threads 128-255 heads 1, 3, ...): thread s (< splits) of a
-    // head fetches split s's max and sum and forms its weight e^(m_s - M);
-    // every thread sums its dim over all splits with loads that are all in
-    // flight at once.
+    // Every split's max and sum go to shared memory once; thread t owns
+    // kDpt adjacent dims (d0 = kDpt t of the [G][128] outputs) and loads them
+    // from every split, all in flight together; then per output
+    // o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s.
     const float* base = p.part + static_cast<int64_t>(g) * p.splits * G * (kD + 2);
     const int64_t stride = static_cast<int64_t>(G) * (kD + 2);
-    constexpr int kHalves = kThreadsA / kD;                // 2: threads 0-127 and 128-255
-    constexpr int kHpt = (G + kHalves - 1) / kHalves;      // heads per thread
-    float v[kHpt][kMaxSplitsK];
+    constexpr int kDpt = G * kD > kComputeThreads ? G * kD / kComputeThreads : 1;
+    static_assert(kDpt * kComputeThreads >= G * kD && kDpt <= 2, "one pass over the outputs");
+    const int d0 = tid * kDpt;
+    const bool mine = d0 < G * kD;
+    const int h = mine ? d0 / kD : 0, dim = d0 % kD;
+    float as[kMaxSplitsK][kDpt];
 #pragma unroll
-    for (int e = 0; e < kHpt; ++e) {
-        const int h = hh + kHalves * e;
-        const float* col = base + static_cast<int64_t>(h < G ? h : 0) * (kD + 2);
-#pragma unroll
-        for (int sidx = 0; sidx < kMaxSplitsK; ++sidx)
-            v[e][sidx] = h < G && sidx < p.splits ? __ldcg(col + sidx * stride + 2 + dim) : 0.f;
-        if (h < G && dim < p.splits) {
-            sm_m[h][dim] = __ldcg(col + dim * stride);
-            sm_l[h][dim] = __ldcg(col + dim * stride + 1);
+    for (int sidx = 0; sidx < kMaxSplitsK; ++sidx) {
+        const float* src = base + sidx * stride + h * (kD + 2) + 2 + dim;
+        if (kDpt == 2) {  // 8-byte aligned: every term of the offset is even
+            const float2 v = mine && sidx < p.splits ? __ldcg(reinterpret_cast<const float2*>(src))
+                                                      : make_float2(0.f, 0.f);
+            as[sidx][0] = v.x;
+            as[sidx][kDpt - 1] = v.y;
+        } else {
+            as[sidx][0] = mine && sidx < p.splits ? __ldcg(src) : 0.f;
         }
     }
-    __syncthreads();
-    float mx[kHpt];
-#pragma unroll
-    for (int e = 0; e < kHpt; ++e) {
-        const int h = hh + kHalves * e;
-        mx[e] = -INFINITY;
-        if (h < G)
-            for (int sidx = 0; sidx < p.splits; ++sidx) mx[e] = fmaxf(mx[e], sm_m[h][sidx]);
+    // (after the acc loads are issued, so that none waits behind these)
+    if (tid < p.splits * G) {
+        const int sidx = tid / G, hh = tid % G;
+        const float mv = __ldcg(base + sidx * stride + hh * (kD + 2));
+        const float lv = __ldcg(base + sidx * stride + hh * (kD + 2) + 1);
+        sm_m[sidx][hh] = mv;
+        sm_l[sidx][hh] = lv;
     }
-    __syncthreads();  // every thread has its maxima
+    compute_bar();
+    if (mine) {
+        float mm = -INFINITY;
 #pragma unroll
-    for (int e = 0; e < kHpt; ++e) {
-        const int h = hh + kHalves * e;
-        if (h < G && dim < p.splits)
-            sm_m[h][dim] = sm_m[h][dim] == -INFINITY ? 0.f : expf(sm_m[h][dim] - mx[e]);
-    }
-    __syncthreads();
+        for (int sidx = 0; sidx < kMaxSplitsK; ++sidx)
+            if (sidx < p.splits) mm = fmaxf(mm, sm_m[sidx][h]);
+        float ll = 0.f, aa[kDpt];
 #pragma unroll
-    for (int e = 0; e < kHpt; ++e) {
-        const int h = hh + kHalves * e;
-        if (h >= G) continue;
-        float ll = 0.f, aa = 0.f;
+        for (int i = 0; i < kDpt; ++i) aa[i] = 0.f;
 #pragma unroll
         for (int sidx = 0; sidx < kMaxSplitsK; ++sidx) {
             if (sidx < p.splits) {
-                ll = fmaf(sm_m[h][sidx], sm_l[h][sidx], ll);
-                aa = fmaf(sm_m[h][sidx], v[e][sidx], aa);
+                const float ms = sm_m[sidx][h];
+                const float c = ms == -INFINITY ? 0.f : ex2_a(ms - mm);
+                ll = fmaf(c, sm_l[sidx][h], ll);
+#pragma unroll
+                for (int i = 0; i < kDpt; ++i) aa[i] = fmaf(c, as[sidx][i], aa[i]);
             }
         }
-        p.o[static_cast<int64_t>(g * G + h) * kD + dim] = f2h_rn(aa / ll);
+#pragma unroll
+        for (int i = 0; i < kDpt; ++i)
+            p.o[static_cast<int64_t>(g * G + h) * kD + dim + i] = f2h_rn(aa[i] / ll);
     }
     if (tid == 0) p.ticket[g] = 0u;
 }
@@ -465,7 +534,7 @@ qg_status launch_decode_attention(const AttentionLaunch& L, cudaStream_t stream)
     p.hkv = L.hkv;
     p.splits = pick_splits(L.hkv, G, L.l_max, dev.num_sms);
     p.theta = L.theta;
-    p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kD)));
+    p.qscale = kLog2e / std::sqrt(static_cast<double>(kD));
     const size_t tickets = (static_cast<size_t>(L.hkv) * 4 + 255) / 256 * 256;
     p.ticket = static_cast<unsigned int*>(L.workspace);
     p.part = reinterpret_cast<float*>(static_cast<char*>(L.workspace) + tickets);

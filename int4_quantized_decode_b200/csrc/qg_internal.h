@@ -106,7 +106,7 @@ struct AttentionLaunch {
 };
 size_t decode_attention_workspace_bytes(int hq, int hkv);
 qg_status launch_decode_attention(const AttentionLaunch& L, cudaStream_t stream);
-unsigned int attention_read_and_clear_error();  // bit 0: position outside [0, l_max)
+unsigned int attention_read_and_clear_error();  // bit 0: position outside [0, l_max); bit 1: a wait expired
 
 // S <= 16 tokens on the tensor cores (qg_gemm_tc.cu): int8 block-32 or int4
 // group-64 weights, plain (Y fp32) or SwiGLU (H fp16).
