@@ -85,7 +85,7 @@ struct TcFmt {
     static constexpr int kGroup = FMT == 0 ? 32 : 64;      // k per scale (and bias)
 };
 
-template <int FMT, int NMAT, bool SPLIT>
+template <int FMT, int NMAT, bool SPLIT, bool SK = false>
 struct TcLayout {
     using F = TcFmt<FMT>;
     static constexpr int kStageBytes = NMAT * kCodeTileBytes + F::kXBoxes * kXBoxBytes;
@@ -107,10 +107,12 @@ struct TcLayout {
     // Two single-weight CTAs fit on an SM (shared memory) and share its 512
     // tensor-memory columns; a gate/up CTA is alone on its SM and takes all.
     static constexpr uint32_t kTmemCols = NMAT == 1 ? 256 : 512;
-    // tensor memory: accumulator c of matrix m at columns 16 (m kAcc + c);
-    // then the A groups, each kGroupSteps x NMAT x 8 columns (16 fp16 of K
-    // per lane and step)
-    static constexpr int kDCols = 16 * kAcc * NMAT;
+    // tensor memory: accumulator c of matrix m at columns 16 (m kAcc + c)
+    // (stream-K: a second set of them, for the CTA's second tile, at + 16
+    // kAcc NMAT); then the A groups, each kGroupSteps x NMAT x 8 columns (16
+    // fp16 of K per lane and step)
+    static constexpr int kDSetCols = 16 * kAcc * NMAT;
+    static constexpr int kDCols = kDSetCols * (SK ? 2 : 1);
     static constexpr int kGroupCols = kGroupSteps * NMAT * 8;
     static constexpr int kAGroups = (static_cast<int>(kTmemCols) - kDCols) / kGroupCols;
     static constexpr int kGroupsPerStage = F::kKSteps / kGroupSteps;  // 1 or 2
@@ -124,6 +126,8 @@ struct TcLayout {
     static_assert(kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
     static_assert(NMAT == 1 || kSmem > 116 * 1024, "a gate/up CTA must be alone on its SM");
     static_assert(NMAT == 2 || kSmem + 2048 <= 113 * 1024, "two single-weight CTAs per SM");
+    static_assert(!SK || (SPLIT && NMAT == 1), "stream-K runs pair tiles in clusters");
+    static_assert(!SK || kRecvBytes >= kPairRows * 2 * 16 * 4, "one pair tile's partial");
 };
 
 struct TcParams {
@@ -322,13 +326,13 @@ __device__ __forceinline__ bool warp_wait_or_abort(uint64_t* bar, uint32_t parit
     return __all_sync(0xffffffffu, ok);
 }
 
-template <int FMT, int NMAT, int EPI, bool SPLIT>
-__global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 1 ? 2 : 1)
+template <int FMT, int NMAT, int EPI, bool SPLIT, bool SK = false>
+__global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT, SK>::kThreads, NMAT == 1 ? 2 : 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_codes0,
                    const __grid_constant__ CUtensorMap tm_codes1,
                    const __grid_constant__ CUtensorMap tm_x, const TcParams p) {
     using F = TcFmt<FMT>;
-    using L = TcLayout<FMT, NMAT, SPLIT>;
+    using L = TcLayout<FMT, NMAT, SPLIT, SK>;
     constexpr int NSTG = L::kStages;
     constexpr int NG = L::kAGroups;
     constexpr int GPS = L::kGroupsPerStage;
@@ -358,16 +362,40 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 
     const uint32_t rank = SPLIT ? cluster_ctarank_tc() : 0u;
     constexpr bool PAIR = EPI == kEpiPair;
     static_assert(!PAIR || NMAT == 1, "a pair tile holds both matrices in one MMA tile");
-    const int64_t tile = blockIdx.x / P;
-    const int64_t row0 = tile * (PAIR ? kPairRows : kTcRows);  // first output row
-    // this CTA's K range: stages [st0, st1) of the row, split as evenly as the
-    // stage count allows
+    static_assert(!SK || PAIR, "stream-K runs pair tiles");
+    constexpr int kTileRows = PAIR ? kPairRows : kTcRows;  // output rows of a tile
+    // This CTA's work: nA stages of tile tA from its stage sA, then (stream-K
+    // only) nB stages of tile tA + 1 from its stage 0.  A split CTA takes the
+    // stages [rank S / P, (rank + 1) S / P) of its tile's S, as evenly as the
+    // stage count allows.  Stream-K: a cluster of P CTAs takes the (P - 1) S
+    // stages of its P - 1 tiles in P equal shares, u = [rank (P - 1) S / P,
+    // (rank + 1) (P - 1) S / P); with S >= P, rank 0 holds the head of the
+    // first tile, rank P - 1 the tail of the last, and every rank r between
+    // them the tail of tile r - 1 and the head of tile r.
     const int total_st = static_cast<int>(p.k / F::kStageK);
-    const int st0 = static_cast<int>(rank) * total_st / P;
-    const int st1 = (static_cast<int>(rank) + 1) * total_st / P;
-    const int64_t kbeg = static_cast<int64_t>(st0) * F::kStageK;
-    const int nstages = st1 - st0;
+    int64_t tA;
+    int sA, nA, nB = 0;
+    if (SK) {
+        const int U = (P - 1) * total_st;
+        const int u0 = static_cast<int>(rank) * U / P;
+        const int u1 = (static_cast<int>(rank) + 1) * U / P;
+        const int t_in = u0 / total_st;  // tile of the cluster the share starts in
+        const int endA = (t_in + 1) * total_st < u1 ? (t_in + 1) * total_st : u1;
+        tA = static_cast<int64_t>(blockIdx.x / P) * (P - 1) + t_in;
+        sA = u0 - t_in * total_st;
+        nA = endA - u0;
+        nB = u1 - endA;
+    } else {
+        tA = blockIdx.x / P;
+        sA = static_cast<int>(rank) * total_st / P;
+        nA = (static_cast<int>(rank) + 1) * total_st / P - sA;
+    }
+    const int64_t row0 = tA * kTileRows;         // first output row of tile tA
+    const int64_t row0B = row0 + kTileRows;      // ... of tile tA + 1
+    const int64_t kbeg = static_cast<int64_t>(sA) * F::kStageK;
+    const int nstages = nA + nB;
     const int ngroups = nstages * GPS;
+    const int gB = nA * GPS;  // first A group of tile tA + 1 (== ngroups without one)
 
     if (threadIdx.x == 0) {
         abort_sh = 0;
@@ -411,7 +439,8 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 
     auto stage_x = [&](int slot) -> uint32_t {
         return sbase + slot * L::kStageBytes + NMAT * kCodeTileBytes;
     };
-    // accumulator c of matrix m; step j of A group g for matrix m
+    // accumulator c of matrix m (of the second set: + kDSetCols); step j of A
+    // group g for matrix m
     auto d_col = [](int m, int c) -> uint32_t { return static_cast<uint32_t>(16 * (m * kAcc + c)); };
     auto a_col = [](int g, int j, int m) -> uint32_t {
         return static_cast<uint32_t>(L::kDCols + g * L::kGroupCols + (j * NMAT + m) * 8);
@@ -423,25 +452,29 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 
         const uint64_t pol_w = l2_policy_evict_first();
         const uint64_t pol_x = l2_policy_evict_last();
         const int code_bytes_per_k = FMT == 0 ? 1 : 0;  // int8: 1 byte per k; int4: 1/2
+        // stage st of this CTA: k offset and first row of its tile
+        auto stage_k0 = [&](int st) -> int64_t {
+            return static_cast<int64_t>(st < nA ? sA + st : st - nA) * F::kStageK;
+        };
         auto code_c0 = [&](int st) -> int {
-            const int64_t k0 = kbeg + static_cast<int64_t>(st) * F::kStageK;
+            const int64_t k0 = stage_k0(st);
             return static_cast<int>(code_bytes_per_k ? k0 : k0 / 2);
         };
         auto issue_codes = [&](int st) {
             const int slot = st % NSTG;
+            const int r0 = static_cast<int>(st < nA ? row0 : row0B);
             mbar_arrive_expect_tx(&full_bar[slot], L::kStageBytes);
-            tma_load_2d(stage_codes(slot, 0), &tm_codes0, code_c0(st), static_cast<int>(row0),
-                        &full_bar[slot], pol_w);
+            tma_load_2d(stage_codes(slot, 0), &tm_codes0, code_c0(st), r0, &full_bar[slot], pol_w);
             if (PAIR)  // up rows below the gate rows (64-row boxes)
                 tma_load_2d(stage_codes(slot, 0) + kPairRows * kCodeBox, &tm_codes1, code_c0(st),
-                            static_cast<int>(row0), &full_bar[slot], pol_w);
+                            r0, &full_bar[slot], pol_w);
             if (NMAT == 2)
-                tma_load_2d(stage_codes(slot, 1), &tm_codes1, code_c0(st), static_cast<int>(row0),
-                            &full_bar[slot], pol_w);
+                tma_load_2d(stage_codes(slot, 1), &tm_codes1, code_c0(st), r0, &full_bar[slot],
+                            pol_w);
         };
         auto issue_x = [&](int st) {
             const int slot = st % NSTG;
-            const int64_t k0 = kbeg + static_cast<int64_t>(st) * F::kStageK;
+            const int64_t k0 = stage_k0(st);
 #pragma unroll
             for (int b = 0; b < F::kXBoxes; ++b)
                 tma_load_2d(stage_x(slot) + b * kXBoxBytes, &tm_x, static_cast<int>(k0 + b * kXBoxK),
@@ -476,7 +509,8 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 
         // accumulates into accumulator j % kAcc, so consecutive MMAs do not
         // wait for one another's result; one commit then releases the group.
         // The whole warp runs the loop and waits; the elected lane issues the
-        // MMAs and their commits.
+        // MMAs and their commits.  Stream-K: the groups of the second tile
+        // accumulate into the second set, which they start afresh.
         for (int g = 0; g < ngroups; ++g) {
             const int st = g / GPS, gi = g % GPS;
             const int slot = st % NSTG;
@@ -484,6 +518,8 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 
             if (gi == 0 && !warp_wait_or_abort(&full_bar[slot], (st / NSTG) & 1, &abort_sh)) break;
             if (!warp_wait_or_abort(&afull_bar[ag], (g / NG) & 1, &abort_sh)) break;
             tc_fence_after();
+            const uint32_t dset = g >= gB ? static_cast<uint32_t>(L::kDSetCols) : 0u;
+            const bool fresh = g == 0 || g == gB;  // the first group of a tile
             if (elect_one()) {
 #pragma unroll
                 for (int j = 0; j < kGroupSteps; ++j) {
@@ -492,8 +528,8 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 
                                                              (kk % 4) * (kKStep * 2));
 #pragma unroll
                     for (int m = 0; m < NMAT; ++m)
-                        tc_mma_ts(tmem + d_col(m, j % kAcc), tmem + a_col(ag, j, m), bdesc,
-                                  kIdescF16M128N16, (g > 0 || j >= kAcc) ? 1u : 0u);
+                        tc_mma_ts(tmem + dset + d_col(m, j % kAcc), tmem + a_col(ag, j, m), bdesc,
+                                  kIdescF16M128N16, (!fresh || j >= kAcc) ? 1u : 0u);
                 }
                 tc_commit(&aempty_bar[ag]);                     // A group free once read
                 if (gi == GPS - 1) tc_commit(&empty_bar[slot]);  // X of this stage read
@@ -515,11 +551,16 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 
         const int rl = quarter * 32 + lane;   // row within the tile
         const int64_t grow_raw = PAIR ? row0 + (rl & (kPairRows - 1)) : row0 + rl;
         const int64_t grow = grow_raw < p.n ? grow_raw : p.n - 1;  // tail rows: discard
+        const int64_t growB = grow_raw + kTileRows < p.n ? grow_raw + kTileRows : p.n - 1;
         const int msrc = PAIR ? rl / kPairRows : 0;                 // pair tile: gate or up
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
         const int64_t sides_per_row = p.k / F::kGroup;
+        // the row's scales (and biases) from this CTA's first stage of tile tA,
+        // and (stream-K) from stage 0 of tile tA + 1
         const uint16_t* srow[NMAT];
         const uint16_t* brow[NMAT];
+        const uint16_t* srowB[NMAT];
+        const uint16_t* browB[NMAT];
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
             // (a select, not an index: a parameter array indexed at run time
@@ -528,13 +569,18 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 
             const uint16_t* bbase = (m + msrc) == 0 ? p.biases[0] : p.biases[1];
             srow[m] = sbase + grow * sides_per_row + kbeg / F::kGroup;
             brow[m] = FMT == 1 ? bbase + grow * sides_per_row + kbeg / F::kGroup : nullptr;
+            srowB[m] = sbase + growB * sides_per_row;
+            browB[m] = FMT == 1 ? bbase + growB * sides_per_row : nullptr;
         }
         // the row's 4 scales (and biases) of a stage: 8 bytes each
         auto load_sides = [&](int st, uint2 (&sv)[NMAT], uint2 (&bv)[NMAT]) {
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
-                sv[m] = __ldg(reinterpret_cast<const uint2*>(srow[m] + st * 4));
-                if (FMT == 1) bv[m] = __ldg(reinterpret_cast<const uint2*>(brow[m] + st * 4));
+                const bool b = SK && st >= nA;
+                const int o = (b ? st - nA : st) * 4;
+                sv[m] = __ldg(reinterpret_cast<const uint2*>((b ? srowB[m] : srow[m]) + o));
+                if (FMT == 1)
+                    bv[m] = __ldg(reinterpret_cast<const uint2*>((b ? browB[m] : brow[m]) + o));
             }
         };
         uint2 sv[NMAT], bv[NMAT], sv_next[NMAT], bv_next[NMAT];
@@ -602,6 +648,7 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 
     // after it has completed.
     griddep_wait();
     float acc[NMAT][16];
+    float accB[16];  // stream-K: the second tile's partial (rank 1)
     const bool epi_warp = warp >= 2 && warp < 6;  // one warp per tensor-memory quarter
     const int quarter = warp & 3;
     const int rl = quarter * 32 + lane;
@@ -610,31 +657,88 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT>::kThreads, NMAT == 
         tc_fence_after();
         __syncwarp();
         // the kAcc partial sums of each matrix, added in accumulator order
-#pragma unroll
-        for (int m = 0; m < NMAT; ++m) {
-            const uint32_t base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        auto load_acc = [&](uint32_t col0, float (&out)[16]) {
+            const uint32_t base = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + col0;
             uint32_t r[kAcc][16];  // every accumulator's load in flight, one wait
 #pragma unroll
-            for (int c = 0; c < kAcc; ++c) tc_ld16_async(base + d_col(m, c), r[c]);
+            for (int c = 0; c < kAcc; ++c) tc_ld16_async(base + d_col(0, c), r[c]);
             tc_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 float v = __uint_as_float(r[0][i]);
 #pragma unroll
                 for (int c = 1; c < kAcc; ++c) v += __uint_as_float(r[c][i]);
-                acc[m][i] = v;
+                out[i] = done ? v : 0.f;
             }
-            if (!done)
+        };
 #pragma unroll
-                for (int i = 0; i < 16; ++i) acc[m][i] = 0.f;
-        }
+        for (int m = 0; m < NMAT; ++m) load_acc(d_col(m, 0), acc[m]);
+        if (SK && nB > 0) load_acc(static_cast<uint32_t>(L::kDSetCols), accB);
         // this warp's tensor-memory reads are complete (tcgen05.wait::ld)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&fin_bar);
     }
 
-    if (SPLIT) {
+    if (SK) {
+        // Stream-K.  Every rank but the first stages the partial of its first
+        // tile as [pair row][gate|up][token] and sends it with one bulk copy
+        // into the receive buffer, onto the receive barrier, of rank - 1, which
+        // owns that tile; every rank but the last owns the tile of its last
+        // stages, adds the partial it receives to its own and stores the tile.
+        constexpr int kPartialFloats = kPairRows * 2 * 16;
+        float* stage = reinterpret_cast<float*>(sgen);       // the stages are free now
+        float* xch = stage + kPartialFloats;                  // the owner's gate/up exchange
+        float* recv = reinterpret_cast<float*>(sgen + NSTG * L::kStageBytes);
+        const bool sends = rank > 0;
+        const bool owns = static_cast<int>(rank) < P - 1;
+        const int ri = rl & (kPairRows - 1), vm = rl / kPairRows;
+        if (epi_warp && sends) {
+            float4* dst = reinterpret_cast<float4*>(stage + (ri * 2 + vm) * 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                dst[i] = make_float4(acc[0][4 * i], acc[0][4 * i + 1], acc[0][4 * i + 2],
+                                     acc[0][4 * i + 3]);
+            // the bulk copy (async proxy) reads what these stores wrote
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        __syncwarp();
+        if (warp >= 2)  // warps 2.. : the staged partial is visible to the sending warp
+            asm volatile("barrier.sync 2, %0;" ::"r"(L::kThreads - 64) : "memory");
+        if (owns && threadIdx.x == 64)
+            mbar_arrive_expect_tx(&recv_bar, static_cast<uint32_t>(kPartialFloats * 4));
+        cluster_wait();  // every peer's receive barrier is initialized
+        if (sends && warp == 2) {
+            if (lane == 0) {
+                const uint32_t q = rank - 1;
+                bulk_s2peer(peer_addr(smem_u32(recv), q), smem_u32(stage),
+                            static_cast<uint32_t>(kPartialFloats * 4),
+                            peer_addr(smem_u32(&recv_bar), q));
+            }
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+        if (owns && epi_warp) {
+            if (!mbar_wait_bounded(&recv_bar, 0) && lane == 0) atomicOr(&g_tc_err, kGemvErrTimeout);
+            // own partial (of the last stages: the second set when there are
+            // two tiles) + the received one, then the pair tile's gate/up
+            // exchange as in the whole-tile path below
+            const float* own = nB > 0 ? accB : acc[0];
+            const int64_t orow0 = nB > 0 ? row0B : row0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) xch[i * kTcRows + rl] = own[i] + recv[(ri * 2 + vm) * 16 + i];
+            __syncwarp();
+            asm volatile("barrier.sync 1, 128;" ::: "memory");
+            for (int e = (warp - 2) * 32 + lane; e < kPairRows * 16; e += 128) {
+                const int tok = e / kPairRows, r = e % kPairRows;
+                const float g = xch[tok * kTcRows + r], u = xch[tok * kTcRows + kPairRows + r];
+                const int64_t grow = orow0 + r;
+                if (tok < p.S && grow < p.n)
+                    p.H[static_cast<int64_t>(tok) * p.n + grow] = f2h_rn(g / (1.0f + expf(-g)) * u);
+            }
+        }
+        // this CTA's copy has read its staged partial before it may exit
+        if (sends && warp == 2) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    } else if (SPLIT) {
         // Split K.  Rank q finishes rows [q RT / P, (q + 1) RT / P) of the
         // tile's RT rows (output rows; pair rows for a pair tile, each with
         // the gate and up vectors).  Every CTA stages its partials in its own
@@ -787,10 +891,10 @@ qg_status make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int
 }
 
 // Shared memory of the kernel variant, and its attributes set once per device.
-template <int FMT, int NMAT, int EPI, bool SPLIT>
+template <int FMT, int NMAT, int EPI, bool SPLIT, bool SK = false>
 qg_status prepare_tc(const DeviceInfo& dev, size_t* smem_out) {
-    using L = TcLayout<FMT, NMAT, SPLIT>;
-    auto kern = gemm_tc_kernel<FMT, NMAT, EPI, SPLIT>;
+    using L = TcLayout<FMT, NMAT, SPLIT, SK>;
+    auto kern = gemm_tc_kernel<FMT, NMAT, EPI, SPLIT, SK>;
     const size_t smem = L::kSmem + 1024;
     if (smem + 2048 > static_cast<size_t>(dev.max_smem_optin)) return QG_ERR_SHAPE;
     static bool attr_done[64] = {false};
@@ -810,7 +914,7 @@ qg_status prepare_tc(const DeviceInfo& dev, size_t* smem_out) {
 
 // Clusters of P CTAs the device holds at once for this kernel (cached per
 // device and P); 0 if the query fails.
-template <int FMT, int NMAT, int EPI, bool SPLIT>
+template <int FMT, int NMAT, int EPI, bool SPLIT, bool SK = false>
 int clusters_per_wave(const DeviceInfo& dev, size_t smem, int P) {
     static int cache[64][kMaxClusterTc + 1] = {{0}};
     if (dev.device < 64 && cache[dev.device][P] != 0) return cache[dev.device][P];
@@ -826,7 +930,7 @@ int clusters_per_wave(const DeviceInfo& dev, size_t smem, int P) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<FMT, NMAT, EPI, SPLIT>, &cfg) !=
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<FMT, NMAT, EPI, SPLIT, SK>, &cfg) !=
         cudaSuccess) {
         cudaGetLastError();  // clear the query's error
         return 0;
@@ -883,6 +987,39 @@ double choose_split(const GemmS16Launch& Lc, const DeviceInfo& dev, size_t smem1
     return best;
 }
 
+// Stream-K for pair tiles: clusters of C CTAs over C - 1 tiles, each CTA
+// (C - 1) / C of a tile, every tile finished by one CTA.  The same model as
+// the split: returns the time it expects for the best C (3..8, C - 1 dividing
+// the tile count, at least C stages per tile), or infinity if none applies.
+template <int FMT>
+double stream_k_time(const GemmS16Launch& Lc, const DeviceInfo& dev, size_t smemSK, int* C_out) {
+    using F = TcFmt<FMT>;
+    const int64_t tiles = (Lc.n + kPairRows - 1) / kPairRows;
+    const int64_t stages = Lc.k / F::kStageK;
+    const double bytes_per_k = FMT == 0 ? 1.0625 : 0.5625;
+    const double tile_kb = kTcRows * static_cast<double>(Lc.k) * bytes_per_k / 1e3;
+    double best = 1e30;
+    *C_out = 0;
+    for (int c = 3; c <= kMaxClusterTc; ++c) {
+        if (tiles % (c - 1) != 0 || stages < c) continue;
+        int cpw = clusters_per_wave<FMT, 1, kEpiPair, true, true>(dev, smemSK, c);
+        if (cpw <= 0) continue;
+        cpw = std::max(2 * cpw, static_cast<int>(0.9 * 2 * dev.num_sms / c));
+        const int64_t clusters = tiles / (c - 1);
+        const int64_t rounds = (clusters + cpw - 1) / cpw;
+        const int64_t per_round = (clusters + rounds - 1) / rounds;
+        const int64_t per_sm = (per_round * c + dev.num_sms - 1) / dev.num_sms;
+        const double rate = (FMT == 0 ? 1.0 : 0.5) * (per_sm >= 2 ? 54.0 : 29.0);
+        const double t = static_cast<double>(rounds) *
+                         (static_cast<double>(per_sm) * tile_kb * (c - 1) / c / rate + 4.6);
+        if (t < best * (1 - 1e-9)) {
+            best = t;
+            *C_out = c;
+        }
+    }
+    return best;
+}
+
 template <int FMT, int NMAT, int EPI>
 qg_status prepare_both(const DeviceInfo& dev, size_t* smem1, size_t* smemP) {
     qg_status st = prepare_tc<FMT, NMAT, EPI, false>(dev, smem1);
@@ -892,7 +1029,7 @@ qg_status prepare_both(const DeviceInfo& dev, size_t* smem1, size_t* smemP) {
 
 template <int FMT, int NMAT, int EPI>
 qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream_t stream,
-                      int P, size_t smem1, size_t smemP) {
+                      int P, size_t smem1, size_t smemP, bool sk = false) {
     constexpr bool PAIR = EPI == kEpiPair;
     constexpr int kMats = PAIR ? 2 : NMAT;
     CUtensorMap mc[2], mx;
@@ -919,11 +1056,11 @@ qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream
     p.n = Lc.n;
     p.k = Lc.k;
     p.S = Lc.S;
-    p.splits = P;
     const int64_t tiles = (Lc.n + (PAIR ? kPairRows : kTcRows) - 1) / (PAIR ? kPairRows : kTcRows);
+    p.splits = P;  // stream-K: P CTAs per P - 1 tiles (smemP is the stream-K kernel's)
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(tiles * P));
+    cfg.gridDim = dim3(static_cast<unsigned>(sk ? tiles / (P - 1) * P : tiles * P));
     cfg.blockDim = dim3(TcLayout<FMT, NMAT, false>::kThreads);
     cfg.dynamicSmemBytes = P > 1 ? smemP : smem1;
     cfg.stream = stream;
@@ -939,6 +1076,9 @@ qg_status launch_tc_t(const GemmS16Launch& Lc, const DeviceInfo& dev, cudaStream
     ++na;
     cfg.attrs = attr;
     cfg.numAttrs = na;
+    if (PAIR && sk)
+        return cuda_status(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<FMT, NMAT, EPI, true, PAIR>,
+                                              mc[0], mc[1], mx, p));
     if (P > 1)
         return cuda_status(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<FMT, NMAT, EPI, true>, mc[0],
                                               mc[1], mx, p));
@@ -963,7 +1103,13 @@ qg_status launch_fmt(const GemmS16Launch& L, const DeviceInfo& dev, cudaStream_t
     }
     qg_status st = prepare_both<FMT, 1, kEpiPair>(dev, &s1, &sP);
     if (st != QG_OK) return st;
-    choose_split<FMT, 1, kEpiPair>(L, dev, s1, sP, &P);
+    const double t_split = choose_split<FMT, 1, kEpiPair>(L, dev, s1, sP, &P);
+    size_t sSK = 0;
+    st = prepare_tc<FMT, 1, kEpiPair, true, true>(dev, &sSK);
+    if (st != QG_OK) return st;
+    int C = 0;
+    if (stream_k_time<FMT>(L, dev, sSK, &C) < t_split)
+        return launch_tc_t<FMT, 1, kEpiPair>(L, dev, stream, C, s1, sSK, true);
     return launch_tc_t<FMT, 1, kEpiPair>(L, dev, stream, P, s1, sP);
 }
 

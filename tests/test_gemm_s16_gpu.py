@@ -57,11 +57,13 @@ def test_gemm_s16_deterministic(cuda, fmt):
 
 
 # gate/up runs as pair tiles (64 gate + 64 up rows per tensor-core tile): the
-# shapes take it whole on one CTA per tile (12288x4096, 9728x2560) and split
-# over clusters (77x512, 1000x2048, 6144x2048, 130x2560), with ragged pair
-# tiles (77, 1000, 130 rows) and S below 16
+# shapes run stream-K (three CTAs of a cluster over two pair tiles: 12288x4096,
+# 12248x4096 with a ragged last tile, 9728x2560) or split K over clusters
+# (77x512, 1000x2048, 6144x2048, 130x2560), with ragged pair tiles (77, 1000,
+# 130, 12248 rows) and S below 16
 @pytest.mark.parametrize("fmt,n,k,S", [(I8, 12288, 4096, 16), (I8, 77, 512, 5), (I8, 1000, 2048, 16),
                                        (I8, 6144, 2048, 16), (I8, 130, 2560, 11),
+                                       (I8, 12248, 4096, 7), (I8, 9728, 2560, 16),
                                        (I4, 12288, 4096, 16), (I4, 77, 512, 5),
                                        (I4, 1000, 2048, 16), (I4, 9728, 2560, 9)])
 def test_swiglu_s16(cuda, fmt, n, k, S):
