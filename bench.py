@@ -115,10 +115,10 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-# The sources of the S=1 and S<=16 kernels whose DRAM traffic profiles/dram_traffic.txt
+# The sources of the S=1, S<=16 and attention kernels whose DRAM traffic profiles/dram_traffic.txt
 # records: a committed traffic figure is used only while these are unchanged.
 KERNEL_SOURCES = ("qg_device.cuh", "qg_gemv.cu", "qg_gemv_impl.cuh", "qg_internal.h",
-                  "qg_gemm_tc.cu")
+                  "qg_gemm_tc.cu", "qg_attention.cu")
 
 
 def csrc_digest() -> str:

@@ -303,6 +303,8 @@ QG_API qg_status qg_rmsnorm_f16(const float* h, const uint16_t* gamma, int64_t k
  *          workspace must be serialized.
  * Accuracy: |o - o_ref| <= 1e-3 * sum_j p_j |V[g][j]| + ulp_f16(o_ref) per
  * element, o_ref the fp64 attention on the same fp16 cache.  Deterministic.
+ * The kernel's waits on its own copies are bounded; one that expires makes
+ * qg_stream_check report QG_ERR_TIMEOUT (o is then undefined).
  * ------------------------------------------------------------------------- */
 QG_API size_t qg_decode_attention_workspace_bytes(int hq, int hkv);
 QG_API qg_status qg_decode_attention(const float* qkv, int hq, int hkv, int d,
