@@ -342,7 +342,8 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT, SK>::kThreads, NMAT
     // a stage's codes are read by one set (int8: one group per stage) or by both
     constexpr int kEmptyArrivals = (GPS == 1 ? NDQ / 2 : NDQ) + 1;
     extern __shared__ unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t full_bar[NSTG];
+    __shared__ __align__(8) uint64_t full_bar[NSTG];   // a stage's codes have landed
+    __shared__ __align__(8) uint64_t xfull_bar[NSTG];  // its X chunk has landed
     __shared__ __align__(8) uint64_t empty_bar[NSTG];
     __shared__ __align__(8) uint64_t afull_bar[NG];
     __shared__ __align__(8) uint64_t aempty_bar[NG];
@@ -401,6 +402,7 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT, SK>::kThreads, NMAT
         abort_sh = 0;
         for (int s = 0; s < NSTG; ++s) {
             mbar_init(&full_bar[s], 1);
+            mbar_init(&xfull_bar[s], 1);
             mbar_init(&empty_bar[s], kEmptyArrivals);
         }
         for (int j = 0; j < NG; ++j) {
@@ -463,7 +465,7 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT, SK>::kThreads, NMAT
         auto issue_codes = [&](int st) {
             const int slot = st % NSTG;
             const int r0 = static_cast<int>(st < nA ? row0 : row0B);
-            mbar_arrive_expect_tx(&full_bar[slot], L::kStageBytes);
+            mbar_arrive_expect_tx(&full_bar[slot], NMAT * kCodeTileBytes);
             tma_load_2d(stage_codes(slot, 0), &tm_codes0, code_c0(st), r0, &full_bar[slot], pol_w);
             if (PAIR)  // up rows below the gate rows (64-row boxes)
                 tma_load_2d(stage_codes(slot, 0) + kPairRows * kCodeBox, &tm_codes1, code_c0(st),
@@ -475,10 +477,11 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT, SK>::kThreads, NMAT
         auto issue_x = [&](int st) {
             const int slot = st % NSTG;
             const int64_t k0 = stage_k0(st);
+            mbar_arrive_expect_tx(&xfull_bar[slot], F::kXBoxes * kXBoxBytes);
 #pragma unroll
             for (int b = 0; b < F::kXBoxes; ++b)
                 tma_load_2d(stage_x(slot) + b * kXBoxBytes, &tm_x, static_cast<int>(k0 + b * kXBoxK),
-                            0, &full_bar[slot], pol_x);
+                            0, &xfull_bar[slot], pol_x);
         };
         // codes of the first stages before the wait on the previous kernel
         const int pre = nstages < NSTG ? nstages : NSTG;
@@ -500,8 +503,10 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT, SK>::kThreads, NMAT
         }
         // drain: every issued copy lands before the CTA may exit (bounded)
         const int first = nstages > NSTG ? nstages - NSTG : 0;
-        for (int st = first; st < nstages; ++st)
+        for (int st = first; st < nstages; ++st) {
             mbar_wait_bounded(&full_bar[st % NSTG], (st / NSTG) & 1);
+            mbar_wait_bounded(&xfull_bar[st % NSTG], (st / NSTG) & 1);
+        }
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA ---
@@ -515,7 +520,7 @@ __global__ void __launch_bounds__(TcLayout<FMT, NMAT, SPLIT, SK>::kThreads, NMAT
             const int st = g / GPS, gi = g % GPS;
             const int slot = st % NSTG;
             const int ag = g % NG;
-            if (gi == 0 && !warp_wait_or_abort(&full_bar[slot], (st / NSTG) & 1, &abort_sh)) break;
+            if (gi == 0 && !warp_wait_or_abort(&xfull_bar[slot], (st / NSTG) & 1, &abort_sh)) break;
             if (!warp_wait_or_abort(&afull_bar[ag], (g / NG) & 1, &abort_sh)) break;
             tc_fence_after();
             const uint32_t dset = g >= gB ? static_cast<uint32_t>(L::kDSetCols) : 0u;
