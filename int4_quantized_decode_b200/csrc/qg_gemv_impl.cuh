@@ -915,7 +915,7 @@ constexpr size_t ring_smem_bytes() {
 }
 
 // Per-CTA shared memory that still lets two CTAs share an SM.
-constexpr size_t kSmemPerCtaBudget = 110 * 1024;
+constexpr size_t kSmemPerCtaBudget = 112 * 1024;
 
 template <int FMT, int NMAT, int RG, int EPI, bool RING>
 qg_status launch_t(Params p, const DeviceInfo& dev, cudaStream_t stream) {
@@ -997,6 +997,17 @@ qg_status launch_pick(const Params& p0, const DeviceInfo& dev, cudaStream_t stre
 // Launch one S=1 call of format FMT.  PLAIN is the single-weight epilogue
 // (kEpiPlain, or kEpiResidual for the residual-stream update); XF adds
 // kEpiNormIn when x is the RMSNorm of an fp32 hidden state.
+// Rows (or gate/up pairs) per warp item times the most items any warp gets:
+// the warp makespan, in rows, of round-robin items over tw warps.  Items of
+// three rows are taken (int8) when they cut that makespan by a quarter or
+// more against the measured rule above: timed on B200, the 2B gate/up (6144
+// pairs on 2368 warps: 4 -> 3 pairs for the busiest warp), the 4B / 8B q|k|v
+// and the 27B o and down, sweeps 2B / 4B / 8B / 27B +2.7 / +2.0 / +0.5 / +6.4%.
+inline int64_t makespan_rows(int64_t n, int rg, int tw) {
+    const int64_t items = (n + rg - 1) / rg;
+    return (items + tw - 1) / tw * rg;
+}
+
 template <int FMT, int PLAIN = kEpiPlain, int XF = 0>
 qg_status dispatch_fmt(const GemvLaunch& L, const Params& p, const DeviceInfo& dev,
                        cudaStream_t stream) {
@@ -1007,7 +1018,10 @@ qg_status dispatch_fmt(const GemvLaunch& L, const Params& p, const DeviceInfo& d
             if constexpr (FMT == 2) {
                 return QG_ERR_FORMAT;  // fp16 weights: GEMV and head only
             } else {
-                if (pick_rg(L.n, 2, tw) == 2)
+                const int rg2 = pick_rg(L.n, 2, tw);
+                if (FMT == 0 && 4 * makespan_rows(L.n, 3, tw) <= 3 * makespan_rows(L.n, rg2, tw))
+                    return launch_pick<FMT, 2, 3, kEpiSwiglu | XF>(p, dev, stream);
+                if (rg2 == 2)
                     return launch_pick<FMT, 2, 2, kEpiSwiglu | XF>(p, dev, stream);
                 return launch_pick<FMT, 2, 1, kEpiSwiglu | XF>(p, dev, stream);
             }
@@ -1018,6 +1032,8 @@ qg_status dispatch_fmt(const GemvLaunch& L, const Params& p, const DeviceInfo& d
             return launch_pick<FMT, 1, 1, kEpiHead | XF>(p, dev, stream);
         }
     }
+    if (FMT == 0 && 4 * makespan_rows(L.n, 3, tw) <= 3 * makespan_rows(L.n, rg, tw))
+        return launch_pick<FMT, 1, 3, PLAIN | XF>(p, dev, stream);
     if (rg == 4) return launch_pick<FMT, 1, 4, PLAIN | XF>(p, dev, stream);
     if (rg == 2) return launch_pick<FMT, 1, 2, PLAIN | XF>(p, dev, stream);
     return launch_pick<FMT, 1, 1, PLAIN | XF>(p, dev, stream);
