@@ -1008,6 +1008,22 @@ inline int64_t makespan_rows(int64_t n, int rg, int tw) {
     return (items + tw - 1) / tw * rg;
 }
 
+// Three-row items (int8) run on the shared-memory ring only, with x by bulk
+// copy unless x is an RMSNorm input; callers check that this fits first.
+template <int NMAT, int EPI>
+bool ring3_fits(const Params& p0) {
+    Params p = p0;
+    p.x_bulk = (EPI & kEpiNormIn) ? 0 : 1;
+    return (p.k / Fmt<0>::kBlock) % 8 == 0 &&
+           x_smem_bytes(0, p) + ring_smem_bytes<0, NMAT, 3>() <= kSmemPerCtaBudget;
+}
+template <int NMAT, int EPI>
+qg_status launch_ring3(const Params& p0, const DeviceInfo& dev, cudaStream_t stream) {
+    Params p = p0;
+    p.x_bulk = (EPI & kEpiNormIn) ? 0 : 1;
+    return launch_t<0, NMAT, 3, EPI, true>(p, dev, stream);
+}
+
 template <int FMT, int PLAIN = kEpiPlain, int XF = 0>
 qg_status dispatch_fmt(const GemvLaunch& L, const Params& p, const DeviceInfo& dev,
                        cudaStream_t stream) {
@@ -1019,8 +1035,11 @@ qg_status dispatch_fmt(const GemvLaunch& L, const Params& p, const DeviceInfo& d
                 return QG_ERR_FORMAT;  // fp16 weights: GEMV and head only
             } else {
                 const int rg2 = pick_rg(L.n, 2, tw);
-                if (FMT == 0 && 4 * makespan_rows(L.n, 3, tw) <= 3 * makespan_rows(L.n, rg2, tw))
-                    return launch_pick<FMT, 2, 3, kEpiSwiglu | XF>(p, dev, stream);
+                if constexpr (FMT == 0) {
+                    if (4 * makespan_rows(L.n, 3, tw) <= 3 * makespan_rows(L.n, rg2, tw) &&
+                        ring3_fits<2, kEpiSwiglu | XF>(p))
+                        return launch_ring3<2, kEpiSwiglu | XF>(p, dev, stream);
+                }
                 if (rg2 == 2)
                     return launch_pick<FMT, 2, 2, kEpiSwiglu | XF>(p, dev, stream);
                 return launch_pick<FMT, 2, 1, kEpiSwiglu | XF>(p, dev, stream);
@@ -1032,8 +1051,11 @@ qg_status dispatch_fmt(const GemvLaunch& L, const Params& p, const DeviceInfo& d
             return launch_pick<FMT, 1, 1, kEpiHead | XF>(p, dev, stream);
         }
     }
-    if (FMT == 0 && 4 * makespan_rows(L.n, 3, tw) <= 3 * makespan_rows(L.n, rg, tw))
-        return launch_pick<FMT, 1, 3, PLAIN | XF>(p, dev, stream);
+    if constexpr (FMT == 0) {
+        if (4 * makespan_rows(L.n, 3, tw) <= 3 * makespan_rows(L.n, rg, tw) &&
+            ring3_fits<1, PLAIN | XF>(p))
+            return launch_ring3<1, PLAIN | XF>(p, dev, stream);
+    }
     if (rg == 4) return launch_pick<FMT, 1, 4, PLAIN | XF>(p, dev, stream);
     if (rg == 2) return launch_pick<FMT, 1, 2, PLAIN | XF>(p, dev, stream);
     return launch_pick<FMT, 1, 1, PLAIN | XF>(p, dev, stream);

@@ -42,7 +42,8 @@ def _case(fmt, n, k, seed, dev):
 
 SHAPES = ([(I8, n, k) for n, k in [(5, 32), (77, 64), (130, 96), (300, 2048), (2050, 6144),
                                     (64, 17408)]] +
-          [(I4, n, k) for n, k in [(5, 64), (77, 128), (130, 192), (300, 2560), (1000, 9728)]])
+          [(I4, n, k) for n, k in [(5, 64), (77, 128), (130, 192), (300, 2560), (1000, 9728),
+                                    (6001, 2560)]])
 
 
 @pytest.mark.parametrize("fmt,n,k", SHAPES)

@@ -21,7 +21,10 @@ I8, I4 = qg.FMT_I8_B32, qg.FMT_I4_G64
 SHAPES_I8 = [(1, 32), (7, 96), (33, 544), (300, 2048), (1000, 2080), (4103, 512),
              (2048, 6144), (9473, 2560), (20000, 1024), (64, 17408)]
 SHAPES_I4 = [(1, 64), (9, 192), (41, 1088), (300, 2560), (1000, 1536), (4103, 1024),
-             (20000, 2048), (64, 9728)]
+             (20000, 2048), (64, 9728),
+             # rows of 32 x + 16 lane granules with 2 and 4 rows per warp item
+             # (the last step of each row pair packed into one warp step)
+             (4103, 2560), (6001, 1536), (3000, 9728)]
 
 
 def _weight(fmt, n, k, seed, dev):
