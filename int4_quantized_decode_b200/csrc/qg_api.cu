@@ -333,11 +333,11 @@ qg_status qg_sweep_plan(const qg_stage* stages, int n_stages, void* workspace, s
     out.n_stages = n_stages;
     // the stream sweep when the plan qualifies (all int8, rows of whole
     // 512-code steps), else the general persistent kernels
-    int depth = 0, xmax = 0;
-    qg_status st = qg::plan_stream(L.data(), n_stages, workspace, ws_bytes, &depth, &xmax);
+    int slots = 0, xmax = 0;
+    qg_status st = qg::plan_stream(L.data(), n_stages, workspace, ws_bytes, &slots, &xmax);
     if (st == QG_OK) {
         out.kernel = qg::kSweepKernelStream;
-        out.reserved[0] = depth;
+        out.reserved[0] = slots;
         out.reserved[1] = xmax;
         *sweep = out;
         return QG_OK;

@@ -66,9 +66,9 @@ qg_status launch_sweep(int kernel, void* ws, int n_stages, cudaStream_t stream);
 // The stream sweep (qg_stream.cu): all-int8 plans whose rows hold whole
 // 512-code steps run as one launch whose weight stream spans the stages.
 size_t stream_workspace_bytes(int n_stages);
-qg_status plan_stream(const GemvLaunch* L, int n, void* ws, size_t ws_bytes, int* depth,
+qg_status plan_stream(const GemvLaunch* L, int n, void* ws, size_t ws_bytes, int* slots,
                       int* xmax);
-qg_status launch_stream(void* ws, int n, int depth, int xmax, cudaStream_t stream);
+qg_status launch_stream(void* ws, int n, int slots, int xmax, cudaStream_t stream);
 unsigned int stream_read_and_clear_error();
 constexpr int kSweepKernelStream = 2;
 

@@ -6,31 +6,37 @@
 // S=1 projections in which each stage needs the whole output of the stage
 // before it ("Qwen3.8-27B ... -- Core AI", The vision path: prefill runs as
 // pipelined S=1 steps).  Only the activation depends on the previous stage,
-// never the weights; so every warp streams its own weight rows through a
-// deep per-lane shared-memory ring whose copy cursor runs straight on into
-// the next stages while the warp waits for the next activation.  With 8-11
-// slots per lane and 15 streaming warps per SM, 110-150 KB of weights per SM
-// are in flight across each stage boundary.
+// never the weights; so one thread per SM streams the SM's share of every
+// stage's weights, in plan order, into a shared-memory ring and never waits
+// for an activation: while the compute warps wait at a stage boundary the
+// ring keeps filling.
 //
-//  * One CTA per SM (cooperative launch): 15 streaming warps + 1 sync warp.
-//  * Items: one or two weight rows (a row or row pair of a projection, or the
-//    gate and up rows of one SwiGLU output).  Item j of a stage goes to CTA
-//    j % G and to warp ((j / G) + rot) % 15 of it; rot turns from stage to
-//    stage so that no warp always gets the extra item.
-//  * Copy cursor: each lane copies 16 bytes of every row's 512-byte step with
-//    cp.async into its warp's ring slot, four lanes copying the step's 16
-//    scales; D - 1 steps stay in flight, across stage boundaries.
-//  * Compute: lane l takes the 8-byte code pieces at 8 l and 256 + 8 l of a
-//    step against x read raw (fp16, as the bulk copy left it) at 16 l and
-//    512 + 16 l: conflict-free, so x needs no re-layout.  Codes become exact
-//    fp16 q (byte permute into 1024 + (q + 128), packed subtraction of 1152)
-//    and the sm_100 mixed-precision FMA accumulates the exact products q x
-//    in fp32; the block scale multiplies each 8-code partial.
-//  * Sync warp: when every warp of its CTA is done with stage s (an
+//  * One CTA per SM (cooperative launch): 16 compute warps, a producer warp
+//    and a sync warp.
+//  * Each CTA owns a contiguous range of every stage's rows (n / G rounded,
+//    so no CTA has more than one row above the average), cut into chunks of
+//    whole rows (a SwiGLU chunk: the same rows of gate and of up) of at most
+//    32 KB of codes, so that every chunk is a few large 1-D bulk copies (on
+//    this GPU a bulk copy costs ~450 cycles of the SM's copy engine whatever
+//    its size, and only copies of 16 KB or more reach the HBM rate).
+//  * Producer: one lane issues each chunk's copies (codes and fp16 scales of
+//    each matrix) into the chunk's ring slot, completing on the slot's
+//    mbarrier; it refills a slot once every compute warp has released it.
+//  * Compute warps: row u of a stage's range belongs to warp u % 16, which
+//    computes it whole (lane l takes the 16 codes at 16 l of each 512-code
+//    step against x[16 l .. 16 l + 16), raw fp16 in shared memory; codes
+//    become exact fp16 q by a byte permute into 1024 + (q + 128) and a packed
+//    subtraction of 1152, and the sm_100 mixed-precision FMA accumulates the
+//    exact products q x in fp32; each block scale multiplies its 16-code
+//    partial; one warp reduction per row).  Every compute warp walks every
+//    chunk in ring order -- waits for its copies, computes its own rows in it,
+//    releases it -- so it sees each slot's fills in order and no parity wait
+//    can match a stale phase.
+//  * Sync warp: when every compute warp of its CTA is done with stage s (an
 //    mbarrier), it arrives on the grid counter of stage s (release), waits
 //    for every CTA (acquire, bounded) and fetches x of stage s + 1 with one
 //    bulk copy into the other half of a double buffer, on an mbarrier the
-//    streaming warps wait on.  It also finishes a head stage's argmax for its
+//    compute warps wait on.  It also finishes a head stage's argmax for its
 //    CTA (atomicMax of an order-preserving key, last-CTA ticket).
 //  * Every wait is bounded; one that gives up sets the device error flag and
 //    the CTA's abort flag, after which the CTA drains its own copies and
@@ -48,27 +54,32 @@ QG_DEFINE_ERROR_FLAG(g_stream_err);
 
 namespace {
 
-constexpr int kSwW = 15;                      // streaming warps per CTA
-constexpr int kSwThreads = (kSwW + 1) * 32;   // + the sync warp
-constexpr int kSwStep = 512;                  // code bytes of one warp step along a row
-constexpr int kSwSlotRow = kSwStep + 32;      // codes + the step's 16 fp16 scales
-constexpr int kSwSlot = 2 * kSwSlotRow;       // a slot holds up to two rows
+constexpr int kSwW = 16;                      // compute warps per CTA
+constexpr int kProdWarp = kSwW;               // the producer warp
+constexpr int kSyncWarp = kSwW + 1;           // the sync warp
+constexpr int kSwThreads = (kSwW + 2) * 32;
+constexpr int kSwStep = 512;                  // codes of one warp step along a row
+constexpr int kChunkCodes = 32768;            // code bytes a ring slot holds
+constexpr int kSlotBytes = kChunkCodes + kChunkCodes / 16;  // + their fp16 scales
+constexpr int kMaxSlots = 8;
+constexpr int kMinSlots = 3;
 constexpr int kSwMaxStages = 320;
-constexpr uint32_t kStreamMagic = 0x32575351u;
+constexpr uint32_t kStreamMagic = 0x34575351u;
 
 enum StreamOp : int32_t { kOpGemv = 0, kOpSwiglu = 1, kOpHead = 2 };
 
 // What the warps' cursors read of a stage (kept in shared memory).
+// Rows are output rows: a SwiGLU row is the pair (gate r, up r).
 struct StreamStage {
     const uint8_t* codes[2];    // gemv/head: [0]; swiglu: gate, up
     const uint16_t* scales[2];
     int32_t n, k;               // rows, columns (k % 512 == 0)
-    int32_t items;              // work items of the stage
     int32_t op;                 // StreamOp
-    int32_t rows;               // rows per item: 1 or 2
-    int32_t rot;                // warp rotation of the item assignment
+    int32_t nmat;               // 1, or 2 for SwiGLU
+    int32_t nrc;                // rows per chunk: nmat * nrc * k <= kChunkCodes
     int32_t nst;                // steps per row: k / 512
     int32_t xext;               // x is a run input: no stage of the plan writes it
+    int32_t pad;
 };
 static_assert(sizeof(StreamStage) == 64, "stage descriptors are 64 bytes");
 
@@ -88,7 +99,7 @@ static_assert(sizeof(StreamOut) == 64, "outputs are 64 bytes");
 struct StreamHeader {
     uint32_t magic;
     int32_t n_stages;
-    int32_t depth;              // ring slots per lane the plan was made for
+    int32_t slots;              // ring slots the plan was made for
     int32_t xmax;               // the largest k of the plan
     uint32_t reserved[60];
 };
@@ -125,8 +136,8 @@ __host__ __device__ constexpr size_t sw_desc_bytes(int n) {
 __host__ __device__ constexpr size_t sw_x_bytes(int xmax) {
     return a256(static_cast<size_t>(xmax) * 2);
 }
-__host__ __device__ constexpr size_t sw_smem(int n, int xmax, int depth) {
-    return sw_desc_bytes(n) + 2 * sw_x_bytes(xmax) + static_cast<size_t>(kSwW) * depth * kSwSlot;
+__host__ __device__ constexpr size_t sw_smem(int n, int xmax, int slots) {
+    return sw_desc_bytes(n) + 2 * sw_x_bytes(xmax) + static_cast<size_t>(slots) * kSlotBytes;
 }
 
 // Expect `bytes` more on the current phase without arriving (the phase then
@@ -168,16 +179,6 @@ __device__ __forceinline__ bool poll_counter(const unsigned int* c, unsigned int
     return true;
 }
 
-__device__ __forceinline__ void cp16(uint32_t dst, const void* src, uint64_t pol) {
-    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst),
-                 "l"(src), "l"(pol)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 __device__ __forceinline__ void bulk_g2s_u32(uint32_t dst, const void* src, uint32_t bytes,
                                              uint64_t* bar, uint64_t policy) {
     asm volatile(
@@ -185,16 +186,6 @@ __device__ __forceinline__ void bulk_g2s_u32(uint32_t dst, const void* src, uint
         " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
         "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
-}
-// Ask L2 to fetch [p, p + bytes) (16-byte aligned, a multiple of 16): a hint
-// with no completion to track.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ uint2 lds64(uint32_t a) {
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
-    return v;
 }
 __device__ __forceinline__ uint4 lds128s(uint32_t a) {
     uint4 v;
@@ -222,17 +213,6 @@ __device__ __forceinline__ void fma_mixed(float& a0, float& a1, uint32_t q2, uin
         : "+f"(a0), "+f"(a1)
         : "r"(q2), "r"(x2));
 }
-// 8 int8 codes against their 8 fp16 x: sum q x with exact products.
-__device__ __forceinline__ float dot8(uint2 c, uint4 x) {
-    float a0 = 0.f, a1 = 0.f;
-    const uint32_t u0 = c.x ^ 0x80808080u, u1 = c.y ^ 0x80808080u;
-    fma_mixed(a0, a1, hsub2s(__byte_perm(u0, 0x64646464u, 0x4140), 0x64806480u), x.x);
-    fma_mixed(a0, a1, hsub2s(__byte_perm(u0, 0x64646464u, 0x4342), 0x64806480u), x.y);
-    fma_mixed(a0, a1, hsub2s(__byte_perm(u1, 0x64646464u, 0x4140), 0x64806480u), x.z);
-    fma_mixed(a0, a1, hsub2s(__byte_perm(u1, 0x64646464u, 0x4342), 0x64806480u), x.w);
-    return a0 + a1;
-}
-
 __device__ __forceinline__ unsigned long long key_of(float v, int idx) {
     uint32_t b = __float_as_uint(v);
     b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);  // order-preserving
@@ -240,51 +220,59 @@ __device__ __forceinline__ unsigned long long key_of(float v, int idx) {
            static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(idx));
 }
 
-// A warp's walk over the plan: stage s, its m-th item there (global item
-// index `item`), and the step within the item's rows.
-struct Cursor {
-    int s, m, step;
-    int64_t item;
-};
-
-// Item m of stage `st` for warp w of CTA cta (-1 if the warp has none).
-__device__ __forceinline__ int64_t item_of(const StreamStage& st, int cta, int w, int G, int m) {
-    const int wr = (w - st.rot + kSwW) % kSwW;  // rot < kSwW
-    const int64_t j = static_cast<int64_t>(cta) +
-                      static_cast<int64_t>(G) * (wr + static_cast<int64_t>(kSwW) * m);
-    return j < st.items ? j : -1;
+// 16 int8 codes (k order, byte 0 first) against their 16 fp16 x (xa: the
+// first 8, xb: the last 8): sum q x with exact products.
+__device__ __forceinline__ float dot16(uint4 c, uint4 xa, uint4 xb) {
+    float a0 = 0.f, a1 = 0.f;
+    const uint32_t u0 = c.x ^ 0x80808080u, u1 = c.y ^ 0x80808080u;
+    const uint32_t u2 = c.z ^ 0x80808080u, u3 = c.w ^ 0x80808080u;
+    fma_mixed(a0, a1, hsub2s(__byte_perm(u0, 0x64646464u, 0x4140), 0x64806480u), xa.x);
+    fma_mixed(a0, a1, hsub2s(__byte_perm(u0, 0x64646464u, 0x4342), 0x64806480u), xa.y);
+    fma_mixed(a0, a1, hsub2s(__byte_perm(u1, 0x64646464u, 0x4140), 0x64806480u), xa.z);
+    fma_mixed(a0, a1, hsub2s(__byte_perm(u1, 0x64646464u, 0x4342), 0x64806480u), xa.w);
+    fma_mixed(a0, a1, hsub2s(__byte_perm(u2, 0x64646464u, 0x4140), 0x64806480u), xb.x);
+    fma_mixed(a0, a1, hsub2s(__byte_perm(u2, 0x64646464u, 0x4342), 0x64806480u), xb.y);
+    fma_mixed(a0, a1, hsub2s(__byte_perm(u3, 0x64646464u, 0x4140), 0x64806480u), xb.z);
+    fma_mixed(a0, a1, hsub2s(__byte_perm(u3, 0x64646464u, 0x4342), 0x64806480u), xb.w);
+    return a0 + a1;
 }
 
-// Position c at the first existing item at or after (c.s, c.m); c.s == n
-// when the plan is exhausted.
-__device__ __forceinline__ void seek(Cursor& c, const StreamStage* st, int n, int cta, int w,
-                                     int G) {
-    c.step = 0;
-    while (c.s < n) {
-        c.item = item_of(st[c.s], cta, w, G, c.m);
-        if (c.item >= 0) return;
-        ++c.s;
-        c.m = 0;
+// One whole row (NR = 1) or a gate/up pair (NR = 2) of a chunk: codes at
+// ca / cb in shared memory (k bytes each), scales at sa / sb (k / 16 bytes);
+// returns this lane's partial sums (the warp reduces them).
+template <int NR>
+__device__ __forceinline__ void row_dot(uint32_t ca, uint32_t cb, uint32_t sa, uint32_t sb,
+                                        uint32_t xs, int nst, int lane, float& acc0,
+                                        float& acc1) {
+    const uint32_t cl = lane * 16, sl = (lane >> 1) * 2, xl = xs + lane * 32;
+#pragma unroll 2
+    for (int st = 0; st < nst; ++st) {
+        const uint4 xa = lds128s(xl + st * (kSwStep * 2));
+        const uint4 xb = lds128s(xl + st * (kSwStep * 2) + 16);
+        const uint4 c0 = lds128s(ca + cl + st * kSwStep);
+        const float s0 = h2f(lds16s(sa + sl + st * 32));
+        acc0 = fmaf(s0, dot16(c0, xa, xb), acc0);
+        if (NR == 2) {
+            const uint4 c1 = lds128s(cb + cl + st * kSwStep);
+            const float s1 = h2f(lds16s(sb + sl + st * 32));
+            acc1 = fmaf(s1, dot16(c1, xa, xb), acc1);
+        }
     }
 }
 
-// Row r (0 or 1) of item j of stage st, clamped into the matrix (a second
-// row past the end is copied and discarded), and the matrix it lies in.
-__device__ __forceinline__ int64_t item_row(const StreamStage& st, int64_t j, int r, int* mat) {
-    if (st.op == kOpSwiglu) {
-        *mat = r;
-        return j;
-    }
-    *mat = 0;
-    const int64_t row = j * st.rows + r;
-    return row < st.n ? row : st.n - 1;
+// This CTA's rows [r0, r0 + R) of stage S.
+__device__ __forceinline__ void rows_of(const StreamStage& S, int cta, int G, int64_t& r0, int& R) {
+    r0 = static_cast<int64_t>(cta) * S.n / G;
+    R = static_cast<int>(static_cast<int64_t>(cta + 1) * S.n / G - r0);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kSwThreads, 1) stream_sweep_kernel(unsigned char* ws, int n) {
+__global__ void __launch_bounds__(kSwThreads, 1) stream_sweep_kernel(unsigned char* ws, int n,
+                                                                     int NS) {
     extern __shared__ __align__(1024) unsigned char smem[];
     __shared__ __align__(8) uint64_t xfull[2];  // x of stage s landed (tx bytes)
-    __shared__ __align__(8) uint64_t sdone[2];  // every streaming warp done with stage s
+    __shared__ __align__(8) uint64_t sdone[2];  // every compute warp done with stage s
+    __shared__ __align__(8) uint64_t full[kMaxSlots];   // a slot's copies landed (tx bytes)
+    __shared__ __align__(8) uint64_t empty[kMaxSlots];  // every compute warp done with a slot
     __shared__ float best_v[2][kSwW];
     __shared__ int best_i[2][kSwW];
     __shared__ volatile int abort_sh;
@@ -292,8 +280,9 @@ __global__ void __launch_bounds__(kSwThreads, 1) stream_sweep_kernel(unsigned ch
     const StreamHeader* hdr = reinterpret_cast<const StreamHeader*>(ws);
     uint32_t dyn_smem;
     asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_smem));
-    if (hdr->magic != kStreamMagic || hdr->n_stages != n || hdr->depth != D ||
-        hdr->xmax < kSwStep || sw_smem(n, hdr->xmax, D) > dyn_smem) {
+    if (hdr->magic != kStreamMagic || hdr->n_stages != n || hdr->slots != NS ||
+        NS < kMinSlots || NS > kMaxSlots || hdr->xmax < kSwStep ||
+        sw_smem(n, hdr->xmax, NS) > dyn_smem) {
         if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(&g_stream_err, kGemvErrBadPlan);
         return;
     }
@@ -320,11 +309,15 @@ __global__ void __launch_bounds__(kSwThreads, 1) stream_sweep_kernel(unsigned ch
         mbar_init(&xfull[1], 1);
         mbar_init(&sdone[0], kSwW);
         mbar_init(&sdone[1], kSwW);
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kSwW);
+        }
         fence_mbar_init();
     }
     __syncthreads();
 
-    if (warp == kSwW) {
+    if (warp == kSyncWarp) {
         // ------------------------------------------------------ sync warp ---
         const uint64_t pol_x = l2_policy_evict_last();
         // x of stage s into its half of the buffer.  A run input may be copied
@@ -426,190 +419,150 @@ __global__ void __launch_bounds__(kSwThreads, 1) stream_sweep_kernel(unsigned ch
                 mbar_wait_bounded(&xfull[s & 1], (s >> 1) & 1);
         }
         __syncwarp();
+    } else if (warp == kProdWarp) {
+        // --------------------------------------------------- producer warp ---
+        // Chunk C of the CTA's ring order goes to slot C % NS, after the
+        // compute warps have released the chunk that slot held (C - NS).
+        if (lane == 0) {
+            const uint64_t pol = l2_policy_evict_first();
+            int slot = 0;
+            uint32_t round = 0;
+            bool ok = true;
+            for (int s = 0; s < n && ok; ++s) {
+                const StreamStage& S = st[s];
+                int64_t r0;
+                int R;
+                rows_of(S, cta, G, r0, R);
+                const int64_t kb = S.k;  // code bytes per row
+                for (int u0 = 0; u0 < R && ok; u0 += S.nrc) {
+                    if (round > 0) {
+                        ok = !abort_sh && mbar_wait_bounded(&empty[slot], (round - 1) & 1);
+                        if (!ok) break;
+                    }
+                    const int rows = min(S.nrc, R - u0);
+                    const int64_t row = r0 + u0;
+                    const uint32_t cbytes = static_cast<uint32_t>(rows * kb);
+                    const uint32_t sbytes = static_cast<uint32_t>(rows * kb / 16);
+                    const uint32_t sb = ring0 + static_cast<uint32_t>(slot) * kSlotBytes;
+                    mbar_arrive_expect_tx(&full[slot], S.nmat * (cbytes + sbytes));
+                    for (int m = 0; m < S.nmat; ++m) {
+                        bulk_g2s_u32(sb + static_cast<uint32_t>(m * S.nrc * kb),
+                                     S.codes[m] + row * kb, cbytes, &full[slot], pol);
+                        bulk_g2s_u32(sb + kChunkCodes + static_cast<uint32_t>(m * S.nrc * kb / 16),
+                                     S.scales[m] + row * (kb / 32), sbytes, &full[slot], pol);
+                    }
+                    if (++slot == NS) {
+                        slot = 0;
+                        ++round;
+                    }
+                }
+            }
+            if (!ok) {
+                if (!abort_sh) atomicOr(&g_stream_err, kGemvErrTimeout);
+                abort_sh = 1;
+            }
+            // the copies issued land before the CTA may exit (bounded)
+            for (int i = 0; i < NS; ++i) {
+                const uint32_t filled = round * NS + slot;  // chunks issued so far
+                const uint32_t c = filled >= static_cast<uint32_t>(NS) ? filled - NS + i : i;
+                if (c < filled) mbar_wait_bounded(&full[c % NS], (c / NS) & 1);
+            }
+        }
+        __syncwarp();
     } else {
-        // ---------------------------------------------------- streaming warp --
-        const uint64_t pol = l2_policy_evict_first();
-        const uint32_t ring = ring0 + static_cast<uint32_t>(warp) * D * kSwSlot;
-        // copy cursor: the item it copies, with this lane's source pointers of
-        // that item's rows (advanced by one step per copy)
-        Cursor cc = {0, 0, 0, -1};
-        seek(cc, st, n, cta, warp, G);
-        int cslot = 0;
-        const uint8_t* cp0 = nullptr;   // row 0 codes, this lane's 16 bytes
-        const uint8_t* cp1 = nullptr;   // row 1 codes
-        const uint16_t* cps = nullptr;  // side lanes 0-3: scales of row lane >> 1, piece lane & 1
-        int cleft = 0;                  // steps of the item left to copy
-        bool ctwo = false;              // the item has two rows
-        auto load_item = [&]() {
-            const StreamStage& S = st[cc.s];
-            int m0, m1;
-            const int64_t r0 = item_row(S, cc.item, 0, &m0);
-            const int64_t r1 = item_row(S, cc.item, 1, &m1);
-            ctwo = S.rows == 2 || S.op == kOpSwiglu;
-            cp0 = S.codes[m0] + r0 * S.k + lane * 16;
-            cp1 = S.codes[m1] + r1 * S.k + lane * 16;
-            if (lane == 0) {
-                // ask L2 for the whole item now: its later steps' copies then
-                // hit L2 instead of waiting out HBM latency one step at a time
-                const uint8_t* c0 = S.codes[m0] + r0 * S.k;
-                const uint8_t* c1 = S.codes[m1] + r1 * S.k;
-                const uint32_t sb = static_cast<uint32_t>(S.k / 16);  // scale bytes per row
-                if (ctwo && m0 == m1 && r1 == r0 + 1) {
-                    prefetch_l2_bulk(c0, static_cast<uint32_t>(2 * S.k));
-                    prefetch_l2_bulk(S.scales[m0] + r0 * (S.k / 32), 2 * sb);
-                } else {
-                    prefetch_l2_bulk(c0, static_cast<uint32_t>(S.k));
-                    prefetch_l2_bulk(S.scales[m0] + r0 * (S.k / 32), sb);
-                    if (ctwo) {
-                        prefetch_l2_bulk(c1, static_cast<uint32_t>(S.k));
-                        prefetch_l2_bulk(S.scales[m1] + r1 * (S.k / 32), sb);
-                    }
-                }
-            }
-            const bool srow1 = (lane >> 1) & 1;
-            cps = S.scales[srow1 ? m1 : m0] + (srow1 ? r1 : r0) * (S.k / 32) + (lane & 1) * 8;
-            cleft = S.nst;
-        };
-        if (cc.s < n) load_item();
-        const bool side_lane = lane < 4;
-        const uint32_t side_off = static_cast<uint32_t>((lane >> 1) * kSwSlotRow + kSwStep + (lane & 1) * 16);
-        auto issue = [&]() {
-            if (cleft > 0) {
-                const uint32_t dst = ring + cslot * kSwSlot + lane * 16;
-                cp16(dst, cp0, pol);
-                if (ctwo) cp16(dst + kSwSlotRow, cp1, pol);
-                if (side_lane && (lane < 2 || ctwo))
-                    cp16(ring + cslot * kSwSlot + side_off, cps, pol);
-                cp0 += kSwStep;
-                cp1 += kSwStep;
-                cps += 16;
-                if (--cleft == 0) {
-                    ++cc.m;
-                    seek(cc, st, n, cta, warp, G);
-                    if (cc.s < n) load_item();
-                }
-            }
-            cp_commit();
-            if (++cslot == D) cslot = 0;
-        };
-#pragma unroll 1
-        for (int d = 0; d < D - 1; ++d) issue();
-
-        // compute cursor
-        Cursor uc = {0, 0, 0, -1};
-        int uslot = 0;
-        int cur = -1;  // the stage whose x this warp has waited for
-        float bv = -FLT_MAX;
-        int bi = INT_MAX;
+        // ----------------------------------------------------- compute warp --
+        int slot = 0;
+        uint32_t ph = 0;  // parity of the current pass over the ring
         bool aborted = false;
-        // stages before (and including) `upto` that this warp has no more
-        // items in: arrive on their completion barriers, in order
-        int arrived = 0;  // stages 0 .. arrived-1 arrived
-        auto arrive_until = [&](int upto) -> bool {
-            for (; arrived < upto; ++arrived) {
-                const int s = arrived;
-                // Arrive for stage s only once x of stage s - 1 has landed: the
-                // sync warp copies it after it has seen stage s - 2 complete,
-                // so the barrier of parity s & 1 is then in stage s's phase
-                // (a warp without items must not run two phases ahead).
-                if (s >= 1 && !mbar_wait_bounded(&xfull[(s - 1) & 1], ((s - 1) >> 1) & 1))
-                    return false;
-                if (st[s].op == kOpHead) {
-                    // best of this warp in stage s (its head rows), then arrive
-                    if (lane == 0) {
-                        best_v[s & 1][warp] = s == cur ? bv : -FLT_MAX;
-                        best_i[s & 1][warp] = s == cur ? bi : INT_MAX;
+        for (int s = 0; s < n && !aborted; ++s) {
+            const StreamStage& S = st[s];
+            const StreamOut& o = outs[s];
+            int64_t r0;
+            int R;
+            rows_of(S, cta, G, r0, R);
+            const int64_t kb = S.k;
+            const uint32_t xs = xbuf0 + (s & 1) * xstride;
+            bool have_x = false;
+            float bv = -FLT_MAX;  // head: this warp's best row of the stage
+            int bidx = INT_MAX;
+            for (int u0 = 0; u0 < R && !aborted; u0 += S.nrc) {
+                const bool okf = mbar_wait_bounded(&full[slot], ph);
+                if (!__all_sync(0xffffffffu, okf)) {
+                    aborted = true;
+                    break;
+                }
+                const int rows = min(S.nrc, R - u0);
+                const uint32_t sb = ring0 + static_cast<uint32_t>(slot) * kSlotBytes;
+                // this warp's rows of the chunk: u = u0 + i with u % kSwW == warp
+                int i = (warp - u0 % kSwW + kSwW) % kSwW;
+                for (; i < rows; i += kSwW) {
+                    if (!have_x) {
+                        const bool okx = !abort_sh && mbar_wait_bounded(&xfull[s & 1], (s >> 1) & 1);
+                        if (!__all_sync(0xffffffffu, okx)) {
+                            aborted = true;
+                            break;
+                        }
+                        have_x = true;
                     }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sdone[s & 1]);
-            }
-            return true;
-        };
-        seek(uc, st, n, cta, warp, G);
-        while (uc.s < n) {
-            const StreamStage& S = st[uc.s];
-            if (uc.s != cur) {
-                // finish the stages before this one, then wait for its x
-                if (!arrive_until(uc.s)) {
-                    aborted = true;
-                    break;
-                }
-                cur = uc.s;
-                bv = -FLT_MAX;
-                bi = INT_MAX;
-                if (abort_sh || !mbar_wait_bounded(&xfull[cur & 1], (cur >> 1) & 1)) {
-                    aborted = true;
-                    break;
-                }
-            }
-            uint32_t xp = xbuf0 + (cur & 1) * xstride + lane * 16;  // this lane's x pieces
-            const bool two = S.op == kOpSwiglu || S.rows == 2;
-            const int nst = S.nst;
-            float acc0 = 0.f, acc1 = 0.f;
-            for (int step = 0; step < nst; ++step) {
-                issue();
-                cp_wait<D - 1>();
-                __syncwarp();  // every lane's copies of this slot are visible
-                const uint32_t slot = ring + uslot * kSwSlot;
-                const uint4 xa = lds128s(xp);
-                const uint4 xb = lds128s(xp + kSwStep);
-                xp += kSwStep * 2;
-                {
-                    const uint2 ca = lds64(slot + lane * 8);
-                    const uint2 cb = lds64(slot + 256 + lane * 8);
-                    const float sa = h2f(lds16s(slot + kSwStep + (lane >> 2) * 2));
-                    const float sb = h2f(lds16s(slot + kSwStep + 16 + (lane >> 2) * 2));
-                    acc0 = fmaf(sa, dot8(ca, xa), fmaf(sb, dot8(cb, xb), acc0));
-                }
-                if (two) {
-                    const uint32_t s1 = slot + kSwSlotRow;
-                    const uint2 ca = lds64(s1 + lane * 8);
-                    const uint2 cb = lds64(s1 + 256 + lane * 8);
-                    const float sa = h2f(lds16s(s1 + kSwStep + (lane >> 2) * 2));
-                    const float sb = h2f(lds16s(s1 + kSwStep + 16 + (lane >> 2) * 2));
-                    acc1 = fmaf(sa, dot8(ca, xa), fmaf(sb, dot8(cb, xb), acc1));
-                }
-                __syncwarp();  // every lane is done with the slot before it is refilled
-                if (++uslot == D) uslot = 0;
-            }
-            acc0 = warp_sum(acc0);
-            acc1 = warp_sum(acc1);
-            if (lane == 0) {
-                const StreamOut& o = outs[uc.s];
-                if (S.op == kOpSwiglu) {
-                    o.h[uc.item] = f2h_rn(acc0 / (1.0f + expf(-acc0)) * acc1);
-                } else {
-#pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        const int64_t row = uc.item * S.rows + r;
-                        if (r < S.rows && row < S.n) {
-                            const float v = r == 0 ? acc0 : acc1;
-                            if (S.op == kOpGemv) {
-                                if (o.y) o.y[row] = v;
-                                if (o.y16) o.y16[row] = f2h_rn(v);
-                            } else {
-                                if (o.logits) o.logits[row] = v;
-                                if (v > bv) {  // rows arrive in increasing order
-                                    bv = v;
-                                    bi = static_cast<int>(row);
-                                }
+                    float acc0 = 0.f, acc1 = 0.f;
+                    const uint32_t ca = sb + static_cast<uint32_t>(i * kb);
+                    const uint32_t sa = sb + kChunkCodes + static_cast<uint32_t>(i * kb / 16);
+                    if (S.op == kOpSwiglu)
+                        row_dot<2>(ca, ca + static_cast<uint32_t>(S.nrc * kb), sa,
+                                   sa + static_cast<uint32_t>(S.nrc * kb / 16), xs, S.nst, lane,
+                                   acc0, acc1);
+                    else
+                        row_dot<1>(ca, ca, sa, sa, xs, S.nst, lane, acc0, acc1);
+                    acc0 = warp_sum(acc0);
+                    if (S.op == kOpSwiglu) acc1 = warp_sum(acc1);
+                    if (lane == 0) {
+                        const int64_t row = r0 + u0 + i;
+                        if (S.op == kOpSwiglu) {
+                            o.h[row] = f2h_rn(acc0 / (1.0f + expf(-acc0)) * acc1);
+                        } else if (S.op == kOpGemv) {
+                            if (o.y) o.y[row] = acc0;
+                            if (o.y16) o.y16[row] = f2h_rn(acc0);
+                        } else {
+                            if (o.logits) o.logits[row] = acc0;
+                            if (acc0 > bv) {  // rows arrive in increasing order
+                                bv = acc0;
+                                bidx = static_cast<int>(row);
                             }
                         }
                     }
                 }
+                if (aborted) break;
+                __syncwarp();  // every lane is done with the slot before it is released
+                if (lane == 0) mbar_arrive(&empty[slot]);
+                if (++slot == NS) {
+                    slot = 0;
+                    ph ^= 1u;
+                }
             }
-            ++uc.m;
-            seek(uc, st, n, cta, warp, G);
-        }
-        if (!aborted && !arrive_until(n)) aborted = true;
-        if (aborted) {
-            if (lane == 0) {
-                if (!abort_sh) atomicOr(&g_stream_err, kGemvErrTimeout);
-                abort_sh = 1;
+            if (aborted) break;
+            // Done with stage s: arrive on its completion barrier.  Only once x
+            // of stage s - 1 has landed: the sync warp copies it after it has
+            // seen stage s - 2 complete, so the barrier of parity s & 1 is then
+            // in stage s's phase (a warp without rows must not run two phases
+            // ahead).
+            if (s >= 1) {
+                const bool okp = mbar_wait_bounded(&xfull[(s - 1) & 1], ((s - 1) >> 1) & 1);
+                if (!__all_sync(0xffffffffu, okp)) {
+                    aborted = true;
+                    break;
+                }
             }
+            if (S.op == kOpHead && lane == 0) {
+                best_v[s & 1][warp] = bv;
+                best_i[s & 1][warp] = bidx;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sdone[s & 1]);
         }
-        cp_wait<0>();  // this lane's copies land before the CTA may exit
+        if (aborted && lane == 0) {
+            if (!abort_sh) atomicOr(&g_stream_err, kGemvErrTimeout);
+            abort_sh = 1;
+        }
         __syncwarp();
     }
 
@@ -632,11 +585,12 @@ __global__ void __launch_bounds__(kSwThreads, 1) stream_sweep_kernel(unsigned ch
 
 size_t stream_workspace_bytes(int n_stages) { return sw_bytes(n_stages); }
 
-// Plan: every stage int8 block-32 with k % 512 == 0, at most kSwMaxStages
-// stages, shared memory for the descriptors, x and the rings at depth 11 or
-// at least 8.  Returns QG_ERR_FORMAT / QG_ERR_SHAPE when the plan does not
-// qualify (the caller then plans the general persistent kernel).
-qg_status plan_stream(const GemvLaunch* L, int n, void* ws, size_t ws_bytes, int* depth_out,
+// Plan: every stage int8 block-32 with k % 512 == 0 and one row (or gate/up
+// pair) within a ring slot, at most kSwMaxStages stages, shared memory for the
+// descriptors, x and at least kMinSlots ring slots.  Returns QG_ERR_FORMAT /
+// QG_ERR_SHAPE when the plan does not qualify (the caller then plans the
+// general persistent kernel).
+qg_status plan_stream(const GemvLaunch* L, int n, void* ws, size_t ws_bytes, int* slots_out,
                       int* xmax_out) {
     DeviceInfo dev;
     qg_status st = device_info(&dev);
@@ -646,22 +600,22 @@ qg_status plan_stream(const GemvLaunch* L, int n, void* ws, size_t ws_bytes, int
     int xmax = 0;
     for (int i = 0; i < n; ++i) {
         if (L[i].fmt != QG_FMT_I8_B32) return QG_ERR_FORMAT;
-        if (L[i].k % kSwStep != 0 || L[i].n > (1LL << 30)) return QG_ERR_SHAPE;
+        const int64_t nmat = L[i].epilogue == kEpiSwiglu ? 2 : 1;
+        if (L[i].k % kSwStep != 0 || L[i].n > (1LL << 30) || nmat * L[i].k > kChunkCodes)
+            return QG_ERR_SHAPE;
+        if (reinterpret_cast<uintptr_t>(L[i].x) % 16 != 0) return QG_ERR_SHAPE;
         if (L[i].k > xmax) xmax = static_cast<int>(L[i].k);
     }
-    int depth = 0;
-    for (int d : {11, 8})
-        if (sw_smem(n, xmax, d) + 1024 <= static_cast<size_t>(dev.max_smem_optin)) {
-            depth = d;
-            break;
-        }
-    if (depth == 0) return QG_ERR_SHAPE;
-    const int G = dev.num_sms;
+    const size_t fixed = sw_smem(n, xmax, 0) + 1024;
+    if (fixed >= static_cast<size_t>(dev.max_smem_optin)) return QG_ERR_SHAPE;
+    int slots = static_cast<int>((static_cast<size_t>(dev.max_smem_optin) - fixed) / kSlotBytes);
+    if (slots > kMaxSlots) slots = kMaxSlots;
+    if (slots < kMinSlots) return QG_ERR_SHAPE;
     std::vector<unsigned char> host(sw_bytes(n), 0);
     StreamHeader* hdr = reinterpret_cast<StreamHeader*>(host.data());
     hdr->magic = kStreamMagic;
     hdr->n_stages = n;
-    hdr->depth = depth;
+    hdr->slots = slots;
     hdr->xmax = xmax;
     StreamStage* S = reinterpret_cast<StreamStage*>(host.data() + sw_stage_off(n));
     StreamOut* O = reinterpret_cast<StreamOut*>(host.data() + sw_out_off(n));
@@ -690,22 +644,13 @@ qg_status plan_stream(const GemvLaunch* L, int n, void* ws, size_t ws_bytes, int
         s.n = static_cast<int32_t>(l.n);
         s.k = static_cast<int32_t>(l.k);
         s.nst = static_cast<int32_t>(l.k / kSwStep);
-        s.rot = static_cast<int32_t>((i * 7) % kSwW);
         const uintptr_t x0 = reinterpret_cast<uintptr_t>(l.x), x1 = x0 + static_cast<uintptr_t>(l.k) * 2;
         s.xext = 1;
         for (const auto& w : written)
             if (x0 < w.second && w.first < x1) s.xext = 0;
-        if (l.epilogue == kEpiSwiglu) {
-            s.op = kOpSwiglu;
-            s.rows = 2;
-            s.items = static_cast<int32_t>(l.n);
-        } else {
-            s.op = l.epilogue == kEpiHead ? kOpHead : kOpGemv;
-            // two rows per item: every ring slot carries two rows' steps (a
-            // warp without an item in a small stage streams ahead instead)
-            s.rows = l.n >= 2 ? 2 : 1;
-            s.items = static_cast<int32_t>((l.n + s.rows - 1) / s.rows);
-        }
+        s.op = l.epilogue == kEpiSwiglu ? kOpSwiglu : (l.epilogue == kEpiHead ? kOpHead : kOpGemv);
+        s.nmat = l.epilogue == kEpiSwiglu ? 2 : 1;
+        s.nrc = static_cast<int32_t>(kChunkCodes / (static_cast<int64_t>(s.nmat) * l.k));
         StreamOut& o = O[i];
         o.x = l.x;
         o.y = l.y;
@@ -719,34 +664,27 @@ qg_status plan_stream(const GemvLaunch* L, int n, void* ws, size_t ws_bytes, int
     }
     st = cuda_status(cudaMemcpy(ws, host.data(), host.size(), cudaMemcpyHostToDevice));
     if (st == QG_OK) {
-        *depth_out = depth;
+        *slots_out = slots;
         *xmax_out = xmax;
     }
     return st;
 }
 
-qg_status launch_stream(void* ws, int n, int depth, int xmax, cudaStream_t stream) {
+qg_status launch_stream(void* ws, int n, int slots, int xmax, cudaStream_t stream) {
     DeviceInfo dev;
     qg_status st = device_info(&dev);
     if (st != QG_OK) return st;
-    if (n < 1 || n > kSwMaxStages || xmax < kSwStep) return QG_ERR_PLAN;
-    void (*kern)(unsigned char*, int);
-    if (depth == 11) {
-        kern = stream_sweep_kernel<11>;
-    } else if (depth == 8) {
-        kern = stream_sweep_kernel<8>;
-    } else {
+    if (n < 1 || n > kSwMaxStages || xmax < kSwStep || slots < kMinSlots || slots > kMaxSlots)
         return QG_ERR_PLAN;
-    }
-    const size_t smem = sw_smem(n, xmax, depth);
+    void (*kern)(unsigned char*, int, int) = stream_sweep_kernel;
+    const size_t smem = sw_smem(n, xmax, slots);
     if (smem + 1024 > static_cast<size_t>(dev.max_smem_optin)) return QG_ERR_PLAN;
-    static size_t attr[2][64] = {{0}};
-    const int ki = depth == 11 ? 0 : 1;
-    if (dev.device >= 64 || attr[ki][dev.device] < smem) {
+    static size_t attr[64] = {0};
+    if (dev.device >= 64 || attr[dev.device] < smem) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return cuda_status(e);
-        if (dev.device < 64) attr[ki][dev.device] = smem;
+        if (dev.device < 64) attr[dev.device] = smem;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(dev.num_sms));
@@ -758,7 +696,7 @@ qg_status launch_stream(void* ws, int n, int depth, int xmax, cudaStream_t strea
     at[0].val.cooperative = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cuda_status(cudaLaunchKernelEx(&cfg, kern, static_cast<unsigned char*>(ws), n));
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, static_cast<unsigned char*>(ws), n, slots));
 }
 
 unsigned int stream_read_and_clear_error() {
