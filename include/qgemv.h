@@ -319,8 +319,14 @@ QG_API qg_status qg_decode_attention(const float* qkv, int hq, int hkv, int d,
  * (qkv -> o -> gate/up + SwiGLU -> down) and the LM head with the greedy
  * argmax ("Qwen3.8-27B ... -- Core AI", The vision path: prefill runs as
  * pipelined S=1 steps).  A sweep is that chain: an ordered list of stages,
- * each one of the S=1 calls above with the same arguments, results and
- * accuracy (the results are bit-identical to those calls).
+ * each one of the S=1 calls above with the same arguments and accuracy.  An
+ * all-int8 plan whose rows hold whole 512-code steps and fit a 32 KB ring
+ * slot (k <= 32768 per weight, a SwiGLU stage's two weights together)
+ * runs on the stream kernel: one CTA per SM, results within the same bound
+ * as the calls and identical from run to run, each row summed in its own
+ * fixed order (not the calls' order).  Other plans run on the general
+ * persistent kernels (two CTAs per SM), whose results are bit-identical to
+ * the calls.
  *
  * Order: stage i + 1 reads its x only after every part of stage i is done,
  * exactly as if the calls were enqueued one after another on one stream, so
@@ -361,8 +367,9 @@ QG_API qg_status qg_decode_attention(const float* qkv, int hq, int hkv, int d,
  *   never while a run that uses the same workspace may still execute.
  *   1 <= n_stages <= 65536.
  * qg_sweep_run -- enqueues one run of the plan on `stream` (asynchronous;
- *   safe to capture in a CUDA graph).  It is a cooperative launch of two
- *   CTAs per SM that must all be resident at once: it fails with
+ *   safe to capture in a CUDA graph).  It is a cooperative launch (one or
+ *   two CTAs per SM, as above) whose CTAs must all be resident at once: it
+ *   fails with
  *   QG_ERR_CUDA if the device cannot host them, and runs must not overlap
  *   other runs of the same workspace.  Between stages the CTAs wait on
  *   counters in the workspace; a wait that has not finished after ~2 s gives
