@@ -2,9 +2,12 @@
 
     python -m int4_quantized_decode_b200.profile_case --op swiglu --n 6144 --k 2048
     python -m int4_quantized_decode_b200.profile_case --op attention --n 16 --k 16384
+    python -m int4_quantized_decode_b200.profile_case --op sweep --decoder qwen3vl-2b
 
 For --op attention, n is the number of query heads (8 kv heads, head_dim 128)
-and k the K/V cache rows; the token sits at the last row.
+and k the K/V cache rows; the token sits at the last row.  --op sweep runs
+the int8 S=1 weight sweep of a decoder as one persistent launch per sweep
+(qg_sweep_run), `--launches` times (n and k unused).
 
 Builds one seeded weight (two for swiglu), quantizes it, and launches the op
 `--launches` times on the current device, then synchronizes.  It prints
@@ -20,19 +23,33 @@ import torch
 from . import qgemv as qg
 from . import workloads as wl
 
-OPS = ("gemv", "swiglu", "head", "s16", "s16swiglu", "quantize", "attention")
+OPS = ("gemv", "swiglu", "head", "s16", "s16swiglu", "quantize", "attention", "sweep")
+DECODERS = {"qwen3vl-2b": wl.QWEN3VL_2B, "qwen3vl-4b": wl.QWEN3VL_4B, "qwen3vl-8b": wl.QWEN3VL_8B}
 
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--op", choices=OPS, required=True)
-    ap.add_argument("--n", type=int, required=True)
-    ap.add_argument("--k", type=int, required=True)
+    ap.add_argument("--n", type=int, default=0)
+    ap.add_argument("--k", type=int, default=0)
+    ap.add_argument("--decoder", choices=sorted(DECODERS), default="qwen3vl-2b")
     ap.add_argument("--fmt", type=int, default=qg.FMT_I8_B32, choices=(0, 1))
     ap.add_argument("--S", type=int, default=16)
     ap.add_argument("--launches", type=int, default=3)
     a = ap.parse_args(argv)
     dev = torch.device("cuda:0")
+    if a.op == "sweep":
+        from .sweep import DecodeSweep
+        sw = DecodeSweep(DECODERS[a.decoder], qg.FMT_I8_B32, qg.FMT_I8_B32, S=1, device=dev)
+        sw.make_plan()
+        torch.cuda.synchronize()
+        for _ in range(a.launches):
+            sw.step(persistent=True)
+        qg.qg_stream_check()
+        print(f"sweep {a.decoder} persistent x{a.launches}")
+        return 0
+    if a.n < 1 or a.k < 1:
+        ap.error("--n and --k are required for this op")
     if a.op == "attention":
         hkv, hd = 8, 128
         kc = wl.act_fp16((hkv, a.k, hd), 11, dev)
