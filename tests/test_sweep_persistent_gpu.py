@@ -318,3 +318,49 @@ def test_decode_sweep_persistent(cuda, dec, body):
         del sw
         gc.collect()
         torch.cuda.empty_cache()
+
+
+def test_stream_sweep_short_plans(cuda):
+    """Plans with fewer rows than CTAs (most CTAs own no rows of a stage, and
+    every CTA still takes part in each stage boundary), a one-stage plan, and
+    rows that exactly fill the stream kernel's 32 KB chunks (a SwiGLU stage of
+    k = 16384: one gate row and one up row per chunk) run on the stream kernel
+    and stay within the oracle's bound, teacher-forced on the x each read."""
+    c = Chain(cuda, I8)
+    a = c.gemv("a", 1, 512, c.x0[:512], fp16_out=True)
+    c.swiglu("b", 3, 512, c.x1[:512])
+    c.head("c", 147, 1024, c.x0)
+    big_x = wl.act_fp16(16384, 13, cuda)
+    c.swiglu("d", 300, 16384, big_x)
+    c.gemv("e", 149, 1024, c.x1)
+    outs = c._alloc()
+    plan = qg.SweepPlan(c.stages(outs), [], cuda)
+    assert plan.sweep.kernel == STREAM
+    for _ in range(2):
+        plan.run()
+        qg.qg_stream_check()
+    for kind, name, Ws, src, _ in c.ops:
+        x = c._x(src, outs)
+        if kind == "swiglu":
+            gr, mg = oracle_gemv(Ws[0], x)
+            ur, mu = oracle_gemv(Ws[1], x)
+            hr, hb = oracle.swiglu(gr, ur, mg, mu, oracle.GEMV_TOL)
+            hd = outs[name][0].cpu().numpy().astype(np.float64)
+            assert np.all(np.abs(hd - hr) <= hb), name
+        else:
+            yr, mag = oracle_gemv(Ws[0], x)
+            assert_within_bound(outs[name][0].cpu().numpy(), yr, mag)
+            if kind == "head":
+                assert oracle.argmax_ok(int(outs[name][1].item()), yr), name
+    # one stage
+    c1 = Chain(cuda, I8)
+    c1.head("h", 5003, 2048, wl.act_fp16(2048, 14, cuda))
+    o1 = c1._alloc()
+    p1 = qg.SweepPlan(c1.stages(o1), [], cuda)
+    assert p1.sweep.kernel == STREAM
+    p1.run()
+    qg.qg_stream_check()
+    Wh = c1.ops[0][2][0]
+    yr, mag = oracle_gemv(Wh, c1._x(c1.ops[0][3], o1))
+    assert_within_bound(o1["h"][0].cpu().numpy(), yr, mag)
+    assert oracle.argmax_ok(int(o1["h"][1].item()), yr)
