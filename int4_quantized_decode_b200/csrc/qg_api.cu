@@ -33,6 +33,8 @@ qg_status device_info(DeviceInfo* out) {
     d.device = dev;
     if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&d.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
             cudaSuccess)
         return cuda_status(cudaErrorInvalidDevice);
     if (dev >= 0 && dev < 64) {

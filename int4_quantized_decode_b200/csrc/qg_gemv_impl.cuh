@@ -700,7 +700,7 @@ struct GridSync {
 // Bytes in flight cost no registers: 3 steps x RG rows x 16 B per lane stay
 // outstanding.  Requires a multiple of 8 scales per row (16-byte pieces).
 // Returns false, with its copies drained, if the wait for x gave up.
-template <int FMT, int NMAT, int RG, int EPI, class SYNC>
+template <int FMT, int NMAT, int RG, int EPI, bool WHOLE = false, class SYNC>
 __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem, SYNC& sync,
                                            float* red_v, int* red_i) {
     using F = Fmt<FMT>;
@@ -797,13 +797,51 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
         }
     };
 
+    // WHOLE: rows of whole steps (every lane has a code vector in every step,
+    // every step has its 16 sides) and at least kRing - 1 steps.  The load
+    // cursor below then moves on to the next item only at step
+    // nst - (kRing - 1) of each item, so the streaming loop needs no per-step
+    // bounds or item tests.  The launcher picks it only for such rows.
+    if constexpr (WHOLE) {
+        if (granules % kLanes != 0 || nst < kRing - 1) {
+            if (threadIdx.x == 0) atomicOr(&g_gemv_err, kGemvErrBadPlan);
+            return false;
+        }
+    }
+    constexpr uint32_t kSlotBytes = ROWS * RL::kPerRow;
+    const uint32_t ring_end = ring + kRing * kSlotBytes;
+    const uint32_t side_ld =
+        side_row * RL::kPerRow + RL::kCodes + side_which * RL::kSide + side_half * 16;
+    uint32_t ld_addr = ring;  // the slot the whole-step cursor fills next
+    auto issue_whole = [&]() {
+        const uint32_t a = ld_addr + lane * 16;
+#pragma unroll
+        for (int j = 0; j < ROWS; ++j) {
+            cp_async16(a + j * RL::kPerRow, lc[j], pol);
+            lc[j] += kStepBytes;
+        }
+        if (side_lane) {
+            cp_async16(ld_addr + side_ld, lside, pol);
+            lside += kStepSides;
+        }
+        ld_addr = ld_addr + kSlotBytes == ring_end ? ring : ld_addr + kSlotBytes;
+    };
+
     // 1) weight prologue (independent of the work before this stage)
     sync.before_prologue();
     if (my_items > 0) set_item(0);
+    if constexpr (WHOLE) {
 #pragma unroll
-    for (int d = 0; d < kRing - 1; ++d) {
-        if (d < total) issue();
-        else cp_async_commit();
+        for (int d = 0; d < kRing - 1; ++d) {
+            if (my_items > 0) issue_whole();
+            cp_async_commit();
+        }
+    } else {
+#pragma unroll
+        for (int d = 0; d < kRing - 1; ++d) {
+            if (d < total) issue();
+            else cp_async_commit();
+        }
     }
     if (lane == 0) prefetch_items<FMT, NMAT, RG>(p, wg, tw, 1, p.prefetch_items - 1, my_items);
 
@@ -843,44 +881,98 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
     for (int j = 0; j < ROWS; ++j) acc[j] = 0.f;
     float best_v = -FLT_MAX;
     int best_i = INT_MAX;
-    int cu_st = 0, cu_item = 0, cu_slot = 0;
-    float h_old = 0.f;
-    for (int t = 0; t < total; ++t) {
-        if (cu_st == 0) h_old = residual_old<RG, EPI>(p, (wg + cu_item * tw) * RG, N, lane);
-        if (t + kRing - 1 < total) issue();
-        else cp_async_commit();
-        cp_async_wait<kRing - 1>();
-        __syncwarp();  // side pieces copied by other lanes are now visible
-        const int g = cu_st * kLanes + lane;
-        if (g < granules) {
-            uint4 xv[F::kPieces];
-            const uint4* xp = xs + x_lane + cu_st * kXStep;
+    // One step of every row of the item from the ring slot at `slot`: the
+    // lane's code vectors and sides, against the x pieces at xp (c1: the sum
+    // of the lane's x, int4).
+    auto compute = [&](uint32_t slot, const uint4* xp, float c1) {
+        uint4 xv[F::kPieces];
 #pragma unroll
-            for (int i = 0; i < F::kPieces; ++i) xv[i] = xp[i * 8];
-            const float c1 = FMT == 1 ? sums[g] : 0.f;
+        for (int i = 0; i < F::kPieces; ++i) xv[i] = xp[i * 8];
+        const uint32_t cl = slot + lane * 16;
+        const uint32_t cs = slot + RL::kCodes + side_off;
 #pragma unroll
-            for (int j = 0; j < ROWS; ++j) {
-                const uint4 c = lds128(slot_codes(cu_slot, j));
-                if (FMT == 2) {
-                    acc[j] += dot8_f16(c, xv);
-                    continue;
-                }
-                const float sc = h2f(lds16(slot_side(cu_slot, j, 0) + side_off));
-                if (FMT == 0) {
-                    acc[j] = fmaf(sc, dot16_i8(c, xv), acc[j]);
-                } else {
-                    const float bi = h2f(lds16(slot_side(cu_slot, j, 1) + side_off));
-                    acc[j] = i4_accumulate(acc[j], sc, bi, c, xv, c1);
-                }
+        for (int j = 0; j < ROWS; ++j) {
+            const uint4 c = lds128(cl + j * RL::kPerRow);
+            if (FMT == 2) {
+                acc[j] += dot8_f16(c, xv);
+                continue;
+            }
+            const float sc = h2f(lds16(cs + j * RL::kPerRow));
+            if (FMT == 0) {
+                acc[j] = fmaf(sc, dot16_i8(c, xv), acc[j]);
+            } else {
+                const float bi = h2f(lds16(cs + j * RL::kPerRow + RL::kSide));
+                acc[j] = i4_accumulate(acc[j], sc, bi, c, xv, c1);
             }
         }
-        __syncwarp();  // every lane is done with this slot before it is refilled
-        if (++cu_slot == kRing) cu_slot = 0;
-        if (++cu_st == nst) {
-            finish_item<NMAT, RG, EPI>(acc, (wg + cu_item * tw) * RG, N, p, lane, best_v, best_i,
-                                       h_old);
-            cu_st = 0;
-            ++cu_item;
+    };
+    if constexpr (WHOLE) {
+        // the cursor filled steps 0 .. kRing - 2 of item 0; in every step it
+        // fills one more, moving to the next item at step nst - (kRing - 1)
+        bool more = my_items > 0;
+        uint32_t cu = ring;
+        for (int il = 0; il < my_items; ++il) {
+            const int64_t r0 = (wg + il * tw) * RG;
+            const float h_old = residual_old<RG, EPI>(p, r0, N, lane);
+            const uint4* xp = xs + x_lane;
+            const float* sp = sums + lane;
+            for (int st = 0; st < nst; ++st) {
+                if (st == nst - (kRing - 1)) {
+                    if (il + 1 < my_items) set_item(il + 1);
+                    else more = false;
+                }
+                if (more) issue_whole();
+                cp_async_commit();
+                cp_async_wait<kRing - 1>();
+                __syncwarp();  // side pieces copied by other lanes are now visible
+                compute(cu, xp, FMT == 1 ? *sp : 0.f);
+                __syncwarp();  // every lane is done with this slot before it is refilled
+                xp += kXStep;
+                sp += kLanes;
+                cu = cu + kSlotBytes == ring_end ? ring : cu + kSlotBytes;
+            }
+            finish_item<NMAT, RG, EPI>(acc, r0, N, p, lane, best_v, best_i, h_old);
+        }
+    } else {
+        int cu_st = 0, cu_item = 0, cu_slot = 0;
+        float h_old = 0.f;
+        for (int t = 0; t < total; ++t) {
+            if (cu_st == 0) h_old = residual_old<RG, EPI>(p, (wg + cu_item * tw) * RG, N, lane);
+            if (t + kRing - 1 < total) issue();
+            else cp_async_commit();
+            cp_async_wait<kRing - 1>();
+            __syncwarp();  // side pieces copied by other lanes are now visible
+            const int g = cu_st * kLanes + lane;
+            if (g < granules) {
+                uint4 xv[F::kPieces];
+                const uint4* xp = xs + x_lane + cu_st * kXStep;
+#pragma unroll
+                for (int i = 0; i < F::kPieces; ++i) xv[i] = xp[i * 8];
+                const float c1 = FMT == 1 ? sums[g] : 0.f;
+#pragma unroll
+                for (int j = 0; j < ROWS; ++j) {
+                    const uint4 c = lds128(slot_codes(cu_slot, j));
+                    if (FMT == 2) {
+                        acc[j] += dot8_f16(c, xv);
+                        continue;
+                    }
+                    const float sc = h2f(lds16(slot_side(cu_slot, j, 0) + side_off));
+                    if (FMT == 0) {
+                        acc[j] = fmaf(sc, dot16_i8(c, xv), acc[j]);
+                    } else {
+                        const float bi = h2f(lds16(slot_side(cu_slot, j, 1) + side_off));
+                        acc[j] = i4_accumulate(acc[j], sc, bi, c, xv, c1);
+                    }
+                }
+            }
+            __syncwarp();  // every lane is done with this slot before it is refilled
+            if (++cu_slot == kRing) cu_slot = 0;
+            if (++cu_st == nst) {
+                finish_item<NMAT, RG, EPI>(acc, (wg + cu_item * tw) * RG, N, p, lane, best_v,
+                                           best_i, h_old);
+                cu_st = 0;
+                ++cu_item;
+            }
         }
     }
     cp_async_wait<0>();
@@ -888,13 +980,13 @@ __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem,
     return true;
 }
 
-template <int FMT, int NMAT, int RG, int EPI>
+template <int FMT, int NMAT, int RG, int EPI, bool WHOLE = false>
 __global__ void __launch_bounds__(kThreads, 2) gemv_ring_kernel(const Params p) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ float red_v[kWarps];
     __shared__ int red_i[kWarps];
     StreamSync sync;
-    ring_stage<FMT, NMAT, RG, EPI>(p, smem, sync, red_v, red_i);
+    ring_stage<FMT, NMAT, RG, EPI, WHOLE>(p, smem, sync, red_v, red_i);
 }
 
 // x's shared memory: the staged fp16 x, its per-granule sums, and the raw
@@ -917,24 +1009,58 @@ constexpr size_t ring_smem_bytes() {
 // Per-CTA shared memory that still lets two CTAs share an SM.
 constexpr size_t kSmemPerCtaBudget = 112 * 1024;
 
+// Rows of at least kWholeMinSteps whole warp steps (512 int8, 1024 int4 or
+// 256 fp16 codes) stream through the ring kernel's whole-step loop, which
+// drops the per-step bounds and item tests: about a fifth of the thread
+// instructions of a one-row-per-item launch (ncu, 2048x6144 int8: 8.1 -> 6.7
+// per weight).  Timed on B200 (graphs of every layer's launches, L2 flushed),
+// it shortened the down projections of the 2B / 4B / 8B / 27B decoders
+// 5.27 -> 4.90, 9.39 -> 8.65, 11.72 -> 10.87 and 24.2 -> 22.3 us and the 27B o
+// (12 steps) 7.92 -> 7.49 us, but lengthened rows of 4-8 steps (2B q|k|v 3.50
+// -> 3.97 us, 8B q|k|v 6.23 -> 7.30 us, 8B o 5.01 -> 5.75 us).
+constexpr int kWholeMinSteps = 12;
+inline bool whole_step_rows(int fmt, int64_t k) {
+    const int64_t step = static_cast<int64_t>(kLanes) *
+                         (fmt == 0 ? Fmt<0>::kCodesPerLane
+                                   : (fmt == 1 ? Fmt<1>::kCodesPerLane : Fmt<2>::kCodesPerLane));
+    return k % step == 0 && k / step >= kWholeMinSteps;
+}
+
 template <int FMT, int NMAT, int RG, int EPI, bool RING>
 qg_status launch_t(Params p, const DeviceInfo& dev, cudaStream_t stream) {
     void (*kern)(Params);  // only the chosen family is instantiated
+    int variant = 0;
     if constexpr (RING) {
-        kern = gemv_ring_kernel<FMT, NMAT, RG, EPI>;
+        if (whole_step_rows(FMT, p.k)) {
+            kern = gemv_ring_kernel<FMT, NMAT, RG, EPI, true>;
+            variant = 1;
+        } else {
+            kern = gemv_ring_kernel<FMT, NMAT, RG, EPI, false>;
+        }
     } else {
         kern = gemv_kernel<FMT, NMAT, RG, EPI>;
     }
     size_t smem = x_smem_bytes(FMT, p) + (RING ? ring_smem_bytes<FMT, NMAT, RG>() : 0);
     if (smem + 1024 > static_cast<size_t>(dev.max_smem_optin)) return QG_ERR_SHAPE;
+    if (variant == 1) {
+        // A whole-step kernel holds fewer registers than the general one (67
+        // against 90 for one int8 row per item), so a third CTA would fit on an
+        // SM, and launches chained by programmatic dependent launch then crowd
+        // the SMs that free first (2B down 4.90 -> 5.93 us).  Its shared-memory
+        // request is padded past a third of the SM's to keep kCtasPerSm per SM.
+        const size_t two_per_sm = (static_cast<size_t>(dev.smem_per_sm) / (kCtasPerSm + 1) + 16) /
+                                  16 * 16;
+        if (smem < two_per_sm && two_per_sm + 1024 <= static_cast<size_t>(dev.max_smem_optin))
+            smem = two_per_sm;
+    }
     // Opt in to exactly the dynamic shared memory this launch needs (static
     // shared memory counts against the same per-block limit).
-    static size_t attr_set[64] = {0};
-    if (dev.device >= 64 || attr_set[dev.device] < smem) {
+    static size_t attr_set[2][64] = {};  // per kernel variant and device
+    if (dev.device >= 64 || attr_set[variant][dev.device] < smem) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return cuda_status(e);
-        if (dev.device < 64) attr_set[dev.device] = smem;
+        if (dev.device < 64) attr_set[variant][dev.device] = smem;
     }
     const int64_t items = (p.n + RG - 1) / RG;
     int64_t grid = (items + kWarps - 1) / kWarps;

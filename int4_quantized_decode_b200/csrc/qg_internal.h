@@ -13,6 +13,7 @@ struct DeviceInfo {
     int device;
     int num_sms;
     int max_smem_optin;  // bytes of dynamic shared memory a CTA may opt into
+    int smem_per_sm;     // bytes of shared memory per SM
 };
 qg_status device_info(DeviceInfo* out);
 
