@@ -1009,16 +1009,16 @@ constexpr size_t ring_smem_bytes() {
 // Per-CTA shared memory that still lets two CTAs share an SM.
 constexpr size_t kSmemPerCtaBudget = 112 * 1024;
 
-// Rows of at least kWholeMinSteps whole warp steps (512 int8, 1024 int4 or
-// 256 fp16 codes) stream through the ring kernel's whole-step loop, which
+// Rows of whole warp steps (512 int8, 1024 int4 or 256 fp16 codes), at least
+// kRing - 1 of them, stream through the ring kernel's whole-step loop, which
 // drops the per-step bounds and item tests: about a fifth of the thread
 // instructions of a one-row-per-item launch (ncu, 2048x6144 int8: 8.1 -> 6.7
-// per weight).  Timed on B200 (graphs of every layer's launches, L2 flushed),
-// it shortened the down projections of the 2B / 4B / 8B / 27B decoders
-// 5.27 -> 4.90, 9.39 -> 8.65, 11.72 -> 10.87 and 24.2 -> 22.3 us and the 27B o
-// (12 steps) 7.92 -> 7.49 us, but lengthened rows of 4-8 steps (2B q|k|v 3.50
-// -> 3.97 us, 8B q|k|v 6.23 -> 7.30 us, 8B o 5.01 -> 5.75 us).
-constexpr int kWholeMinSteps = 12;
+// per weight).  Timed on B200 (graphs of every layer's launches, L2 flushed):
+// down projections of the 2B / 4B / 8B / 27B decoders 5.19 -> 4.83,
+// 9.34 -> 8.48, 11.72 -> 10.89 and 24.3 -> 22.7 us, then, for rows of 4-10
+// steps, 4B q|k|v 4.63 -> 4.55, o 4.67 -> 4.54, 8B q|k|v 6.20 -> 5.99, o
+// 4.99 -> 4.72, 8B int4 gate/up 17.6 -> 17.0 us.
+constexpr int kWholeMinSteps = kRing - 1;
 inline bool whole_step_rows(int fmt, int64_t k) {
     const int64_t step = static_cast<int64_t>(kLanes) *
                          (fmt == 0 ? Fmt<0>::kCodesPerLane
