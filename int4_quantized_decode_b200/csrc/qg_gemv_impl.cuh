@@ -699,6 +699,9 @@ struct GridSync {
 // scales (and biases) as 16-byte pieces, read by the warp after a __syncwarp.
 // Bytes in flight cost no registers: 3 steps x RG rows x 16 B per lane stay
 // outstanding.  Requires a multiple of 8 scales per row (16-byte pieces).
+// WHOLE selects the loop for rows of at least kRing - 1 whole steps (see
+// below); both loops add the same products in the same order, so the two
+// variants give bit-identical results.
 // Returns false, with its copies drained, if the wait for x gave up.
 template <int FMT, int NMAT, int RG, int EPI, bool WHOLE = false, class SYNC>
 __device__ __forceinline__ bool ring_stage(const Params& p, unsigned char* smem, SYNC& sync,
