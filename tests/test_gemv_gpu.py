@@ -22,12 +22,17 @@ SHAPES_I8 = [(1, 32), (7, 96), (33, 544), (300, 2048), (1000, 2080), (4103, 512)
              (2048, 6144), (9473, 2560), (20000, 1024), (64, 17408),
              # three rows per warp item would cut the busiest warp's rows, but their
              # ring does not fit beside this x: the launcher falls back to fewer rows
-             (6144, 17408)]
+             (6144, 17408),
+             # rows of exactly three whole steps (the whole-step loop's copy cursor
+             # moves to the next item at each item's first step), 3-4 items per warp
+             (30000, 1536)]
 SHAPES_I4 = [(1, 64), (9, 192), (41, 1088), (300, 2560), (1000, 1536), (4103, 1024),
              (20000, 2048), (64, 9728),
              # rows of 32 x + 16 lane granules with 2 and 4 rows per warp item
              # (the last step of each row pair packed into one warp step)
-             (4103, 2560), (6001, 1536), (3000, 9728)]
+             (4103, 2560), (6001, 1536), (3000, 9728),
+             # three whole int4 steps per row, 1-2 items per warp
+             (12000, 3072)]
 
 
 def _weight(fmt, n, k, seed, dev):
@@ -89,7 +94,8 @@ def test_gemv_one_hot_and_ones_closed_forms(cuda):
 
 @pytest.mark.parametrize("fmt,n,k", [(I8, 1, 32), (I8, 45, 2048), (I8, 6144, 2048),
                                      (I8, 3000, 2080), (I4, 77, 2560), (I4, 9728, 2560),
-                                     (I8, 17408, 5120), (I8, 6144, 12288)])
+                                     (I8, 17408, 5120), (I8, 6144, 12288), (I8, 9000, 1536),
+                                     (I4, 5000, 3072)])
 def test_gate_up_swiglu_s1(cuda, fmt, n, k):
     wg, Wg = _weight(fmt, n, k, 31, cuda)
     wu, Wu = _weight(fmt, n, k, 32, cuda)
